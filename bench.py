@@ -1,0 +1,481 @@
+#!/usr/bin/env python
+"""Benchmark of the context-sparse decode hot path on B200.
+
+Metric: sparse decode us/step and effective HBM GB/s at 50x sparsity vs dense
+decode ("Inference Time Context Sparsity: Illusion or Opportunity?",
+gist.science summary, section 3.C: sparse decode kernels against dense decode,
+traffic O(k d) instead of O(N d)).
+
+One step runs the whole path on one batch of the workload:
+  exact top-k indexer (score + select) -> sparse decode on the selected rows
+  -> dense decode on the same cache (the comparator),
+each leg bracketed by CUDA events on the launching stream, with a 256 MiB
+write (twice the 126 MB L2) before each leg so every leg reads from HBM.
+`value` is the sparse-decode leg (the metric); the other legs are reported
+beside it.  Multi-GPU runs are weak scaling: every rank decodes its own batch
+(no data-path collective), the timings are the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference] [--config NAME]
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode µs/step and effective HBM GB/s at 50× sparsity vs dense decode"
+UNIT = "µs/step"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["native", "reference"], default="native")
+    p.add_argument("--config", default="llama3_8b")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(cfg, k):
+    return {
+        "workload": f"{cfg.name}: {cfg.description}",
+        "batch": cfg.batch, "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": 128,
+        "context": cfg.max_seq_len, "k": k, "tokens_per_seq": cfg.tokens_per_seq,
+        "l2": "flushed before every timed leg (256 MiB device write)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# Clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for r in csv.reader(io.StringIO(self.out or "")):
+            if len(r) < 9:
+                continue
+            try:
+                rows.append([x.strip() for x in r])
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace('.', '', 1).isdigit())
+        smax = max((float(r[2]) for r in rows if r[2].replace('.', '', 1).isdigit()), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j].lower().startswith("active")})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# Helpers
+# ---------------------------------------------------------------------------
+def source_sha(name):
+    path = os.path.join(ROOT, "top_sparse_decode_topk_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str, source: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("source_sha") != source_sha(source):
+            return None
+        return float(e["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def unique_rows(idx, token_seq, hkv, group, max_len):
+    """Distinct (sequence, kv head, token) rows named by the index lists."""
+    import torch
+    T, Hq, K = idx.shape
+    b = token_seq.view(T, 1, 1).long()
+    g = (torch.arange(Hq, device=idx.device) // group).view(1, Hq, 1)
+    key = (b * hkv + g) * max_len + idx.long()
+    key = key[idx >= 0]
+    return int(torch.unique(key).numel())
+
+
+def time_cpu_oracle(w, k, budget_s=10.0):
+    """The oracle on the host cores: exact top-k plus sparse attention for a sample of
+    (sequence, kv head) groups, repeated until `budget_s`; extrapolated to the step."""
+    import numpy as np
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:
+        limiter = None
+    import oracle
+    cfg = w.cfg
+    G = cfg.group
+    scale = 1.0 / math.sqrt(128)
+    rng = np.random.default_rng(0)
+    groups = [(int(rng.integers(cfg.batch)), int(rng.integers(cfg.num_kv_heads))) for _ in range(2)]
+    data = []
+    for b, g in groups:
+        K = oracle.from_bf16_bits(w.logical_kv_bits(b, g, "k"))
+        V = oracle.from_bf16_bits(w.logical_kv_bits(b, g, "v"))
+        for t in range(int(w.q_indptr[b]), int(w.q_indptr[b + 1])):
+            L = int(w.kv_len[t])
+            for h in range(g * G, (g + 1) * G):
+                data.append((oracle.from_bf16_bits(w.q_bits[t, h]), K[:L], V[:L]))
+    nlists = len(data)
+    total_lists = len(w.kv_len) * cfg.num_q_heads
+    kk = w.k_per_token(k)
+    idxs = [oracle.exact_topk(oracle.attention_scores(q, Kb), int(kk[0])) for q, Kb, _ in data]
+    # top-k
+    t0 = time.perf_counter()
+    reps_topk = 0
+    while True:
+        for q, Kb, _ in data:
+            oracle.exact_topk(oracle.attention_scores(q, Kb), int(kk[0]))
+        reps_topk += 1
+        if time.perf_counter() - t0 > budget_s / 2:
+            break
+    topk_s = (time.perf_counter() - t0) / reps_topk
+    # sparse attention over the selected lists
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for (q, Kb, Vb), ix in zip(data, idxs):
+            oracle.sparse_attention(q, Kb, Vb, ix, scale)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s / 2:
+            break
+    sparse_s = (time.perf_counter() - t0) / reps
+    f = total_lists / nlists
+    return {
+        "sparse_us_per_step": sparse_s * f * 1e6,
+        "topk_us_per_step": topk_s * f * 1e6,
+        "cores": 1,
+        "sample": f"{nlists} of {total_lists} (token, head) lists ({len(groups)} (sequence, kv head) groups), "
+                  f"{reps} repetitions of the sparse attention and {reps_topk} of the top-k in "
+                  f"~{budget_s:.0f} s, extrapolated linearly to the full step",
+    }
+
+
+# ---------------------------------------------------------------------------
+# Native arm
+# ---------------------------------------------------------------------------
+def run_native(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import top_sparse_decode_topk_b200 as tsd
+    from top_sparse_decode_topk_b200 import workload as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from top_sparse_decode_topk_b200.build import build
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    tsd.load_library()
+
+    cfg = W.CONFIGS[args.config]
+    k = cfg.ks[0] if cfg.ks else None
+    w = W.make_workload(cfg, seed=rank)
+    dw = W.to_device(w, dev)
+    contiguous = cfg.layout == "contiguous"
+    cache = tsd.KVCache(dw.k, dw.v, dw.seq_lens, max_seq_len=cfg.max_seq_len,
+                        page_table=None if contiguous else dw.page_table)
+    multi = cfg.tokens_per_seq > 1
+    scale = 1.0 / math.sqrt(128)
+    queries = tsd.Queries(dw.q, q_indptr=dw.q_indptr if multi else None, max_tokens_per_seq=cfg.tokens_per_seq,
+                          causal=cfg.causal, sm_scale=scale)
+    kpt = w.k_per_token(k)
+    k_max = int(kpt.max())
+    kpt_dev = None if k is not None else torch.from_numpy(kpt).to(dev)
+    out_dtype = torch.float32 if cfg.out_dtype == "f32" else torch.bfloat16
+    ws = tsd.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    idx_buf = torch.empty((len(w.kv_len), cfg.num_q_heads, k_max), dtype=torch.int32, device=dev)
+    cnt_buf = torch.empty((len(w.kv_len), cfg.num_q_heads), dtype=torch.int32, device=dev)
+
+    def leg_topk():
+        tsd.topk_select(cache, queries, k_max, k_per_token=kpt_dev, out_idx=idx_buf, out_count=cnt_buf, workspace=ws)
+
+    def leg_sparse():
+        return tsd.sparse_decode(cache, queries, idx_buf, out_dtype=out_dtype, workspace=ws)
+
+    def leg_dense():
+        return tsd.dense_decode(cache, queries, out_dtype=out_dtype, workspace=ws)
+
+    legs = [leg_topk, leg_sparse, leg_dense]
+    for _ in range(max(3, args.warmup)):
+        for leg in legs:
+            flush.fill_(1)
+            leg()
+    torch.cuda.synchronize()
+    if tsd.read_device_status(ws) != 0:
+        raise RuntimeError("device status bits set during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for s in range(args.steps):
+            for j, leg in enumerate(legs):
+                flush.fill_(1)
+                ev[s][2 * j].record(stream)
+                leg()
+                ev[s][2 * j + 1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = np.array([[ev[s][2 * j].elapsed_time(ev[s][2 * j + 1]) for j in range(3)] for s in range(args.steps)])
+    mean_ms = ms.mean(axis=0)
+    t = torch.tensor(mean_ms.tolist(), dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    topk_ms, sparse_ms, dense_ms = t.tolist()
+
+    # algorithmic bytes (per rank; every rank has the same shapes)
+    T, Hq, Hkv, G = len(w.kv_len), cfg.num_q_heads, cfg.num_kv_heads, cfg.group
+    U = unique_rows(idx_buf, torch.from_numpy(w.token_seq).to(dev), Hkv, G, cfg.max_seq_len)
+    entries = int((idx_buf >= 0).sum().item())
+    out_bytes = 4 if out_dtype == torch.float32 else 2
+    q_bytes = T * Hq * 128 * 2
+    o_bytes = T * Hq * 128 * out_bytes
+    sparse_bytes = U * 512 + q_bytes + o_bytes
+    ctx_rows = int(sum(int(L) for L in w.seq_lens)) * Hkv
+    dense_bytes = ctx_rows * 512 + q_bytes + o_bytes
+    topk_bytes = ctx_rows * 256 + q_bytes + T * Hq * k_max * 4
+    index_bytes = T * Hq * k_max * 4
+    hbm, peak_kind = peaks()
+    gbs = lambda b, ms_: b / (ms_ * 1e-3) / 1e9
+    sparse_gbs, dense_gbs, topk_gbs = gbs(sparse_bytes, sparse_ms), gbs(dense_bytes, dense_ms), gbs(topk_bytes, topk_ms)
+
+    # end to end through the public API with pinned host buffers
+    q_host = dw.q.cpu().pin_memory()
+    idx_host = idx_buf.cpu().pin_memory()
+    out_host = torch.empty((T, Hq, 128), dtype=out_dtype).pin_memory()
+    lse_host = torch.empty((T, Hq), dtype=torch.float32).pin_memory()
+    hq = tsd.Queries(q_host, q_indptr=dw.q_indptr if multi else None, max_tokens_per_seq=cfg.tokens_per_seq,
+                     causal=cfg.causal, sm_scale=scale)
+    e2e_ms, e2e_idx_ms = [], []
+    for s in range(args.warmup + args.steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        tsd.sparse_decode(cache, hq, idx_host, out=out_host, lse=lse_host, workspace=ws)
+        b.record(stream)
+        flush.fill_(1)
+        c, d = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c.record(stream)
+        idx_d, _ = tsd.topk_select(cache, hq, k_max, k_per_token=kpt_dev, out_idx=idx_buf, out_count=cnt_buf,
+                                   workspace=ws)
+        tsd.sparse_decode(cache, hq, idx_d, out=out_host, lse=lse_host, workspace=ws)
+        d.record(stream)
+        torch.cuda.synchronize()
+        if s >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+            e2e_idx_ms.append(c.elapsed_time(d))
+    e = torch.tensor([float(np.mean(e2e_ms)), float(np.mean(e2e_idx_ms))], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e, op=dist.ReduceOp.MAX)
+    e2e_us, e2e_idx_us = (x * 1e3 for x in e.tolist())
+    if tsd.read_device_status(ws) != 0:
+        raise RuntimeError("device status bits set during the timed run")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_cpu_oracle(w, k)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    cl = clocks.summary()
+    traffic = ncu_traffic("sparse_decode_kernel", cfg.name, "tsd_decode.cu")
+    line = {
+        "metric": METRIC,
+        "value": round(sparse_ms * 1e3, 3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(topk_ms + sparse_ms + dense_ms, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "storage_dtype": "bf16",
+        "data": "synthetic (seeded Philox N(0,1) bf16 K/V/q with planted needles/sink/window)"
+                if cfg.planted else "synthetic (seeded Philox N(0,1) bf16 K/V/q)",
+        "config": workload_desc(cfg, k_max),
+        "legs_us": {"topk_select": round(topk_ms * 1e3, 3), "sparse_decode": round(sparse_ms * 1e3, 3),
+                    "dense_decode": round(dense_ms * 1e3, 3)},
+        "effective_gbs": round(sparse_gbs, 1),
+        "speedup_vs_dense": round(dense_ms / sparse_ms, 3),
+        "speedup_vs_dense_with_indexer": round(dense_ms / (sparse_ms + topk_ms), 3),
+        "roofline": {"bound": "hbm", "achieved": round(sparse_gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(sparse_gbs / hbm, 4), "traffic": traffic,
+                     "kernel": "sparse_decode_kernel", "peak_source": f"{peak_kind} copy bandwidth",
+                     "frac_of_nominal_8tbs": round(sparse_gbs / NOMINAL_HBM_GBS, 4),
+                     "algorithmic_bytes": sparse_bytes, "unique_rows": U, "entries": entries,
+                     "index_bytes_not_counted": index_bytes},
+        "rooflines_other": {
+            "topk_select": {"achieved": round(topk_gbs, 1), "frac": round(topk_gbs / hbm, 4),
+                            "algorithmic_bytes": topk_bytes, "kernels": ["topk_score_kernel", "topk_select_kernel"]},
+            "dense_decode": {"achieved": round(dense_gbs, 1), "frac": round(dense_gbs / hbm, 4),
+                             "algorithmic_bytes": dense_bytes, "kernels": ["dense_decode_kernel"]},
+        },
+        "e2e": {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": q_bytes + index_bytes,
+                "d2h_bytes_per_step": o_bytes + T * Hq * 4,
+                "what": "tsd.sparse_decode with pinned host q and index lists in, host out and lse back"},
+        "e2e_with_indexer": {"value": round(e2e_idx_us, 3), "unit": UNIT, "h2d_bytes_per_step": q_bytes,
+                             "d2h_bytes_per_step": o_bytes + T * Hq * 4,
+                             "what": "host q in -> topk_select -> sparse_decode -> host out and lse"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": cl,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = {"value": round(cpu["sparse_us_per_step"], 1), "unit": UNIT, "cores": cpu["cores"],
+                                "kind": "oracle", "sample": cpu["sample"],
+                                "topk_us_per_step": round(cpu["topk_us_per_step"], 1)}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the CPU oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from top_sparse_decode_topk_b200 import workload as W
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:
+        pass
+    cfg = W.CONFIGS[args.config]
+    k = cfg.ks[0] if cfg.ks else None
+    w = W.make_workload(cfg, seed=0)
+    G = cfg.group
+    scale = 1.0 / math.sqrt(128)
+    rng = np.random.default_rng(0)
+    groups = [(int(rng.integers(cfg.batch)), int(rng.integers(cfg.num_kv_heads))) for _ in range(2)]
+    kk = w.k_per_token(k)
+    data = []
+    for b, g in groups:
+        K = oracle.from_bf16_bits(w.logical_kv_bits(b, g, "k"))
+        V = oracle.from_bf16_bits(w.logical_kv_bits(b, g, "v"))
+        for t in range(int(w.q_indptr[b]), int(w.q_indptr[b + 1])):
+            L = int(w.kv_len[t])
+            for h in range(g * G, (g + 1) * G):
+                q = oracle.from_bf16_bits(w.q_bits[t, h])
+                idx = oracle.exact_topk(oracle.attention_scores(q, K[:L]), int(kk[t]))
+                data.append((q, K[:L], V[:L], idx))
+    total = len(w.kv_len) * cfg.num_q_heads
+    f = total / len(data)
+    times = []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        for q, Kb, Vb, idx in data:
+            oracle.sparse_attention(q, Kb, Vb, idx, scale)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt * f * 1e6)
+    v = float(np.mean(times))
+    sample = (f"{len(data)} of {total} (token, head) lists ({len(groups)} (sequence, kv head) groups) per step, "
+              f"extrapolated linearly to the full step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1e3, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_desc(cfg, int(kk.max())),
+        "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

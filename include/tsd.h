@@ -1,0 +1,183 @@
+/*
+ * tsd.h -- C ABI of the B200 context-sparse decode attention library (libtsd.so).
+ *
+ * The operations come from "Inference Time Context Sparsity: Illusion or
+ * Opportunity?" (gist.science technical summary, section 2 "Oracle Top-K" and
+ * "Hardware implementation", section 3.C "Kernel speed-ups" and "Bandwidth
+ * efficiency"):
+ *   - tsd_topk_select : exact top-k token selection per (query token, q head)
+ *                       over the whole KV cache ("Oracle Top-K");
+ *   - tsd_sparse_decode: decode attention that reads only the selected K/V rows,
+ *                       which may differ per token, per query and per head
+ *                       (traffic O(k d) instead of O(N d));
+ *   - tsd_dense_decode : the dense decode attention it is measured against
+ *                       (O(N d) traffic).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers are DEVICE pointers unless the comment says "host".  The caller
+ *    owns every buffer; the library allocates nothing and keeps no state
+ *    between calls.  Calls are asynchronous on the given stream.
+ *  - head_dim must be 128.  num_q_heads must be a multiple of num_kv_heads;
+ *    q head h reads kv head h / (num_q_heads / num_kv_heads).
+ *  - Host-checkable errors return a status without launching anything.
+ *    Problems only the device can see (an index outside [0, kv_len), a list
+ *    that is not ascending, a page id outside [0, num_pages), a sequence length
+ *    above max_seq_len) never fault: the offending entry is skipped and a bit is
+ *    OR-ed into the status word at the start of the workspace; read it with
+ *    tsd_read_device_status.
+ *  - Workspace: each call takes (ws, ws_bytes) of at least the size returned by
+ *    the matching *_workspace_size function.  Its first part must be zero when a
+ *    call starts; every call leaves it zero again, so zero it once (cudaMemset or
+ *    tsd_workspace_init) after allocating it and again whenever the cache or
+ *    query shape changes.  Calls that share a workspace must not overlap in time.
+ *  - Thread safety: calls with distinct workspaces may run concurrently.
+ */
+#ifndef TSD_H_
+#define TSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tsd_stream_t; /* same type as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  TSD_OK = 0,
+  TSD_ERR_INVALID_ARGUMENT = 1,    /* null pointer, negative size, inconsistent shape */
+  TSD_ERR_UNSUPPORTED = 2,         /* head_dim != 128, page_size not a power of two, dtype */
+  TSD_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_size result */
+  TSD_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+  TSD_ERR_DEVICE_STATUS = 5        /* returned by tsd_read_device_status when a bit is set */
+} tsd_status;
+
+typedef enum { TSD_BF16 = 0, TSD_F32 = 1 } tsd_dtype;
+
+/* Bits of the device status word. */
+enum {
+  TSD_DEV_BAD_INDEX = 1u << 0, /* an index entry was < -1 or >= kv_len of its query; skipped */
+  TSD_DEV_UNSORTED = 1u << 1,  /* an index list was not ascending where it was read          */
+  TSD_DEV_BAD_PAGE = 1u << 2,  /* a page-table entry was outside [0, num_pages); row skipped */
+  TSD_DEV_BAD_SEQ = 1u << 3    /* seq_len outside [0, max_seq_len] or a bad q_indptr; the
+                                  affected sequence is treated as empty                      */
+};
+
+typedef enum {
+  /* k, v: [num_pages][num_kv_heads][page_size][head_dim] bf16 ("HND" pages).
+     Token i of sequence b lives in page page_table[b * max_pages_per_seq + i / page_size],
+     slot i % page_size.  page_size must be a power of two. */
+  TSD_LAYOUT_PAGED = 0,
+  /* k, v: [batch][num_kv_heads][max_seq_len][head_dim] bf16; page_table must be NULL. */
+  TSD_LAYOUT_CONTIGUOUS = 1
+} tsd_layout;
+
+/* A bf16 KV cache. */
+typedef struct {
+  const void* k;               /* device, bf16, layout above */
+  const void* v;               /* device, bf16, same layout as k */
+  int32_t layout;              /* tsd_layout */
+  int32_t num_kv_heads;        /* Hkv >= 1 */
+  int32_t head_dim;            /* must be 128 */
+  int32_t page_size;           /* paged: power of two >= 1; contiguous: ignored */
+  const int32_t* page_table;   /* device int32 [batch][max_pages_per_seq] (paged), else NULL */
+  int32_t max_pages_per_seq;   /* paged: >= ceil(max_seq_len / page_size) */
+  int64_t num_pages;           /* paged: number of physical pages in k and v */
+  const int32_t* seq_lens;     /* device int32 [batch]: tokens cached per sequence */
+  int32_t batch;               /* number of sequences B >= 1 */
+  int32_t max_seq_len;         /* host bound on every seq_lens[b] (>= 1) */
+} tsd_kv_cache;
+
+/* The decode queries of one step. */
+typedef struct {
+  const void* q;               /* device [num_tokens][num_q_heads][head_dim], q_dtype */
+  int32_t q_dtype;             /* TSD_BF16 or TSD_F32 */
+  int32_t num_q_heads;         /* Hq, a multiple of num_kv_heads */
+  int32_t num_tokens;          /* T: query tokens over all sequences */
+  const int32_t* q_indptr;     /* device int32 [batch+1]: tokens of sequence b are
+                                  q_indptr[b] .. q_indptr[b+1]-1; NULL means one token per
+                                  sequence (T == batch) */
+  int32_t max_tokens_per_seq;  /* host bound on q_indptr[b+1]-q_indptr[b] (1 when q_indptr is NULL) */
+  int32_t causal;              /* nonzero: token j of the n_b tokens of sequence b sees
+                                  kv_len = seq_lens[b] - n_b + j + 1 tokens; zero: it sees
+                                  all seq_lens[b] tokens */
+  float sm_scale;              /* softmax scale, usually 1/sqrt(head_dim) */
+} tsd_queries;
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t tsd_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* tsd_status_string(tsd_status s);
+
+/* Zero `bytes` bytes of a workspace on `stream` (cudaMemsetAsync). */
+tsd_status tsd_workspace_init(void* ws, size_t bytes, tsd_stream_t stream);
+
+/* Host: bytes of workspace tsd_topk_select needs for these shapes (0 on invalid input). */
+size_t tsd_topk_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max);
+
+/*
+ * Exact top-k token selection ("Oracle Top-K", pages section 2).
+ * For each query token t (of sequence b) and q head h (kv head g):
+ *   s_i = sum_d q[t,h,d] * K[b,g,i,d], accumulated in fp32 from bf16 inputs, for i < kv_len(t);
+ *   keep the k_t = min(k, kv_len(t)) tokens with the largest s_i, ties to the lower index,
+ *   where k = k_per_token[t] if k_per_token is non-NULL, else k_max (k_per_token[t] is
+ *   clamped to [0, k_max]).  The softmax scale is not applied (it does not change the order).
+ * out_idx  : device int32 [T][Hq][k_max]; the k_t kept token indices in ascending order,
+ *            then -1 up to k_max.
+ * out_count: device int32 [T][Hq] or NULL; receives k_t.
+ * k_max >= 1.  Errors: INVALID_ARGUMENT, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA.
+ */
+tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                           const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count,
+                           void* ws, size_t ws_bytes, tsd_stream_t stream);
+
+/* Host: bytes of workspace tsd_sparse_decode needs for these shapes (0 on invalid input). */
+size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries,
+                                        int32_t k_max);
+
+/*
+ * Sparse decode attention over per-(token, head) index lists (pages section 2,
+ * "Hardware implementation"; section 3.C).  For each query token t and q head h:
+ *   z_i = sm_scale * q[t,h] . K[b,g,i]   for every entry i of idx[t][h][0..k_max)
+ *   out[t,h] = sum_i exp(z_i - M) V[b,g,i] / sum_i exp(z_i - M),   M = max_i z_i
+ *   lse[t,h] = M + ln sum_i exp(z_i - M)       (natural log of the scaled scores)
+ * idx: device int32 [T][Hq][k_max].  Each list holds token indices in non-decreasing order
+ *   (as tsd_topk_select writes them), followed by -1 padding; every entry is one term, so a
+ *   repeated token counts once per occurrence.  Entries >= kv_len(t) or < -1 are skipped and
+ *   set TSD_DEV_BAD_INDEX; an observed descending pair sets TSD_DEV_UNSORTED (the result for
+ *   such a list is unspecified).  Rows shared by several lists of one kv head (the q heads of a
+ *   GQA group and the query tokens of one sequence) are loaded from memory once.
+ * out: device [T][Hq][128] of out_dtype (TSD_BF16 or TSD_F32).  An empty list gives zeros.
+ * lse: device f32 [T][Hq] or NULL; -inf for an empty list.
+ */
+tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queries,
+                             const int32_t* idx, int32_t k_max, void* out, int32_t out_dtype,
+                             float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream);
+
+/* Host: bytes of workspace tsd_dense_decode needs for these shapes (0 on invalid input). */
+size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries);
+
+/*
+ * Dense decode attention (the baseline of pages section 3.C): tsd_sparse_decode with the
+ * list {0, 1, ..., kv_len(t)-1} for every (t, h), streamed page by page.
+ * out, lse: as tsd_sparse_decode.
+ */
+tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* queries, void* out,
+                            int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                            tsd_stream_t stream);
+
+/*
+ * Copy the device status word of `ws` to *flags (host), clear it, and synchronize `stream`.
+ * Returns TSD_OK when no bit was set, TSD_ERR_DEVICE_STATUS when one was, TSD_ERR_CUDA on a
+ * CUDA failure.
+ */
+tsd_status tsd_read_device_status(void* ws, tsd_stream_t stream, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSD_H_ */

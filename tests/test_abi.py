@@ -1,0 +1,150 @@
+"""The C-ABI library without a GPU: it loads, exports what include/tsd.h declares,
+and rejects bad arguments on the host before launching anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import top_sparse_decode_topk_b200 as tsd
+from top_sparse_decode_topk_b200 import _KvCacheC, _QueriesC
+from top_sparse_decode_topk_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tsd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return tsd.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tsd_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_path(lib):
+    names = declared_functions()
+    for need in ("tsd_topk_select", "tsd_sparse_decode", "tsd_dense_decode", "tsd_read_device_status"):
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # the binding declares the same set
+    assert set(declared_functions()) == set(tsd.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.tsd_version() >= 100
+    assert tsd.status_string(0) == "TSD_OK"
+    assert tsd.status_string(3) == "TSD_ERR_WORKSPACE_TOO_SMALL"
+    assert tsd.status_string(99) == "TSD_UNKNOWN_STATUS"
+
+
+FAKE = 0x7F0000000000   # 256-byte aligned, never dereferenced by the host checks
+
+
+def make_cache(**kw):
+    c = _KvCacheC()
+    c.k, c.v = FAKE, FAKE + 0x100000
+    c.layout = kw.get("layout", 0)
+    c.num_kv_heads = kw.get("hkv", 8)
+    c.head_dim = kw.get("head_dim", 128)
+    c.page_size = kw.get("page_size", 16)
+    c.page_table = kw.get("page_table", FAKE + 0x200000)
+    c.max_pages_per_seq = kw.get("max_pages", 2048)
+    c.num_pages = kw.get("num_pages", 8 * 2048)
+    c.seq_lens = FAKE + 0x300000
+    c.batch = kw.get("batch", 8)
+    c.max_seq_len = kw.get("max_seq_len", 32768)
+    return c
+
+
+def make_queries(**kw):
+    q = _QueriesC()
+    q.q = kw.get("q", FAKE + 0x400000)
+    q.q_dtype = kw.get("q_dtype", 0)
+    q.num_q_heads = kw.get("hq", 32)
+    q.num_tokens = kw.get("tokens", 8)
+    q.q_indptr = kw.get("q_indptr", None)
+    q.max_tokens_per_seq = kw.get("max_tokens", 1)
+    q.causal = 1
+    q.sm_scale = kw.get("sm_scale", 0.088)
+    return q
+
+
+def sparse(lib, c, q, k_max=655, ws_bytes=1 << 40, out_dtype=0, idx=FAKE + 0x500000):
+    return lib.tsd_sparse_decode(ctypes.byref(c), ctypes.byref(q), idx, k_max, FAKE + 0x600000, out_dtype,
+                                 None, FAKE + 0x700000, ws_bytes, None)
+
+
+def test_workspace_sizes(lib):
+    c, q = make_cache(), make_queries()
+    s1 = lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 655)
+    s2 = lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 13107)
+    d = lib.tsd_dense_decode_workspace_size(ctypes.byref(c), ctypes.byref(q))
+    t = lib.tsd_topk_workspace_size(ctypes.byref(c), ctypes.byref(q), 655)
+    assert 0 < s1 <= s2 and d > 0
+    # top-k holds one fp32 score per (token, head, position)
+    assert t >= 8 * 32 * 32768 * 4
+    bad = make_cache(head_dim=64)
+    assert lib.tsd_sparse_decode_workspace_size(ctypes.byref(bad), ctypes.byref(q), 655) == 0
+    assert lib.tsd_topk_workspace_size(ctypes.byref(c), ctypes.byref(q), 0) == 0
+
+
+@pytest.mark.parametrize("mutate,status", [
+    (dict(head_dim=64), tsd.TSD_ERR_UNSUPPORTED),
+    (dict(page_size=24), tsd.TSD_ERR_UNSUPPORTED),
+    (dict(hkv=5), tsd.TSD_ERR_INVALID_ARGUMENT),        # 32 % 5 != 0
+    (dict(batch=0), tsd.TSD_ERR_INVALID_ARGUMENT),
+    (dict(max_pages=10), tsd.TSD_ERR_INVALID_ARGUMENT),  # 10 * 16 < max_seq_len
+    (dict(layout=7), tsd.TSD_ERR_INVALID_ARGUMENT),
+    (dict(page_table=None), tsd.TSD_ERR_INVALID_ARGUMENT),
+])
+def test_cache_errors_before_launch(lib, mutate, status):
+    assert sparse(lib, make_cache(**mutate), make_queries()) == status
+
+
+@pytest.mark.parametrize("mutate,status", [
+    (dict(tokens=7), tsd.TSD_ERR_INVALID_ARGUMENT),      # no q_indptr: T must equal batch
+    (dict(q_dtype=9), tsd.TSD_ERR_UNSUPPORTED),
+    (dict(sm_scale=0.0), tsd.TSD_ERR_INVALID_ARGUMENT),
+    (dict(q=FAKE + 8), tsd.TSD_ERR_INVALID_ARGUMENT),    # misaligned rows
+    (dict(q=None), tsd.TSD_ERR_INVALID_ARGUMENT),
+])
+def test_query_errors_before_launch(lib, mutate, status):
+    assert sparse(lib, make_cache(), make_queries(**mutate)) == status
+
+
+def test_other_errors_before_launch(lib):
+    c, q = make_cache(), make_queries()
+    assert sparse(lib, c, q, ws_bytes=1024) == tsd.TSD_ERR_WORKSPACE_TOO_SMALL
+    assert sparse(lib, c, q, k_max=0) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert sparse(lib, c, q, idx=None) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert sparse(lib, c, q, out_dtype=5) == tsd.TSD_ERR_UNSUPPORTED
+    assert lib.tsd_sparse_decode(None, ctypes.byref(q), FAKE, 8, FAKE, 0, None, FAKE, 1 << 40, None) == \
+        tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_dense_decode(ctypes.byref(c), ctypes.byref(q), FAKE, 0, None, FAKE, 16, None) == \
+        tsd.TSD_ERR_WORKSPACE_TOO_SMALL
+    assert lib.tsd_topk_select(ctypes.byref(c), ctypes.byref(q), 655, None, FAKE, None, FAKE, 16, None) == \
+        tsd.TSD_ERR_WORKSPACE_TOO_SMALL
+    assert lib.tsd_topk_select(ctypes.byref(c), ctypes.byref(q), 655, None, None, None, FAKE, 1 << 40, None) == \
+        tsd.TSD_ERR_INVALID_ARGUMENT
+    flags = ctypes.c_uint32(0)
+    assert lib.tsd_read_device_status(None, None, ctypes.byref(flags)) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_workspace_init(None, 0, None) == tsd.TSD_OK
+    assert lib.tsd_workspace_init(None, 16, None) == tsd.TSD_ERR_INVALID_ARGUMENT
+
+
+def test_multi_token_queries_need_bounds(lib):
+    c = make_cache(batch=32)
+    q = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=0)
+    assert sparse(lib, c, q) == tsd.TSD_ERR_INVALID_ARGUMENT
+    q = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=4)
+    assert lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 2622) > 0

@@ -1,0 +1,414 @@
+"""B200-native context-sparse decode attention: exact top-k indexer + sparse decode.
+
+Thin Python binding over the C ABI of ``libtsd.so`` (include/tsd.h).  Every
+step of the attention path runs in the library's CUDA kernels; this module only
+marshals arguments (torch tensors -> device pointers, shapes, the stream) and
+moves host tensors to and from the device when a caller passes them.  PyTorch
+supplies device memory and streams.
+
+The operations follow "Inference Time Context Sparsity: Illusion or
+Opportunity?" (gist.science technical summary, section 2 "Oracle Top-K" and
+"Hardware implementation", section 3.C):
+
+    idx, count = topk_select(cache, queries, k_max)     # exact top-k per (token, head)
+    out, lse   = sparse_decode(cache, queries, idx)      # attention over the kept rows
+    out, lse   = dense_decode(cache, queries)            # attention over every row
+
+There is no fallback: if ``libtsd.so`` is missing or a call fails, an
+exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+__all__ = [
+    "KVCache", "Queries", "Workspace", "TsdError", "topk_select", "sparse_decode", "dense_decode",
+    "read_device_status", "library_path", "load_library", "DEV_BAD_INDEX", "DEV_UNSORTED",
+    "DEV_BAD_PAGE", "DEV_BAD_SEQ",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+
+TSD_OK, TSD_ERR_INVALID_ARGUMENT, TSD_ERR_UNSUPPORTED = 0, 1, 2
+TSD_ERR_WORKSPACE_TOO_SMALL, TSD_ERR_CUDA, TSD_ERR_DEVICE_STATUS = 3, 4, 5
+TSD_BF16, TSD_F32 = 0, 1
+LAYOUT_PAGED, LAYOUT_CONTIGUOUS = 0, 1
+DEV_BAD_INDEX, DEV_UNSORTED, DEV_BAD_PAGE, DEV_BAD_SEQ = 1, 2, 4, 8
+
+
+class TsdError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class _KvCacheC(ctypes.Structure):
+    _fields_ = [
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("layout", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("page_table", ctypes.c_void_p), ("max_pages_per_seq", ctypes.c_int32),
+        ("num_pages", ctypes.c_int64), ("seq_lens", ctypes.c_void_p), ("batch", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32),
+    ]
+
+
+class _QueriesC(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("q_dtype", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+        ("num_tokens", ctypes.c_int32), ("q_indptr", ctypes.c_void_p),
+        ("max_tokens_per_seq", ctypes.c_int32), ("causal", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+    ]
+
+
+EXPORTS = {
+    "tsd_version": (ctypes.c_int32, []),
+    "tsd_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "tsd_workspace_init": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tsd_topk_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32]),
+    "tsd_topk_select": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_size_t, ctypes.c_void_p]),
+    "tsd_sparse_decode_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
+                                                           ctypes.c_int32]),
+    "tsd_sparse_decode": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_void_p,
+                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tsd_dense_decode_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC)]),
+    "tsd_dense_decode": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_void_p,
+                                        ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                        ctypes.c_void_p]),
+    "tsd_read_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+}
+
+_LIB = None
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libtsd.so")
+
+
+def load_library():
+    """Load libtsd.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing; build it with `python -m top_sparse_decode_topk_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in EXPORTS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def status_string(s: int) -> str:
+    return load_library().tsd_status_string(int(s)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != TSD_OK:
+        raise TsdError(status, what)
+
+
+# ---------------------------------------------------------------------------
+# Descriptors
+# ---------------------------------------------------------------------------
+@dataclass
+class KVCache:
+    """A bf16 KV cache on one CUDA device.
+
+    paged:      k, v [num_pages, num_kv_heads, page_size, 128]; page_table int32 [B, max_pages];
+    contiguous: k, v [B, num_kv_heads, max_seq_len, 128]; page_table None.
+    seq_lens: int32 [B] on the device; max_seq_len: host bound on every entry.
+    """
+    k: "object"
+    v: "object"
+    seq_lens: "object"
+    max_seq_len: int
+    page_table: "object" = None
+
+    def __post_init__(self):
+        import torch
+        if self.k.dtype != torch.bfloat16 or self.v.dtype != torch.bfloat16:
+            raise TypeError("k and v must be bfloat16")
+        if self.k.dim() != 4 or self.k.shape != self.v.shape or self.k.shape[-1] != 128:
+            raise ValueError("k and v must have the same 4-d shape with head_dim 128")
+        if not (self.k.is_contiguous() and self.v.is_contiguous()):
+            raise ValueError("k and v must be contiguous")
+        if self.seq_lens.dtype != torch.int32 or self.seq_lens.device != self.k.device:
+            raise ValueError("seq_lens must be int32 on the cache's device")
+        if self.page_table is None and int(self.max_seq_len) != int(self.k.shape[2]):
+            raise ValueError("contiguous cache: max_seq_len must equal k.shape[2] (the token stride)")
+        if self.page_table is not None:
+            if self.page_table.dtype != torch.int32 or self.page_table.dim() != 2:
+                raise ValueError("page_table must be an int32 [batch, max_pages] tensor")
+            self.page_table = self.page_table.contiguous()
+
+    @property
+    def device(self):
+        return self.k.device
+
+    @property
+    def batch(self) -> int:
+        return int(self.seq_lens.shape[0])
+
+    @property
+    def num_kv_heads(self) -> int:
+        return int(self.k.shape[1])
+
+    def c_struct(self) -> _KvCacheC:
+        c = _KvCacheC()
+        c.k = self.k.data_ptr()
+        c.v = self.v.data_ptr()
+        c.num_kv_heads = self.num_kv_heads
+        c.head_dim = int(self.k.shape[3])
+        c.seq_lens = self.seq_lens.data_ptr()
+        c.batch = self.batch
+        c.max_seq_len = int(self.max_seq_len)
+        if self.page_table is None:
+            c.layout = LAYOUT_CONTIGUOUS
+            c.page_size = int(self.k.shape[2])
+            c.page_table = None
+            c.max_pages_per_seq = 1
+            c.num_pages = int(self.k.shape[0])
+        else:
+            c.layout = LAYOUT_PAGED
+            c.page_size = int(self.k.shape[2])
+            c.page_table = self.page_table.data_ptr()
+            c.max_pages_per_seq = int(self.page_table.shape[1])
+            c.num_pages = int(self.k.shape[0])
+        return c
+
+
+@dataclass
+class Queries:
+    """Decode queries q [T, Hq, 128] (bf16 or fp32).
+
+    q_indptr (int32 [B+1] on the device) gives the tokens of each sequence; None
+    means one token per sequence.  max_tokens_per_seq bounds q_indptr's gaps.
+    """
+    q: "object"
+    q_indptr: "object" = None
+    max_tokens_per_seq: int = 1
+    causal: bool = True
+    sm_scale: Optional[float] = None
+
+    def c_struct(self) -> _QueriesC:
+        import torch
+        if self.q.dim() != 3 or self.q.shape[-1] != 128 or not self.q.is_contiguous():
+            raise ValueError("q must be a contiguous [T, Hq, 128] tensor")
+        if self.q.dtype not in (torch.bfloat16, torch.float32):
+            raise TypeError("q must be bfloat16 or float32")
+        c = _QueriesC()
+        c.q = self.q.data_ptr()
+        c.q_dtype = TSD_BF16 if self.q.dtype == torch.bfloat16 else TSD_F32
+        c.num_q_heads = int(self.q.shape[1])
+        c.num_tokens = int(self.q.shape[0])
+        c.q_indptr = None if self.q_indptr is None else self.q_indptr.data_ptr()
+        c.max_tokens_per_seq = 1 if self.q_indptr is None else int(self.max_tokens_per_seq)
+        c.causal = 1 if self.causal else 0
+        c.sm_scale = float(self.sm_scale if self.sm_scale is not None else 1.0 / math.sqrt(128))
+        return c
+
+
+class Workspace:
+    """Device scratch for the library calls (zero-initialised; the library keeps its
+    leading region zero between calls).  Grows on demand; re-zeroed when the
+    cache/query shapes change."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+        self.key = None
+
+    def get(self, nbytes: int, key, stream) -> "object":
+        import torch
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            self.key = key
+        elif key != self.key:
+            _check(load_library().tsd_workspace_init(self.buf.data_ptr(), self.buf.numel(), stream), "workspace_init")
+            self.key = key
+        return self.buf
+
+
+_DEFAULT_WS = {}
+
+
+def _ws(workspace: Optional[Workspace], device) -> Workspace:
+    if workspace is not None:
+        return workspace
+    key = str(device)
+    if key not in _DEFAULT_WS:
+        _DEFAULT_WS[key] = Workspace(device)
+    return _DEFAULT_WS[key]
+
+
+def _stream_ptr(stream, device):
+    import torch
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return s, ctypes.c_void_p(s.cuda_stream)
+
+
+def _shape_key(cache: KVCache, queries: Queries):
+    return (cache.batch, cache.num_kv_heads, int(queries.q.shape[1]), int(queries.q.shape[0]),
+            queries.max_tokens_per_seq if queries.q_indptr is not None else 1, int(cache.max_seq_len))
+
+
+def _to_device(t, device, stream):
+    """Host tensors are copied to `device` on `stream` (asynchronously from pinned memory)."""
+    import torch
+    if t is None or t.device == device:
+        return t
+    with torch.cuda.stream(stream):
+        return t.to(device, non_blocking=True)
+
+
+def _on_device_queries(queries: Queries, device, stream) -> Queries:
+    if queries.q.device == device and (queries.q_indptr is None or queries.q_indptr.device == device):
+        return queries
+    return Queries(q=_to_device(queries.q, device, stream), q_indptr=_to_device(queries.q_indptr, device, stream),
+                   max_tokens_per_seq=queries.max_tokens_per_seq, causal=queries.causal, sm_scale=queries.sm_scale)
+
+
+# ---------------------------------------------------------------------------
+# Operations
+# ---------------------------------------------------------------------------
+def topk_select(cache: KVCache, queries: Queries, k_max: int, k_per_token=None, out_idx=None, out_count=None,
+                workspace: Optional[Workspace] = None, stream=None) -> Tuple["object", "object"]:
+    """Exact top-k token indices per (query token, q head): int32 [T, Hq, k_max]
+    ascending, -1 padded, and the per-list counts int32 [T, Hq]."""
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    queries = _on_device_queries(queries, dev, s)
+    k_per_token = _to_device(k_per_token, dev, s)
+    cs, qs = cache.c_struct(), queries.c_struct()
+    T, Hq = int(queries.q.shape[0]), int(queries.q.shape[1])
+    if out_idx is None:
+        out_idx = torch.empty((T, Hq, k_max), dtype=torch.int32, device=dev)
+    if out_count is None:
+        out_count = torch.empty((T, Hq), dtype=torch.int32, device=dev)
+    if k_per_token is not None and (k_per_token.dtype != torch.int32 or k_per_token.numel() != T):
+        raise ValueError("k_per_token must be int32 [T]")
+    nbytes = lib.tsd_topk_workspace_size(ctypes.byref(cs), ctypes.byref(qs), int(k_max))
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_topk_workspace_size")
+    ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, queries), sp)
+    _check(lib.tsd_topk_select(ctypes.byref(cs), ctypes.byref(qs), int(k_max),
+                               None if k_per_token is None else k_per_token.data_ptr(),
+                               out_idx.data_ptr(), out_count.data_ptr(), ws.data_ptr(), ws.numel(), sp),
+           "tsd_topk_select")
+    return out_idx, out_count
+
+
+def _out_buffers(queries, out, out_dtype, lse, dev):
+    import torch
+    T, Hq = int(queries.q.shape[0]), int(queries.q.shape[1])
+    host_out = None
+    if out is not None and out.device != dev:
+        host_out = out
+        out = None
+    if out is None:
+        out = torch.empty((T, Hq, 128), dtype=out_dtype, device=dev)
+    if out.dtype not in (torch.bfloat16, torch.float32) or not out.is_contiguous():
+        raise TypeError("out must be a contiguous bfloat16 or float32 tensor")
+    host_lse = None
+    if lse is True:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    elif lse is not None and lse is not False and lse.device != dev:
+        host_lse = lse
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    elif lse is False:
+        lse = None
+    return out, host_out, lse, host_lse
+
+
+def _finish(out, host_out, lse, host_lse, stream):
+    import torch
+    with torch.cuda.stream(stream):
+        if host_out is not None:
+            host_out.copy_(out, non_blocking=True)
+            out = host_out
+        if host_lse is not None:
+            host_lse.copy_(lse, non_blocking=True)
+            lse = host_lse
+    return out, lse
+
+
+def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=None, lse=True,
+                  workspace: Optional[Workspace] = None, stream=None):
+    """Attention of each (token, head) over the rows of its index list.
+
+    idx: int32 [T, Hq, k_max], each list non-decreasing then -1 padded (as
+    topk_select writes it).  Returns (out [T, Hq, 128], lse [T, Hq] or None).
+    Host (CPU) inputs are copied in and a host `out`/`lse` is filled on return
+    (asynchronously from/to pinned memory, ordered on `stream`).
+    """
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    queries = _on_device_queries(queries, dev, s)
+    idx = _to_device(idx, dev, s)
+    if idx.dtype != torch.int32 or idx.dim() != 3 or not idx.is_contiguous():
+        raise ValueError("idx must be a contiguous int32 [T, Hq, k_max] tensor")
+    out_dtype = out_dtype or (out.dtype if out is not None else torch.bfloat16)
+    out, host_out, lse, host_lse = _out_buffers(queries, out, out_dtype, lse, dev)
+    cs, qs = cache.c_struct(), queries.c_struct()
+    k_max = int(idx.shape[2])
+    nbytes = lib.tsd_sparse_decode_workspace_size(ctypes.byref(cs), ctypes.byref(qs), k_max)
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_sparse_decode_workspace_size")
+    ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, queries), sp)
+    _check(lib.tsd_sparse_decode(ctypes.byref(cs), ctypes.byref(qs), idx.data_ptr(), k_max, out.data_ptr(),
+                                 TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32,
+                                 None if lse is None else lse.data_ptr(), ws.data_ptr(), ws.numel(), sp),
+           "tsd_sparse_decode")
+    return _finish(out, host_out, lse, host_lse, s)
+
+
+def dense_decode(cache: KVCache, queries: Queries, out=None, out_dtype=None, lse=True,
+                 workspace: Optional[Workspace] = None, stream=None):
+    """Dense decode attention over every visible token (the comparator)."""
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    queries = _on_device_queries(queries, dev, s)
+    out_dtype = out_dtype or (out.dtype if out is not None else torch.bfloat16)
+    out, host_out, lse, host_lse = _out_buffers(queries, out, out_dtype, lse, dev)
+    cs, qs = cache.c_struct(), queries.c_struct()
+    nbytes = lib.tsd_dense_decode_workspace_size(ctypes.byref(cs), ctypes.byref(qs))
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_dense_decode_workspace_size")
+    ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, queries), sp)
+    _check(lib.tsd_dense_decode(ctypes.byref(cs), ctypes.byref(qs), out.data_ptr(),
+                                TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32,
+                                None if lse is None else lse.data_ptr(), ws.data_ptr(), ws.numel(), sp),
+           "tsd_dense_decode")
+    return _finish(out, host_out, lse, host_lse, s)
+
+
+def read_device_status(workspace: Optional[Workspace] = None, device=None, stream=None) -> int:
+    """Read and clear the device status bits of a workspace (synchronises the stream)."""
+    import torch
+    lib = load_library()
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    ws = _ws(workspace, dev)
+    if ws.buf is None:
+        return 0
+    s, sp = _stream_ptr(stream, ws.buf.device)
+    flags = ctypes.c_uint32(0)
+    rc = lib.tsd_read_device_status(ws.buf.data_ptr(), sp, ctypes.byref(flags))
+    if rc not in (TSD_OK, TSD_ERR_DEVICE_STATUS):
+        raise TsdError(rc, "tsd_read_device_status")
+    return int(flags.value)

@@ -1,0 +1,280 @@
+// extern "C" entry points of libtsd: host-side validation, work decomposition,
+// workspace layout and kernel launches.  See include/tsd.h for the contract.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "tsd.h"
+#include "tsd_common.cuh"
+#include "tsd_plan.h"
+
+#include "tsd_args.h"
+
+namespace tsd {
+cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream);
+cudaError_t launch_dense_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream);
+cudaError_t launch_topk(const TopkArgs& a, int nwin, int batch, int hkv, int num_lists, cudaStream_t stream);
+}  // namespace tsd
+
+using namespace tsd;
+
+namespace {
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int log2i(int x) {
+  int s = 0;
+  while ((1 << s) < x) ++s;
+  return s;
+}
+
+// Host validation of the descriptors; fills the kernel views and shape summary.
+tsd_status check_inputs(const tsd_kv_cache* c, const tsd_queries* q, KvView* kv, QView* qv, Shapes* sh) {
+  if (c == nullptr || q == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  if (c->head_dim != kHeadDim) return TSD_ERR_UNSUPPORTED;
+  if (c->k == nullptr || c->v == nullptr || c->seq_lens == nullptr || q->q == nullptr)
+    return TSD_ERR_INVALID_ARGUMENT;
+  if (c->batch < 1 || c->num_kv_heads < 1 || c->max_seq_len < 1) return TSD_ERR_INVALID_ARGUMENT;
+  if (q->num_q_heads < 1 || q->num_q_heads % c->num_kv_heads != 0) return TSD_ERR_INVALID_ARGUMENT;
+  if (q->num_tokens < 1) return TSD_ERR_INVALID_ARGUMENT;
+  if (q->q_dtype != TSD_BF16 && q->q_dtype != TSD_F32) return TSD_ERR_UNSUPPORTED;
+  int max_tokens = q->max_tokens_per_seq;
+  if (q->q_indptr == nullptr) {
+    if (q->num_tokens != c->batch) return TSD_ERR_INVALID_ARGUMENT;
+    max_tokens = 1;
+  } else if (max_tokens < 1 || max_tokens > q->num_tokens) {
+    return TSD_ERR_INVALID_ARGUMENT;
+  }
+  if (!(q->sm_scale > 0.f) || q->sm_scale != q->sm_scale) return TSD_ERR_INVALID_ARGUMENT;
+  // 16-byte alignment of the row streams
+  if (((uintptr_t)c->k & 15) || ((uintptr_t)c->v & 15) || ((uintptr_t)q->q & 15)) return TSD_ERR_INVALID_ARGUMENT;
+
+  memset(kv, 0, sizeof(*kv));
+  kv->k = static_cast<const uint16_t*>(c->k);
+  kv->v = static_cast<const uint16_t*>(c->v);
+  kv->seq_lens = c->seq_lens;
+  kv->hkv = c->num_kv_heads;
+  kv->max_seq_len = c->max_seq_len;
+  kv->batch = c->batch;
+  if (c->layout == TSD_LAYOUT_PAGED) {
+    if (c->page_table == nullptr || !is_pow2(c->page_size)) return c->page_table ? TSD_ERR_UNSUPPORTED : TSD_ERR_INVALID_ARGUMENT;
+    if ((int64_t)c->max_pages_per_seq * c->page_size < c->max_seq_len) return TSD_ERR_INVALID_ARGUMENT;
+    if (c->num_pages < 1) return TSD_ERR_INVALID_ARGUMENT;
+    // physical rows are addressed with 32-bit row numbers
+    if ((double)c->num_pages * c->num_kv_heads * c->page_size >= 4294967295.0) return TSD_ERR_UNSUPPORTED;
+    kv->page_table = c->page_table;
+    kv->page_shift = log2i(c->page_size);
+    kv->max_pages = c->max_pages_per_seq;
+    kv->num_pages = c->num_pages;
+  } else if (c->layout == TSD_LAYOUT_CONTIGUOUS) {
+    if (c->page_table != nullptr) return TSD_ERR_INVALID_ARGUMENT;
+    if ((double)c->batch * c->num_kv_heads * c->max_seq_len >= 4294967295.0) return TSD_ERR_UNSUPPORTED;
+    kv->page_table = nullptr;
+    kv->num_pages = c->batch;
+  } else {
+    return TSD_ERR_INVALID_ARGUMENT;
+  }
+  memset(qv, 0, sizeof(*qv));
+  qv->q = q->q;
+  qv->q_f32 = q->q_dtype == TSD_F32;
+  qv->hq = q->num_q_heads;
+  qv->num_tokens = q->num_tokens;
+  qv->q_indptr = q->q_indptr;
+  qv->max_tokens = max_tokens;
+  qv->causal = q->causal != 0;
+  qv->sm_scale = q->sm_scale;
+
+  sh->batch = c->batch;
+  sh->hkv = c->num_kv_heads;
+  sh->hq = q->num_q_heads;
+  sh->group = q->num_q_heads / c->num_kv_heads;
+  sh->tokens = q->num_tokens;
+  sh->max_tokens = max_tokens;
+  sh->max_seq_len = c->max_seq_len;
+  return TSD_OK;
+}
+
+tsd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSD_OK : TSD_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t tsd_version(void) { return 100; }
+
+const char* tsd_status_string(tsd_status s) {
+  switch (s) {
+    case TSD_OK: return "TSD_OK";
+    case TSD_ERR_INVALID_ARGUMENT: return "TSD_ERR_INVALID_ARGUMENT";
+    case TSD_ERR_UNSUPPORTED: return "TSD_ERR_UNSUPPORTED";
+    case TSD_ERR_WORKSPACE_TOO_SMALL: return "TSD_ERR_WORKSPACE_TOO_SMALL";
+    case TSD_ERR_CUDA: return "TSD_ERR_CUDA";
+    case TSD_ERR_DEVICE_STATUS: return "TSD_ERR_DEVICE_STATUS";
+  }
+  return "TSD_UNKNOWN_STATUS";
+}
+
+tsd_status tsd_workspace_init(void* ws, size_t bytes, tsd_stream_t stream) {
+  if (ws == nullptr && bytes > 0) return TSD_ERR_INVALID_ARGUMENT;
+  if (bytes == 0) return TSD_OK;
+  return cuda_status(cudaMemsetAsync(ws, 0, bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t tsd_topk_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max) {
+  KvView kv; QView qv; Shapes sh;
+  if (k_max < 1) return 0;
+  // shape-only validation: device pointers may be NULL when only sizing
+  tsd_kv_cache c = *cache;
+  tsd_queries q = *queries;
+  static const uint16_t dummy[8] = {0};
+  if (c.k == nullptr) c.k = dummy;
+  if (c.v == nullptr) c.v = dummy;
+  if (c.seq_lens == nullptr) c.seq_lens = reinterpret_cast<const int32_t*>(dummy);
+  if (c.layout == TSD_LAYOUT_PAGED && c.page_table == nullptr) c.page_table = reinterpret_cast<const int32_t*>(dummy);
+  if (q.q == nullptr) q.q = dummy;
+  if (check_inputs(&c, &q, &kv, &qv, &sh) != TSD_OK) return 0;
+  return topk_layout(sh).total;
+}
+
+static tsd_status sizes_for(const tsd_kv_cache* cache, const tsd_queries* queries, Shapes* sh) {
+  if (cache == nullptr || queries == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  KvView kv; QView qv;
+  tsd_kv_cache c = *cache;
+  tsd_queries q = *queries;
+  static const uint16_t dummy[8] = {0};
+  if (c.k == nullptr) c.k = dummy;
+  if (c.v == nullptr) c.v = dummy;
+  if (c.seq_lens == nullptr) c.seq_lens = reinterpret_cast<const int32_t*>(dummy);
+  if (c.layout == TSD_LAYOUT_PAGED && c.page_table == nullptr) c.page_table = reinterpret_cast<const int32_t*>(dummy);
+  if (q.q == nullptr) q.q = dummy;
+  return check_inputs(&c, &q, &kv, &qv, sh);
+}
+
+size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max) {
+  Shapes sh;
+  if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return 0;
+  const SparsePlan p = plan_sparse(sh, k_max);
+  return decode_layout(sh, p.nsplit).total;
+}
+
+size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries) {
+  Shapes sh;
+  if (sizes_for(cache, queries, &sh) != TSD_OK) return 0;
+  const DensePlan p = plan_dense(sh);
+  return decode_layout(sh, p.nsplit).total;
+}
+
+tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                           const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count, void* ws,
+                           size_t ws_bytes, tsd_stream_t stream) {
+  KvView kv; QView qv; Shapes sh;
+  tsd_status st = check_inputs(cache, queries, &kv, &qv, &sh);
+  if (st != TSD_OK) return st;
+  if (k_max < 1 || out_idx == nullptr || ws == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  if (((uintptr_t)ws & 255) != 0) return TSD_ERR_INVALID_ARGUMENT;
+  const TopkLayout lay = topk_layout(sh);
+  if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
+  TopkArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kv = kv;
+  a.qv = qv;
+  a.k_max = k_max;
+  a.k_per_token = k_per_token;
+  a.out_idx = out_idx;
+  a.out_count = out_count;
+  a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
+  a.score_stride = lay.score_stride;
+  a.lists_per_cta = (int)(sh.group * sh.max_tokens < kMaxListsPerCta ? sh.group * sh.max_tokens : kMaxListsPerCta);
+  a.list_groups = list_groups(sh);
+  a.window = kScoreTokensPerCta;
+  a.status = static_cast<uint32_t*>(ws);
+  const int nwin = (int)((sh.max_seq_len + a.window - 1) / a.window);
+  return cuda_status(launch_topk(a, nwin, (int)sh.batch, (int)sh.hkv, (int)(sh.tokens * sh.hq),
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static tsd_status decode_common(const tsd_kv_cache* cache, const tsd_queries* queries, void* out,
+                                int32_t out_dtype, float* lse, void* ws, size_t ws_bytes, KvView* kv,
+                                QView* qv, Shapes* sh) {
+  tsd_status st = check_inputs(cache, queries, kv, qv, sh);
+  if (st != TSD_OK) return st;
+  if (out == nullptr || ws == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return TSD_ERR_UNSUPPORTED;
+  if (((uintptr_t)ws & 255) != 0) return TSD_ERR_INVALID_ARGUMENT;
+  (void)ws_bytes;
+  (void)lse;
+  return TSD_OK;
+}
+
+tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
+                             int32_t k_max, void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                             tsd_stream_t stream) {
+  KvView kv; QView qv; Shapes sh;
+  tsd_status st = decode_common(cache, queries, out, out_dtype, lse, ws, ws_bytes, &kv, &qv, &sh);
+  if (st != TSD_OK) return st;
+  if (idx == nullptr || k_max < 1) return TSD_ERR_INVALID_ARGUMENT;
+  if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
+  const SparsePlan p = plan_sparse(sh, k_max);
+  const DecodeLayout lay = decode_layout(sh, p.nsplit);
+  if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kv = kv;
+  a.qv = qv;
+  a.idx = idx;
+  a.k_max = k_max;
+  a.span = p.entries;
+  a.nsplit = p.nsplit;
+  a.lists_per_cta = p.lists_per_cta;
+  a.list_groups = p.list_groups;
+  a.out = out;
+  a.out_f32 = out_dtype == TSD_F32;
+  a.lse = lse;
+  a.status = static_cast<uint32_t*>(ws);
+  a.counters = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_counters);
+  a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.off_ml);
+  a.part_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_acc);
+  return cuda_status(launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* queries, void* out, int32_t out_dtype,
+                            float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream) {
+  KvView kv; QView qv; Shapes sh;
+  tsd_status st = decode_common(cache, queries, out, out_dtype, lse, ws, ws_bytes, &kv, &qv, &sh);
+  if (st != TSD_OK) return st;
+  const DensePlan p = plan_dense(sh);
+  const DecodeLayout lay = decode_layout(sh, p.nsplit);
+  if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kv = kv;
+  a.qv = qv;
+  a.idx = nullptr;
+  a.k_max = 0;
+  a.span = p.window;
+  a.nsplit = p.nsplit;
+  a.lists_per_cta = p.lists_per_cta;
+  a.list_groups = p.list_groups;
+  a.out = out;
+  a.out_f32 = out_dtype == TSD_F32;
+  a.lse = lse;
+  a.status = static_cast<uint32_t*>(ws);
+  a.counters = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_counters);
+  a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.off_ml);
+  a.part_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_acc);
+  return cuda_status(launch_dense_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tsd_status tsd_read_device_status(void* ws, tsd_stream_t stream, uint32_t* flags) {
+  if (ws == nullptr || flags == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return TSD_ERR_CUDA;
+  *flags = host;
+  return host ? TSD_ERR_DEVICE_STATUS : TSD_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// Kernel argument blocks of libtsd (passed by value to the kernels).
+#pragma once
+
+#include <stdint.h>
+
+#include "tsd_common.cuh"
+
+namespace tsd {
+
+struct DecodeArgs {
+  KvView kv;
+  QView qv;
+  const int32_t* idx;   // sparse: [T][Hq][k_max]; dense: unused
+  int32_t k_max;
+  int32_t span;         // sparse: entries per list per split (E); dense: tokens per window (W)
+  int32_t nsplit;
+  int32_t lists_per_cta;
+  int32_t list_groups;
+  void* out;
+  int32_t out_f32;
+  float* lse;
+  uint32_t* status;
+  uint32_t* counters;
+  float2* part_ml;
+  float* part_acc;
+};
+
+struct TopkArgs {
+  KvView kv;
+  QView qv;
+  int32_t k_max;
+  const int32_t* k_per_token;
+  int32_t* out_idx;
+  int32_t* out_count;
+  float* scores;
+  int64_t score_stride;
+  int32_t lists_per_cta;
+  int32_t list_groups;
+  int32_t window;
+  uint32_t* status;
+};
+
+}  // namespace tsd

@@ -1,0 +1,178 @@
+// Device-side helpers shared by the sm_100a kernels of libtsd.
+//
+// Storage: K and V are bf16 rows of 128 elements (256 bytes per (token, kv head)),
+// either in HND pages [page][kv head][slot][128] or contiguous
+// [sequence][kv head][token][128].  All arithmetic is fp32.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tsd_plan.h"
+
+namespace tsd {
+
+constexpr int kHeadDim = 128;
+constexpr uint32_t kInvalidRow = 0xFFFFFFFFu;
+
+// ---------------------------------------------------------------------------
+// Views passed by value to the kernels
+// ---------------------------------------------------------------------------
+struct KvView {
+  const uint16_t* k;
+  const uint16_t* v;
+  const int32_t* page_table;  // nullptr for the contiguous layout
+  const int32_t* seq_lens;
+  int64_t num_pages;
+  int32_t hkv;
+  int32_t page_shift;         // log2(page_size) (paged)
+  int32_t max_pages;          // page-table row stride (paged)
+  int32_t max_seq_len;
+  int32_t batch;
+};
+
+struct QView {
+  const void* q;
+  int32_t q_f32;              // 1: fp32 queries, 0: bf16
+  int32_t hq;
+  int32_t num_tokens;
+  const int32_t* q_indptr;    // nullptr: token b belongs to sequence b
+  int32_t max_tokens;         // host bound on tokens per sequence
+  int32_t causal;
+  float sm_scale;
+};
+
+// Physical row (units of 128 elements) of token i of (sequence b, kv head g), or
+// kInvalidRow when its page id is out of range (the caller flags TSD_DEV_BAD_PAGE).
+__device__ __forceinline__ uint32_t kv_row(const KvView& kv, int b, int g, int i) {
+  if (kv.page_table == nullptr) {
+    return (uint32_t)(((int64_t)b * kv.hkv + g) * kv.max_seq_len + i);
+  }
+  const int32_t page = __ldg(kv.page_table + (int64_t)b * kv.max_pages + (i >> kv.page_shift));
+  if (page < 0 || (int64_t)page >= kv.num_pages) return kInvalidRow;
+  const int32_t mask = (1 << kv.page_shift) - 1;
+  return (uint32_t)((((int64_t)page * kv.hkv + g) << kv.page_shift) | (i & mask));
+}
+
+// Tokens [t0, t0 + n) of sequence b, validated against the host bounds.  A bad
+// descriptor makes the sequence empty and raises TSD_DEV_BAD_SEQ.
+struct SeqInfo {
+  int t0;
+  int n;        // query tokens of the sequence
+  int len;      // cached tokens (seq_lens[b])
+};
+
+__device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {
+  atomicOr(status, bits);
+}
+
+__device__ __forceinline__ SeqInfo seq_info(const KvView& kv, const QView& qv, int b, uint32_t* status,
+                                            bool report) {
+  SeqInfo s;
+  int len = __ldg(kv.seq_lens + b);
+  int t0, t1;
+  if (qv.q_indptr != nullptr) {
+    t0 = __ldg(qv.q_indptr + b);
+    t1 = __ldg(qv.q_indptr + b + 1);
+  } else {
+    t0 = b;
+    t1 = b + 1;
+  }
+  bool bad = len < 0 || len > kv.max_seq_len || t0 < 0 || t1 < t0 || t1 > qv.num_tokens ||
+             (t1 - t0) > qv.max_tokens;
+  if (bad) {
+    if (report) flag_status(status, TSD_DEV_BAD_SEQ_BIT);
+    s.t0 = 0; s.n = 0; s.len = 0;
+    return s;
+  }
+  s.t0 = t0; s.n = t1 - t0; s.len = len;
+  return s;
+}
+
+// Tokens visible to query j (0-based) of the n tokens of a sequence with len cached tokens.
+__device__ __forceinline__ int kv_len_of(const QView& qv, const SeqInfo& s, int j) {
+  int L = qv.causal ? s.len - s.n + j + 1 : s.len;
+  return L < 0 ? 0 : L;
+}
+
+// ---------------------------------------------------------------------------
+// Numerics
+// ---------------------------------------------------------------------------
+// 2^x via the hardware approximation (ex2.approx, documented PTX instruction).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two bf16 packed in a 32-bit word -> two fp32 (exact: bf16 is the top half of fp32).
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  f[0] = bf16lo(u.x); f[1] = bf16hi(u.x);
+  f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
+  f[4] = bf16lo(u.z); f[5] = bf16hi(u.z);
+  f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
+}
+
+// fp32 -> bf16 bits, round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u = __float_as_uint(f);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// Order-preserving map of an fp32 score onto uint32 (larger score -> larger key);
+// -0.0 is folded onto +0.0 so that equal scores tie on the index.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t u = __float_as_uint(s);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// Asynchronous global->shared copies (cp.async, 16 bytes, L2-only caching)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide exclusive scan of one int per thread (blockDim.x == NT, multiple of 32)
+// ---------------------------------------------------------------------------
+template <int NT>
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tmp /* >= NT/32 + 1 */, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < NT / 32 ? warp_tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < NT / 32) warp_tmp[lane] = w;   // inclusive prefix of warp totals
+    if (lane == NT / 32 - 1) warp_tmp[NT / 32] = w;
+  }
+  __syncthreads();
+  int excl = x - v + (warp > 0 ? warp_tmp[warp - 1] : 0);
+  *total = warp_tmp[NT / 32];
+  __syncthreads();
+  return excl;
+}
+
+}  // namespace tsd

@@ -290,11 +290,16 @@ def _random_unit_orthogonal(rng: np.random.Generator, ref: np.ndarray) -> np.nda
     return _unit(z)
 
 
-def make_workload(cfg: DecodeConfig, seed: int = 0) -> HostWorkload:
-    """Build the host-side description of one seeded workload (no bulk K/V)."""
+def make_workload(cfg: DecodeConfig, seed: int = 0, seq_lens: Optional[Sequence[int]] = None) -> HostWorkload:
+    """Build the host-side description of one seeded workload (no bulk K/V).
+
+    `seq_lens` overrides the configuration's lengths (each <= cfg.max_seq_len).
+    """
     B, Hq, Hkv, G = cfg.batch, cfg.num_q_heads, cfg.num_kv_heads, cfg.group
-    D = HEAD_DIM
-    if cfg.seq_len is not None:
+    if seq_lens is not None:
+        seq_lens = np.asarray(seq_lens, dtype=np.int32)
+        assert seq_lens.shape == (B,) and int(seq_lens.max()) <= cfg.max_seq_len
+    elif cfg.seq_len is not None:
         seq_lens = np.full(B, cfg.seq_len, dtype=np.int32)
     else:
         lo, hi = cfg.seq_len_range
@@ -412,28 +417,16 @@ def zipf_page_run_indices(w: HostWorkload, k: int, alpha: float = 1.1, seed_purp
         P = -(-L // ps)
         if b not in perms:
             perms[b] = rng.permutation(-(-int(w.seq_lens[b]) // ps))
-        page_of_rank = [p for p in perms[b] if p < P]
+        page_of_rank = perms[b][perms[b] < P]
         wts = np.arange(1, P + 1, dtype=np.float64) ** (-alpha)
         wts /= wts.sum()
         n = min(k, L)
+        draw = min(P, -(-n // ps) + 2)
         for h in range(Hq):
-            need_pages = min(P, -(-n // ps) + 1)
-            ranks = rng.choice(P, size=need_pages, replace=False, p=wts)
-            toks: List[int] = []
-            for r in ranks:
-                p = page_of_rank[r]
-                slots = range(p * ps, min((p + 1) * ps, L))
-                for s in slots:
-                    if len(toks) < n:
-                        toks.append(s)
-                if len(toks) >= n:
-                    break
-            if len(toks) < n:   # short last page: fill from further ranks in order
-                for p in page_of_rank:
-                    for s in range(p * ps, min((p + 1) * ps, L)):
-                        if len(toks) < n and s not in toks:
-                            toks.append(s)
-            out[t, h, :n] = np.sort(np.array(toks, dtype=np.int32))
+            ranks = rng.choice(P, size=draw, replace=False, p=wts)
+            toks = page_of_rank[ranks][:, None] * ps + np.arange(ps)[None, :]
+            toks = toks[toks < L][:n]
+            out[t, h, :n] = np.sort(toks).astype(np.int32)
     return out
 
 
@@ -489,7 +482,8 @@ def to_device(w: HostWorkload, device="cuda", stream=None) -> DeviceWorkload:
     lib = _fill_lib()
     for tensor, tid in ((k, TENSOR_K), (v, TENSOR_V)):
         rc = lib.tsdw_fill_kv(tensor.data_ptr(), table.data_ptr(), page_table.data_ptr(),
-                              seq_lens.data_ptr(), cfg.batch, cfg.num_kv_heads, w.page_size,
+                              seq_lens.data_ptr(), cfg.batch, cfg.num_kv_heads,
+                              0 if cfg.layout == "contiguous" else w.page_size,
                               w.max_pages_per_seq, cfg.max_seq_len,
                               w.seed & 0xFFFFFFFF, w.seed >> 32, tid, ctypes.c_void_p(s.cuda_stream))
         if rc != 0:
