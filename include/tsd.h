@@ -170,6 +170,28 @@ tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* querie
                             tsd_stream_t stream);
 
 /*
+ * Sparse decode for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this entry point: it exists for callers such as a plugin running inside
+ * another runtime that owns all device memory, or a decode loop that must not call
+ * cudaMalloc (which synchronizes the device) and cannot pass a workspace down to here.
+ * It computes exactly what tsd_sparse_decode computes (same arguments and results) but
+ * allocates nothing and takes no workspace: its scratch lives in a 16 MiB array inside the
+ * library, which every GPU that loads the library holds until the process exits.
+ *  - Shapes whose scratch exceeds 16 MiB return TSD_ERR_WORKSPACE_TOO_SMALL without
+ *    launching (16 MiB covers e.g. 8 sequences x 32 q heads at k = 655).
+ *  - The first call on each device looks up the array's device address with that device
+ *    current; make that first call before any stream capture.
+ *  - Every call shares the one array and clears its status word and merge counters on
+ *    `stream` before launching: calls that overlap on the GPU (other streams, other host
+ *    threads) race and must be serialized by the caller.
+ *  - status: device uint32 the kernel ORs TSD_DEV_* bits into, or NULL to drop them (the
+ *    caller clears it; it cannot be read with tsd_read_device_status).
+ */
+tsd_status tsd_sparse_decode_static_ws(const tsd_kv_cache* cache, const tsd_queries* queries,
+                                       const int32_t* idx, int32_t k_max, void* out, int32_t out_dtype,
+                                       float* lse, uint32_t* status, tsd_stream_t stream);
+
+/*
  * Copy the device status word of `ws` to *flags (host), clear it, and synchronize `stream`.
  * Returns TSD_OK when no bit was set, TSD_ERR_DEVICE_STATUS when one was, TSD_ERR_CUDA on a
  * CUDA failure.

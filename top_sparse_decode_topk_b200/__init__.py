@@ -83,6 +83,9 @@ EXPORTS = {
                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.c_void_p]),
     "tsd_read_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "tsd_sparse_decode_static_ws": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
+                                                   ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 _LIB = None

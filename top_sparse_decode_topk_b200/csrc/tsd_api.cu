@@ -278,3 +278,38 @@ tsd_status tsd_read_device_status(void* ws, tsd_stream_t stream, uint32_t* flags
 }
 
 }  // extern "C"
+
+namespace tsd {
+
+// Validation and argument setup for tsd_sparse_decode_static_ws (tsd_static_ws.cu): the
+// same checks and work decomposition as tsd_sparse_decode, minus the workspace pointers,
+// plus the bytes the layout needs (`ws_needed`) and the size of its zero region.
+tsd_status prepare_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
+                                 int32_t k_max, void* out, int32_t out_dtype, float* lse, DecodeArgs* a,
+                                 Shapes* sh, size_t* ws_needed, size_t* zero_bytes) {
+  KvView kv; QView qv;
+  tsd_status st = check_inputs(cache, queries, &kv, &qv, sh);
+  if (st != TSD_OK) return st;
+  if (out == nullptr || idx == nullptr || k_max < 1) return TSD_ERR_INVALID_ARGUMENT;
+  if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return TSD_ERR_UNSUPPORTED;
+  if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
+  const SparsePlan p = plan_sparse(*sh, k_max);
+  const DecodeLayout lay = decode_layout(*sh, p.nsplit);
+  memset(a, 0, sizeof(*a));
+  a->kv = kv;
+  a->qv = qv;
+  a->idx = idx;
+  a->k_max = k_max;
+  a->span = p.entries;
+  a->nsplit = p.nsplit;
+  a->lists_per_cta = p.lists_per_cta;
+  a->list_groups = p.list_groups;
+  a->out = out;
+  a->out_f32 = out_dtype == TSD_F32;
+  a->lse = lse;
+  *ws_needed = lay.total;
+  *zero_bytes = zero_region_bytes(*sh);
+  return TSD_OK;
+}
+
+}  // namespace tsd
