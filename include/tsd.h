@@ -61,8 +61,10 @@ enum {
   TSD_DEV_BAD_INDEX = 1u << 0, /* an index entry was < -1 or >= kv_len of its query; skipped */
   TSD_DEV_UNSORTED = 1u << 1,  /* an index list was not ascending where it was read          */
   TSD_DEV_BAD_PAGE = 1u << 2,  /* a page-table entry was outside [0, num_pages); row skipped */
-  TSD_DEV_BAD_SEQ = 1u << 3    /* seq_len outside [0, max_seq_len] or a bad q_indptr; the
-                                  affected sequence is treated as empty                      */
+  TSD_DEV_BAD_SEQ = 1u << 3,   /* seq_len outside [0, max_seq_len] or a bad q_indptr; the
+                                  outputs of the affected sequence are not written          */
+  TSD_DEV_TIMEOUT = 1u << 4    /* a bounded wait inside a kernel gave up (an asynchronous
+                                  copy never completed); the results are not valid          */
 };
 
 typedef enum {

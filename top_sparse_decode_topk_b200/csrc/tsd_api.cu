@@ -234,6 +234,7 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
   a.counters = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_counters);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.off_ml);
   a.part_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_acc);
+  a.sched = static_cast<uint32_t*>(ws) + 1;
   return cuda_status(launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
 }
 

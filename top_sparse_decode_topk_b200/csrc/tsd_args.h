@@ -20,6 +20,7 @@ struct DecodeArgs {
   int32_t out_f32;
   float* lse;
   uint32_t* status;
+  uint32_t* sched;      // sparse: [0] work-unit counter, [1] finished-CTA counter (zero region)
   uint32_t* counters;
   float2* part_ml;
   float* part_acc;

@@ -38,7 +38,6 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kTileBytes = kRowsPerTile * 2 * 256;          // K rows then V rows
 constexpr int kRingBytes = kStages * kTileBytes;
 constexpr int kCombFloats = 132;                             // m, l, pad, pad, acc[128]
-constexpr int kMaxTiles = kMaxEntriesPerCta / kRowsPerTile;  // tiles per sparse CTA
 
 
 // List m of a CTA -> (token, q head).  Lists are ordered token-major inside a sequence:
@@ -258,270 +257,174 @@ __device__ void finish_lists(const DecodeArgs& a, const SeqInfo& si, int b, int 
 // ---------------------------------------------------------------------------
 // Sparse decode
 // ---------------------------------------------------------------------------
+// Scattered 256-byte rows are gathered straight into registers: a half-warp (16 lanes,
+// one 16-byte load each) owns a K row and a V row at a time, U rows in flight per
+// half-warp.  Measured on B200, this reaches the copy bandwidth for random 256-byte rows
+// at large sizes, while staging the same rows through shared memory (cp.async 16 B or
+// one 256-byte bulk copy per row) is 25-35% slower at every size.
+//
+// Work unit: (sequence b, kv head g, list group lg, split) -- up to 16 lists (q heads of
+// the GQA group x decode tokens of the sequence) and E consecutive entries of each.  The
+// grid is persistent (CTAs per SM x SMs); CTAs take units from a global counter, so the
+// tail is at most one small unit.  Within a unit every list gets P = 16 / lists
+// half-warps; each takes 16-entry chunks of its list in turn (chunk c -> part c % P), so
+// all lists of the kv head walk the token range together and a row picked by several of
+// them is read from DRAM once and served to the others from L1/L2.
+//
+// Per entry (half-warp): the 128-dim dot is 8 FMA per lane plus a 4-step shuffle
+// reduction; the online softmax keeps (max, sum, 8 output dims per lane) in registers.
+// At the end of a unit the parts of each list are combined, the split's partial is
+// written, and the last CTA to finish a (b, g, lg) merges its splits.
+constexpr int kSpU = 4;                 // rows in flight per half-warp
+constexpr int kSpThreads = 256;         // 16 half-warps
+
 struct SparseSmem {
-  unsigned char ring[kRingBytes];              // also the combine buffer at the end
-  uint32_t ent_tok[kMaxEntriesPerCta];         // compacted entries, list m at m*E
-  uint16_t ent_slot[kMaxEntriesPerCta];        // unique-row slot of each entry
-  uint32_t rowaddr[kMaxEntriesPerCta];         // physical row of each slot
-  uint32_t bitmap[kBitmapWords];
-  int wbase[kBitmapWords];
-  uint16_t bnd[kMaxListsPerCta][kMaxTiles + 1];  // first entry of each tile, per list
-  int list_n[kMaxListsPerCta];
-  int list_off[kMaxListsPerCta + 1];
-  int scan_tmp[kDecodeThreads / 32 + 1];
-  int tmin, tmax, nunique;
+  float comb[16 * kCombFloats];         // one state per half-warp
   float mx[kMaxListsPerCta], lsum[kMaxListsPerCta];
+  int unit;
 };
-static_assert(kStages * kTileBytes >= kMaxListsPerCta * kCombFloats * 4, "combine buffer must fit the ring");
 
-__device__ __forceinline__ void load_tile(SparseSmem& S, const KvView& kv, int tile, int nunique) {
-  const int stage = tile % kStages;
-  unsigned char* base = S.ring + stage * kTileBytes;
-#pragma unroll
-  for (int q = 0; q < (kRowsPerTile * 32) / kDecodeThreads; ++q) {
-    const int id = threadIdx.x + q * kDecodeThreads;
-    const int r = id >> 5, which = (id >> 4) & 1, ch = id & 15;
-    const int slot = tile * kRowsPerTile + r;
-    if (slot < nunique) {
-      const uint32_t row = S.rowaddr[slot];
-      if (row != kInvalidRow) {
-        const uint16_t* src = (which ? kv.v : kv.k) + (int64_t)row * kHeadDim + ch * 8;
-        cp_async16(base + which * (kRowsPerTile * 256) + r * 256 + ch * 16, src);
-      }
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kDecodeThreads, 2) sparse_decode_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  SparseSmem& S = *reinterpret_cast<SparseSmem*>(smem_raw);
-
-  const int split = blockIdx.x;
-  const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
-  const int b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int E = a.span;
-
-  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, split == 0 && g == 0 && lg == 0 && threadIdx.x == 0);
+__global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs a) {
+  __shared__ __align__(16) SparseSmem S;
+  const int lane = threadIdx.x & 31;
+  const int hw = threadIdx.x >> 4, l = threadIdx.x & 15;
+  const unsigned hmask = 0xFFFFu << (lane & 16);
   const int G = a.qv.hq / a.kv.hkv;
-  int nlists = si.n * G - lg * a.lists_per_cta;
-  if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
-  if (nlists <= 0) return;   // uniform over the whole (b, g, lg) unit: no merge is owed
+  const int E = a.span;
+  const int total_units = a.nsplit * a.list_groups * a.kv.hkv * a.kv.batch;
+  const float scale = a.qv.sm_scale * kLog2e;
+  uint32_t* work = a.sched;       // unit counter and finished-CTA counter (zero between calls)
+  uint32_t* done = a.sched + 1;
 
-  // ---- 1. entries: load, validate, compact (warp per list) ----
-  for (int m = warp; m < nlists; m += kDecodeThreads / 32) {
-    const ListRef r = list_ref(a, si, g, lg, m);
-    const int32_t* lst = a.idx + ((int64_t)r.t * a.qv.hq + r.h) * a.k_max;
-    const int e0 = split * E;
-    int e1 = e0 + E;
-    if (e1 > a.k_max) e1 = a.k_max;
-    uint32_t prev = (e0 > 0) ? (uint32_t)__ldg(lst + e0 - 1) : 0u;
-    int count = 0;
-    uint32_t bad = 0;
-    for (int base = e0; base < e1; base += 32) {
-      const int e = base + lane;
-      const int32_t v = e < e1 ? __ldg(lst + e) : -1;
-      uint32_t before = __shfl_up_sync(0xFFFFFFFFu, (uint32_t)v, 1);
-      if (lane == 0) before = prev;
-      if (e < e1 && (e > 0) && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
-      if (e < e1 && (v < -1 || v >= r.kvlen)) bad |= TSD_DEV_BAD_INDEX;
-      const bool ok = e < e1 && v >= 0 && v < r.kvlen;
-      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, ok);
-      if (ok) S.ent_tok[m * E + count + __popc(bal & ((1u << lane) - 1))] = (uint32_t)v;
-      count += __popc(bal);
-      prev = __shfl_sync(0xFFFFFFFFu, (uint32_t)v, 31);
-    }
-    bad = __reduce_or_sync(0xFFFFFFFFu, bad);
-    if (lane == 0) {
-      S.list_n[m] = count;
-      if (bad) flag_status(a.status, bad);
-    }
-  }
-  if (threadIdx.x == 0) {
-    S.tmin = 0x7FFFFFFF;
-    S.tmax = -1;
-  }
-  __syncthreads();
-
-  // ---- 2. token span of the chunk ----
-  {
-    int lo = 0x7FFFFFFF, hi = -1;
-    for (int m = 0; m < nlists; ++m) {
-      const int n = S.list_n[m];
-      for (int e = threadIdx.x; e < n; e += kDecodeThreads) {
-        const int v = (int)S.ent_tok[m * E + e];
-        lo = min(lo, v);
-        hi = max(hi, v);
-      }
-    }
-    lo = __reduce_min_sync(0xFFFFFFFFu, lo);
-    hi = __reduce_max_sync(0xFFFFFFFFu, hi);
-    if (lane == 0) {
-      atomicMin(&S.tmin, lo);
-      atomicMax(&S.tmax, hi);
-    }
-  }
-  if (threadIdx.x == 0) {
-    int off = 0;
-    for (int m = 0; m < nlists; ++m) {
-      S.list_off[m] = off;
-      off += S.list_n[m];
-    }
-    S.list_off[nlists] = off;
-  }
-  __syncthreads();
-
-  // ---- 3. deduplicate rows: bitmap over the span, prefix popcount -> slots ----
-  const int tmin = S.tmin;
-  const int span = S.tmax - tmin + 1;
-  int nunique;
-  if (S.tmax >= 0 && span <= kBitmapWords * 32) {
-    const int nwords = (span + 31) >> 5;
-    for (int w = threadIdx.x; w < nwords; w += kDecodeThreads) S.bitmap[w] = 0u;
+  for (;;) {
+    if (threadIdx.x == 0) S.unit = (int)atomicAdd(work, 1u);
     __syncthreads();
-    for (int m = 0; m < nlists; ++m) {
-      const int n = S.list_n[m];
-      for (int e = threadIdx.x; e < n; e += kDecodeThreads) {
-        const int o = (int)S.ent_tok[m * E + e] - tmin;
-        atomicOr(&S.bitmap[o >> 5], 1u << (o & 31));
-      }
-    }
+    const int unit = S.unit;
     __syncthreads();
-    constexpr int kWordsPerThread = kBitmapWords / kDecodeThreads;
-    int cnt = 0;
+    if (unit >= total_units) break;
+    const int split = unit % a.nsplit;
+    int rest = unit / a.nsplit;
+    const int lg = rest % a.list_groups;
+    rest /= a.list_groups;
+    const int g = rest % a.kv.hkv;
+    const int b = rest / a.kv.hkv;
+    const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, split == 0 && g == 0 && lg == 0 && threadIdx.x == 0);
+    int nlists = si.n * G - lg * a.lists_per_cta;
+    if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
+    if (nlists <= 0) continue;   // the same for every split of this (b, g, lg): no merge is owed
+
+    const int P = 16 / nlists;                 // half-warps per list
+    const int my_list = hw / P, my_part = hw % P;
+    const bool active = my_list < nlists;
+    float m_run = -CUDART_INF_F, l_run = 0.f, acc[8];
 #pragma unroll
-    for (int j = 0; j < kWordsPerThread; ++j) {
-      const int w = threadIdx.x * kWordsPerThread + j;
-      cnt += (w < nwords) ? __popc(S.bitmap[w]) : 0;
-    }
-    int total;
-    int run = block_exclusive_scan<kDecodeThreads>(cnt, S.scan_tmp, &total);
-#pragma unroll
-    for (int j = 0; j < kWordsPerThread; ++j) {
-      const int w = threadIdx.x * kWordsPerThread + j;
-      if (w < nwords) {
-        S.wbase[w] = run;
-        // physical rows of the unique tokens, in token order
-        uint32_t bits = S.bitmap[w];
-        int slot = run;
-        while (bits) {
-          const int bit = __ffs(bits) - 1;
-          bits &= bits - 1;
-          const int tok = tmin + w * 32 + bit;
-          const uint32_t row = kv_row(a.kv, b, g, tok);
-          if (row == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
-          S.rowaddr[slot++] = row;
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+
+    if (active) {
+      const ListRef r = list_ref(a, si, g, lg, my_list);
+      // this lane's 8 query dims [8l, 8l+8), scaled so that dots are base-2 softmax units
+      float q[8];
+      {
+        const int64_t qb = ((int64_t)r.t * a.qv.hq + r.h) * kHeadDim + 8 * l;
+        if (a.qv.q_f32) {
+          const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.qv.q) + qb);
+          const float4 x = __ldg(p), y = __ldg(p + 1);
+          q[0] = x.x; q[1] = x.y; q[2] = x.z; q[3] = x.w; q[4] = y.x; q[5] = y.y; q[6] = y.z; q[7] = y.w;
+        } else {
+          unpack8(__ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.qv.q) + qb)), q);
         }
-        run += __popc(S.bitmap[w]);
-      }
-    }
-    nunique = total;
-    __syncthreads();
-    for (int m = 0; m < nlists; ++m) {
-      const int n = S.list_n[m];
-      for (int e = threadIdx.x; e < n; e += kDecodeThreads) {
-        const int o = (int)S.ent_tok[m * E + e] - tmin;
-        const uint32_t word = S.bitmap[o >> 5];
-        S.ent_slot[m * E + e] = (uint16_t)(S.wbase[o >> 5] + __popc(word & ((1u << (o & 31)) - 1u)));
-      }
-    }
-  } else {
-    // span too wide for the bitmap: every entry is its own row (no dedupe)
-    nunique = S.list_off[nlists];
-    for (int m = 0; m < nlists; ++m) {
-      const int n = S.list_n[m];
-      for (int e = threadIdx.x; e < n; e += kDecodeThreads) {
-        const int slot = S.list_off[m] + e;
-        const uint32_t row = kv_row(a.kv, b, g, (int)S.ent_tok[m * E + e]);
-        if (row == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
-        S.rowaddr[slot] = row;
-        S.ent_slot[m * E + e] = (uint16_t)slot;
-      }
-    }
-  }
-  const int ntiles = (nunique + kRowsPerTile - 1) / kRowsPerTile;
-  // ---- 4. tile boundaries of every list: bnd[m][i] = first entry with slot >= i*R ----
-  for (int i = threadIdx.x; i < nlists * (kMaxTiles + 1); i += kDecodeThreads) {
-    const int m = i / (kMaxTiles + 1), tt = i % (kMaxTiles + 1);
-    if (tt <= ntiles) S.bnd[m][tt] = (uint16_t)S.list_n[m];
-  }
-  __syncthreads();
-  for (int m = 0; m < nlists; ++m) {
-    const int n = S.list_n[m];
-    for (int e = threadIdx.x; e < n; e += kDecodeThreads) {
-      const int ti = S.ent_slot[m * E + e] / kRowsPerTile;
-      const int lo = (e == 0) ? 0 : S.ent_slot[m * E + e - 1] / kRowsPerTile + 1;
-      for (int tt = lo; tt <= ti; ++tt) S.bnd[m][tt] = (uint16_t)e;
-    }
-  }
-  // prefetch the first tiles while the boundaries settle
-  // (rowaddr is complete: it was written before the previous barrier)
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < ntiles) load_tile(S, a.kv, s, nunique);
-    cp_async_commit();
-  }
-
-  // ---- 5. lane-group roles: list m = group / P, part p = group % P ----
-  const int group = threadIdx.x >> 3, l8 = threadIdx.x & 7;
-  const int P = 32 / nlists;                    // parts per list (>= 1)
-  const int my_list = group / P, my_part = group % P;
-  const bool has_list = my_list < nlists;
-  float q[16];
-  SoftState st;
-  soft_init(st);
-  {
-    const ListRef r = list_ref(a, si, g, lg, has_list ? my_list : 0);
-    const float scale = a.qv.sm_scale * kLog2e;
-    load_q16(a.qv, r.t, r.h, l8, scale, q);
-  }
-
-  // ---- 6. main loop over tiles ----
-  for (int tile = 0; tile < ntiles; ++tile) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (tile + kStages - 1 < ntiles) load_tile(S, a.kv, tile + kStages - 1, nunique);
-    cp_async_commit();
-
-    const unsigned char* kbase = S.ring + (tile % kStages) * kTileBytes;
-    const unsigned char* vbase = kbase + kRowsPerTile * 256;
-    int ea = 0, eb = 0, first = 0, cnt = 0;
-    if (has_list) {
-      ea = S.bnd[my_list][tile];
-      eb = S.bnd[my_list][tile + 1];
-      const int n = S.list_n[my_list];
-      ea = min(ea, n);
-      eb = min(max(eb, ea), n);
-      first = ea + ((my_part - ea) % P + P) % P;
-      cnt = eb > first ? (eb - first + P - 1) / P : 0;
-    }
-    int nmax = cnt;
-    nmax = max(nmax, __shfl_xor_sync(0xFFFFFFFFu, nmax, 8));
-    nmax = max(nmax, __shfl_xor_sync(0xFFFFFFFFu, nmax, 16));
-    for (int it = 0; it < nmax; ++it) {
-      const int e = first + it * P;
-      bool active = it < cnt;
-      int r = 0;
-      if (active) {
-        const int slot = S.ent_slot[my_list * E + e];
-        r = slot - tile * kRowsPerTile;
-        if (r < 0 || r >= kRowsPerTile || S.rowaddr[slot] == kInvalidRow) {
-          active = false;
-          r = 0;
+        for (int j = 0; j < 8; ++j) q[j] *= scale;
+      }
+      const int32_t* lst = a.idx + ((int64_t)r.t * a.qv.hq + r.h) * a.k_max;
+      const int e0 = split * E;
+      const int e1 = min(e0 + E, a.k_max);
+      const int nchunks = (e1 - e0 + 15) >> 4;
+      uint32_t bad = 0;
+      for (int c = my_part; c < nchunks; c += P) {
+        // entry of this lane, its predecessor, validity and physical row
+        const int e = e0 + 16 * c + l;
+        const int32_t v = e < e1 ? __ldg(lst + e) : -1;
+        uint32_t before = __shfl_up_sync(hmask, (uint32_t)v, 1, 16);
+        if (l == 0) before = (e > 0) ? (uint32_t)__ldg(lst + e - 1) : 0u;
+        if (e < e1 && e > 0 && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
+        if (e < e1 && (v < -1 || v >= r.kvlen)) bad |= TSD_DEV_BAD_INDEX;
+        uint32_t row = kInvalidRow;
+        if (e < e1 && v >= 0 && v < r.kvlen) {
+          row = kv_row(a.kv, b, g, v);
+          if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
+        }
+        // the chunk's 16 rows, U at a time
+#pragma unroll
+        for (int j0 = 0; j0 < 16; j0 += kSpU) {
+          uint32_t rr[kSpU];
+          uint4 kr[kSpU], vr[kSpU];
+#pragma unroll
+          for (int u = 0; u < kSpU; ++u) {
+            rr[u] = __shfl_sync(hmask, row, j0 + u, 16);
+            if (rr[u] != kInvalidRow) {
+              kr[u] = __ldg(reinterpret_cast<const uint4*>(a.kv.k + (int64_t)rr[u] * kHeadDim) + l);
+              vr[u] = __ldg(reinterpret_cast<const uint4*>(a.kv.v + (int64_t)rr[u] * kHeadDim) + l);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kSpU; ++u) {
+            if (rr[u] == kInvalidRow) continue;    // uniform over the half-warp
+            float kf[8], vf[8];
+            unpack8(kr[u], kf);
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+              s0 = fmaf(q[j], kf[j], s0);
+              s1 = fmaf(q[j + 1], kf[j + 1], s1);
+            }
+            float s = s0 + s1;
+            s += __shfl_xor_sync(hmask, s, 1);
+            s += __shfl_xor_sync(hmask, s, 2);
+            s += __shfl_xor_sync(hmask, s, 4);
+            s += __shfl_xor_sync(hmask, s, 8);
+            if (s > m_run) {
+              const float alpha = fast_exp2(m_run - s);
+              l_run *= alpha;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) acc[j] *= alpha;
+              m_run = s;
+            }
+            const float p = fast_exp2(s - m_run);
+            l_run += p;
+            unpack8(vr[u], vf);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = fmaf(p, vf[j], acc[j]);
+          }
         }
       }
-      const float s = group_dot(kbase + r * 256, l8, q);
-      if (active) soft_update(st, s, vbase + r * 256, l8);
+      bad |= __shfl_xor_sync(hmask, bad, 1);
+      bad |= __shfl_xor_sync(hmask, bad, 2);
+      bad |= __shfl_xor_sync(hmask, bad, 4);
+      bad |= __shfl_xor_sync(hmask, bad, 8);
+      if (l == 0 && bad) flag_status(a.status, bad);
+      // this half-warp's state -> combine buffer entry (list * P + part)
+      float* ce = S.comb + (size_t)(my_list * P + my_part) * kCombFloats;
+      if (l == 0) {
+        ce[0] = m_run;
+        ce[1] = l_run;
+      }
+      *reinterpret_cast<float4*>(ce + 4 + 8 * l) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float4*>(ce + 8 + 8 * l) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+    __syncthreads();
+    finish_lists(a, si, b, g, lg, split, nlists, P, S.comb, S.mx, S.lsum);
+    __syncthreads();
+  }
+  // the last CTA out resets the unit counters for the next call
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t prev = atomicAdd(done, 1u);
+    if (prev == gridDim.x - 1) {
+      atomicExch(work, 0u);
+      atomicExch(done, 0u);
     }
   }
-  cp_async_wait<0>();
-  __syncthreads();
-
-  // ---- 7. combine parts, write partial / output, merge splits ----
-  float* comb = reinterpret_cast<float*>(S.ring);
-  if (has_list) soft_store(comb, my_list * P + my_part, st, l8);
-  __syncthreads();
-  finish_lists(a, si, b, g, lg, split, nlists, P, comb, S.mx, S.lsum);
 }
 
 // ---------------------------------------------------------------------------
@@ -670,15 +573,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) dense_decode_kernel(DecodeA
 // Host launchers
 // ---------------------------------------------------------------------------
 cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
-  const size_t smem = sizeof(SparseSmem);
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int ctas_per_sm = 0, sms = 0;
+  if (ctas_per_sm == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, sparse_decode_kernel, kSpThreads, 0);
     if (e != cudaSuccess) return e;
-    configured = true;
+    if (ctas_per_sm < 1) ctas_per_sm = 1;
   }
-  dim3 grid(a.nsplit, hkv * a.list_groups, batch);
-  sparse_decode_kernel<<<grid, kDecodeThreads, smem, stream>>>(a);
+  const int units = a.nsplit * a.list_groups * hkv * batch;
+  int grid = ctas_per_sm * sms;
+  if (grid > units) grid = units;
+  sparse_decode_kernel<<<grid, kSpThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,7 +1,8 @@
 // Work decomposition and workspace layout of libtsd (host and device).
 //
 // Workspace layout (bytes from the start; every region 256-byte aligned):
-//   [0, 256)              header: device status word (uint32) at offset 0
+//   [0, 256)              header: device status word (uint32) at offset 0; sparse-decode
+//                         work-unit counter at byte 4 and finished-CTA counter at byte 8
 //   counters              uint32 [batch][num_kv_heads][group * max_tokens]: arrival counters
 //                         of the split-K merge, one per list group (zero between calls)
 //   -- everything above is the "zero region": it must be zero when a call starts and every
@@ -21,12 +22,14 @@
 namespace tsd {
 
 constexpr int kMaxListsPerCta = 32;     // query lists (token x q head) handled by one CTA
+constexpr int kSparseMaxLists = 16;     // sparse decode: lists per work unit (one half-warp each at least)
 constexpr int kDecodeThreads = 256;     // 8 warps = 32 groups of 8 lanes
 constexpr int kRowsPerTile = 16;        // K/V rows per pipeline stage
 constexpr int kStages = 4;              // cp.async pipeline depth
-constexpr int kMaxEntriesPerCta = 2048; // sparse: lists x entries per CTA
+constexpr int kMaxEntriesPerCta = 1024; // sparse: lists x entries per CTA
 constexpr int kBitmapWords = 1024;      // sparse: dedupe bitmap spans 32768 tokens
 constexpr int kMaxSplits = 256;         // split-K partials per (token, head)
+constexpr int kSparseEntriesTarget = 256;  // sparse: entries (all lists) a CTA aims for
 constexpr int kScoreThreads = 256;
 constexpr int kSelectThreads = 512;
 constexpr int kScoreTokensPerCta = 1024;
@@ -62,17 +65,16 @@ struct SparsePlan {
 inline SparsePlan plan_sparse(const Shapes& s, int k_max) {
   SparsePlan p;
   const int64_t m = s.group * s.max_tokens;
-  int lists = (int)(m < kMaxListsPerCta ? m : kMaxListsPerCta);
+  int lists = (int)(m < kSparseMaxLists ? m : kSparseMaxLists);
   const int kr = (k_max + 15) / 16 * 16;
-  int e = (512 / lists + 15) / 16 * 16;
+  int e = (kSparseEntriesTarget / lists + 15) / 16 * 16;
   if (e < 16) e = 16;
   if (e > kr) e = kr;
   int ns = (k_max + e - 1) / e;
-  if (ns > kMaxSplits) {   // long lists: grow the chunk, then shrink the list group to fit
-    e = ((k_max + kMaxSplits - 1) / kMaxSplits + 15) / 16 * 16;
+  if (ns > kMaxSplits) {
+    e = ((k_max + kMaxSplits - 1) / kMaxSplits + 15) / 16 * 16;   // long lists: bigger chunks
     ns = (k_max + e - 1) / e;
   }
-  if (lists * e > kMaxEntriesPerCta) lists = kMaxEntriesPerCta / e > 0 ? kMaxEntriesPerCta / e : 1;
   p.lists_per_cta = lists;
   p.list_groups = (int)((m + lists - 1) / lists);
   p.entries = e;
