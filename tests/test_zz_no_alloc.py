@@ -65,15 +65,23 @@ def test_static_ws_matches_workspace_entry_point():
 
 
 def test_static_ws_rejects_shapes_beyond_its_size():
+    """A shape whose scratch exceeds the array is refused before anything is launched.
+
+    The descriptors hold placeholder addresses, so the entry point must not launch: the
+    test first checks through the sizing function (host only) that the shape needs far
+    more than 16 MiB, and calls the entry point only then."""
     lib = tsd.load_library()
     c = tsd._KvCacheC()
     c.k, c.v = 0x7F0000000000, 0x7F0000100000
     c.layout, c.num_kv_heads, c.head_dim, c.page_size = 0, 8, 128, 16
-    c.page_table, c.max_pages_per_seq, c.num_pages = 0x7F0000200000, 8192, 32 * 8192
-    c.seq_lens, c.batch, c.max_seq_len = 0x7F0000300000, 32, 131072
+    c.page_table, c.max_pages_per_seq, c.num_pages = 0x7F0000200000, 8192, 512 * 8192
+    c.seq_lens, c.batch, c.max_seq_len = 0x7F0000300000, 512, 131072
     q = tsd._QueriesC()
-    q.q, q.q_dtype, q.num_q_heads, q.num_tokens = 0x7F0000400000, 0, 32, 128
+    q.q, q.q_dtype, q.num_q_heads, q.num_tokens = 0x7F0000400000, 0, 32, 2048
     q.q_indptr, q.max_tokens_per_seq, q.causal, q.sm_scale = 0x7F0000500000, 4, 1, 0.088
+    need = lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 2622)
+    # 2048 tokens x 32 heads of split-K rows alone are 34 MB; refuse to call otherwise
+    assert need > 2 * (16 << 20), f"shape no longer exceeds the static array ({need} bytes): not calling"
     rc = lib.tsd_sparse_decode_static_ws(ctypes.byref(c), ctypes.byref(q), 0x7F0000600000, 2622, 0x7F0000700000,
                                          tsd.TSD_BF16, None, None, None)
     assert rc == tsd.TSD_ERR_WORKSPACE_TOO_SMALL

@@ -225,8 +225,8 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
   a.k_max = k_max;
   a.span = p.entries;
   a.nsplit = p.nsplit;
-  a.lists_per_cta = p.lists_per_cta;
-  a.list_groups = p.list_groups;
+  a.lists_per_cta = p.lists;
+  a.list_groups = 1;
   a.out = out;
   a.out_f32 = out_dtype == TSD_F32;
   a.lse = lse;
@@ -303,8 +303,8 @@ tsd_status prepare_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* q
   a->k_max = k_max;
   a->span = p.entries;
   a->nsplit = p.nsplit;
-  a->lists_per_cta = p.lists_per_cta;
-  a->list_groups = p.list_groups;
+  a->lists_per_cta = p.lists;
+  a->list_groups = 1;
   a->out = out;
   a->out_f32 = out_dtype == TSD_F32;
   a->lse = lse;

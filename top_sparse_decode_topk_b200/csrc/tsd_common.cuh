@@ -192,6 +192,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                : "memory");
 }
 
+// Asynchronous prefetch of `bytes` (multiple of 16, 16-byte aligned) from global memory
+// into L2; it holds no register or shared-memory resources while in flight.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Block-wide exclusive scan of one int per thread (blockDim.x == NT, multiple of 32)
 // ---------------------------------------------------------------------------

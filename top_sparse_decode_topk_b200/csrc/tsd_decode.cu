@@ -245,9 +245,20 @@ __device__ void finish_lists(const DecodeArgs& a, const SeqInfo& si, int b, int 
     float A = 0.f;
     if (L > 0.f) {
       const int64_t pbase = ((int64_t)r.t * a.qv.hq + r.h) * a.nsplit;
-      for (int c = 0; c < a.nsplit; ++c) {
-        const float w = fast_exp2(__ldcg(&a.part_ml[pbase + c]).x - mx);
-        if (w > 0.f) A = fmaf(w, __ldcg(&a.part_acc[(pbase + c) * kHeadDim + d]), A);
+      // 8 splits at a time with independent loads (one L2 round trip per 8 splits)
+      for (int c0 = 0; c0 < a.nsplit; c0 += 8) {
+        float mm[8], aa[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int c = c0 + u;
+          mm[u] = c < a.nsplit ? __ldcg(&a.part_ml[pbase + c]).x : -CUDART_INF_F;
+          aa[u] = c < a.nsplit ? __ldcg(&a.part_acc[(pbase + c) * kHeadDim + d]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float w = fast_exp2(mm[u] - mx);   // 0 for empty splits (mm = -inf)
+          A = fmaf(w, aa[u], A);
+        }
       }
     }
     store_out(a, r.t, r.h, d, L > 0.f ? A / L : 0.f);
@@ -257,174 +268,230 @@ __device__ void finish_lists(const DecodeArgs& a, const SeqInfo& si, int b, int 
 // ---------------------------------------------------------------------------
 // Sparse decode
 // ---------------------------------------------------------------------------
-// Scattered 256-byte rows are gathered straight into registers: a half-warp (16 lanes,
-// one 16-byte load each) owns a K row and a V row at a time, U rows in flight per
-// half-warp.  Measured on B200, this reaches the copy bandwidth for random 256-byte rows
-// at large sizes, while staging the same rows through shared memory (cp.async 16 B or
-// one 256-byte bulk copy per row) is 25-35% slower at every size.
-//
-// Work unit: (sequence b, kv head g, list group lg, split) -- up to 16 lists (q heads of
-// the GQA group x decode tokens of the sequence) and E consecutive entries of each.  The
-// grid is persistent (CTAs per SM x SMs); CTAs take units from a global counter, so the
-// tail is at most one small unit.  Within a unit every list gets P = 16 / lists
-// half-warps; each takes 16-entry chunks of its list in turn (chunk c -> part c % P), so
-// all lists of the kv head walk the token range together and a row picked by several of
-// them is read from DRAM once and served to the others from L1/L2.
-//
-// Per entry (half-warp): the 128-dim dot is 8 FMA per lane plus a 4-step shuffle
-// reduction; the online softmax keeps (max, sum, 8 output dims per lane) in registers.
-// At the end of a unit the parts of each list are combined, the split's partial is
-// written, and the last CTA to finish a (b, g, lg) merges its splits.
-constexpr int kSpU = 4;                 // rows in flight per half-warp
-constexpr int kSpThreads = 256;         // 16 half-warps
+// Design, from measurements on B200:
+//  * Scattered 256-byte rows are gathered with 16-byte loads straight into registers.
+//    For random 256-byte rows this reaches the copy bandwidth at large sizes; staging
+//    them in shared memory (cp.async, one bulk copy per row, or TMA gather4) is slower
+//    unless 4-6 CTAs per SM are resident.
+//  * What sets the gather rate is how many warps are issuing loads, so the work is cut
+//    into many small independent tasks: one half-warp (16 lanes x 16 bytes = one row)
+//    takes a chunk of E entries of one list (token x q head) and nothing else.  There is
+//    no block-level synchronisation and no shared memory.
+//  * Tasks are numbered (sequence, kv head, chunk, list) so that the lists of one kv head
+//    -- the q heads of a GQA group and the decode tokens of the sequence -- read the same
+//    token range in the same CTA at the same time: a row picked by several of them is
+//    read from DRAM once and served to the others from L1/L2.
+// Per row the half-warp computes a 128-dim dot (8 FMA per lane + a 4-step shuffle
+// reduction); its online softmax state (max, sum, 8 output dims per lane) is updated once
+// per batch of U rows in flight.  Each task writes its partial state; the last task of a list
+// to arrive (a per-list counter) merges them with log-sum-exp.  A list that fits one
+// task is written directly.
+constexpr int kSpThreads = 256;   // 16 half-warps, one task each
+constexpr int kSpU = 4;           // rows in flight per half-warp
 
-struct SparseSmem {
-  float comb[16 * kCombFloats];         // one state per half-warp
-  float mx[kMaxListsPerCta], lsum[kMaxListsPerCta];
-  int unit;
-};
+__device__ __forceinline__ void row_fetch(const DecodeArgs& a, uint32_t row, int l, uint4& k, uint4& v) {
+  if (row != kInvalidRow) {
+    k = __ldg(reinterpret_cast<const uint4*>(a.kv.k + (int64_t)row * kHeadDim) + l);
+    v = __ldg(reinterpret_cast<const uint4*>(a.kv.v + (int64_t)row * kHeadDim) + l);
+  }
+}
+
+// Online-softmax update of a half-warp's state with a batch of U rows at once: the U
+// scores are reduced together (independent shuffle chains), then one max, one rescale
+// and U independent exponentials -- the serial chain is per batch, not per row.
+template <int U>
+__device__ __forceinline__ void batch_update(const uint4* kq, const uint4* vq, const uint32_t* rr, const float* q,
+                                             float& m_run, float& l_run, float* acc, unsigned hmask) {
+  float s[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    float kf[8];
+    unpack8(kq[u], kf);
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      s0 = fmaf(q[j], kf[j], s0);
+      s1 = fmaf(q[j + 1], kf[j + 1], s1);
+    }
+    s[u] = s0 + s1;
+  }
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+    for (int u = 0; u < U; ++u) s[u] += __shfl_xor_sync(hmask, s[u], o);
+  float mb = -CUDART_INF_F;
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+    if (rr[u] != kInvalidRow) mb = fmaxf(mb, s[u]);
+  if (mb == -CUDART_INF_F) return;   // no valid row in the batch (uniform over the half-warp)
+  const float m_new = fmaxf(m_run, mb);
+  const float alpha = fast_exp2(m_run - m_new);   // 0 on the first batch (m_run = -inf)
+  l_run *= alpha;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] *= alpha;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const float p = rr[u] != kInvalidRow ? fast_exp2(s[u] - m_new) : 0.f;
+    l_run += p;
+    float vf[8];
+    unpack8(vq[u], vf);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = fmaf(p, vf[j], acc[j]);
+  }
+  m_run = m_new;
+}
 
 __global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs a) {
-  __shared__ __align__(16) SparseSmem S;
   const int lane = threadIdx.x & 31;
-  const int hw = threadIdx.x >> 4, l = threadIdx.x & 15;
+  const int l = threadIdx.x & 15;
   const unsigned hmask = 0xFFFFu << (lane & 16);
   const int G = a.qv.hq / a.kv.hkv;
-  const int E = a.span;
-  const int total_units = a.nsplit * a.list_groups * a.kv.hkv * a.kv.batch;
+  const int M = a.lists_per_cta;   // list slots per (sequence, kv head): G x max tokens per sequence
+  const int C = a.nsplit;          // tasks (chunks) per list
+  const int E = a.span;            // entries per task
+  const int64_t task = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4);
+  const int64_t total = (int64_t)a.kv.batch * a.kv.hkv * C * M;
+  if (task >= total) return;
+  const int m = (int)(task % M);
+  int64_t rest = task / M;
+  const int c = (int)(rest % C);
+  rest /= C;
+  const int g = (int)(rest % a.kv.hkv);
+  const int b = (int)(rest / a.kv.hkv);
+
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, c == 0 && g == 0 && m == 0 && l == 0);
+  const int j = m / G;
+  if (j >= si.n) return;           // no such list (fewer decode tokens in this sequence)
+  const int t = si.t0 + j, h = g * G + (m - j * G);
+  const int kvlen = kv_len_of(a.qv, si, j);
+  const int64_t list_id = (int64_t)t * a.qv.hq + h;
   const float scale = a.qv.sm_scale * kLog2e;
-  uint32_t* work = a.sched;       // unit counter and finished-CTA counter (zero between calls)
-  uint32_t* done = a.sched + 1;
 
-  for (;;) {
-    if (threadIdx.x == 0) S.unit = (int)atomicAdd(work, 1u);
-    __syncthreads();
-    const int unit = S.unit;
-    __syncthreads();
-    if (unit >= total_units) break;
-    const int split = unit % a.nsplit;
-    int rest = unit / a.nsplit;
-    const int lg = rest % a.list_groups;
-    rest /= a.list_groups;
-    const int g = rest % a.kv.hkv;
-    const int b = rest / a.kv.hkv;
-    const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, split == 0 && g == 0 && lg == 0 && threadIdx.x == 0);
-    int nlists = si.n * G - lg * a.lists_per_cta;
-    if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
-    if (nlists <= 0) continue;   // the same for every split of this (b, g, lg): no merge is owed
-
-    const int P = 16 / nlists;                 // half-warps per list
-    const int my_list = hw / P, my_part = hw % P;
-    const bool active = my_list < nlists;
-    float m_run = -CUDART_INF_F, l_run = 0.f, acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-
-    if (active) {
-      const ListRef r = list_ref(a, si, g, lg, my_list);
-      // this lane's 8 query dims [8l, 8l+8), scaled so that dots are base-2 softmax units
-      float q[8];
-      {
-        const int64_t qb = ((int64_t)r.t * a.qv.hq + r.h) * kHeadDim + 8 * l;
-        if (a.qv.q_f32) {
-          const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.qv.q) + qb);
-          const float4 x = __ldg(p), y = __ldg(p + 1);
-          q[0] = x.x; q[1] = x.y; q[2] = x.z; q[3] = x.w; q[4] = y.x; q[5] = y.y; q[6] = y.z; q[7] = y.w;
-        } else {
-          unpack8(__ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.qv.q) + qb)), q);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) q[j] *= scale;
-      }
-      const int32_t* lst = a.idx + ((int64_t)r.t * a.qv.hq + r.h) * a.k_max;
-      const int e0 = split * E;
-      const int e1 = min(e0 + E, a.k_max);
-      const int nchunks = (e1 - e0 + 15) >> 4;
-      uint32_t bad = 0;
-      for (int c = my_part; c < nchunks; c += P) {
-        // entry of this lane, its predecessor, validity and physical row
-        const int e = e0 + 16 * c + l;
-        const int32_t v = e < e1 ? __ldg(lst + e) : -1;
-        uint32_t before = __shfl_up_sync(hmask, (uint32_t)v, 1, 16);
-        if (l == 0) before = (e > 0) ? (uint32_t)__ldg(lst + e - 1) : 0u;
-        if (e < e1 && e > 0 && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
-        if (e < e1 && (v < -1 || v >= r.kvlen)) bad |= TSD_DEV_BAD_INDEX;
-        uint32_t row = kInvalidRow;
-        if (e < e1 && v >= 0 && v < r.kvlen) {
-          row = kv_row(a.kv, b, g, v);
-          if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
-        }
-        // the chunk's 16 rows, U at a time
-#pragma unroll
-        for (int j0 = 0; j0 < 16; j0 += kSpU) {
-          uint32_t rr[kSpU];
-          uint4 kr[kSpU], vr[kSpU];
-#pragma unroll
-          for (int u = 0; u < kSpU; ++u) {
-            rr[u] = __shfl_sync(hmask, row, j0 + u, 16);
-            if (rr[u] != kInvalidRow) {
-              kr[u] = __ldg(reinterpret_cast<const uint4*>(a.kv.k + (int64_t)rr[u] * kHeadDim) + l);
-              vr[u] = __ldg(reinterpret_cast<const uint4*>(a.kv.v + (int64_t)rr[u] * kHeadDim) + l);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < kSpU; ++u) {
-            if (rr[u] == kInvalidRow) continue;    // uniform over the half-warp
-            float kf[8], vf[8];
-            unpack8(kr[u], kf);
-            float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < 8; j += 2) {
-              s0 = fmaf(q[j], kf[j], s0);
-              s1 = fmaf(q[j + 1], kf[j + 1], s1);
-            }
-            float s = s0 + s1;
-            s += __shfl_xor_sync(hmask, s, 1);
-            s += __shfl_xor_sync(hmask, s, 2);
-            s += __shfl_xor_sync(hmask, s, 4);
-            s += __shfl_xor_sync(hmask, s, 8);
-            if (s > m_run) {
-              const float alpha = fast_exp2(m_run - s);
-              l_run *= alpha;
-#pragma unroll
-              for (int j = 0; j < 8; ++j) acc[j] *= alpha;
-              m_run = s;
-            }
-            const float p = fast_exp2(s - m_run);
-            l_run += p;
-            unpack8(vr[u], vf);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = fmaf(p, vf[j], acc[j]);
-          }
-        }
-      }
-      bad |= __shfl_xor_sync(hmask, bad, 1);
-      bad |= __shfl_xor_sync(hmask, bad, 2);
-      bad |= __shfl_xor_sync(hmask, bad, 4);
-      bad |= __shfl_xor_sync(hmask, bad, 8);
-      if (l == 0 && bad) flag_status(a.status, bad);
-      // this half-warp's state -> combine buffer entry (list * P + part)
-      float* ce = S.comb + (size_t)(my_list * P + my_part) * kCombFloats;
-      if (l == 0) {
-        ce[0] = m_run;
-        ce[1] = l_run;
-      }
-      *reinterpret_cast<float4*>(ce + 4 + 8 * l) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      *reinterpret_cast<float4*>(ce + 8 + 8 * l) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  // this lane's 8 query dims [8l, 8l+8), scaled so that dots are base-2 softmax units
+  float q[8];
+  {
+    const int64_t qb = list_id * kHeadDim + 8 * l;
+    if (a.qv.q_f32) {
+      const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.qv.q) + qb);
+      const float4 x = __ldg(p), y = __ldg(p + 1);
+      q[0] = x.x; q[1] = x.y; q[2] = x.z; q[3] = x.w; q[4] = y.x; q[5] = y.y; q[6] = y.z; q[7] = y.w;
+    } else {
+      unpack8(__ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.qv.q) + qb)), q);
     }
-    __syncthreads();
-    finish_lists(a, si, b, g, lg, split, nlists, P, S.comb, S.mx, S.lsum);
-    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] *= scale;
   }
-  // the last CTA out resets the unit counters for the next call
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const uint32_t prev = atomicAdd(done, 1u);
-    if (prev == gridDim.x - 1) {
-      atomicExch(work, 0u);
-      atomicExch(done, 0u);
+
+  const int32_t* lst = a.idx + list_id * a.k_max;
+  const int e0 = c * E;
+  const int e1 = min(e0 + E, a.k_max);
+  float m_run = -CUDART_INF_F, l_run = 0.f, acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  uint32_t bad = 0;
+  for (int base = e0; base < e1; base += 16) {
+    // this lane's entry: index, predecessor check, validity, physical row
+    const int e = base + l;
+    const int32_t v = e < e1 ? __ldg(lst + e) : -1;
+    uint32_t before = __shfl_up_sync(hmask, (uint32_t)v, 1, 16);
+    if (l == 0 && e > 0 && e < e1) before = (uint32_t)__ldg(lst + e - 1);
+    if (e < e1 && e > 0 && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
+    if (e < e1 && (v < -1 || v >= kvlen)) bad |= TSD_DEV_BAD_INDEX;
+    uint32_t row = kInvalidRow;
+    if (e < e1 && v >= 0 && v < kvlen) {
+      row = kv_row(a.kv, b, g, v);
+      if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
+    }
+    // the 16 rows, U at a time
+#pragma unroll
+    for (int j0 = 0; j0 < 16; j0 += kSpU) {
+      uint32_t rr[kSpU];
+      uint4 kq[kSpU], vq[kSpU];
+#pragma unroll
+      for (int u = 0; u < kSpU; ++u) {
+        rr[u] = __shfl_sync(hmask, row, j0 + u, 16);
+        kq[u] = make_uint4(0, 0, 0, 0);
+        vq[u] = make_uint4(0, 0, 0, 0);
+        row_fetch(a, rr[u], l, kq[u], vq[u]);
+      }
+      batch_update<kSpU>(kq, vq, rr, q, m_run, l_run, acc, hmask);
     }
   }
+  bad |= __shfl_xor_sync(hmask, bad, 1);
+  bad |= __shfl_xor_sync(hmask, bad, 2);
+  bad |= __shfl_xor_sync(hmask, bad, 4);
+  bad |= __shfl_xor_sync(hmask, bad, 8);
+  if (l == 0 && bad) flag_status(a.status, bad);
+
+  if (C == 1) {   // the whole list in one task
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, acc[i] * inv);
+    if (l == 0 && a.lse != nullptr) a.lse[list_id] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -CUDART_INF_F;
+    return;
+  }
+  // partial of this task, then the per-list arrival count
+  const int64_t pidx = list_id * C + c;
+  if (l == 0) a.part_ml[pidx] = make_float2(m_run, l_run);
+  float4* pa = reinterpret_cast<float4*>(a.part_acc + pidx * kHeadDim + 8 * l);
+  pa[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  pa[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  __threadfence();
+  __syncwarp(hmask);
+  uint32_t prev = 0;
+  if (l == 0) {
+    prev = atomicAdd(a.counters + list_id, 1u);
+    if (prev == (uint32_t)(C - 1)) atomicExch(a.counters + list_id, 0u);   // leave it zero for the next call
+  }
+  prev = __shfl_sync(hmask, prev, 0, 16);
+  if (prev != (uint32_t)(C - 1)) return;
+  __threadfence();
+  // last task of the list: merge its C partials (lanes over splits for the max and sum,
+  // then 8 output dims per lane with independent loads)
+  const float2* ml = a.part_ml + list_id * C;
+  float mx = -CUDART_INF_F;
+  for (int i = l; i < C; i += 16) mx = fmaxf(mx, __ldcg(&ml[i]).x);
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 4));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 8));
+  float L = 0.f;
+  float o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  if (mx != -CUDART_INF_F) {
+    for (int i = l; i < C; i += 16) {
+      const float2 x = __ldcg(&ml[i]);
+      L = fmaf(fast_exp2(x.x - mx), x.y, L);
+    }
+    L += __shfl_xor_sync(hmask, L, 1);
+    L += __shfl_xor_sync(hmask, L, 2);
+    L += __shfl_xor_sync(hmask, L, 4);
+    L += __shfl_xor_sync(hmask, L, 8);
+    for (int c0 = 0; c0 < C; c0 += 4) {
+      float w[4];
+      float4 x0[4], x1[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int cc = c0 + u;
+        w[u] = cc < C ? fast_exp2(__ldcg(&ml[cc]).x - mx) : 0.f;
+        const float4* src = reinterpret_cast<const float4*>(a.part_acc + (list_id * C + (cc < C ? cc : 0)) * kHeadDim + 8 * l);
+        x0[u] = __ldcg(src);
+        x1[u] = __ldcg(src + 1);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        o[0] = fmaf(w[u], x0[u].x, o[0]); o[1] = fmaf(w[u], x0[u].y, o[1]);
+        o[2] = fmaf(w[u], x0[u].z, o[2]); o[3] = fmaf(w[u], x0[u].w, o[3]);
+        o[4] = fmaf(w[u], x1[u].x, o[4]); o[5] = fmaf(w[u], x1[u].y, o[5]);
+        o[6] = fmaf(w[u], x1[u].z, o[6]); o[7] = fmaf(w[u], x1[u].w, o[7]);
+      }
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, o[i] * inv);
+  if (l == 0 && a.lse != nullptr) a.lse[list_id] = L > 0.f ? (mx + log2f(L)) * kLn2 : -CUDART_INF_F;
 }
 
 // ---------------------------------------------------------------------------
@@ -573,19 +640,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) dense_decode_kernel(DecodeA
 // Host launchers
 // ---------------------------------------------------------------------------
 cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
-  static int ctas_per_sm = 0, sms = 0;
-  if (ctas_per_sm == 0) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, sparse_decode_kernel, kSpThreads, 0);
-    if (e != cudaSuccess) return e;
-    if (ctas_per_sm < 1) ctas_per_sm = 1;
-  }
-  const int units = a.nsplit * a.list_groups * hkv * batch;
-  int grid = ctas_per_sm * sms;
-  if (grid > units) grid = units;
-  sparse_decode_kernel<<<grid, kSpThreads, 0, stream>>>(a);
+  const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
+  const int64_t grid = (tasks + 15) / 16;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  sparse_decode_kernel<<<(unsigned)grid, kSpThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

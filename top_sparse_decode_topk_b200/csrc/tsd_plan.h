@@ -3,8 +3,8 @@
 // Workspace layout (bytes from the start; every region 256-byte aligned):
 //   [0, 256)              header: device status word (uint32) at offset 0; sparse-decode
 //                         work-unit counter at byte 4 and finished-CTA counter at byte 8
-//   counters              uint32 [batch][num_kv_heads][group * max_tokens]: arrival counters
-//                         of the split-K merge, one per list group (zero between calls)
+//   counters              uint32, one per list (token x q head): arrival counters of the
+//                         split-K merge (zero between calls)
 //   -- everything above is the "zero region": it must be zero when a call starts and every
 //      call leaves it zero --
 //   decode partials       float2 [T][Hq][nsplit] (running max, running sum; base-2 units)
@@ -29,7 +29,6 @@ constexpr int kStages = 4;              // cp.async pipeline depth
 constexpr int kMaxEntriesPerCta = 1024; // sparse: lists x entries per CTA
 constexpr int kBitmapWords = 1024;      // sparse: dedupe bitmap spans 32768 tokens
 constexpr int kMaxSplits = 256;         // split-K partials per (token, head)
-constexpr int kSparseEntriesTarget = 256;  // sparse: entries (all lists) a CTA aims for
 constexpr int kScoreThreads = 256;
 constexpr int kSelectThreads = 512;
 constexpr int kScoreTokensPerCta = 1024;
@@ -45,38 +44,45 @@ inline int list_groups(const Shapes& s) {
   return (int)((m + kMaxListsPerCta - 1) / kMaxListsPerCta);
 }
 
-// Room for one counter per list, enough for any split of the lists into groups.
+// Room for one arrival counter per list (token x q head), which also covers one per
+// (sequence, kv head, list group).
 inline size_t zero_region_bytes(const Shapes& s) {
-  return 256 + align256((size_t)s.batch * s.hkv * s.group * s.max_tokens * sizeof(uint32_t));
+  const int64_t toks = s.batch * s.max_tokens > s.tokens ? s.batch * s.max_tokens : s.tokens;
+  return 256 + align256((size_t)toks * s.hq * sizeof(uint32_t));
 }
 
 // Longest index list tsd_sparse_decode accepts (kMaxSplits chunks of at most
 // kMaxEntriesPerCta entries).
 constexpr int kMaxSparseK = kMaxSplits * kMaxEntriesPerCta;
 
-// Sparse decode: entries per list per CTA (E) and number of splits.
+// Sparse decode: every list (token x q head) is cut into C tasks of E entries (E a
+// multiple of 16); a task is one half-warp.  E grows with the workload so that the task
+// count stays near kSparseTaskTarget (a few per resident half-warp of a B200: enough to
+// keep every SM issuing gathers, few enough that the split-K partials stay small), and
+// C stays <= kMaxSplits.
 struct SparsePlan {
-  int lists_per_cta;
-  int list_groups;
+  int lists;     // list slots per (sequence, kv head): G x max tokens per sequence
   int entries;   // E
-  int nsplit;
+  int nsplit;    // C
 };
+
+constexpr int64_t kSparseTaskTarget = 2 * 148 * 48;
 
 inline SparsePlan plan_sparse(const Shapes& s, int k_max) {
   SparsePlan p;
-  const int64_t m = s.group * s.max_tokens;
-  int lists = (int)(m < kSparseMaxLists ? m : kSparseMaxLists);
-  const int kr = (k_max + 15) / 16 * 16;
-  int e = (kSparseEntriesTarget / lists + 15) / 16 * 16;
+  p.lists = (int)(s.group * s.max_tokens);
+  const double total = (double)s.tokens * s.hq * k_max;
+  int e = (int)(total / kSparseTaskTarget);
+  e = (e + 15) / 16 * 16;
   if (e < 16) e = 16;
+  if (e > 1024) e = 1024;
+  const int kr = (k_max + 15) / 16 * 16;
   if (e > kr) e = kr;
   int ns = (k_max + e - 1) / e;
   if (ns > kMaxSplits) {
-    e = ((k_max + kMaxSplits - 1) / kMaxSplits + 15) / 16 * 16;   // long lists: bigger chunks
+    e = ((k_max + kMaxSplits - 1) / kMaxSplits + 15) / 16 * 16;
     ns = (k_max + e - 1) / e;
   }
-  p.lists_per_cta = lists;
-  p.list_groups = (int)((m + lists - 1) / lists);
   p.entries = e;
   p.nsplit = ns;
   return p;
