@@ -6,24 +6,11 @@
 // index list -- which may differ per token, per query and per head -- so that
 // the bytes read fall from O(N d) to O(k d).  Dense decode attends to every row.
 //
-// Work unit (one CTA): sequence b, kv head g, a group of up to 32 query lists
-// (q heads of the GQA group x decode tokens of the sequence) and one split of
-// the work: a chunk of E consecutive entries of every list (sparse) or a window
-// of W consecutive tokens (dense).
-//
-// Sparse CTA, in order:
-//   1. load the chunk's entries of every list, validate and compact them;
-//   2. deduplicate the rows across lists with a bitmap over the chunk's token
-//      span (one bit per token; a prefix popcount gives each row its slot), so
-//      a row picked by several heads or tokens is loaded once;
-//   3. stream the unique rows through a 4-stage cp.async ring of 16-row tiles
-//      (16-byte copies; K and V rows are 256 bytes each);
-//   4. 32 lane-groups of 8 lanes walk the lists: each entry's score is a 16-wide
-//      fp32 dot per lane reduced over the group with 3 shuffles, followed by an
-//      online-softmax update of the group's (max, sum, 128-wide row) state;
-//   5. combine the groups of a list, write the split's partial, and the last
-//      CTA of the (b, g, list group) to arrive merges the splits (log-sum-exp).
-// No CTA ever waits on another: the merge is done by whichever arrives last.
+// Sparse decode: one half-warp per task (16+ entries of one list); rows gathered into
+// registers; batched online softmax; per-list split-K merge by the last task to finish.
+// Dense decode: one CTA per (sequence, kv head, list group, window of W tokens); rows
+// staged through a cp.async ring; CTA-level partials merged by the last CTA of the unit.
+// No kernel ever waits on another CTA: merges are done by whichever arrives last.
 #include <cuda_runtime.h>
 #include <math_constants.h>
 #include <stdint.h>
@@ -341,6 +328,83 @@ __device__ __forceinline__ void batch_update(const uint4* kq, const uint4* vq, c
   m_run = m_new;
 }
 
+// End of a task: a list that fits one task is written directly; otherwise the task's
+// partial state is stored, and the last task of the list to arrive (per-list counter)
+// merges the C partials with log-sum-exp.  Called by the 16 lanes of one half-warp
+// (hmask), lane l holding output dims [8l, 8l+8).
+__device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id, int t, int h, int C, int c,
+                                            float m_run, float l_run, const float* acc, int l, unsigned hmask) {
+  if (C == 1) {   // the whole list in one task
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, acc[i] * inv);
+    if (l == 0 && a.lse != nullptr) a.lse[list_id] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -CUDART_INF_F;
+    return;
+  }
+  // partial of this task, then the per-list arrival count
+  const int64_t pidx = list_id * C + c;
+  if (l == 0) a.part_ml[pidx] = make_float2(m_run, l_run);
+  float4* pa = reinterpret_cast<float4*>(a.part_acc + pidx * kHeadDim + 8 * l);
+  pa[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  pa[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  __threadfence();
+  __syncwarp(hmask);
+  uint32_t prev = 0;
+  if (l == 0) {
+    prev = atomicAdd(a.counters + list_id, 1u);
+    if (prev == (uint32_t)(C - 1)) atomicExch(a.counters + list_id, 0u);   // leave it zero for the next call
+  }
+  prev = __shfl_sync(hmask, prev, 0, 16);
+  if (prev != (uint32_t)(C - 1)) return;
+  __threadfence();
+  // last task of the list: merge its C partials (lanes over splits for the max and sum,
+  // then 8 output dims per lane with independent loads)
+  const float2* ml = a.part_ml + list_id * C;
+  float mx = -CUDART_INF_F;
+  for (int i = l; i < C; i += 16) mx = fmaxf(mx, __ldcg(&ml[i]).x);
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 4));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 8));
+  float L = 0.f;
+  float o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  if (mx != -CUDART_INF_F) {
+    for (int i = l; i < C; i += 16) {
+      const float2 x = __ldcg(&ml[i]);
+      L = fmaf(fast_exp2(x.x - mx), x.y, L);
+    }
+    L += __shfl_xor_sync(hmask, L, 1);
+    L += __shfl_xor_sync(hmask, L, 2);
+    L += __shfl_xor_sync(hmask, L, 4);
+    L += __shfl_xor_sync(hmask, L, 8);
+    for (int c0 = 0; c0 < C; c0 += 4) {
+      float w[4];
+      float4 x0[4], x1[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int cc = c0 + u;
+        w[u] = cc < C ? fast_exp2(__ldcg(&ml[cc]).x - mx) : 0.f;
+        const float4* src = reinterpret_cast<const float4*>(a.part_acc + (list_id * C + (cc < C ? cc : 0)) * kHeadDim + 8 * l);
+        x0[u] = __ldcg(src);
+        x1[u] = __ldcg(src + 1);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        o[0] = fmaf(w[u], x0[u].x, o[0]); o[1] = fmaf(w[u], x0[u].y, o[1]);
+        o[2] = fmaf(w[u], x0[u].z, o[2]); o[3] = fmaf(w[u], x0[u].w, o[3]);
+        o[4] = fmaf(w[u], x1[u].x, o[4]); o[5] = fmaf(w[u], x1[u].y, o[5]);
+        o[6] = fmaf(w[u], x1[u].z, o[6]); o[7] = fmaf(w[u], x1[u].w, o[7]);
+      }
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, o[i] * inv);
+  if (l == 0 && a.lse != nullptr) a.lse[list_id] = L > 0.f ? (mx + log2f(L)) * kLn2 : -CUDART_INF_F;
+}
+
 __global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs a) {
   const int lane = threadIdx.x & 31;
   const int l = threadIdx.x & 15;
@@ -423,75 +487,7 @@ __global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs
   bad |= __shfl_xor_sync(hmask, bad, 8);
   if (l == 0 && bad) flag_status(a.status, bad);
 
-  if (C == 1) {   // the whole list in one task
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, acc[i] * inv);
-    if (l == 0 && a.lse != nullptr) a.lse[list_id] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -CUDART_INF_F;
-    return;
-  }
-  // partial of this task, then the per-list arrival count
-  const int64_t pidx = list_id * C + c;
-  if (l == 0) a.part_ml[pidx] = make_float2(m_run, l_run);
-  float4* pa = reinterpret_cast<float4*>(a.part_acc + pidx * kHeadDim + 8 * l);
-  pa[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  pa[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  __threadfence();
-  __syncwarp(hmask);
-  uint32_t prev = 0;
-  if (l == 0) {
-    prev = atomicAdd(a.counters + list_id, 1u);
-    if (prev == (uint32_t)(C - 1)) atomicExch(a.counters + list_id, 0u);   // leave it zero for the next call
-  }
-  prev = __shfl_sync(hmask, prev, 0, 16);
-  if (prev != (uint32_t)(C - 1)) return;
-  __threadfence();
-  // last task of the list: merge its C partials (lanes over splits for the max and sum,
-  // then 8 output dims per lane with independent loads)
-  const float2* ml = a.part_ml + list_id * C;
-  float mx = -CUDART_INF_F;
-  for (int i = l; i < C; i += 16) mx = fmaxf(mx, __ldcg(&ml[i]).x);
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 2));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 8));
-  float L = 0.f;
-  float o[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) o[i] = 0.f;
-  if (mx != -CUDART_INF_F) {
-    for (int i = l; i < C; i += 16) {
-      const float2 x = __ldcg(&ml[i]);
-      L = fmaf(fast_exp2(x.x - mx), x.y, L);
-    }
-    L += __shfl_xor_sync(hmask, L, 1);
-    L += __shfl_xor_sync(hmask, L, 2);
-    L += __shfl_xor_sync(hmask, L, 4);
-    L += __shfl_xor_sync(hmask, L, 8);
-    for (int c0 = 0; c0 < C; c0 += 4) {
-      float w[4];
-      float4 x0[4], x1[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int cc = c0 + u;
-        w[u] = cc < C ? fast_exp2(__ldcg(&ml[cc]).x - mx) : 0.f;
-        const float4* src = reinterpret_cast<const float4*>(a.part_acc + (list_id * C + (cc < C ? cc : 0)) * kHeadDim + 8 * l);
-        x0[u] = __ldcg(src);
-        x1[u] = __ldcg(src + 1);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        o[0] = fmaf(w[u], x0[u].x, o[0]); o[1] = fmaf(w[u], x0[u].y, o[1]);
-        o[2] = fmaf(w[u], x0[u].z, o[2]); o[3] = fmaf(w[u], x0[u].w, o[3]);
-        o[4] = fmaf(w[u], x1[u].x, o[4]); o[5] = fmaf(w[u], x1[u].y, o[5]);
-        o[6] = fmaf(w[u], x1[u].z, o[6]); o[7] = fmaf(w[u], x1[u].w, o[7]);
-      }
-    }
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, o[i] * inv);
-  if (l == 0 && a.lse != nullptr) a.lse[list_id] = L > 0.f ? (mx + log2f(L)) * kLn2 : -CUDART_INF_F;
+  finish_task(a, list_id, t, h, C, c, m_run, l_run, acc, l, hmask);
 }
 
 // ---------------------------------------------------------------------------

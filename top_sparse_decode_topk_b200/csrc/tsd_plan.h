@@ -71,6 +71,7 @@ constexpr int64_t kSparseTaskTarget = 2 * 148 * 48;
 inline SparsePlan plan_sparse(const Shapes& s, int k_max) {
   SparsePlan p;
   p.lists = (int)(s.group * s.max_tokens);
+
   const double total = (double)s.tokens * s.hq * k_max;
   int e = (int)(total / kSparseTaskTarget);
   e = (e + 15) / 16 * 16;
