@@ -1,18 +1,23 @@
 // extern "C" entry points of libtsd: host-side validation, work decomposition,
 // workspace layout and kernel launches.  See include/tsd.h for the contract.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "tsd.h"
 #include "tsd_common.cuh"
 #include "tsd_plan.h"
 
 #include "tsd_args.h"
+#include "tsd_kvtile.cuh"
 
 namespace tsd {
 cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream);
-cudaError_t launch_dense_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream);
+cudaError_t launch_dense_decode(const DecodeArgs& a, const KvMaps& maps, int batch, int hkv, cudaStream_t stream);
 cudaError_t launch_topk(const TopkArgs& a, int nwin, int batch, int hkv, int num_lists, cudaStream_t stream);
 }  // namespace tsd
 
@@ -95,6 +100,50 @@ tsd_status check_inputs(const tsd_kv_cache* c, const tsd_queries* q, KvView* kv,
 }
 
 tsd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TSD_OK : TSD_ERR_CUDA; }
+
+// Tensor maps of the K and V caches seen as [rows][128] bf16 with a {64, box_rows} box and
+// 128-byte swizzling, for the TMA loads of the dense-tile kernels.  Caches whose pages
+// are smaller than 8 tokens do not use them (their tiles are copied with cp.async).
+tsd_status make_kv_maps(const tsd_kv_cache* c, KvMaps* maps) {
+  memset(maps, 0, sizeof(*maps));
+  int64_t rows;
+  int box_rows;
+  if (c->layout == TSD_LAYOUT_CONTIGUOUS) {
+    rows = (int64_t)c->batch * c->num_kv_heads * c->max_seq_len;
+    box_rows = 16;
+  } else {
+    if (c->page_size < 8) return TSD_OK;
+    rows = c->num_pages * c->num_kv_heads * c->page_size;
+    box_rows = c->page_size < 16 ? c->page_size : 16;
+  }
+  if (rows >= (int64_t)1 << 31) return TSD_ERR_UNSUPPORTED;
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (encode == nullptr) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return TSD_ERR_CUDA;
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const void* ptrs[2] = {c->k, c->v};
+  CUtensorMap* out[2] = {&maps->k, &maps->v};
+  for (int i = 0; i < 2; ++i) {
+    const CUresult r = encode(out[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptrs[i]), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return TSD_ERR_CUDA;
+  }
+  return TSD_OK;
+}
 
 }  // namespace
 
@@ -263,7 +312,10 @@ tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* querie
   a.counters = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_counters);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.off_ml);
   a.part_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_acc);
-  return cuda_status(launch_dense_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
+  KvMaps maps;
+  st = make_kv_maps(cache, &maps);
+  if (st != TSD_OK) return st;
+  return cuda_status(launch_dense_decode(a, maps, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tsd_status tsd_read_device_status(void* ws, tsd_stream_t stream, uint32_t* flags) {

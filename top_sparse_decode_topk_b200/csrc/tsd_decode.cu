@@ -17,13 +17,12 @@
 
 #include "tsd_args.h"
 #include "tsd_common.cuh"
+#include "tsd_kvtile.cuh"
 
 namespace tsd {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr int kTileBytes = kRowsPerTile * 2 * 256;          // K rows then V rows
-constexpr int kRingBytes = kStages * kTileBytes;
 constexpr int kCombFloats = 132;                             // m, l, pad, pad, acc[128]
 
 
@@ -491,145 +490,241 @@ __global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs
 }
 
 // ---------------------------------------------------------------------------
-// Dense decode: every token of [split*W, split*W + W) for all lists of the CTA.
-// Lane-groups hold 2 lists each ("sets"); the groups of a set split the tile's rows.
+// Dense decode on tensor cores
 // ---------------------------------------------------------------------------
-constexpr int kDenseHeadsPerGroup = 2;
+// One CTA per (sequence b, kv head g, list group lg, window of W tokens): up to 16 lists
+// (q heads of the GQA group x decode tokens) are the rows of the mma M dimension.  A
+// producer warp streams 64-token K/V tiles through a 3-stage ring (TMA, see tsd_kvtile.cuh);
+// each of the 4 consumer warps takes 16 tokens of every tile:
+//   S = q K^T (16 x 16, 8 k-steps of mma.m16n8k16), scaled to base-2 softmax units in fp32,
+//   masked past each list's kv_len; online softmax per query row (quad shuffles);
+//   O += P V with P split into bf16 hi + lo (two MMAs, ~16-bit weights) and V read with
+//   transposing ldmatrix.
+// The 4 warp states of each list are combined at the end and merged across windows like the
+// sparse path's CTA partials.
+constexpr int kDnStages = 3;
+constexpr int kDnConsumers = 4;
+constexpr int kDnThreads = 32 * (kDnConsumers + 1);
+constexpr int kDnStageBytes = 2 * kTileBytesKV;   // K then V
 
 struct DenseSmem {
-  unsigned char ring[kRingBytes + 2048];   // ring; combine buffer (needs 32*2*132 floats)
-  uint32_t rowaddr[kStages][kRowsPerTile];
-  float mx[kMaxListsPerCta], lsum[kMaxListsPerCta];
+  alignas(1024) unsigned char stage[kDnStages][kDnStageBytes];   // also the combine buffer
+  uint64_t full[kDnStages];
+  uint64_t empty[kDnStages];
+  uint32_t abort;
+  float mx[16], lsum[16];
 };
-static_assert(kRingBytes + 2048 >= 32 * kDenseHeadsPerGroup * kCombFloats * 4, "dense combine buffer");
+static_assert(kDnStages * kDnStageBytes >= 16 * kDnConsumers * kCombFloats * 4, "dense combine buffer");
 
-__device__ __forceinline__ void dense_load_tile(DenseSmem& S, const KvView& kv, int b, int g, int tok0,
-                                                int tile, int ntok, uint32_t* status) {
-  const int stage = tile % kStages;
-  unsigned char* base = S.ring + stage * kTileBytes;
-  const int first = tok0 + tile * kRowsPerTile;
-#pragma unroll
-  for (int q = 0; q < (kRowsPerTile * 32) / kDecodeThreads; ++q) {
-    const int id = threadIdx.x + q * kDecodeThreads;
-    const int r = id >> 5, which = (id >> 4) & 1, ch = id & 15;
-    const int tok = first + r;
-    if (tok - tok0 < ntok) {
-      const uint32_t row = kv_row(kv, b, g, tok);
-      if (row != kInvalidRow) {
-        const uint16_t* src = (which ? kv.v : kv.k) + (int64_t)row * kHeadDim + ch * 8;
-        cp_async16(base + which * (kRowsPerTile * 256) + r * 256 + ch * 16, src);
-      }
-      if (which == 0 && ch == 0) {
-        S.rowaddr[stage][r] = row;
-        if (row == kInvalidRow) flag_status(status, TSD_DEV_BAD_PAGE);
-      }
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kDecodeThreads, 2) dense_decode_kernel(DecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  DenseSmem& S = *reinterpret_cast<DenseSmem*>(smem_raw);
-
+template <bool QF32>
+__global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(DecodeArgs a, const __grid_constant__ KvMaps maps) {
+  extern __shared__ __align__(1024) unsigned char smem_dn[];
+  DenseSmem& S = *reinterpret_cast<DenseSmem*>(smem_dn);
   const int split = blockIdx.x;
   const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
   const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, split == 0 && g == 0 && lg == 0 && threadIdx.x == 0);
   const int G = a.qv.hq / a.kv.hkv;
   int nlists = si.n * G - lg * a.lists_per_cta;
   if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
   if (nlists <= 0) return;
-
   const int tok0 = split * a.span;
-  int ntok = si.len - tok0;
-  if (ntok > a.span) ntok = a.span;
-  if (ntok < 0) ntok = 0;
-  const int ntiles = (ntok + kRowsPerTile - 1) / kRowsPerTile;
-
-#pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < ntiles) dense_load_tile(S, a.kv, b, g, tok0, s, ntok, a.status);
-    cp_async_commit();
+  const int tok_end = min(tok0 + a.span, si.len);
+  const int ntiles = tok_end > tok0 ? (tok_end - tok0 + kTileTok - 1) / kTileTok : 0;
+  const bool use_tma = a.kv.page_table == nullptr || a.kv.page_shift >= 3;
+  // the swizzled tiles need 1024-byte alignment; refuse to run rather than mis-address them
+  if (smem_u32(S.stage[0]) & 1023u) {
+    if (threadIdx.x == 0) flag_status(a.status, TSD_DEV_TIMEOUT);
+    return;
   }
 
-  const int group = threadIdx.x >> 3, l8 = threadIdx.x & 7;
-  const int nsets = (nlists + kDenseHeadsPerGroup - 1) / kDenseHeadsPerGroup;
-  const int PG = 32 / nsets;   // groups per set (nsets <= 16 -> PG >= 2)
-  const int my_set = group / PG, my_part = group % PG;
-  const bool has_set = my_set < nsets;
-
-  float q[kDenseHeadsPerGroup][16];
-  SoftState st[kDenseHeadsPerGroup];
-  int kvlen[kDenseHeadsPerGroup];
-  const float scale = a.qv.sm_scale * kLog2e;
-#pragma unroll
-  for (int hh = 0; hh < kDenseHeadsPerGroup; ++hh) {
-    soft_init(st[hh]);
-    const int m = my_set * kDenseHeadsPerGroup + hh;
-    const ListRef r = list_ref(a, si, g, lg, (has_set && m < nlists) ? m : 0);
-    kvlen[hh] = (has_set && m < nlists) ? r.kvlen : 0;
-    load_q16(a.qv, r.t, r.h, l8, scale, q[hh]);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDnStages; ++s) {
+      mbar_init(&S.full[s], use_tma ? 1 : 32);
+      mbar_init(&S.empty[s], kDnConsumers);
+    }
+    mbar_fence_init();
+    S.abort = 0;
   }
+  __syncthreads();
 
-  for (int tile = 0; tile < ntiles; ++tile) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (tile + kStages - 1 < ntiles) dense_load_tile(S, a.kv, b, g, tok0, tile + kStages - 1, ntok, a.status);
-    cp_async_commit();
+  // per warp state: rows r0 = lane/4 and r0 + 8
+  float o[16][4];
+  float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_run[2] = {0.f, 0.f};
 
-    const int stage = tile % kStages;
-    const unsigned char* kbase = S.ring + stage * kTileBytes;
-    const unsigned char* vbase = kbase + kRowsPerTile * 256;
-    const int rows = min(kRowsPerTile, ntok - tile * kRowsPerTile);
-    // rows r = my_part, my_part + PG, ...: the loop bound is the same for every group
-    for (int r0 = 0; r0 < kRowsPerTile; r0 += PG) {
-      const int r = r0 + my_part;
-      const bool row_ok = has_set && r < rows && S.rowaddr[stage][r < kRowsPerTile ? r : 0] != kInvalidRow;
-      const int rr = (r < kRowsPerTile) ? r : 0;
-      const int tok = tok0 + tile * kRowsPerTile + rr;
-      const unsigned char* krow = kbase + rr * 256;
-      uint4 k0 = *reinterpret_cast<const uint4*>(krow + 16 * l8);
-      uint4 k1 = *reinterpret_cast<const uint4*>(krow + 128 + 16 * l8);
-      float kf[16];
-      unpack8(k0, kf);
-      unpack8(k1, kf + 8);
-      float s[kDenseHeadsPerGroup];
-#pragma unroll
-      for (int hh = 0; hh < kDenseHeadsPerGroup; ++hh) {
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          s0 = fmaf(q[hh][j], kf[j], s0);
-          s1 = fmaf(q[hh][8 + j], kf[8 + j], s1);
+  if (warp == kDnConsumers) {
+    // producer
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int s = tile % kDnStages;
+      if (tile >= kDnStages) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&S.empty[s], ((tile / kDnStages) - 1) & 1);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
+            flag_status(a.status, TSD_DEV_TIMEOUT);
+            atomicOr(&S.abort, 1u);
+          }
+          break;
         }
-        s[hh] = s0 + s1;
       }
-#pragma unroll
-      for (int hh = 0; hh < kDenseHeadsPerGroup; ++hh) {
-        s[hh] += __shfl_xor_sync(0xFFFFFFFFu, s[hh], 1);
-        s[hh] += __shfl_xor_sync(0xFFFFFFFFu, s[hh], 2);
-        s[hh] += __shfl_xor_sync(0xFFFFFFFFu, s[hh], 4);
+      unsigned char* kd = S.stage[s];
+      unsigned char* vd = S.stage[s] + kTileBytesKV;
+      const int tok = tok0 + tile * kTileTok;
+      if (use_tma) {
+        if (lane == 0) {
+          // the expected bytes must be registered before the loads can complete the phase
+          const int bp = a.kv.page_table == nullptr ? 16 : min(16, 1 << a.kv.page_shift);
+          const int rows = min(kTileTok, tok_end - tok);
+          uint32_t want = 0;
+          for (int r = 0; r < rows; r += bp) want += 4 * bp * 128;
+          mbar_arrive_expect_tx(&S.full[s], want);
+          const uint32_t got = tile_issue_tma(a.kv, &maps.k, &maps.v, b, g, tok, tok_end, kd, vd, &S.full[s], a.status);
+          // rows skipped for a bad page never arrive: complete them so the phase still ends
+          if (got < want) asm volatile("{\n .reg .b64 st;\n mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n}\n" ::"r"(smem_u32(&S.full[s])), "r"(want - got) : "memory");
+        }
+      } else {
+        tile_issue_cpasync(a.kv, b, g, tok, tok_end, kd, vd, lane, a.status);
+        cp_async_mbar_arrive(&S.full[s]);
       }
-      if (row_ok) {
+    }
+    if (lane == 0) {
+      for (int tile = (ntiles > kDnStages ? ntiles - kDnStages : 0); tile < ntiles; ++tile)
+        if (!mbar_wait(&S.full[tile % kDnStages], (tile / kDnStages) & 1)) flag_status(a.status, TSD_DEV_TIMEOUT);
+    }
+  } else {
+    const int w = warp;
+    const float scale2 = a.qv.sm_scale * kLog2e;
+    QFrags<QF32> qf;
+    load_q_frags<QF32>(a.qv, si, g, G, lg * a.lists_per_cta, nlists, lane, qf);
+    int kvl[2];
 #pragma unroll
-        for (int hh = 0; hh < kDenseHeadsPerGroup; ++hh)
-          if (tok < kvlen[hh]) soft_update(st[hh], s[hh], vbase + rr * 256, l8);
+    for (int hr = 0; hr < 2; ++hr) {
+      const int m = (lane >> 2) + 8 * hr;
+      kvl[hr] = m < nlists ? kv_len_of(a.qv, si, (lg * a.lists_per_cta + m) / G) : 0;
+    }
+#pragma unroll
+    for (int nd = 0; nd < 16; ++nd) o[nd][0] = o[nd][1] = o[nd][2] = o[nd][3] = 0.f;
+    const int i4 = lane >> 3, rr = lane & 7;
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int s = tile % kDnStages;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&S.full[s], (tile / kDnStages) & 1);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok || S.abort) {
+        if (lane == 0 && !ok) flag_status(a.status, TSD_DEV_TIMEOUT);
+        break;
+      }
+      const unsigned char* kt = S.stage[s];
+      const unsigned char* vt = S.stage[s] + kTileBytesKV;
+      float sc[2][4];
+      qk_tile<QF32>(qf, kt, w, lane, sc);
+      // scale, mask, online softmax per query row
+      const int tbase = tok0 + tile * kTileTok + 16 * w + 2 * (lane & 3);
+      float p[2][4];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        float mloc = -CUDART_INF_F;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int tk = tbase + 8 * nt + j;
+            float v = sc[nt][2 * hr + j] * scale2;
+            if (tk >= kvl[hr] || tk >= tok_end) v = -CUDART_INF_F;
+            sc[nt][2 * hr + j] = v;
+            mloc = fmaxf(mloc, v);
+          }
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xFFFFFFFFu, mloc, 1));
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xFFFFFFFFu, mloc, 2));
+        const float mnew = fmaxf(m_run[hr], mloc);
+        const float alpha = mnew == -CUDART_INF_F ? 1.f : fast_exp2(m_run[hr] - mnew);
+        float ps = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float v = sc[nt][2 * hr + j];
+            const float pv = v == -CUDART_INF_F ? 0.f : fast_exp2(v - mnew);
+            p[nt][2 * hr + j] = pv;
+            ps += pv;
+          }
+        l_run[hr] = l_run[hr] * alpha + ps;
+        m_run[hr] = mnew;
+#pragma unroll
+        for (int nd = 0; nd < 16; ++nd) {
+          o[nd][2 * hr] *= alpha;
+          o[nd][2 * hr + 1] *= alpha;
+        }
+      }
+      // V rows of this warp's slice past the window end are stale shared memory or cache
+      // slots beyond the sequence (possibly non-finite): zero them so that 0 * V stays 0
+      const int slice0 = tok0 + tile * kTileTok + 16 * w;
+      const bool zeroed = slice0 + 16 > tok_end;
+      if (zeroed) {
+        unsigned char* vw = S.stage[s] + kTileBytesKV;
+        for (int i = lane; i < 16 * 16; i += 32) {   // 16 rows x (2 halves x 8 chunks of 16 B)
+          const int r = i >> 4, hc = i & 15;
+          if (slice0 + r >= tok_end)
+            *reinterpret_cast<uint4*>(vw + (hc >> 3) * kHalfBytes + sw128(16 * w + r, hc & 7)) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+      }
+      // P (16 x 16) as the A operand: hi and lo bf16 parts
+      uint32_t ph[4], pl[4];
+      split_bf16(p[0][0], p[0][1], ph[0], pl[0]);
+      split_bf16(p[0][2], p[0][3], ph[1], pl[1]);
+      split_bf16(p[1][0], p[1][1], ph[2], pl[2]);
+      split_bf16(p[1][2], p[1][3], ph[3], pl[3]);
+      const uint32_t vbase = smem_u32(vt);
+      const int tokrow = 16 * w + ((i4 & 1) << 3) + rr;
+#pragma unroll
+      for (int nd = 0; nd < 16; nd += 2) {
+        const int dc = nd + (i4 >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vbase + (dc >> 3) * kHalfBytes + sw128(tokrow, dc & 7), b0, b1, b2, b3);
+        mma_bf16(o[nd], ph, b0, b1);
+        mma_bf16(o[nd], pl, b0, b1);
+        mma_bf16(o[nd + 1], ph, b2, b3);
+        mma_bf16(o[nd + 1], pl, b2, b3);
+      }
+      __syncwarp();
+      // order this warp's generic-proxy writes before the stage's next TMA refill
+      if (zeroed) asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      if (lane == 0) mbar_arrive(&S.empty[s]);
+    }
+    // row sums over the quad
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      l_run[hr] += __shfl_xor_sync(0xFFFFFFFFu, l_run[hr], 1);
+      l_run[hr] += __shfl_xor_sync(0xFFFFFFFFu, l_run[hr], 2);
+    }
+  }
+  __syncthreads();
+  // combine buffer: entry (list m, part = warp)
+  float* comb = reinterpret_cast<float*>(S.stage[0]);
+  if (warp < kDnConsumers) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int m = (lane >> 2) + 8 * hr;
+      if (m < nlists) {
+        float* e = comb + (size_t)(m * kDnConsumers + warp) * kCombFloats;
+        if ((lane & 3) == 0) {
+          e[0] = m_run[hr];
+          e[1] = l_run[hr];
+        }
+#pragma unroll
+        for (int nd = 0; nd < 16; ++nd) {
+          const int d = nd * 8 + 2 * (lane & 3);
+          e[4 + d] = o[nd][2 * hr];
+          e[4 + d + 1] = o[nd][2 * hr + 1];
+        }
       }
     }
   }
-  cp_async_wait<0>();
   __syncthreads();
-
-  float* comb = reinterpret_cast<float*>(S.ring);
-  if (has_set) {
-#pragma unroll
-    for (int hh = 0; hh < kDenseHeadsPerGroup; ++hh) {
-      const int m = my_set * kDenseHeadsPerGroup + hh;
-      if (m < nlists) soft_store(comb, m * PG + my_part, st[hh], l8);
-    }
-  }
-  __syncthreads();
-  finish_lists(a, si, b, g, lg, split, nlists, PG, comb, S.mx, S.lsum);
+  finish_lists(a, si, b, g, lg, split, nlists, kDnConsumers, comb, S.mx, S.lsum);
 }
 
 // ---------------------------------------------------------------------------
@@ -643,16 +738,22 @@ cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaSt
   return cudaGetLastError();
 }
 
-cudaError_t launch_dense_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
+cudaError_t launch_dense_decode(const DecodeArgs& a, const KvMaps& maps, int batch, int hkv, cudaStream_t stream) {
   const size_t smem = sizeof(DenseSmem);
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(dense_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(dense_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(dense_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 grid(a.nsplit, hkv * a.list_groups, batch);
-  dense_decode_kernel<<<grid, kDecodeThreads, smem, stream>>>(a);
+  if (a.qv.q_f32) {
+    dense_decode_kernel<true><<<grid, kDnThreads, smem, stream>>>(a, maps);
+  } else {
+    dense_decode_kernel<false><<<grid, kDnThreads, smem, stream>>>(a, maps);
+  }
   return cudaGetLastError();
 }
 

@@ -89,7 +89,8 @@ inline SparsePlan plan_sparse(const Shapes& s, int k_max) {
   return p;
 }
 
-// Dense decode: tokens per CTA window and number of windows.
+// Dense decode: up to 16 lists per CTA (the mma M dimension) and a window of W tokens (a
+// multiple of the 64-token tile), sized for about four waves of 2 CTAs per SM.
 struct DensePlan {
   int lists_per_cta;
   int list_groups;
@@ -97,19 +98,24 @@ struct DensePlan {
   int nsplit;
 };
 
+constexpr int kDenseMaxLists = 16;
+constexpr int kDenseTargetCtas = 4 * 296;
+
 inline DensePlan plan_dense(const Shapes& s) {
   DensePlan p;
-  int64_t m = s.group * s.max_tokens;
-  p.lists_per_cta = (int)(m < kMaxListsPerCta ? m : kMaxListsPerCta);
-  p.list_groups = list_groups(s);
-  int w = 1024;
-  int ns = (int)((s.max_seq_len + w - 1) / w);
-  while (ns > kMaxSplits) {
-    w *= 2;
-    ns = (int)((s.max_seq_len + w - 1) / w);
-  }
-  p.window = w;
-  p.nsplit = ns;
+  const int64_t m = s.group * s.max_tokens;
+  p.lists_per_cta = (int)(m < kDenseMaxLists ? m : kDenseMaxLists);
+  p.list_groups = (int)((m + p.lists_per_cta - 1) / p.lists_per_cta);
+  const int64_t units = s.batch * s.hkv * p.list_groups;
+  int64_t ns = (kDenseTargetCtas + units - 1) / units;
+  const int64_t max_ns = (s.max_seq_len + 63) / 64;
+  if (ns > max_ns) ns = max_ns;
+  if (ns > kMaxSplits) ns = kMaxSplits;
+  if (ns < 1) ns = 1;
+  int64_t w = (s.max_seq_len + ns - 1) / ns;
+  w = (w + 63) / 64 * 64;
+  p.window = (int)w;
+  p.nsplit = (int)((s.max_seq_len + w - 1) / w);
   return p;
 }
 
