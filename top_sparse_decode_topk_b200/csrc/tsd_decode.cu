@@ -502,22 +502,25 @@ __global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs
 //   transposing ldmatrix.
 // The 4 warp states of each list are combined at the end and merged across windows like the
 // sparse path's CTA partials.
-constexpr int kDnStages = 3;
+constexpr int kDnStages = 2;
 constexpr int kDnConsumers = 4;
 constexpr int kDnThreads = 32 * (kDnConsumers + 1);
 constexpr int kDnStageBytes = 2 * kTileBytesKV;   // K then V
 
 struct DenseSmem {
   alignas(1024) unsigned char stage[kDnStages][kDnStageBytes];   // also the combine buffer
+  alignas(1024) unsigned char qhi[kQTileBytes];
+  alignas(1024) unsigned char qlo[kQTileBytes];
   uint64_t full[kDnStages];
   uint64_t empty[kDnStages];
   uint32_t abort;
   float mx[16], lsum[16];
 };
 static_assert(kDnStages * kDnStageBytes >= 16 * kDnConsumers * kCombFloats * 4, "dense combine buffer");
+static_assert(sizeof(DenseSmem) + 1024 <= 75 * 1024, "three dense CTAs per SM");
 
 template <bool QF32>
-__global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(DecodeArgs a, const __grid_constant__ KvMaps maps) {
+__global__ void __launch_bounds__(kDnThreads, 3) dense_decode_kernel(DecodeArgs a, const __grid_constant__ KvMaps maps) {
   extern __shared__ __align__(1024) unsigned char smem_dn[];
   DenseSmem& S = *reinterpret_cast<DenseSmem*>(smem_dn);
   const int split = blockIdx.x;
@@ -547,6 +550,7 @@ __global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(DecodeArgs 
     mbar_fence_init();
     S.abort = 0;
   }
+  store_q_tile(a.qv, si, g, G, lg * a.lists_per_cta, nlists, S.qhi, QF32 ? S.qlo : nullptr, threadIdx.x, kDnThreads);
   __syncthreads();
 
   // per warp state: rows r0 = lane/4 and r0 + 8
@@ -554,7 +558,10 @@ __global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(DecodeArgs 
   float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_run[2] = {0.f, 0.f};
 
   if (warp == kDnConsumers) {
-    // producer
+    // producer: box coordinates prefetched 32 at a time, TMA issued by lane 0
+    BoxRows br;
+    const int bp = tma_box_rows(a.kv);
+    if (use_tma) box_rows_init(br, a.kv, b, g, tok0, tok_end, bp, lane, a.status);
     for (int tile = 0; tile < ntiles; ++tile) {
       const int s = tile % kDnStages;
       if (tile >= kDnStages) {
@@ -573,17 +580,18 @@ __global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(DecodeArgs 
       unsigned char* vd = S.stage[s] + kTileBytesKV;
       const int tok = tok0 + tile * kTileTok;
       if (use_tma) {
-        if (lane == 0) {
-          // the expected bytes must be registered before the loads can complete the phase
-          const int bp = a.kv.page_table == nullptr ? 16 : min(16, 1 << a.kv.page_shift);
-          const int rows = min(kTileTok, tok_end - tok);
-          uint32_t want = 0;
-          for (int r = 0; r < rows; r += bp) want += 4 * bp * 128;
-          mbar_arrive_expect_tx(&S.full[s], want);
-          const uint32_t got = tile_issue_tma(a.kv, &maps.k, &maps.v, b, g, tok, tok_end, kd, vd, &S.full[s], a.status);
-          // rows skipped for a bad page never arrive: complete them so the phase still ends
-          if (got < want) asm volatile("{\n .reg .b64 st;\n mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n}\n" ::"r"(smem_u32(&S.full[s])), "r"(want - got) : "memory");
-        }
+        // the expected bytes must be registered before the loads can complete the phase
+        const int rows = min(kTileTok, tok_end - tok);
+        const uint32_t want = (uint32_t)((rows + bp - 1) / bp) * 4 * bp * 128;
+        if (lane == 0) mbar_arrive_expect_tx(&S.full[s], want);
+        __syncwarp();
+        const uint32_t got = tile_issue_tma(a.kv, &maps.k, &maps.v, br, b, g, tok0, tok_end, tile, kd, vd, &S.full[s],
+                                            lane, a.status);
+        // boxes skipped for a bad page never arrive: complete their bytes so the phase ends
+        if (lane == 0 && got < want)
+          asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(&S.full[s])),
+                       "r"(want - got)
+                       : "memory");
       } else {
         tile_issue_cpasync(a.kv, b, g, tok, tok_end, kd, vd, lane, a.status);
         cp_async_mbar_arrive(&S.full[s]);
@@ -596,8 +604,6 @@ __global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(DecodeArgs 
   } else {
     const int w = warp;
     const float scale2 = a.qv.sm_scale * kLog2e;
-    QFrags<QF32> qf;
-    load_q_frags<QF32>(a.qv, si, g, G, lg * a.lists_per_cta, nlists, lane, qf);
     int kvl[2];
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
@@ -619,7 +625,7 @@ __global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(DecodeArgs 
       const unsigned char* kt = S.stage[s];
       const unsigned char* vt = S.stage[s] + kTileBytesKV;
       float sc[2][4];
-      qk_tile<QF32>(qf, kt, w, lane, sc);
+      qk_tile<QF32>(S.qhi, S.qlo, kt, w, lane, sc);
       // scale, mask, online softmax per query row
       const int tbase = tok0 + tile * kTileTok + 16 * w + 2 * (lane & 3);
       float p[2][4];

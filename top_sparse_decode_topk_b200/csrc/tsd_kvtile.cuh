@@ -32,36 +32,72 @@ struct KvMaps {
   CUtensorMap v;
 };
 
-// Load the tokens [tok, min(tok + 64, tok_end)) of (b, g) into one stage.
-// K goes to kdst (16 KB, 1024-byte aligned), V to vdst (or nothing when vdst is null).
-// TMA path: called by one lane; returns the bytes the stage's barrier must expect.
+// Box rows of the TMA tensor maps: 16-token boxes, or one page when pages are 8 tokens.
+__device__ __forceinline__ int tma_box_rows(const KvView& kv) {
+  return kv.page_table == nullptr ? 16 : min(16, 1 << kv.page_shift);
+}
+
+// Row coordinate (in the [rows][128] view) of the box that starts at token t of (b, g):
+// -1 past tok_end, -2 for a bad page (flagged).
+__device__ __forceinline__ int tma_box_y(const KvView& kv, int b, int g, int t, int tok_end, uint32_t* status) {
+  if (t >= tok_end) return -1;
+  if (kv.page_table == nullptr) return (b * kv.hkv + g) * kv.max_seq_len + t;
+  const int32_t page = __ldg(kv.page_table + (int64_t)b * kv.max_pages + (t >> kv.page_shift));
+  if (page < 0 || (int64_t)page >= kv.num_pages) {
+    flag_status(status, TSD_DEV_BAD_PAGE);
+    return -2;
+  }
+  return (int)((((int64_t)page * kv.hkv + g) << kv.page_shift) | (t & ((1 << kv.page_shift) - 1)));
+}
+
+// Producer-warp view of the box coordinates of a window: lane i holds the coordinate of box
+// 32 s + i of the current segment s and prefetches segment s + 1, so page-table lookups
+// cost one round trip per 32 boxes and are off the issue path.
+struct BoxRows {
+  int cur, nxt, seg;
+};
+
+__device__ __forceinline__ void box_rows_init(BoxRows& br, const KvView& kv, int b, int g, int tok0, int tok_end,
+                                              int bp, int lane, uint32_t* status) {
+  br.seg = 0;
+  br.cur = tma_box_y(kv, b, g, tok0 + lane * bp, tok_end, status);
+  br.nxt = tma_box_y(kv, b, g, tok0 + (32 + lane) * bp, tok_end, status);
+}
+
+// Coordinate of box `box` of the window; all 32 lanes must call it with the same box.
+__device__ __forceinline__ int box_rows_get(BoxRows& br, const KvView& kv, int b, int g, int tok0, int tok_end, int bp,
+                                            int lane, int box, uint32_t* status) {
+  const int seg = box >> 5;
+  while (br.seg < seg) {
+    br.cur = br.nxt;
+    ++br.seg;
+    br.nxt = tma_box_y(kv, b, g, tok0 + ((br.seg + 1) * 32 + lane) * bp, tok_end, status);
+  }
+  return __shfl_sync(0xFFFFFFFFu, br.cur, box & 31);
+}
+
+// Issue the TMA loads of one 64-token tile (all 32 lanes call it; lane 0 issues) and
+// return the bytes issued (valid on lane 0).
 __device__ __forceinline__ uint32_t tile_issue_tma(const KvView& kv, const CUtensorMap* tmk, const CUtensorMap* tmv,
-                                                   int b, int g, int tok, int tok_end, unsigned char* kdst,
-                                                   unsigned char* vdst, uint64_t* bar, uint32_t* status) {
-  const int bp = kv.page_table == nullptr ? 16 : min(16, 1 << kv.page_shift);   // box rows
+                                                   BoxRows& br, int b, int g, int tok0, int tok_end, int tile,
+                                                   unsigned char* kdst, unsigned char* vdst, uint64_t* bar, int lane,
+                                                   uint32_t* status) {
+  const int bp = tma_box_rows(kv);
   uint32_t bytes = 0;
   for (int r = 0; r < kTileTok; r += bp) {
-    const int t = tok + r;
-    if (t >= tok_end) break;
-    int y;
-    if (kv.page_table == nullptr) {
-      y = (b * kv.hkv + g) * kv.max_seq_len + t;
-    } else {
-      const int32_t page = __ldg(kv.page_table + (int64_t)b * kv.max_pages + (t >> kv.page_shift));
-      if (page < 0 || (int64_t)page >= kv.num_pages) {
-        flag_status(status, TSD_DEV_BAD_PAGE);
-        continue;
+    const int box = (tile * kTileTok + r) / bp;
+    const int y = box_rows_get(br, kv, b, g, tok0, tok_end, bp, lane, box, status);
+    if (y == -1) break;
+    if (y < 0) continue;
+    if (lane == 0) {
+      tma_load_2d(kdst + r * 128, tmk, 0, y, bar);
+      tma_load_2d(kdst + kHalfBytes + r * 128, tmk, 64, y, bar);
+      if (vdst != nullptr) {
+        tma_load_2d(vdst + r * 128, tmv, 0, y, bar);
+        tma_load_2d(vdst + kHalfBytes + r * 128, tmv, 64, y, bar);
       }
-      y = (int)((((int64_t)page * kv.hkv + g) << kv.page_shift) | (t & ((1 << kv.page_shift) - 1)));
     }
-    tma_load_2d(kdst + r * 128, tmk, 0, y, bar);
-    tma_load_2d(kdst + kHalfBytes + r * 128, tmk, 64, y, bar);
-    bytes += 2 * bp * 128;
-    if (vdst != nullptr) {
-      tma_load_2d(vdst + r * 128, tmv, 0, y, bar);
-      tma_load_2d(vdst + kHalfBytes + r * 128, tmv, 64, y, bar);
-      bytes += 2 * bp * 128;
-    }
+    bytes += (vdst != nullptr ? 4 : 2) * bp * 128;
   }
   return bytes;
 }
@@ -89,53 +125,53 @@ __device__ __forceinline__ void tile_issue_cpasync(const KvView& kv, int b, int 
   }
 }
 
-// Query fragments (mma A operand, 16 rows x 128 dims): row m is list m of the CTA (token
-// j = m / G of the sequence, q head g * G + m % G); rows >= nlists are zero.  For fp32
-// queries the lo parts carry q - bf16(q).
-template <bool QF32>
-struct QFrags {
-  uint32_t hi[8][4];
-  uint32_t lo[QF32 ? 8 : 1][4];
-};
+// Query tile (mma A operand, 16 rows x 128 dims) in shared memory, laid out like a K tile
+// (two 128-byte halves of [16 rows][128 B], 128-byte swizzled): row m is list m of the CTA
+// (token j = m / G of the sequence, q head g * G + m % G); rows >= nlists are zero.  For
+// fp32 queries a second tile holds the bf16 remainders q - bf16(q).
+constexpr int kQHalfBytes = 16 * 128;
+constexpr int kQTileBytes = 2 * kQHalfBytes;
 
-template <bool QF32>
-__device__ __forceinline__ void load_q_frags(const QView& qv, const SeqInfo& si, int g, int G, int m0, int nlists,
-                                             int lane, QFrags<QF32>& f) {
-  const int r0 = lane >> 2, kk = (lane & 3) * 2;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int m = r0 + 8 * half;
-    const bool ok = m < nlists;
-    const int mg = m0 + m;
-    const int j = mg / G;
-    const int64_t base = ((int64_t)(si.t0 + j) * qv.hq + g * G + (mg - j * G)) * kHeadDim;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-      for (int hk = 0; hk < 2; ++hk) {
-        const int d = ks * 16 + kk + 8 * hk;
-        uint32_t hi = 0, lo = 0;
-        if (ok) {
-          if (QF32) {
-            const float2 x = __ldg(reinterpret_cast<const float2*>(reinterpret_cast<const float*>(qv.q) + base + d));
-            split_bf16(x.x, x.y, hi, lo);
-          } else {
-            hi = __ldg(reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(qv.q) + base + d));
-          }
-        }
-        // a0 = (row r0, k lo), a1 = (row r0 + 8, k lo), a2 = (row r0, k hi), a3 = (row r0 + 8, k hi)
-        f.hi[ks][half + 2 * hk] = hi;
-        if (QF32) f.lo[ks][half + 2 * hk] = lo;
+// Called by `nthreads` threads (index tid): fills qhi (and qlo when non-null).
+__device__ __forceinline__ void store_q_tile(const QView& qv, const SeqInfo& si, int g, int G, int m0, int nlists,
+                                             unsigned char* qhi, unsigned char* qlo, int tid, int nthreads) {
+  for (int i = tid; i < 16 * 16; i += nthreads) {   // 16 rows x 16 chunks of 8 dims
+    const int m = i >> 4, ch = i & 15;
+    uint4 hi = make_uint4(0, 0, 0, 0), lo = make_uint4(0, 0, 0, 0);
+    if (m < nlists) {
+      const int mg = m0 + m;
+      const int j = mg / G;
+      const int64_t base = ((int64_t)(si.t0 + j) * qv.hq + g * G + (mg - j * G)) * kHeadDim + ch * 8;
+      if (qv.q_f32) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(qv.q) + base));
+        const float4 y = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(qv.q) + base + 4));
+        split_bf16(x.x, x.y, hi.x, lo.x);
+        split_bf16(x.z, x.w, hi.y, lo.y);
+        split_bf16(y.x, y.y, hi.z, lo.z);
+        split_bf16(y.z, y.w, hi.w, lo.w);
+      } else {
+        hi = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(qv.q) + base));
       }
     }
+    const uint32_t off = (ch >> 3) * kQHalfBytes + sw128(m, ch & 7);
+    *reinterpret_cast<uint4*>(qhi + off) = hi;
+    if (qlo != nullptr) *reinterpret_cast<uint4*>(qlo + off) = lo;
   }
+}
+
+// A fragment of k-step ks from a query tile.
+__device__ __forceinline__ void q_frag(const unsigned char* qt, int ks, int lane, uint32_t* a) {
+  const int i4 = lane >> 3;
+  const int row = ((i4 & 1) << 3) + (lane & 7);
+  const int chunk = ((ks & 3) << 1) + (i4 >> 1);
+  ldsm_x4(smem_u32(qt) + (ks >> 2) * kQHalfBytes + sw128(row, chunk), a[0], a[1], a[2], a[3]);
 }
 
 // S(16 queries x 16 tokens) of one warp: tokens [16 w, 16 w + 16) of the tile in stage K.
 // S[nt][0..1] = (query lane/4, tokens 8 nt + 2 (lane%4) + {0,1}); S[nt][2..3] = query lane/4 + 8.
 template <bool QF32>
-__device__ __forceinline__ void qk_tile(const QFrags<QF32>& f, const unsigned char* ktile, int w, int lane,
-                                        float S[2][4]) {
+__device__ __forceinline__ void qk_tile(const unsigned char* qhi, const unsigned char* qlo, const unsigned char* ktile,
+                                        int w, int lane, float S[2][4]) {
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -148,11 +184,14 @@ __device__ __forceinline__ void qk_tile(const QFrags<QF32>& f, const unsigned ch
     const int chunk = ((ks & 3) << 1) + (i4 & 1);
     uint32_t b00, b01, b10, b11;
     ldsm_x4(kbase + (ks >> 2) * kHalfBytes + sw128(tokrow, chunk), b00, b01, b10, b11);
-    mma_bf16(S[0], f.hi[ks], b00, b01);
-    mma_bf16(S[1], f.hi[ks], b10, b11);
+    uint32_t a[4];
+    q_frag(qhi, ks, lane, a);
+    mma_bf16(S[0], a, b00, b01);
+    mma_bf16(S[1], a, b10, b11);
     if (QF32) {
-      mma_bf16(S[0], f.lo[ks], b00, b01);
-      mma_bf16(S[1], f.lo[ks], b10, b11);
+      q_frag(qlo, ks, lane, a);
+      mma_bf16(S[0], a, b00, b01);
+      mma_bf16(S[1], a, b10, b11);
     }
   }
 }
