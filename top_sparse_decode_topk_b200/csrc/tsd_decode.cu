@@ -8,8 +8,9 @@
 //
 // Sparse decode: one half-warp per task (16+ entries of one list); rows gathered into
 // registers; batched online softmax; per-list split-K merge by the last task to finish.
-// Dense decode: one CTA per (sequence, kv head, list group, window of W tokens); rows
-// staged through a cp.async ring; CTA-level partials merged by the last CTA of the unit.
+// Dense decode: one CTA per (sequence, kv head, list group, window of W tokens); 64-token
+// K/V tiles arrive by TMA in a 2-stage shared-memory ring and q K^T and P V run on the
+// tensor cores; CTA-level partials are merged by the last CTA of the unit.
 // No kernel ever waits on another CTA: merges are done by whichever arrives last.
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -47,97 +48,6 @@ __device__ __forceinline__ ListRef list_ref(const DecodeArgs& a, const SeqInfo& 
   r.h = g * G + (mg - j * G);
   r.kvlen = kv_len_of(a.qv, si, j);
   return r;
-}
-
-// Load 16 query values of list (t, h) owned by lane `l8` of a group: dims
-// [8*l8, 8*l8+8) and [64+8*l8, 64+8*l8+8), pre-multiplied by scale*log2(e) so that
-// dot products come out in base-2 softmax units.
-__device__ __forceinline__ void load_q16(const QView& qv, int t, int h, int l8, float scale, float* q) {
-  const int64_t base = ((int64_t)t * qv.hq + h) * kHeadDim;
-  if (qv.q_f32) {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(qv.q) + base);
-    float4 a0 = __ldg(p + 2 * l8), a1 = __ldg(p + 2 * l8 + 1);
-    float4 b0 = __ldg(p + 16 + 2 * l8), b1 = __ldg(p + 16 + 2 * l8 + 1);
-    float v[16] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w,
-                   b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-    for (int j = 0; j < 16; ++j) q[j] = v[j] * scale;
-  } else {
-    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(qv.q) + base);
-    uint4 a0 = __ldg(p + l8), b0 = __ldg(p + 8 + l8);
-    float v[16];
-    unpack8(a0, v);
-    unpack8(b0, v + 8);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) q[j] = v[j] * scale;
-  }
-}
-
-// Dot of a 256-byte bf16 row in shared memory with the lane's 16 query values,
-// summed over the 8 lanes of the group (full-warp shuffles: call warp-uniformly).
-__device__ __forceinline__ float group_dot(const unsigned char* row, int l8, const float* q) {
-  uint4 k0 = *reinterpret_cast<const uint4*>(row + 16 * l8);
-  uint4 k1 = *reinterpret_cast<const uint4*>(row + 128 + 16 * l8);
-  float kf[16];
-  unpack8(k0, kf);
-  unpack8(k1, kf + 8);
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    s0 = fmaf(q[j], kf[j], s0);
-    s1 = fmaf(q[8 + j], kf[8 + j], s1);
-  }
-  float s = s0 + s1;
-  s += __shfl_xor_sync(0xFFFFFFFFu, s, 1);
-  s += __shfl_xor_sync(0xFFFFFFFFu, s, 2);
-  s += __shfl_xor_sync(0xFFFFFFFFu, s, 4);
-  return s;
-}
-
-// Online-softmax state of one lane-group for one list.
-struct SoftState {
-  float m, l;
-  float acc[16];
-};
-
-__device__ __forceinline__ void soft_init(SoftState& st) {
-  st.m = -CUDART_INF_F;
-  st.l = 0.f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) st.acc[j] = 0.f;
-}
-
-__device__ __forceinline__ void soft_update(SoftState& st, float s, const unsigned char* vrow, int l8) {
-  if (s > st.m) {
-    const float alpha = fast_exp2(st.m - s);
-    st.l *= alpha;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) st.acc[j] *= alpha;
-    st.m = s;
-  }
-  const float p = fast_exp2(s - st.m);
-  st.l += p;
-  uint4 v0 = *reinterpret_cast<const uint4*>(vrow + 16 * l8);
-  uint4 v1 = *reinterpret_cast<const uint4*>(vrow + 128 + 16 * l8);
-  float vf[16];
-  unpack8(v0, vf);
-  unpack8(v1, vf + 8);
-#pragma unroll
-  for (int j = 0; j < 16; ++j) st.acc[j] = fmaf(p, vf[j], st.acc[j]);
-}
-
-// Write a group's state into the combine buffer entry `slot` (lane l8 owns 16 dims).
-__device__ __forceinline__ void soft_store(float* comb, int slot, const SoftState& st, int l8) {
-  float* e = comb + (size_t)slot * kCombFloats;
-  if (l8 == 0) {
-    e[0] = st.m;
-    e[1] = st.l;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    e[4 + 8 * l8 + j] = st.acc[j];
-    e[4 + 64 + 8 * l8 + j] = st.acc[8 + j];
-  }
 }
 
 __device__ __forceinline__ void store_out(const DecodeArgs& a, int t, int h, int d, float v) {
@@ -494,7 +404,7 @@ __global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs
 // ---------------------------------------------------------------------------
 // One CTA per (sequence b, kv head g, list group lg, window of W tokens): up to 16 lists
 // (q heads of the GQA group x decode tokens) are the rows of the mma M dimension.  A
-// producer warp streams 64-token K/V tiles through a 3-stage ring (TMA, see tsd_kvtile.cuh);
+// producer warp streams 64-token K/V tiles through a 2-stage ring (TMA, see tsd_kvtile.cuh);
 // each of the 4 consumer warps takes 16 tokens of every tile:
 //   S = q K^T (16 x 16, 8 k-steps of mma.m16n8k16), scaled to base-2 softmax units in fp32,
 //   masked past each list's kv_len; online softmax per query row (quad shuffles);
