@@ -18,7 +18,8 @@
 namespace tsd {
 cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream);
 cudaError_t launch_dense_decode(const DecodeArgs& a, const KvMaps& maps, int batch, int hkv, cudaStream_t stream);
-cudaError_t launch_topk(const TopkArgs& a, int nwin, int batch, int hkv, int num_lists, cudaStream_t stream);
+cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int batch, int hkv, int num_lists,
+                        cudaStream_t stream);
 }  // namespace tsd
 
 using namespace tsd;
@@ -233,12 +234,15 @@ tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries
   a.out_count = out_count;
   a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
   a.score_stride = lay.score_stride;
-  a.lists_per_cta = (int)(sh.group * sh.max_tokens < kMaxListsPerCta ? sh.group * sh.max_tokens : kMaxListsPerCta);
-  a.list_groups = list_groups(sh);
-  a.window = kScoreTokensPerCta;
+  const DensePlan p = plan_dense(sh);   // scoring streams K in the dense path's tiles and windows
+  a.lists_per_cta = p.lists_per_cta;
+  a.list_groups = p.list_groups;
+  a.window = p.window;
   a.status = static_cast<uint32_t*>(ws);
-  const int nwin = (int)((sh.max_seq_len + a.window - 1) / a.window);
-  return cuda_status(launch_topk(a, nwin, (int)sh.batch, (int)sh.hkv, (int)(sh.tokens * sh.hq),
+  KvMaps maps;
+  st = make_kv_maps(cache, &maps);
+  if (st != TSD_OK) return st;
+  return cuda_status(launch_topk(a, maps, p.nsplit, (int)sh.batch, (int)sh.hkv, (int)(sh.tokens * sh.hq),
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -237,13 +237,13 @@ __device__ __forceinline__ void batch_update(const uint4* kq, const uint4* vq, c
   m_run = m_new;
 }
 
-// End of a task: a list that fits one task is written directly; otherwise the task's
-// partial state is stored, and the last task of the list to arrive (per-list counter)
-// merges the C partials with log-sum-exp.  Called by the 16 lanes of one half-warp
-// (hmask), lane l holding output dims [8l, 8l+8).
+// End of a list's work in one CTA: a list whose tasks all ran in this CTA is written
+// directly; otherwise this CTA's partial state (partial c of C) is stored, and the last CTA
+// of the list to arrive (per-list counter) merges the C partials with log-sum-exp.  Called
+// by the 16 lanes of one half-warp (hmask), lane l holding output dims [8l, 8l+8).
 __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id, int t, int h, int C, int c,
                                             float m_run, float l_run, const float* acc, int l, unsigned hmask) {
-  if (C == 1) {   // the whole list in one task
+  if (C == 1) {   // the whole list in one CTA
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, acc[i] * inv);
@@ -251,7 +251,7 @@ __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id
     return;
   }
   // partial of this task, then the per-list arrival count
-  const int64_t pidx = list_id * C + c;
+  const int64_t pidx = list_id * a.nsplit + c;
   if (l == 0) a.part_ml[pidx] = make_float2(m_run, l_run);
   float4* pa = reinterpret_cast<float4*>(a.part_acc + pidx * kHeadDim + 8 * l);
   pa[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -268,7 +268,7 @@ __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id
   __threadfence();
   // last task of the list: merge its C partials (lanes over splits for the max and sum,
   // then 8 output dims per lane with independent loads)
-  const float2* ml = a.part_ml + list_id * C;
+  const float2* ml = a.part_ml + list_id * a.nsplit;
   float mx = -CUDART_INF_F;
   for (int i = l; i < C; i += 16) mx = fmaxf(mx, __ldcg(&ml[i]).x);
   mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 1));
@@ -295,7 +295,8 @@ __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id
       for (int u = 0; u < 4; ++u) {
         const int cc = c0 + u;
         w[u] = cc < C ? fast_exp2(__ldcg(&ml[cc]).x - mx) : 0.f;
-        const float4* src = reinterpret_cast<const float4*>(a.part_acc + (list_id * C + (cc < C ? cc : 0)) * kHeadDim + 8 * l);
+        const float4* src =
+            reinterpret_cast<const float4*>(a.part_acc + (list_id * a.nsplit + (cc < C ? cc : 0)) * kHeadDim + 8 * l);
         x0[u] = __ldcg(src);
         x1[u] = __ldcg(src + 1);
       }
@@ -315,88 +316,129 @@ __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id
 }
 
 __global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs a) {
+  // task states of the CTA's 16 half-warps, combined per list before anything leaves the CTA
+  __shared__ float2 s_ml[16];
+  __shared__ __align__(16) float s_acc[16][kHeadDim];
+  __shared__ int64_t s_list[16];
   const int lane = threadIdx.x & 31;
   const int l = threadIdx.x & 15;
+  const int hw = threadIdx.x >> 4;
   const unsigned hmask = 0xFFFFu << (lane & 16);
   const int G = a.qv.hq / a.kv.hkv;
   const int M = a.lists_per_cta;   // list slots per (sequence, kv head): G x max tokens per sequence
   const int C = a.nsplit;          // tasks (chunks) per list
   const int E = a.span;            // entries per task
-  const int64_t task = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4);
+  const int64_t task = (int64_t)blockIdx.x * 16 + hw;
   const int64_t total = (int64_t)a.kv.batch * a.kv.hkv * C * M;
-  if (task >= total) return;
-  const int m = (int)(task % M);
-  int64_t rest = task / M;
+  const int64_t tk = task < total ? task : total - 1;
+  const int m = (int)(tk % M);
+  int64_t rest = tk / M;
   const int c = (int)(rest % C);
   rest /= C;
   const int g = (int)(rest % a.kv.hkv);
   const int b = (int)(rest / a.kv.hkv);
 
-  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, c == 0 && g == 0 && m == 0 && l == 0);
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, task == tk && c == 0 && g == 0 && m == 0 && l == 0);
   const int j = m / G;
-  if (j >= si.n) return;           // no such list (fewer decode tokens in this sequence)
+  const bool valid = task < total && j < si.n;   // no list for slots past this sequence's tokens
   const int t = si.t0 + j, h = g * G + (m - j * G);
-  const int kvlen = kv_len_of(a.qv, si, j);
-  const int64_t list_id = (int64_t)t * a.qv.hq + h;
-  const float scale = a.qv.sm_scale * kLog2e;
-
-  // this lane's 8 query dims [8l, 8l+8), scaled so that dots are base-2 softmax units
-  float q[8];
-  {
-    const int64_t qb = list_id * kHeadDim + 8 * l;
-    if (a.qv.q_f32) {
-      const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.qv.q) + qb);
-      const float4 x = __ldg(p), y = __ldg(p + 1);
-      q[0] = x.x; q[1] = x.y; q[2] = x.z; q[3] = x.w; q[4] = y.x; q[5] = y.y; q[6] = y.z; q[7] = y.w;
-    } else {
-      unpack8(__ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.qv.q) + qb)), q);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) q[i] *= scale;
-  }
-
-  const int32_t* lst = a.idx + list_id * a.k_max;
-  const int e0 = c * E;
-  const int e1 = min(e0 + E, a.k_max);
+  const int64_t list_id = valid ? (int64_t)t * a.qv.hq + h : -1;
   float m_run = -CUDART_INF_F, l_run = 0.f, acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  uint32_t bad = 0;
-  for (int base = e0; base < e1; base += 16) {
-    // this lane's entry: index, predecessor check, validity, physical row
-    const int e = base + l;
-    const int32_t v = e < e1 ? __ldg(lst + e) : -1;
-    uint32_t before = __shfl_up_sync(hmask, (uint32_t)v, 1, 16);
-    if (l == 0 && e > 0 && e < e1) before = (uint32_t)__ldg(lst + e - 1);
-    if (e < e1 && e > 0 && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
-    if (e < e1 && (v < -1 || v >= kvlen)) bad |= TSD_DEV_BAD_INDEX;
-    uint32_t row = kInvalidRow;
-    if (e < e1 && v >= 0 && v < kvlen) {
-      row = kv_row(a.kv, b, g, v);
-      if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
-    }
-    // the 16 rows, U at a time
-#pragma unroll
-    for (int j0 = 0; j0 < 16; j0 += kSpU) {
-      uint32_t rr[kSpU];
-      uint4 kq[kSpU], vq[kSpU];
-#pragma unroll
-      for (int u = 0; u < kSpU; ++u) {
-        rr[u] = __shfl_sync(hmask, row, j0 + u, 16);
-        kq[u] = make_uint4(0, 0, 0, 0);
-        vq[u] = make_uint4(0, 0, 0, 0);
-        row_fetch(a, rr[u], l, kq[u], vq[u]);
-      }
-      batch_update<kSpU>(kq, vq, rr, q, m_run, l_run, acc, hmask);
-    }
-  }
-  bad |= __shfl_xor_sync(hmask, bad, 1);
-  bad |= __shfl_xor_sync(hmask, bad, 2);
-  bad |= __shfl_xor_sync(hmask, bad, 4);
-  bad |= __shfl_xor_sync(hmask, bad, 8);
-  if (l == 0 && bad) flag_status(a.status, bad);
 
-  finish_task(a, list_id, t, h, C, c, m_run, l_run, acc, l, hmask);
+  if (valid) {
+    const int kvlen = kv_len_of(a.qv, si, j);
+    const float scale = a.qv.sm_scale * kLog2e;
+    // this lane's 8 query dims [8l, 8l+8), scaled so that dots are base-2 softmax units
+    float q[8];
+    {
+      const int64_t qb = list_id * kHeadDim + 8 * l;
+      if (a.qv.q_f32) {
+        const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.qv.q) + qb);
+        const float4 x = __ldg(p), y = __ldg(p + 1);
+        q[0] = x.x; q[1] = x.y; q[2] = x.z; q[3] = x.w; q[4] = y.x; q[5] = y.y; q[6] = y.z; q[7] = y.w;
+      } else {
+        unpack8(__ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.qv.q) + qb)), q);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] *= scale;
+    }
+
+    const int32_t* lst = a.idx + list_id * a.k_max;
+    const int e0 = c * E;
+    const int e1 = min(e0 + E, a.k_max);
+    uint32_t bad = 0;
+    for (int base = e0; base < e1; base += 16) {
+      // this lane's entry: index, predecessor check, validity, physical row
+      const int e = base + l;
+      const int32_t v = e < e1 ? __ldg(lst + e) : -1;
+      uint32_t before = __shfl_up_sync(hmask, (uint32_t)v, 1, 16);
+      if (l == 0 && e > 0 && e < e1) before = (uint32_t)__ldg(lst + e - 1);
+      if (e < e1 && e > 0 && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
+      if (e < e1 && (v < -1 || v >= kvlen)) bad |= TSD_DEV_BAD_INDEX;
+      uint32_t row = kInvalidRow;
+      if (e < e1 && v >= 0 && v < kvlen) {
+        row = kv_row(a.kv, b, g, v);
+        if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
+      }
+      // the 16 rows, U at a time
+#pragma unroll
+      for (int j0 = 0; j0 < 16; j0 += kSpU) {
+        uint32_t rr[kSpU];
+        uint4 kq[kSpU], vq[kSpU];
+#pragma unroll
+        for (int u = 0; u < kSpU; ++u) {
+          rr[u] = __shfl_sync(hmask, row, j0 + u, 16);
+          kq[u] = make_uint4(0, 0, 0, 0);
+          vq[u] = make_uint4(0, 0, 0, 0);
+          row_fetch(a, rr[u], l, kq[u], vq[u]);
+        }
+        batch_update<kSpU>(kq, vq, rr, q, m_run, l_run, acc, hmask);
+      }
+    }
+    bad |= __shfl_xor_sync(hmask, bad, 1);
+    bad |= __shfl_xor_sync(hmask, bad, 2);
+    bad |= __shfl_xor_sync(hmask, bad, 4);
+    bad |= __shfl_xor_sync(hmask, bad, 8);
+    if (l == 0 && bad) flag_status(a.status, bad);
+  }
+
+  if (C == 1) {   // every list is one task (uniform over the grid)
+    if (valid) finish_task(a, list_id, t, h, 1, 0, m_run, l_run, acc, l, hmask);
+    return;
+  }
+  // Chunks c, c+1, ... of a list are M tasks apart, so a CTA holds up to 16/M consecutive
+  // chunks of each of its lists.  Their states are combined here, and each list leaves the
+  // CTA as a single partial: the cross-CTA merge reads (16/M)x fewer partials.
+  if (l == 0) {
+    s_ml[hw] = make_float2(m_run, l_run);
+    s_list[hw] = list_id;
+  }
+  *reinterpret_cast<float4*>(&s_acc[hw][8 * l]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  *reinterpret_cast<float4*>(&s_acc[hw][8 * l + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  __syncthreads();
+  if (!valid || (hw >= M && s_list[hw - M] == list_id)) return;   // not the first chunk of its list here
+  for (int o = hw + M; o < 16 && s_list[o] == list_id; o += M) {
+    const float2 x = s_ml[o];
+    const float mn = fmaxf(m_run, x.x);
+    if (mn == -CUDART_INF_F) continue;
+    const float wa = fast_exp2(m_run - mn), wb = fast_exp2(x.x - mn);
+    l_run = l_run * wa + x.y * wb;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = acc[i] * wa + s_acc[o][8 * l + i] * wb;
+    m_run = mn;
+  }
+  // partials of the list = CTAs that hold one of its chunks (with M <= 16 every CTA from the
+  // first chunk's to the last chunk's holds one); this CTA's partial index
+  int parts = C, part = c;
+  if (M <= 16) {
+    const int64_t first = (((int64_t)b * a.kv.hkv + g) * C) * M + m;
+    const int64_t last = first + (int64_t)(C - 1) * M;
+    parts = (int)((last >> 4) - (first >> 4) + 1);
+    part = (int)((int64_t)blockIdx.x - (first >> 4));
+  }
+  finish_task(a, list_id, t, h, parts, part, m_run, l_run, acc, l, hmask);
 }
 
 // ---------------------------------------------------------------------------
@@ -468,49 +510,8 @@ __global__ void __launch_bounds__(kDnThreads, 3) dense_decode_kernel(DecodeArgs 
   float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F}, l_run[2] = {0.f, 0.f};
 
   if (warp == kDnConsumers) {
-    // producer: box coordinates prefetched 32 at a time, TMA issued by lane 0
-    BoxRows br;
-    const int bp = tma_box_rows(a.kv);
-    if (use_tma) box_rows_init(br, a.kv, b, g, tok0, tok_end, bp, lane, a.status);
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int s = tile % kDnStages;
-      if (tile >= kDnStages) {
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(&S.empty[s], ((tile / kDnStages) - 1) & 1);
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (!ok) {
-          if (lane == 0) {
-            flag_status(a.status, TSD_DEV_TIMEOUT);
-            atomicOr(&S.abort, 1u);
-          }
-          break;
-        }
-      }
-      unsigned char* kd = S.stage[s];
-      unsigned char* vd = S.stage[s] + kTileBytesKV;
-      const int tok = tok0 + tile * kTileTok;
-      if (use_tma) {
-        // the expected bytes must be registered before the loads can complete the phase
-        const int rows = min(kTileTok, tok_end - tok);
-        const uint32_t want = (uint32_t)((rows + bp - 1) / bp) * 4 * bp * 128;
-        if (lane == 0) mbar_arrive_expect_tx(&S.full[s], want);
-        __syncwarp();
-        const uint32_t got = tile_issue_tma(a.kv, &maps.k, &maps.v, br, b, g, tok0, tok_end, tile, kd, vd, &S.full[s],
-                                            lane, a.status);
-        // boxes skipped for a bad page never arrive: complete their bytes so the phase ends
-        if (lane == 0 && got < want)
-          asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(&S.full[s])),
-                       "r"(want - got)
-                       : "memory");
-      } else {
-        tile_issue_cpasync(a.kv, b, g, tok, tok_end, kd, vd, lane, a.status);
-        cp_async_mbar_arrive(&S.full[s]);
-      }
-    }
-    if (lane == 0) {
-      for (int tile = (ntiles > kDnStages ? ntiles - kDnStages : 0); tile < ntiles; ++tile)
-        if (!mbar_wait(&S.full[tile % kDnStages], (tile / kDnStages) & 1)) flag_status(a.status, TSD_DEV_TIMEOUT);
-    }
+    produce_tiles<kDnStages, kDnStageBytes, true>(a.kv, maps, b, g, tok0, tok_end, ntiles, &S.stage[0][0], S.full,
+                                                  S.empty, &S.abort, use_tma, lane, a.status);
   } else {
     const int w = warp;
     const float scale2 = a.qv.sm_scale * kLog2e;
@@ -525,13 +526,7 @@ __global__ void __launch_bounds__(kDnThreads, 3) dense_decode_kernel(DecodeArgs 
     const int i4 = lane >> 3, rr = lane & 7;
     for (int tile = 0; tile < ntiles; ++tile) {
       const int s = tile % kDnStages;
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(&S.full[s], (tile / kDnStages) & 1);
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok || S.abort) {
-        if (lane == 0 && !ok) flag_status(a.status, TSD_DEV_TIMEOUT);
-        break;
-      }
+      if (!consume_wait<kDnStages>(S.full, &S.abort, tile, lane, a.status)) break;
       const unsigned char* kt = S.stage[s];
       const unsigned char* vt = S.stage[s] + kTileBytesKV;
       float sc[2][4];

@@ -125,6 +125,79 @@ __device__ __forceinline__ void tile_issue_cpasync(const KvView& kv, int b, int 
   }
 }
 
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Producer warp of a tile ring (all 32 lanes call it).  Streams tiles [0, ntiles) of the
+// window [tok0, tok_end) of (sequence b, kv head g) into stage tile % NST: K at the start of
+// the stage and, WITH_V, V kTileBytesKV after it.  `full[s]` counts the bytes of a fill
+// (TMA) or the 32 lanes' copies (cp.async); `empty[s]` the consumer warps' releases.  Every
+// wait is bounded: on a timeout the producer flags TSD_DEV_TIMEOUT, raises `abort` and
+// stops.  Before returning it waits for its last fills to land, so that no copy into shared
+// memory is in flight when the CTA ends.
+template <int NST, int STAGE_BYTES, bool WITH_V>
+__device__ __forceinline__ void produce_tiles(const KvView& kv, const KvMaps& maps, int b, int g, int tok0,
+                                              int tok_end, int ntiles, unsigned char* stages, uint64_t* full,
+                                              uint64_t* empty, uint32_t* abort, bool use_tma, int lane,
+                                              uint32_t* status) {
+  constexpr uint32_t kLoadsPerBox = WITH_V ? 4 : 2;
+  BoxRows br;
+  const int bp = tma_box_rows(kv);
+  if (use_tma) box_rows_init(br, kv, b, g, tok0, tok_end, bp, lane, status);
+  int issued = 0;
+  for (int tile = 0; tile < ntiles; ++tile) {
+    const int s = tile % NST;
+    if (tile >= NST) {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&empty[s], ((tile / NST) - 1) & 1);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) {
+        if (lane == 0) {
+          flag_status(status, TSD_DEV_TIMEOUT);
+          atomicOr(abort, 1u);
+        }
+        break;
+      }
+    }
+    unsigned char* kd = stages + (size_t)s * STAGE_BYTES;
+    unsigned char* vd = WITH_V ? kd + kTileBytesKV : nullptr;
+    const int tok = tok0 + tile * kTileTok;
+    if (use_tma) {
+      // the expected bytes must be registered before the loads can complete the phase
+      const int rows = min(kTileTok, tok_end - tok);
+      const uint32_t want = (uint32_t)((rows + bp - 1) / bp) * kLoadsPerBox * bp * 128;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], want);
+      __syncwarp();
+      const uint32_t got = tile_issue_tma(kv, &maps.k, &maps.v, br, b, g, tok0, tok_end, tile, kd, vd, &full[s], lane,
+                                          status);
+      // boxes skipped for a bad page never arrive: complete their bytes so the phase ends
+      if (lane == 0 && got < want) mbar_complete_tx(&full[s], want - got);
+    } else {
+      tile_issue_cpasync(kv, b, g, tok, tok_end, kd, vd, lane, status);
+      cp_async_mbar_arrive(&full[s]);
+    }
+    issued = tile + 1;
+  }
+  if (lane == 0) {
+    for (int tile = (issued > NST ? issued - NST : 0); tile < issued; ++tile)
+      if (!mbar_wait(&full[tile % NST], (tile / NST) & 1)) flag_status(status, TSD_DEV_TIMEOUT);
+  }
+}
+
+// Consumer warp: wait (bounded) for tile `tile` of the ring.  False on a timeout (flagged)
+// or when the producer has given up.
+template <int NST>
+__device__ __forceinline__ bool consume_wait(uint64_t* full, const uint32_t* abort, int tile, int lane,
+                                             uint32_t* status) {
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(&full[tile % NST], (tile / NST) & 1);
+  ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+  if (!ok && lane == 0) flag_status(status, TSD_DEV_TIMEOUT);
+  return ok && *reinterpret_cast<const volatile uint32_t*>(abort) == 0u;
+}
+
 // Query tile (mma A operand, 16 rows x 128 dims) in shared memory, laid out like a K tile
 // (two 128-byte halves of [16 rows][128 B], 128-byte swizzled): row m is list m of the CTA
 // (token j = m / G of the sequence, q head g * G + m % G); rows >= nlists are zero.  For

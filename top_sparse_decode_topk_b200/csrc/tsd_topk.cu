@@ -24,156 +24,111 @@
 
 #include "tsd_args.h"
 #include "tsd_common.cuh"
+#include "tsd_kvtile.cuh"
 
 namespace tsd {
 
-constexpr int kScoreRows = 32;                   // rows per tile
-constexpr int kScoreStages = 4;
-constexpr int kScoreTileBytes = kScoreRows * 256;
-constexpr int kHeadsPerScoreGroup = 4;
 constexpr int kSelBins = 2048;
 constexpr int kCandMax = 8192;
 constexpr int kSelPerThread = 16;                 // scores per thread per tile (4 x float4)
 
 
 // ---------------------------------------------------------------------------
-// Scoring
+// Scoring on tensor cores
 // ---------------------------------------------------------------------------
+// One CTA per (sequence b, kv head g, list group lg, window of W tokens).  A producer warp
+// streams 64-token K tiles through a 4-stage ring (TMA, tsd_kvtile.cuh); each of the 4
+// consumer warps scores 16 tokens of every tile against the CTA's 16 query rows with
+// mma.m16n8k16 (bf16 inputs, fp32 accumulation; fp32 queries as bf16 hi + lo) and writes
+// the unscaled fp32 dots of tokens below each list's kv_len.
+constexpr int kScStages = 4;
+constexpr int kScConsumers = 4;
+constexpr int kScThreads = 32 * (kScConsumers + 1);
+
 struct ScoreSmem {
-  unsigned char ring[kScoreStages * kScoreTileBytes];
-  uint32_t rowaddr[kScoreStages][kScoreRows];
+  alignas(1024) unsigned char stage[kScStages][kTileBytesKV];
+  alignas(1024) unsigned char qhi[kQTileBytes];
+  alignas(1024) unsigned char qlo[kQTileBytes];
+  uint64_t full[kScStages];
+  uint64_t empty[kScStages];
+  uint32_t abort;
 };
+static_assert(sizeof(ScoreSmem) + 1024 <= 75 * 1024, "three scoring CTAs per SM");
 
-__device__ __forceinline__ void score_load_tile(ScoreSmem& S, const KvView& kv, int b, int g, int tok0,
-                                                int tile, int ntok, uint32_t* status) {
-  const int stage = tile % kScoreStages;
-  unsigned char* base = S.ring + stage * kScoreTileBytes;
-  const int first = tok0 + tile * kScoreRows;
-#pragma unroll
-  for (int q = 0; q < (kScoreRows * 16) / kScoreThreads; ++q) {
-    const int id = threadIdx.x + q * kScoreThreads;
-    const int r = id >> 4, ch = id & 15;
-    const int tok = first + r;
-    if (tok - tok0 < ntok) {
-      const uint32_t row = kv_row(kv, b, g, tok);
-      if (row != kInvalidRow) cp_async16(base + r * 256 + ch * 16, kv.k + (int64_t)row * kHeadDim + ch * 8);
-      if (ch == 0) {
-        S.rowaddr[stage][r] = row;
-        if (row == kInvalidRow) flag_status(status, TSD_DEV_BAD_PAGE);
-      }
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kScoreThreads, 2) topk_score_kernel(TopkArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>(smem_raw);
+template <bool QF32>
+__global__ void __launch_bounds__(kScThreads, 3) topk_score_kernel(TopkArgs a, const __grid_constant__ KvMaps maps) {
+  extern __shared__ __align__(1024) unsigned char smem_sc[];
+  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>(smem_sc);
   const int win = blockIdx.x;
   const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
   const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, win == 0 && g == 0 && lg == 0 && threadIdx.x == 0);
   const int G = a.qv.hq / a.kv.hkv;
   int nlists = si.n * G - lg * a.lists_per_cta;
   if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
   if (nlists <= 0) return;
   const int tok0 = win * a.window;
-  int ntok = si.len - tok0;
-  if (ntok > a.window) ntok = a.window;
-  if (ntok <= 0) return;
-  const int ntiles = (ntok + kScoreRows - 1) / kScoreRows;
-
-#pragma unroll
-  for (int s = 0; s < kScoreStages - 1; ++s) {
-    if (s < ntiles) score_load_tile(S, a.kv, b, g, tok0, s, ntok, a.status);
-    cp_async_commit();
+  const int tok_end = min(tok0 + a.window, si.len);
+  if (tok_end <= tok0) return;
+  const int ntiles = (tok_end - tok0 + kTileTok - 1) / kTileTok;
+  const bool use_tma = a.kv.page_table == nullptr || a.kv.page_shift >= 3;
+  // the swizzled tiles need 1024-byte alignment; refuse to run rather than mis-address them
+  if (smem_u32(S.stage[0]) & 1023u) {
+    if (threadIdx.x == 0) flag_status(a.status, TSD_DEV_TIMEOUT);
+    return;
   }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kScStages; ++s) {
+      mbar_init(&S.full[s], use_tma ? 1 : 32);
+      mbar_init(&S.empty[s], kScConsumers);
+    }
+    mbar_fence_init();
+    S.abort = 0;
+  }
+  store_q_tile(a.qv, si, g, G, lg * a.lists_per_cta, nlists, S.qhi, QF32 ? S.qlo : nullptr, threadIdx.x, kScThreads);
+  __syncthreads();
 
-  const int group = threadIdx.x >> 3, l8 = threadIdx.x & 7;
-  const int nsets = (nlists + kHeadsPerScoreGroup - 1) / kHeadsPerScoreGroup;   // <= 8
-  const int PG = 32 / nsets;
-  const int my_set = group / PG, my_part = group % PG;
-  const bool has_set = my_set < nsets;
-
-  // the 4 query vectors of this group's set; lane l8 holds dims [8*l8, +8) and [64+8*l8, +8)
-  float q[kHeadsPerScoreGroup][16];
-  int kvlen[kHeadsPerScoreGroup];
-  int64_t srow[kHeadsPerScoreGroup];
+  if (warp == kScConsumers) {
+    produce_tiles<kScStages, kTileBytesKV, false>(a.kv, maps, b, g, tok0, tok_end, ntiles, &S.stage[0][0], S.full,
+                                                  S.empty, &S.abort, use_tma, lane, a.status);
+    return;
+  }
+  // this lane's query rows m = lane/4 and lane/4 + 8: visible length and score row
+  int kvl[2];
+  float* srow[2];
 #pragma unroll
-  for (int hh = 0; hh < kHeadsPerScoreGroup; ++hh) {
-    const int m = my_set * kHeadsPerScoreGroup + hh;
-    const bool ok = has_set && m < nlists;
-    const int mg = lg * a.lists_per_cta + (ok ? m : 0);
-    const int j = mg / G;
-    const int t = si.t0 + j, h = g * G + (mg - j * G);
-    kvlen[hh] = ok ? kv_len_of(a.qv, si, j) : 0;
-    srow[hh] = ((int64_t)t * a.qv.hq + h) * a.score_stride;
-    const int64_t base = ((int64_t)t * a.qv.hq + h) * kHeadDim;
-    if (a.qv.q_f32) {
-      const float* p = reinterpret_cast<const float*>(a.qv.q) + base;
-#pragma unroll
-      for (int j2 = 0; j2 < 8; ++j2) {
-        q[hh][j2] = __ldg(p + 8 * l8 + j2);
-        q[hh][8 + j2] = __ldg(p + 64 + 8 * l8 + j2);
-      }
-    } else {
-      const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.qv.q) + base);
-      unpack8(__ldg(p + l8), q[hh]);
-      unpack8(__ldg(p + 8 + l8), q[hh] + 8);
+  for (int hr = 0; hr < 2; ++hr) {
+    const int m = (lane >> 2) + 8 * hr;
+    kvl[hr] = 0;
+    srow[hr] = a.scores;
+    if (m < nlists) {
+      const int mg = lg * a.lists_per_cta + m;
+      const int j = mg / G;
+      kvl[hr] = min(kv_len_of(a.qv, si, j), tok_end);
+      srow[hr] = a.scores + ((int64_t)(si.t0 + j) * a.qv.hq + g * G + (mg - j * G)) * a.score_stride;
     }
   }
-  // after the transposed reduction lane l8 holds the dot of head ((l8>>2)&1)*2 + ((l8>>1)&1)
-  const int my_head = ((l8 >> 2) & 1) * 2 + ((l8 >> 1) & 1);
-  int my_kvlen = kvlen[0];
-  int64_t my_srow = srow[0];
-#pragma unroll
-  for (int hh = 1; hh < kHeadsPerScoreGroup; ++hh)
-    if (my_head == hh) { my_kvlen = kvlen[hh]; my_srow = srow[hh]; }
-
   for (int tile = 0; tile < ntiles; ++tile) {
-    cp_async_wait<kScoreStages - 2>();
-    __syncthreads();
-    if (tile + kScoreStages - 1 < ntiles) score_load_tile(S, a.kv, b, g, tok0, tile + kScoreStages - 1, ntok, a.status);
-    cp_async_commit();
-    const int stage = tile % kScoreStages;
-    const unsigned char* kbase = S.ring + stage * kScoreTileBytes;
-    const int rows = min(kScoreRows, ntok - tile * kScoreRows);
-    for (int r0 = 0; r0 < kScoreRows; r0 += PG) {
-      const int r = r0 + my_part;
-      const int rr = r < kScoreRows ? r : 0;
-      const unsigned char* krow = kbase + rr * 256;
-      uint4 k0 = *reinterpret_cast<const uint4*>(krow + 16 * l8);
-      uint4 k1 = *reinterpret_cast<const uint4*>(krow + 128 + 16 * l8);
-      float kf[16];
-      unpack8(k0, kf);
-      unpack8(k1, kf + 8);
-      float v[kHeadsPerScoreGroup];
+    if (!consume_wait<kScStages>(S.full, &S.abort, tile, lane, a.status)) break;
+    float sc[2][4];
+    qk_tile<QF32>(S.qhi, S.qlo, S.stage[tile % kScStages], warp, lane, sc);
+    const int tbase = tok0 + tile * kTileTok + 16 * warp + 2 * (lane & 3);
 #pragma unroll
-      for (int hh = 0; hh < kHeadsPerScoreGroup; ++hh) {
-        float s0 = 0.f, s1 = 0.f;
+    for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          s0 = fmaf(q[hh][j], kf[j], s0);
-          s1 = fmaf(q[hh][8 + j], kf[8 + j], s1);
+      for (int nt = 0; nt < 2; ++nt) {
+        const int tk = tbase + 8 * nt;   // even: the pair (tk, tk + 1) is 8-byte aligned
+        if (tk + 1 < kvl[hr]) {
+          *reinterpret_cast<float2*>(srow[hr] + tk) = make_float2(sc[nt][2 * hr], sc[nt][2 * hr + 1]);
+        } else if (tk < kvl[hr]) {
+          srow[hr][tk] = sc[nt][2 * hr];
         }
-        v[hh] = s0 + s1;
       }
-      // transposed butterfly: 4 partial dots over 8 lanes -> one full dot per lane pair
-      const bool hi4 = (l8 & 4) != 0;
-      float a0 = hi4 ? v[2] : v[0], a1 = hi4 ? v[3] : v[1];
-      float s0 = hi4 ? v[0] : v[2], s1 = hi4 ? v[1] : v[3];
-      a0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 4);
-      a1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 4);
-      const bool hi2 = (l8 & 2) != 0;
-      float c = hi2 ? a1 : a0, d = hi2 ? a0 : a1;
-      c += __shfl_xor_sync(0xFFFFFFFFu, d, 2);
-      c += __shfl_xor_sync(0xFFFFFFFFu, c, 1);
-      const int tok = tok0 + tile * kScoreRows + rr;
-      const bool ok = has_set && r < rows && (l8 & 1) == 0 && tok < my_kvlen &&
-                      S.rowaddr[stage][rr] != kInvalidRow;
-      if (ok) a.scores[my_srow + tok] = c;
-    }
+    // the stores consume every fragment read from the stage: release it to the producer
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.empty[tile % kScStages]);
   }
-  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -386,18 +341,26 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
-cudaError_t launch_topk(const TopkArgs& a, int nwin, int batch, int hkv, int num_lists, cudaStream_t stream) {
+cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int batch, int hkv, int num_lists,
+                        cudaStream_t stream) {
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(topk_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(ScoreSmem));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SelectSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_score_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)sizeof(ScoreSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SelectSmem));
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 g1(nwin, hkv * a.list_groups, batch);
-  topk_score_kernel<<<g1, kScoreThreads, sizeof(ScoreSmem), stream>>>(a);
+  if (a.qv.q_f32) {
+    topk_score_kernel<true><<<g1, kScThreads, sizeof(ScoreSmem), stream>>>(a, maps);
+  } else {
+    topk_score_kernel<false><<<g1, kScThreads, sizeof(ScoreSmem), stream>>>(a, maps);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   topk_select_kernel<<<num_lists, kSelectThreads, sizeof(SelectSmem), stream>>>(a);
