@@ -48,6 +48,9 @@ def parse():
     p.add_argument("--impl", choices=["native", "reference"], default="native")
     p.add_argument("--config", default="llama3_8b")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--record-traffic", metavar="NCU_CSV",
+                   help="write profiles/dram_traffic.json for --config from an ncu --csv log of "
+                        "dram__bytes_read.sum, dram__bytes_write.sum and gpu__time_duration.sum (no GPU work)")
     return p.parse_args()
 
 
@@ -125,13 +128,22 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # Helpers
 # ---------------------------------------------------------------------------
-def source_sha(name):
-    path = os.path.join(ROOT, "top_sparse_decode_topk_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+# files whose contents decide the sparse kernel and its launch shape
+SPARSE_SOURCES = ["tsd_decode.cu", "tsd_plan.h", "tsd_common.cuh"]
 
 
-def ncu_traffic(kernel: str, workload: str, source: str):
+def source_sha(names):
+    """Hash of the kernel sources (file names under csrc/, or one name), in order."""
+    if isinstance(names, str):
+        names = [names]
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "top_sparse_decode_topk_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str, source):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
@@ -144,6 +156,56 @@ def ncu_traffic(kernel: str, workload: str, source: str):
         return float(e["bytes_per_launch"])
     except Exception:
         return None
+
+
+# kernel -> the csrc files that decide its code and launch shape
+KERNEL_SOURCES = {
+    "sparse_decode_kernel": SPARSE_SOURCES,
+    "dense_decode_kernel": ["tsd_decode.cu", "tsd_plan.h", "tsd_common.cuh", "tsd_kvtile.cuh"],
+    "topk_score_kernel": ["tsd_topk.cu", "tsd_plan.h", "tsd_common.cuh", "tsd_kvtile.cuh"],
+    "topk_select_kernel": ["tsd_topk.cu", "tsd_plan.h", "tsd_common.cuh"],
+}
+
+
+def record_traffic(csv_path: str, workload: str):
+    """Fold one ncu --csv metric log into profiles/dram_traffic.json (first launch of each kernel)."""
+    import csv
+    with open(csv_path) as f:
+        rows = list(csv.reader(f))
+    head = [i for i, r in enumerate(rows) if r and r[0] == "ID"][0]
+    h = rows[head]
+    got = {}
+    for r in rows[head + 1:]:
+        d = dict(zip(h, r))
+        name = d.get("Kernel Name", "")
+        kern = next((k for k in KERNEL_SOURCES if k in name), None)
+        if kern is None:
+            continue
+        e = got.setdefault(kern, {"id": d["ID"]})
+        if e["id"] != d["ID"]:
+            continue   # a later launch of the same kernel
+        e[d["Metric Name"]] = float(d["Metric Value"].replace(",", ""))
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            out = json.load(f)
+    except Exception:
+        out = {}
+    out["_about"] = ("DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of one captured "
+                     "launch per kernel in the first timed step of the bench, L2 flushed before it; bench.py "
+                     "uses a kernel's figure as roofline.traffic only while source_sha still matches its sources.")
+    for kern, e in got.items():
+        rd, wr = e.get("dram__bytes_read.sum"), e.get("dram__bytes_write.sum")
+        if rd is None or wr is None:
+            continue
+        out.setdefault(kern, {})[workload] = {
+            "bytes_per_launch": rd + wr, "read": rd, "write": wr,
+            "duration_us": round(e.get("gpu__time_duration.sum", float("nan")) / 1e3, 3),
+            "sources": KERNEL_SOURCES[kern], "source_sha": source_sha(KERNEL_SOURCES[kern])}
+    with open(path, "w") as f:
+        json.dump(out, f, indent=1)
+    print(json.dumps({k: v for k, v in out.items() if k != "_about"}, indent=1))
+
 
 
 def unique_rows(idx, token_seq, hkv, group, max_len):
@@ -361,7 +423,7 @@ def run_native(args):
         return
 
     cl = clocks.summary()
-    traffic = ncu_traffic("sparse_decode_kernel", cfg.name, "tsd_decode.cu")
+    traffic = ncu_traffic("sparse_decode_kernel", cfg.name, SPARSE_SOURCES)
     line = {
         "metric": METRIC,
         "value": round(sparse_ms * 1e3, 3),
@@ -471,7 +533,9 @@ def run_reference(args):
 
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.config)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_native(args)

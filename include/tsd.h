@@ -136,7 +136,10 @@ tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries
                            const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count,
                            void* ws, size_t ws_bytes, tsd_stream_t stream);
 
-/* Host: bytes of workspace tsd_sparse_decode needs for these shapes (0 on invalid input). */
+/* Host: bytes of workspace tsd_sparse_decode needs for these shapes on the current device
+ * (0 on invalid input).  The work split, and so the size, depends on the device's SM count:
+ * size the workspace with the device that will run the calls current (148 SMs are assumed
+ * when no device can be queried). */
 size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries,
                                         int32_t k_max);
 

@@ -186,6 +186,29 @@ size_t tsd_topk_workspace_size(const tsd_kv_cache* cache, const tsd_queries* que
   return topk_layout(sh).total;
 }
 
+// SM count of the current device: the sparse plan sizes its grid to the resident CTAs.  A
+// B200's 148 when no device can be queried (host-only sizing calls on a machine without one).
+static int current_sm_count() {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static int cache[kMaxDev] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();
+    return 148;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 static tsd_status sizes_for(const tsd_kv_cache* cache, const tsd_queries* queries, Shapes* sh) {
   if (cache == nullptr || queries == nullptr) return TSD_ERR_INVALID_ARGUMENT;
   KvView kv; QView qv;
@@ -203,7 +226,7 @@ static tsd_status sizes_for(const tsd_kv_cache* cache, const tsd_queries* querie
 size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max) {
   Shapes sh;
   if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return 0;
-  const SparsePlan p = plan_sparse(sh, k_max);
+  const SparsePlan p = plan_sparse(sh, k_max, current_sm_count());
   return decode_layout(sh, p.nsplit).total;
 }
 
@@ -267,7 +290,7 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
   if (st != TSD_OK) return st;
   if (idx == nullptr || k_max < 1) return TSD_ERR_INVALID_ARGUMENT;
   if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
-  const SparsePlan p = plan_sparse(sh, k_max);
+  const SparsePlan p = plan_sparse(sh, k_max, current_sm_count());
   const DecodeLayout lay = decode_layout(sh, p.nsplit);
   if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
   DecodeArgs a;
@@ -350,7 +373,7 @@ tsd_status prepare_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* q
   if (out == nullptr || idx == nullptr || k_max < 1) return TSD_ERR_INVALID_ARGUMENT;
   if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return TSD_ERR_UNSUPPORTED;
   if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
-  const SparsePlan p = plan_sparse(*sh, k_max);
+  const SparsePlan p = plan_sparse(*sh, k_max, current_sm_count());
   const DecodeLayout lay = decode_layout(*sh, p.nsplit);
   memset(a, 0, sizeof(*a));
   a->kv = kv;

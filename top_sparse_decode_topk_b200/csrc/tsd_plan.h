@@ -56,36 +56,44 @@ inline size_t zero_region_bytes(const Shapes& s) {
 constexpr int kMaxSparseK = kMaxSplits * kMaxEntriesPerCta;
 
 // Sparse decode: every list (token x q head) is cut into C tasks of E entries (E a
-// multiple of 16); a task is one half-warp.  E grows with the workload so that the task
-// count stays near kSparseTaskTarget (a few per resident half-warp of a B200: enough to
-// keep every SM issuing gathers, few enough that the split-K partials stay small), and
-// C stays <= kMaxSplits.
+// multiple of 16); a task is one half-warp and a CTA runs 16 tasks.  Every task takes about
+// the same time, so a grid that spills a little into a second wave of resident CTAs costs
+// nearly a whole extra wave.  The plan therefore takes the smallest E whose tasks fit one
+// wave (kSpCtasPerSm CTAs on each SM).  When even one task per list leaves that wave well
+// under-filled (many lists, as with several decode tokens per sequence), it cuts the lists
+// finer instead, about two tasks per resident half-warp, and lets the lists of unequal
+// length even out.  C stays <= kMaxSplits either way.
 struct SparsePlan {
   int lists;     // list slots per (sequence, kv head): G x max tokens per sequence
   int entries;   // E
   int nsplit;    // C
 };
 
-constexpr int64_t kSparseTaskTarget = 2 * 148 * 48;
+constexpr int kSpCtasPerSm = 3;   // resident sparse-decode CTAs per SM (its launch bounds)
 
-inline SparsePlan plan_sparse(const Shapes& s, int k_max) {
+inline SparsePlan plan_sparse(const Shapes& s, int k_max, int num_sms) {
   SparsePlan p;
   p.lists = (int)(s.group * s.max_tokens);
-
-  const double total = (double)s.tokens * s.hq * k_max;
-  int e = (int)(total / kSparseTaskTarget);
-  e = (e + 15) / 16 * 16;
-  if (e < 16) e = 16;
-  if (e > 1024) e = 1024;
+  const int64_t slots = (int64_t)num_sms * kSpCtasPerSm;
+  const int64_t units = s.batch * s.hkv * p.lists;
   const int kr = (k_max + 15) / 16 * 16;
-  if (e > kr) e = kr;
-  int ns = (k_max + e - 1) / e;
-  if (ns > kMaxSplits) {
-    e = ((k_max + kMaxSplits - 1) / kMaxSplits + 15) / 16 * 16;
-    ns = (k_max + e - 1) / e;
+  int e = 16;
+  for (; e < kr; e += 16) {
+    const int64_t ns = (k_max + e - 1) / e;
+    if (ns <= kMaxSplits && (units * ns + 15) / 16 <= slots) break;
+  }
+  const int64_t ctas = (units * ((k_max + e - 1) / e) + 15) / 16;
+  if (4 * ctas < 3 * slots) {   // one wave would be under-filled: about two tasks per half-warp
+    const double total = (double)s.tokens * s.hq * k_max;
+    e = (int)(total / (2.0 * 16.0 * (double)slots));
+    e = (e + 15) / 16 * 16;
+    if (e < 16) e = 16;
+    if (e > 1024) e = 1024;
+    if (e > kr) e = kr;
+    if ((k_max + e - 1) / e > kMaxSplits) e = ((k_max + kMaxSplits - 1) / kMaxSplits + 15) / 16 * 16;
   }
   p.entries = e;
-  p.nsplit = ns;
+  p.nsplit = (k_max + e - 1) / e;
   return p;
 }
 
