@@ -21,28 +21,14 @@
 
 namespace tsd {
 
-constexpr int kMaxListsPerCta = 32;     // query lists (token x q head) handled by one CTA
-constexpr int kSparseMaxLists = 16;     // sparse decode: lists per work unit (one half-warp each at least)
-constexpr int kDecodeThreads = 256;     // 8 warps = 32 groups of 8 lanes
-constexpr int kRowsPerTile = 16;        // K/V rows per pipeline stage
-constexpr int kStages = 4;              // cp.async pipeline depth
-constexpr int kMaxEntriesPerCta = 1024; // sparse: lists x entries per CTA
-constexpr int kBitmapWords = 1024;      // sparse: dedupe bitmap spans 32768 tokens
 constexpr int kMaxSplits = 256;         // split-K partials per (token, head)
-constexpr int kScoreThreads = 256;
-constexpr int kSelectThreads = 512;
-constexpr int kScoreTokensPerCta = 1024;
+constexpr int kMaxEntriesPerSplit = 1024;  // bound used for the largest supported k
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Shapes {
   int64_t batch, hkv, hq, group, tokens, max_tokens, max_seq_len;
 };
-
-inline int list_groups(const Shapes& s) {
-  int64_t m = s.group * s.max_tokens;
-  return (int)((m + kMaxListsPerCta - 1) / kMaxListsPerCta);
-}
 
 // Room for one arrival counter per list (token x q head), which also covers one per
 // (sequence, kv head, list group).
@@ -52,8 +38,8 @@ inline size_t zero_region_bytes(const Shapes& s) {
 }
 
 // Longest index list tsd_sparse_decode accepts (kMaxSplits chunks of at most
-// kMaxEntriesPerCta entries).
-constexpr int kMaxSparseK = kMaxSplits * kMaxEntriesPerCta;
+// kMaxEntriesPerSplit entries).
+constexpr int kMaxSparseK = kMaxSplits * kMaxEntriesPerSplit;
 
 // Sparse decode: every list (token x q head) is cut into C tasks of E entries (E a
 // multiple of 16); a task is one half-warp and a CTA runs 16 tasks.  Every task takes about

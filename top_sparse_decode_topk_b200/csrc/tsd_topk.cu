@@ -6,13 +6,11 @@
 // and the kept indices are written in ascending order.
 //
 // Two kernels:
-//  * topk_score_kernel -- one CTA per (sequence, kv head, list group, 1024-token
-//    window).  K rows stream through a 4-stage cp.async ring of 32-row tiles;
-//    each row is read from HBM once and scored against every query of the GQA
-//    group and every decode token of the sequence (up to 32 lists per CTA).
-//    Lane-groups of 8 lanes hold 4 query vectors (16 dims per lane) and reduce
-//    the 4 dots with a 4-shuffle transposed butterfly.  Scores are fp32
-//    (bf16 x bf16 products are exact in fp32; only the sum rounds).
+//  * topk_score_kernel -- one CTA per (sequence, kv head, list group of <= 16 lists, window of
+//    tokens).  A producer warp streams 64-token K tiles into shared memory with TMA; four
+//    consumer warps score them against the lists' queries on the tensor cores (mma.sync,
+//    bf16 in, fp32 accumulate) and write fp32 scores.  Each K row is read from HBM once for
+//    every query of the GQA group and every decode token of the sequence.
 //  * topk_select_kernel -- one CTA per (t, h).  Scores map to order-preserving
 //    uint32 keys; an 11-bit histogram finds the bin holding the k-th key,
 //    further digit passes narrow it until the candidates fit shared memory, a
@@ -28,6 +26,7 @@
 
 namespace tsd {
 
+constexpr int kSelectThreads = 512;   // one CTA per (token, head)
 constexpr int kSelBins = 2048;
 constexpr int kCandMax = 8192;
 constexpr int kSelPerThread = 16;                 // scores per thread per tile (4 x float4)
