@@ -280,6 +280,32 @@ def time_cpu_oracle(w, k, budget_s=10.0):
 # ---------------------------------------------------------------------------
 # Native arm
 # ---------------------------------------------------------------------------
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's workload: every rank decodes its own batch of sequences (weak scaling)."""
+    return rank
+
+
+def max_over_ranks(values, device):
+    """Element-wise MAX of per-rank timings over the process group (identity on one process).
+    Every rank must call it with the same number of values, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def sum_over_ranks(values, device):
+    """Element-wise SUM over the process group (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.tolist()
+
+
 def run_native(args):
     import numpy as np
     import torch
@@ -306,7 +332,7 @@ def run_native(args):
 
     cfg = W.CONFIGS[args.config]
     k = cfg.ks[0] if cfg.ks else None
-    w = W.make_workload(cfg, seed=rank)
+    w = W.make_workload(cfg, seed=rank_seed(rank))
     dw = W.to_device(w, dev)
     contiguous = cfg.layout == "contiguous"
     cache = tsd.KVCache(dw.k, dw.v, dw.seq_lens, max_seq_len=cfg.max_seq_len,
@@ -359,10 +385,7 @@ def run_native(args):
         dist.barrier()
     ms = np.array([[ev[s][2 * j].elapsed_time(ev[s][2 * j + 1]) for j in range(3)] for s in range(args.steps)])
     mean_ms = ms.mean(axis=0)
-    t = torch.tensor(mean_ms.tolist(), dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    topk_ms, sparse_ms, dense_ms = t.tolist()
+    topk_ms, sparse_ms, dense_ms = max_over_ranks(mean_ms.tolist(), dev)
 
     # algorithmic bytes (per rank; every rank has the same shapes)
     T, Hq, Hkv, G = len(w.kv_len), cfg.num_q_heads, cfg.num_kv_heads, cfg.group
@@ -377,8 +400,13 @@ def run_native(args):
     topk_bytes = ctx_rows * 256 + q_bytes + T * Hq * k_max * 4
     index_bytes = T * Hq * k_max * 4
     hbm, peak_kind = peaks()
+    # whole-job bytes (each rank decodes its own batch) over the slowest rank's time; the
+    # roofline is per GPU: the job's bytes per GPU over that time
+    job_sparse, job_dense, job_topk = sum_over_ranks([sparse_bytes, dense_bytes, topk_bytes], dev)
     gbs = lambda b, ms_: b / (ms_ * 1e-3) / 1e9
-    sparse_gbs, dense_gbs, topk_gbs = gbs(sparse_bytes, sparse_ms), gbs(dense_bytes, dense_ms), gbs(topk_bytes, topk_ms)
+    job_sparse_gbs = gbs(job_sparse, sparse_ms)
+    sparse_gbs, dense_gbs, topk_gbs = (gbs(job_sparse / world, sparse_ms), gbs(job_dense / world, dense_ms),
+                                       gbs(job_topk / world, topk_ms))
 
     # end to end through the public API with pinned host buffers
     q_host = dw.q.cpu().pin_memory()
@@ -405,10 +433,7 @@ def run_native(args):
         if s >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
             e2e_idx_ms.append(c.elapsed_time(d))
-    e = torch.tensor([float(np.mean(e2e_ms)), float(np.mean(e2e_idx_ms))], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e, op=dist.ReduceOp.MAX)
-    e2e_us, e2e_idx_us = (x * 1e3 for x in e.tolist())
+    e2e_us, e2e_idx_us = (x * 1e3 for x in max_over_ranks([np.mean(e2e_ms), np.mean(e2e_idx_ms)], dev))
     if tsd.read_device_status(ws) != 0:
         raise RuntimeError("device status bits set during the timed run")
 
@@ -442,7 +467,8 @@ def run_native(args):
         "config": workload_desc(cfg, k_max),
         "legs_us": {"topk_select": round(topk_ms * 1e3, 3), "sparse_decode": round(sparse_ms * 1e3, 3),
                     "dense_decode": round(dense_ms * 1e3, 3)},
-        "effective_gbs": round(sparse_gbs, 1),
+        "effective_gbs": round(job_sparse_gbs, 1),
+        "effective_gbs_per_gpu": round(sparse_gbs, 1),
         "speedup_vs_dense": round(dense_ms / sparse_ms, 3),
         "speedup_vs_dense_with_indexer": round(dense_ms / (sparse_ms + topk_ms), 3),
         "roofline": {"bound": "hbm", "achieved": round(sparse_gbs, 1), "peak": hbm, "unit": "GB/s",

@@ -1,0 +1,71 @@
+"""Host logic of the multi-process bench on CPU: two gloo ranks, no GPU.
+
+The decode path has no exchange between GPUs: each rank decodes its own batch (weak
+scaling), and the ranks only meet to time the job, taking the slowest rank's time and
+summing the bytes moved.  These tests run that logic in two processes over gloo, and the
+reference arm under torchrun, where rank 0 alone prints the line.
+"""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out_dir: str):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    from top_sparse_decode_topk_b200 import workload as W
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        mx = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 5.0], "cpu")
+        sm = bench.sum_over_ranks([100.0 * (rank + 1), 1.0], "cpu")
+        w = W.make_workload(W.CONFIGS["tiny"], seed=bench.rank_seed(rank))
+        digest = int(np.bitwise_xor.reduce(w.q_bits.reshape(-1).astype(np.uint64)))
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"max": mx, "sum": sm, "q_digest": digest}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_reduce_timings_and_own_their_batches(tmp_path):
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True, start_method="spawn")
+    r0 = json.load(open(tmp_path / "rank0.json"))
+    r1 = json.load(open(tmp_path / "rank1.json"))
+    for r in (r0, r1):
+        assert r["max"] == [2.0, 10.0, 5.0]          # slowest rank per leg
+        assert r["sum"] == [300.0, 2.0]              # bytes of the whole job
+    assert r0["q_digest"] != r1["q_digest"]          # each rank decodes a different batch
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--config", "tiny", "--gpus", "2", "--steps", "1", "--warmup", "0"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
