@@ -17,6 +17,10 @@ Opportunity?" (gist.science technical summary, section 2 "Oracle Top-K" and
   (one term per list entry), giving the output row and its log-sum-exp.
 * ``dense_attention``: the same over every visible token (the dense-decode
   baseline whose O(N d) traffic sparse decoding reduces to O(k d)).
+* ``channel_importance``, ``choose_channels``, ``label_scores`` (``label.py``): the
+  Double-Sparsity-style approximate indexer the pages use to price indexing (section
+  3.C): a few "label" channels per kv head chosen by magnitude, approximate scores over
+  them; its selection is ``exact_topk`` of those scores.
 * ``topk_sets_agree``: the acceptance rule for a GPU top-k set (exact set
   equality except for tokens whose score is within a relative band of the
   k-th score).
@@ -33,3 +37,4 @@ from .attention import (  # noqa: F401
     sparse_attention,
 )
 from .compare import topk_sets_agree, output_errors  # noqa: F401
+from .label import channel_importance, choose_channels, label_scores  # noqa: F401
