@@ -203,6 +203,61 @@ tsd_status tsd_sparse_decode_static_ws(const tsd_kv_cache* cache, const tsd_quer
  */
 tsd_status tsd_read_device_status(void* ws, tsd_stream_t stream, uint32_t* flags);
 
+/* ---------------------------------------------------------------------------------------
+ * Label-channel approximate indexer (Double-Sparsity-style).
+ *
+ * The pages ("Inference Time Context Sparsity: Illusion or Opportunity?", gist.science
+ * summary, section 3.C "Indexing overhead") price the indexer in front of sparse decode by
+ * simulating Double Sparsity: every token is scored with only a few "label" channels of
+ * its key, held in a compact cache, and the top k of those approximate scores are kept.
+ * The pages fix neither the channel count nor the choice; this library takes r channels
+ * per kv head (r in {8, 16, 32}) with the largest total |q_d K_{i,d}| over a calibration
+ * set (ties to the lower channel index), in ascending order.
+ * --------------------------------------------------------------------------------------- */
+
+/* Host: bytes of the label cache for `cache` and r channels: one row of r bf16 values per K
+ * row, same layout and row numbering as K (paged: [num_pages][Hkv][page_size][r];
+ * contiguous: [B][Hkv][max_seq_len][r]).  0 on invalid input. */
+size_t tsd_label_cache_bytes(const tsd_kv_cache* cache, int32_t r);
+
+/* Host: workspace bytes of tsd_label_channels (0 on invalid input). */
+size_t tsd_label_channels_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries);
+
+/*
+ * Offline calibration: choose r label channels per kv head from the queries and the cache.
+ * importance[g][d] = sum over sequences b of (sum over the queries t of b and q heads h of
+ * group g of |q[t,h,d]|) x (sum over tokens i < seq_lens[b] of |K[b,g,i,d]|), accumulated in
+ * fp64 in a fixed order (deterministic); the r largest per g, ties to the lower d.
+ * channels: device int32 [Hkv][r], ascending per kv head.  The first 4 bytes of ws receive
+ * the device status (bad page or length); the workspace needs no zeroing.
+ * Errors: INVALID_ARGUMENT (r not in {8, 16, 32}, null pointers), WORKSPACE_TOO_SMALL, CUDA.
+ */
+tsd_status tsd_label_channels(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t r,
+                              int32_t* channels, void* ws, size_t ws_bytes, tsd_stream_t stream);
+
+/*
+ * Build the label cache: label_k[row][j] = K[row][channels[g][j]] for every K row (rows of
+ * unused slots included).  channels: device int32 [Hkv][r] in [0, 128) (an entry outside
+ * that range reads channel 0 and sets TSD_DEV_BAD_INDEX in *status).  label_k: device, at
+ * least tsd_label_cache_bytes(cache, r) bytes, 16-byte aligned.  status: device uint32 or
+ * NULL.  Errors: INVALID_ARGUMENT, UNSUPPORTED (r), CUDA.
+ */
+tsd_status tsd_label_cache_build(const tsd_kv_cache* cache, const int32_t* channels, int32_t r, void* label_k,
+                                 uint32_t* status, tsd_stream_t stream);
+
+/*
+ * Approximate top-k: as tsd_topk_select, but the score of token i for (t, h) is
+ * s~_i = sum over j < r of q[t,h,channels[g][j]] * label_k[row(i)][j] (unscaled fp32), and
+ * the k largest s~ are kept (ties to the lower index, ascending, -1 padded).  The cache
+ * supplies the page table, lengths and shapes; label_k is the tsd_label_cache_build output
+ * for the same channels.  Workspace: tsd_topk_workspace_size bytes, zeroed as described
+ * above.  Errors: as tsd_topk_select, plus UNSUPPORTED for r not in {8, 16, 32}.
+ */
+tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k, const int32_t* channels,
+                                 int32_t r, const tsd_queries* queries, int32_t k_max, const int32_t* k_per_token,
+                                 int32_t* out_idx, int32_t* out_count, void* ws, size_t ws_bytes,
+                                 tsd_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,6 +28,7 @@ from typing import Optional, Tuple
 
 __all__ = [
     "KVCache", "Queries", "Workspace", "TsdError", "topk_select", "sparse_decode", "dense_decode",
+    "LabelIndex", "label_channels", "label_cache_build", "topk_select_label",
     "read_device_status", "library_path", "load_library", "DEV_BAD_INDEX", "DEV_UNSORTED",
     "DEV_BAD_PAGE", "DEV_BAD_SEQ",
 ]
@@ -86,6 +87,16 @@ EXPORTS = {
     "tsd_sparse_decode_static_ws": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
                                                    ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
                                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "tsd_label_cache_bytes": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.c_int32]),
+    "tsd_label_channels_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC)]),
+    "tsd_label_channels": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
+                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tsd_label_cache_build": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.c_void_p, ctypes.c_int32,
+                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "tsd_topk_select_label": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_int32, ctypes.POINTER(_QueriesC), ctypes.c_int32,
+                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_size_t, ctypes.c_void_p]),
 }
 
 _LIB = None
@@ -310,6 +321,81 @@ def topk_select(cache: KVCache, queries: Queries, k_max: int, k_per_token=None, 
                                None if k_per_token is None else k_per_token.data_ptr(),
                                out_idx.data_ptr(), out_count.data_ptr(), ws.data_ptr(), ws.numel(), sp),
            "tsd_topk_select")
+    return out_idx, out_count
+
+
+# ---------------------------------------------------------------------------
+# Label-channel approximate indexer (Double-Sparsity-style)
+# ---------------------------------------------------------------------------
+@dataclass
+class LabelIndex:
+    """Label channels int32 [Hkv, r] and the label cache (bf16, r values per K row)."""
+    channels: "object"
+    label_k: "object"
+    r: int
+
+
+def label_channels(cache: KVCache, queries: Queries, r: int = 16, out=None, stream=None):
+    """Offline choice of r label channels per kv head (int32 [Hkv, r], ascending)."""
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    queries = _on_device_queries(queries, dev, s)
+    cs, qs = cache.c_struct(), queries.c_struct()
+    if out is None:
+        out = torch.empty((cache.num_kv_heads, r), dtype=torch.int32, device=dev)
+    nbytes = lib.tsd_label_channels_workspace_size(ctypes.byref(cs), ctypes.byref(qs))
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_label_channels_workspace_size")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(lib.tsd_label_channels(ctypes.byref(cs), ctypes.byref(qs), int(r), out.data_ptr(), ws.data_ptr(),
+                                  ws.numel(), sp), "tsd_label_channels")
+    return out
+
+
+def label_cache_build(cache: KVCache, channels, status=None, stream=None) -> LabelIndex:
+    """The compact label cache for `channels` (int32 [Hkv, r] on the cache's device)."""
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    r = int(channels.shape[1])
+    cs = cache.c_struct()
+    nbytes = lib.tsd_label_cache_bytes(ctypes.byref(cs), r)
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_label_cache_bytes")
+    label = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
+    channels = channels.to(dev).to(torch.int32).contiguous()
+    _check(lib.tsd_label_cache_build(ctypes.byref(cs), channels.data_ptr(), r, label.data_ptr(),
+                                     None if status is None else status.data_ptr(), sp), "tsd_label_cache_build")
+    return LabelIndex(channels=channels, label_k=label, r=r)
+
+
+def topk_select_label(cache: KVCache, index: LabelIndex, queries: Queries, k_max: int, k_per_token=None,
+                      out_idx=None, out_count=None, workspace: Optional[Workspace] = None, stream=None):
+    """Approximate top-k over the label channels: int32 [T, Hq, k_max] ascending, -1 padded, and counts."""
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    queries = _on_device_queries(queries, dev, s)
+    k_per_token = _to_device(k_per_token, dev, s)
+    cs, qs = cache.c_struct(), queries.c_struct()
+    T, Hq = int(queries.q.shape[0]), int(queries.q.shape[1])
+    if out_idx is None:
+        out_idx = torch.empty((T, Hq, k_max), dtype=torch.int32, device=dev)
+    if out_count is None:
+        out_count = torch.empty((T, Hq), dtype=torch.int32, device=dev)
+    nbytes = lib.tsd_topk_workspace_size(ctypes.byref(cs), ctypes.byref(qs), int(k_max))
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_topk_workspace_size")
+    ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, queries), sp)
+    _check(lib.tsd_topk_select_label(ctypes.byref(cs), index.label_k.data_ptr(), index.channels.data_ptr(),
+                                     int(index.r), ctypes.byref(qs), int(k_max),
+                                     None if k_per_token is None else k_per_token.data_ptr(),
+                                     out_idx.data_ptr(), out_count.data_ptr(), ws.data_ptr(), ws.numel(), sp),
+           "tsd_topk_select_label")
     return out_idx, out_count
 
 

@@ -20,6 +20,13 @@ cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaSt
 cudaError_t launch_dense_decode(const DecodeArgs& a, const KvMaps& maps, int batch, int hkv, cudaStream_t stream);
 cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int batch, int hkv, int num_lists,
                         cudaStream_t stream);
+size_t label_channels_ws_bytes(int64_t batch, int64_t hkv);
+cudaError_t launch_label_channels(const KvView& kv, const QView& qv, int r, int32_t* channels, void* ws,
+                                  cudaStream_t stream);
+cudaError_t launch_label_build(const KvView& kv, const int32_t* channels, int r, int64_t rows, uint16_t* label,
+                               uint32_t* status, cudaStream_t stream);
+cudaError_t launch_label_topk(const TopkArgs& a, const uint16_t* label, const int32_t* channels, int r, int nwin,
+                              int batch, int hkv, int num_lists, cudaStream_t stream);
 }  // namespace tsd
 
 using namespace tsd;
@@ -343,6 +350,106 @@ tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* querie
   st = make_kv_maps(cache, &maps);
   if (st != TSD_OK) return st;
   return cuda_status(launch_dense_decode(a, maps, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------------------
+// Label-channel approximate indexer
+// ---------------------------------------------------------------------------
+static bool label_r_ok(int32_t r) { return r == 8 || r == 16 || r == 32; }
+
+// The cache descriptor alone, validated through check_inputs with a stand-in query set.
+static tsd_status check_cache_only(const tsd_kv_cache* cache, KvView* kv, Shapes* sh) {
+  if (cache == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  tsd_queries q;
+  memset(&q, 0, sizeof(q));
+  q.q = cache->k;
+  q.q_dtype = TSD_BF16;
+  q.num_q_heads = cache->num_kv_heads;
+  q.num_tokens = cache->batch;
+  q.sm_scale = 1.f;
+  QView qv;
+  return check_inputs(cache, &q, kv, &qv, sh);
+}
+
+static int64_t cache_rows(const tsd_kv_cache* c) {
+  return c->layout == TSD_LAYOUT_CONTIGUOUS ? (int64_t)c->batch * c->num_kv_heads * c->max_seq_len
+                                            : c->num_pages * c->num_kv_heads * c->page_size;
+}
+
+size_t tsd_label_cache_bytes(const tsd_kv_cache* cache, int32_t r) {
+  KvView kv; Shapes sh;
+  if (!label_r_ok(r)) return 0;
+  tsd_kv_cache c;
+  if (cache == nullptr) return 0;
+  c = *cache;
+  static const uint16_t dummy[8] = {0};
+  if (c.k == nullptr) c.k = dummy;
+  if (c.v == nullptr) c.v = dummy;
+  if (c.seq_lens == nullptr) c.seq_lens = reinterpret_cast<const int32_t*>(dummy);
+  if (c.layout == TSD_LAYOUT_PAGED && c.page_table == nullptr) c.page_table = reinterpret_cast<const int32_t*>(dummy);
+  if (check_cache_only(&c, &kv, &sh) != TSD_OK) return 0;
+  return (size_t)cache_rows(&c) * r * sizeof(uint16_t);
+}
+
+size_t tsd_label_channels_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries) {
+  Shapes sh;
+  if (sizes_for(cache, queries, &sh) != TSD_OK) return 0;
+  return label_channels_ws_bytes(sh.batch, sh.hkv);
+}
+
+tsd_status tsd_label_channels(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t r, int32_t* channels,
+                              void* ws, size_t ws_bytes, tsd_stream_t stream) {
+  KvView kv; QView qv; Shapes sh;
+  tsd_status st = check_inputs(cache, queries, &kv, &qv, &sh);
+  if (st != TSD_OK) return st;
+  if (!label_r_ok(r) || channels == nullptr || ws == nullptr || ((uintptr_t)ws & 255) != 0)
+    return TSD_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < label_channels_ws_bytes(sh.batch, sh.hkv)) return TSD_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(launch_label_channels(kv, qv, r, channels, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tsd_status tsd_label_cache_build(const tsd_kv_cache* cache, const int32_t* channels, int32_t r, void* label_k,
+                                 uint32_t* status, tsd_stream_t stream) {
+  KvView kv; Shapes sh;
+  tsd_status st = check_cache_only(cache, &kv, &sh);
+  if (st != TSD_OK) return st;
+  if (!label_r_ok(r)) return TSD_ERR_UNSUPPORTED;
+  if (channels == nullptr || label_k == nullptr || ((uintptr_t)label_k & 15) != 0) return TSD_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_label_build(kv, channels, r, cache_rows(cache), static_cast<uint16_t*>(label_k), status,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k, const int32_t* channels, int32_t r,
+                                 const tsd_queries* queries, int32_t k_max, const int32_t* k_per_token,
+                                 int32_t* out_idx, int32_t* out_count, void* ws, size_t ws_bytes,
+                                 tsd_stream_t stream) {
+  KvView kv; QView qv; Shapes sh;
+  tsd_status st = check_inputs(cache, queries, &kv, &qv, &sh);
+  if (st != TSD_OK) return st;
+  if (!label_r_ok(r)) return TSD_ERR_UNSUPPORTED;
+  if (k_max < 1 || out_idx == nullptr || ws == nullptr || label_k == nullptr || channels == nullptr)
+    return TSD_ERR_INVALID_ARGUMENT;
+  if (((uintptr_t)ws & 255) != 0 || ((uintptr_t)label_k & 15) != 0) return TSD_ERR_INVALID_ARGUMENT;
+  const TopkLayout lay = topk_layout(sh);
+  if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
+  TopkArgs a;
+  memset(&a, 0, sizeof(a));
+  a.kv = kv;
+  a.qv = qv;
+  a.k_max = k_max;
+  a.k_per_token = k_per_token;
+  a.out_idx = out_idx;
+  a.out_count = out_count;
+  a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
+  a.score_stride = lay.score_stride;
+  const DensePlan p = plan_dense(sh);
+  a.lists_per_cta = p.lists_per_cta;
+  a.list_groups = p.list_groups;
+  a.window = p.window;
+  a.status = static_cast<uint32_t*>(ws);
+  return cuda_status(launch_label_topk(a, static_cast<const uint16_t*>(label_k), channels, r, p.nsplit,
+                                       (int)sh.batch, (int)sh.hkv, (int)(sh.tokens * sh.hq),
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tsd_status tsd_read_device_status(void* ws, tsd_stream_t stream, uint32_t* flags) {

@@ -1,0 +1,245 @@
+// Label-channel approximate indexer (Double-Sparsity-style) for sm_100a.
+//
+// Operation ("Inference Time Context Sparsity: Illusion or Opportunity?", gist.science
+// summary, section 3.C, indexing overhead): the pages price the indexer in front of sparse
+// decode with Double Sparsity -- every token is scored with only a few "label" channels of
+// its key, kept in a compact cache, and the top k of those approximate scores are kept.
+// The channel count and choice are not on the pages; here r channels per kv head with the
+// largest total |q_d K_{i,d}| over the calibration pairs (ties to the lower channel), and
+// the top-k of s~_i = sum over the label channels of q_d K_{i,d}.
+//
+// Kernels:
+//  * label_ksum_kernel    -- per (sequence, kv head, token split): sums of |K[., d]| (fp32
+//                            per thread, a fixed reduction order: deterministic).
+//  * label_choose_kernel  -- per kv head: importance_d = sum_b (sum_{t in b, h in g} |q_{t,h,d}|)
+//                            x (sum_i |K_{b,g,i,d}|) in fp64, then the r largest, ascending.
+//  * label_build_kernel   -- gathers the label channels of every cache row into the compact
+//                            label cache (same row numbering as K, r bf16 per row).
+//  * label_score_kernel<R> -- per (sequence, kv head, list group, token window): reads the
+//                            2R-byte label rows once for every list of the GQA group and writes
+//                            fp32 approximate scores; the exact select kernel then picks top-k.
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "tsd_args.h"
+#include "tsd_common.cuh"
+
+namespace tsd {
+
+constexpr int kLblSplits = 16;       // token splits per (sequence, kv head) for the |K| sums
+constexpr int kLblThreads = 256;
+
+// ---------------------------------------------------------------------------
+// Channel choice (offline calibration)
+// ---------------------------------------------------------------------------
+// partial[((b * hkv + g) * kLblSplits + s) * 128 + d] = sum over this split's tokens of |K|.
+__global__ void __launch_bounds__(kLblThreads) label_ksum_kernel(KvView kv, float* partial, uint32_t* status) {
+  __shared__ float red[kLblThreads / 16][kHeadDim];
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int l = threadIdx.x & 15, rgrp = threadIdx.x >> 4;   // 16 row groups x 16 lanes of 8 dims
+  int len = __ldg(kv.seq_lens + b);
+  if (len < 0 || len > kv.max_seq_len) {
+    if (threadIdx.x == 0 && s == 0 && g == 0) flag_status(status, TSD_DEV_BAD_SEQ);
+    len = 0;
+  }
+  const int per = (len + kLblSplits - 1) / kLblSplits;
+  const int i0 = s * per, i1 = min(len, i0 + per);
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int i = i0 + rgrp; i < i1; i += kLblThreads / 16) {
+    const uint32_t row = kv_row(kv, b, g, i);
+    if (row == kInvalidRow) {
+      if (l == 0) flag_status(status, TSD_DEV_BAD_PAGE);
+      continue;
+    }
+    float f[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(kv.k + (int64_t)row * kHeadDim) + l), f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += fabsf(f[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[rgrp][8 * l + j] = acc[j];
+  __syncthreads();
+  if (threadIdx.x < kHeadDim) {
+    float t = 0.f;
+    for (int r = 0; r < kLblThreads / 16; ++r) t += red[r][threadIdx.x];
+    partial[(((int64_t)b * kv.hkv + g) * kLblSplits + s) * kHeadDim + threadIdx.x] = t;
+  }
+}
+
+// One CTA of 128 threads (thread d = channel d) per kv head g.
+__global__ void __launch_bounds__(kHeadDim) label_choose_kernel(KvView kv, QView qv, const float* partial, int r,
+                                                                int32_t* channels) {
+  __shared__ double imp[kHeadDim];
+  __shared__ int warp_sel[kHeadDim / 32];
+  const int g = blockIdx.x, d = threadIdx.x;
+  const int G = qv.hq / kv.hkv;
+  double total = 0.0;
+  for (int b = 0; b < kv.batch; ++b) {
+    int t0 = b, t1 = b + 1;
+    if (qv.q_indptr != nullptr) {
+      t0 = __ldg(qv.q_indptr + b);
+      t1 = __ldg(qv.q_indptr + b + 1);
+    }
+    t0 = max(0, t0);
+    t1 = min(t1, qv.num_tokens);
+    double qs = 0.0;
+    for (int t = t0; t < t1; ++t)
+      for (int h = g * G; h < (g + 1) * G; ++h) {
+        const int64_t e = ((int64_t)t * qv.hq + h) * kHeadDim + d;
+        const float x = qv.q_f32 ? __ldg(reinterpret_cast<const float*>(qv.q) + e)
+                                 : __uint_as_float((uint32_t)__ldg(reinterpret_cast<const uint16_t*>(qv.q) + e) << 16);
+        qs += fabs((double)x);
+      }
+    double ks = 0.0;
+    for (int s = 0; s < kLblSplits; ++s) ks += (double)partial[(((int64_t)b * kv.hkv + g) * kLblSplits + s) * kHeadDim + d];
+    total += qs * ks;
+  }
+  imp[d] = total;
+  __syncthreads();
+  int rank = 0;   // channels ahead of d: larger importance, or equal with a lower index
+  for (int e = 0; e < kHeadDim; ++e) rank += (imp[e] > total) || (imp[e] == total && e < d);
+  const bool sel = rank < r;
+  const unsigned ball = __ballot_sync(0xFFFFFFFFu, sel);
+  if ((d & 31) == 0) warp_sel[d >> 5] = __popc(ball);
+  __syncthreads();
+  int pos = __popc(ball & ((1u << (d & 31)) - 1u));
+  for (int w = 0; w < (d >> 5); ++w) pos += warp_sel[w];
+  if (sel) channels[(int64_t)g * r + pos] = d;
+}
+
+// ---------------------------------------------------------------------------
+// Label cache: out[row * r + j] = K[row * 128 + channels[g(row) * r + j]]
+// ---------------------------------------------------------------------------
+__global__ void label_build_kernel(KvView kv, const int32_t* channels, int r, int64_t rows, uint16_t* label,
+                                   uint32_t* status) {
+  const int64_t n = rows * r;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = e / r;
+    const int j = (int)(e - row * r);
+    const int g = kv.page_table != nullptr ? (int)((row >> kv.page_shift) % kv.hkv)
+                                           : (int)((row / kv.max_seq_len) % kv.hkv);
+    int c = __ldg(channels + (int64_t)g * r + j);
+    if (c < 0 || c >= kHeadDim) {
+      if (status != nullptr) flag_status(status, TSD_DEV_BAD_INDEX);
+      c = 0;
+    }
+    label[e] = __ldg(kv.k + row * kHeadDim + c);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Approximate scores
+// ---------------------------------------------------------------------------
+// One CTA per (window, kv head x list group, sequence); each thread scores tokens
+// tok0 + threadIdx.x, + 256, ... against up to 16 lists whose label queries sit in shared
+// memory.  Unscaled fp32 dots; bf16 x bf16 products are exact, only the R-term sum rounds.
+template <int R>
+__global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, const uint16_t* label,
+                                                                  const int32_t* channels) {
+  __shared__ float qs[16][R];
+  __shared__ int kvl[16];
+  __shared__ int64_t srow[16];
+  const int win = blockIdx.x;
+  const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
+  const int b = blockIdx.z;
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, win == 0 && g == 0 && lg == 0 && threadIdx.x == 0);
+  const int G = a.qv.hq / a.kv.hkv;
+  int nlists = si.n * G - lg * a.lists_per_cta;
+  if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
+  if (nlists <= 0) return;
+  const int tok0 = win * a.window;
+  const int tok_end = min(tok0 + a.window, si.len);
+  if (tok_end <= tok0) return;
+  for (int e = threadIdx.x; e < 16 * R; e += kLblThreads) {
+    const int m = e / R, j = e - (e / R) * R;
+    float v = 0.f;
+    if (m < nlists) {
+      const int mg = lg * a.lists_per_cta + m;
+      const int jt = mg / G;
+      const int h = g * G + (mg - jt * G);
+      int c = __ldg(channels + (int64_t)g * R + j);
+      if (c < 0 || c >= kHeadDim) {
+        flag_status(a.status, TSD_DEV_BAD_INDEX);
+        c = 0;
+      }
+      const int64_t qe = ((int64_t)(si.t0 + jt) * a.qv.hq + h) * kHeadDim + c;
+      v = a.qv.q_f32 ? __ldg(reinterpret_cast<const float*>(a.qv.q) + qe)
+                     : __uint_as_float((uint32_t)__ldg(reinterpret_cast<const uint16_t*>(a.qv.q) + qe) << 16);
+      if (j == 0) {
+        kvl[m] = min(kv_len_of(a.qv, si, jt), tok_end);
+        srow[m] = ((int64_t)(si.t0 + jt) * a.qv.hq + h) * a.score_stride;
+      }
+    }
+    qs[m][j] = v;
+  }
+  __syncthreads();
+  for (int tok = tok0 + threadIdx.x; tok < tok_end; tok += kLblThreads) {
+    const uint32_t row = kv_row(a.kv, b, g, tok);
+    if (row == kInvalidRow) {
+      flag_status(a.status, TSD_DEV_BAD_PAGE);
+      continue;
+    }
+    float kf[R];
+    const uint4* src = reinterpret_cast<const uint4*>(label + (int64_t)row * R);
+#pragma unroll
+    for (int c = 0; c < R / 8; ++c) unpack8(__ldg(src + c), kf + 8 * c);
+    for (int m = 0; m < nlists; ++m) {
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < R; j += 2) {
+        s0 = fmaf(qs[m][j], kf[j], s0);
+        s1 = fmaf(qs[m][j + 1], kf[j + 1], s1);
+      }
+      if (tok < kvl[m]) a.scores[srow[m] + tok] = s0 + s1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+size_t label_channels_ws_bytes(int64_t batch, int64_t hkv) {
+  return 256 + (size_t)batch * hkv * kLblSplits * kHeadDim * sizeof(float);
+}
+
+cudaError_t launch_label_channels(const KvView& kv, const QView& qv, int r, int32_t* channels, void* ws,
+                                  cudaStream_t stream) {
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);
+  label_ksum_kernel<<<dim3(kLblSplits, kv.hkv, kv.batch), kLblThreads, 0, stream>>>(kv, partial, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  label_choose_kernel<<<kv.hkv, kHeadDim, 0, stream>>>(kv, qv, partial, r, channels);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_label_build(const KvView& kv, const int32_t* channels, int r, int64_t rows, uint16_t* label,
+                               uint32_t* status, cudaStream_t stream) {
+  const int64_t n = rows * r;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  if (blocks < 1) blocks = 1;
+  label_build_kernel<<<(unsigned)blocks, 256, 0, stream>>>(kv, channels, r, rows, label, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_select_only(const TopkArgs& a, int num_lists, cudaStream_t stream);
+
+cudaError_t launch_label_topk(const TopkArgs& a, const uint16_t* label, const int32_t* channels, int r, int nwin,
+                              int batch, int hkv, int num_lists, cudaStream_t stream) {
+  dim3 grid(nwin, hkv * a.list_groups, batch);
+  switch (r) {
+    case 8: label_score_kernel<8><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
+    case 16: label_score_kernel<16><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
+    case 32: label_score_kernel<32><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
+    default: return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_topk_select_only(a, num_lists, stream);
+}
+
+}  // namespace tsd

@@ -366,4 +366,17 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
   return cudaGetLastError();
 }
 
+// The selection alone, over scores another kernel wrote into the workspace (the label indexer).
+cudaError_t launch_topk_select_only(const TopkArgs& a, int num_lists, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e =
+        cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SelectSmem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  topk_select_kernel<<<num_lists, kSelectThreads, sizeof(SelectSmem), stream>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace tsd
