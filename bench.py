@@ -408,6 +408,49 @@ def run_native(args):
     sparse_gbs, dense_gbs, topk_gbs = (gbs(job_sparse / world, sparse_ms), gbs(job_dense / world, dense_ms),
                                        gbs(job_topk / world, topk_ms))
 
+    # label-channel (Double-Sparsity-style) indexer: offline calibration once, then the
+    # decode-step cost of approximate top-k + sparse decode against dense decode over a
+    # sparsity sweep, next to the exact indexer's
+    def timed(fn, reps):
+        out = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            fn()
+            b_.record(stream)
+            torch.cuda.synchronize()
+            out.append(a_.elapsed_time(b_))
+        return float(np.mean(out[1:])) if len(out) > 1 else out[0]
+
+    r_label = 16
+    t_cal = timed(lambda: tsd.label_channels(cache, queries, r_label), 2)
+    channels = tsd.label_channels(cache, queries, r_label)
+    label_index = tsd.label_cache_build(cache, channels)
+    torch.cuda.synchronize()
+    curve = []
+    reps = max(4, args.steps // 4 + 1)
+    for x in (2, 5, 10, 20, 50, 100, 200):
+        kx = W.k_for_sparsity(cfg.max_seq_len, x)
+        ibuf = torch.empty((T, Hq, kx), dtype=torch.int32, device=dev)
+        cbuf = torch.empty((T, Hq), dtype=torch.int32, device=dev)
+        t_lab = timed(lambda: tsd.topk_select_label(cache, label_index, queries, kx, out_idx=ibuf, out_count=cbuf,
+                                                    workspace=ws), reps)
+        t_ex = timed(lambda: tsd.topk_select(cache, queries, kx, out_idx=ibuf, out_count=cbuf, workspace=ws), reps)
+        t_sp = timed(lambda: tsd.sparse_decode(cache, queries, ibuf, out_dtype=out_dtype, workspace=ws), reps)
+        t_lab, t_ex, t_sp = max_over_ranks([t_lab, t_ex, t_sp], dev)
+        curve.append({"sparsity": x, "k": kx, "label_topk_us": round(t_lab * 1e3, 2),
+                      "exact_topk_us": round(t_ex * 1e3, 2), "sparse_us": round(t_sp * 1e3, 2),
+                      "net_speedup_label": round(dense_ms / (t_lab + t_sp), 3),
+                      "net_speedup_exact": round(dense_ms / (t_ex + t_sp), 3)})
+    if tsd.read_device_status(ws) != 0:
+        raise RuntimeError("device status bits set in the label-indexer sweep")
+    label_line = {"r": r_label, "calibration_us": round(max_over_ranks([t_cal], dev)[0] * 1e3, 1),
+                  "label_cache_bytes": int(label_index.label_k.numel() * 2),
+                  "dense_us": round(dense_ms * 1e3, 3), "curve": curve,
+                  "what": "label top-k (r channels per kv head, exact top-k of the approximate scores) and "
+                          "exact top-k, each plus sparse decode, against dense decode on the same cache"}
+
     # end to end through the public API with pinned host buffers
     q_host = dw.q.cpu().pin_memory()
     idx_host = idx_buf.cpu().pin_memory()
@@ -489,6 +532,7 @@ def run_native(args):
         "e2e_with_indexer": {"value": round(e2e_idx_us, 3), "unit": UNIT, "h2d_bytes_per_step": q_bytes,
                              "d2h_bytes_per_step": o_bytes + T * Hq * 4,
                              "what": "host q in -> topk_select -> sparse_decode -> host out and lse"},
+        "label_indexer": label_line,
         "gpu_launches": 4 * args.steps,
         "clocks": cl,
     }
