@@ -7,7 +7,8 @@ oracle (lower token index first, "Oracle Top-K" in section 2 of the pages' summa
 result must equal the oracle's list exactly, not just within the rounding band.  With two
 distinct rows a tie group holds about half of a 32768-token list, more candidates than the
 selection gathers in one place, so the full three-round radix path runs; with five rows the
-candidate path runs.
+candidate path runs; with 200 rows the groups are small enough for the sampled-threshold
+path, and the k-th score still falls inside a group of about 160 equal scores.
 """
 
 import math
@@ -48,7 +49,7 @@ def _tied_cache(n_distinct: int, seed: int):
     return K, q
 
 
-@pytest.mark.parametrize("n_distinct", [2, 5])
+@pytest.mark.parametrize("n_distinct", [2, 5, 200])
 def test_topk_ties_go_to_lower_indices(n_distinct):
     import torch
     K, q = _tied_cache(n_distinct, seed=11 + n_distinct)
@@ -59,7 +60,7 @@ def test_topk_ties_go_to_lower_indices(n_distinct):
     cache = tsd.KVCache(kd, vd, lens, max_seq_len=N, page_table=None)
     queries = tsd.Queries(torch.from_numpy(q).to(torch.bfloat16).cuda(), sm_scale=1.0 / math.sqrt(D))
     G = HQ // HKV
-    for k in (1, 1000, 9000, 20000, 32768):
+    for k in (1, 100, 1000, 9000, 20000, 32768):
         idx, cnt = tsd.topk_select(cache, queries, k)
         torch.cuda.synchronize()
         idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()

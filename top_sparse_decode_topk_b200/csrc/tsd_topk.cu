@@ -28,7 +28,7 @@ namespace tsd {
 
 constexpr int kSelectThreads = 512;   // one CTA per (token, head)
 constexpr int kSelBins = 2048;
-constexpr int kCandMax = 8192;
+constexpr int kCandMax = 16384;
 constexpr int kSelPerThread = 16;                 // scores per thread per tile (4 x float4)
 
 
@@ -178,6 +178,135 @@ __device__ __forceinline__ void load16(const float* row, int i0, int L, float* f
   }
 }
 
+// Fast path for lists much longer than k: a threshold from a sample, then ONE pass over the
+// scores.  The r-th largest key lo of a 1024-score strided sample, with r the sample's expected
+// count above the k-th score plus 4 standard deviations, has at least k scores at or above it;
+// one ordered pass copies every (index, key) with key >= lo into shared memory in index order;
+// the exact radix select and the ordered output then run over those few thousand entries
+// only.  Returns false, having written nothing, when the sample says too many keys would be
+// kept or the pass kept more than fit or fewer than k: the caller then runs the full passes.
+constexpr int kFastMinL = 4096;
+constexpr int kFastSample = 1024;
+constexpr int kFastCap = kCandMax / 2;   // kept entries: keys in cand[0, cap), indices in cand[cap, 2 cap)
+
+__device__ bool select_fast(SelectSmem& S, const float* row, int L, int k, int32_t* out, int k_max) {
+  uint32_t* ckey = S.cand;
+  uint32_t* cidx = S.cand + kFastCap;
+  // ---- the r_lo-th largest of a strided sample of keys ----
+  const float mean = (float)kFastSample * (float)k / (float)L;
+  const int r_lo = (int)ceilf(mean + 4.f * sqrtf(mean) + 8.f);
+  if (r_lo >= kFastSample || (int64_t)r_lo * L > (int64_t)kFastCap * kFastSample * 3 / 4) return false;
+  for (int s = threadIdx.x; s < kFastSample; s += kSelectThreads)
+    ckey[s] = score_key(__ldcg(row + (int)(((int64_t)s * L) / kFastSample)));
+  uint32_t prefix = 0u;
+  int need = r_lo, shift = 32;
+  while (shift > 0) {
+    const int nb = shift >= 11 ? 11 : shift;
+    shift -= nb;
+    const bool first = shift + nb == 32;
+    for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[i] = 0u;
+    __syncthreads();
+    for (int c = threadIdx.x; c < kFastSample; c += kSelectThreads) {
+      const uint32_t key = ckey[c];
+      if (first || (key >> (shift + nb)) == prefix) atomicAdd(&S.hist[(key >> shift) & ((1u << nb) - 1u)], 1u);
+    }
+    __syncthreads();
+    select_bin(S, 1 << nb, need);
+    prefix = (prefix << nb) | (uint32_t)S.found_bin;
+    need -= S.found_above;
+    __syncthreads();
+  }
+  const uint32_t lo_key = prefix;
+
+  // ---- one ordered pass: every key >= lo, in index order ----
+  const int tile_elems = kSelectThreads * kSelPerThread;
+  int kept = 0;
+  for (int base = 0; base < L; base += tile_elems) {
+    const int i0 = base + threadIdx.x * kSelPerThread;
+    float f[kSelPerThread];
+    load16(row, i0, L, f);
+    uint32_t keys[kSelPerThread];
+    int n = 0;
+#pragma unroll
+    for (int j = 0; j < kSelPerThread; ++j) {
+      keys[j] = score_key(f[j]);
+      n += (i0 + j < L && keys[j] >= lo_key);
+    }
+    int tot;
+    int pos = kept + block_exclusive_scan<kSelectThreads>(n, S.scan_tmp, &tot);
+#pragma unroll
+    for (int j = 0; j < kSelPerThread; ++j)
+      if (i0 + j < L && keys[j] >= lo_key) {
+        if (pos < kFastCap) {
+          ckey[pos] = keys[j];
+          cidx[pos] = (uint32_t)(i0 + j);
+        }
+        ++pos;
+      }
+    kept += tot;
+  }
+  __syncthreads();
+  if (kept > kFastCap || kept < k) return false;
+
+  // ---- exact k-th key among the kept entries ----
+  prefix = 0u;
+  need = k;
+  shift = 32;
+  while (shift > 0) {
+    const int nb = shift >= 11 ? 11 : shift;
+    shift -= nb;
+    const bool first = shift + nb == 32;
+    for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[i] = 0u;
+    __syncthreads();
+    for (int c = threadIdx.x; c < kept; c += kSelectThreads) {
+      const uint32_t key = ckey[c];
+      if (first || (key >> (shift + nb)) == prefix) atomicAdd(&S.hist[(key >> shift) & ((1u << nb) - 1u)], 1u);
+    }
+    __syncthreads();
+    select_bin(S, 1 << nb, need);
+    prefix = (prefix << nb) | (uint32_t)S.found_bin;
+    need -= S.found_above;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+  const int need_eq = need;
+
+  // ---- ordered output over the kept entries ----
+  constexpr int kPer = (kFastCap + kSelectThreads - 1) / kSelectThreads;
+  const int c0 = threadIdx.x * kPer;
+  int neq = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) neq += (c0 + j < kept && ckey[c0 + j] == T);
+  int eq_total;
+  int eq_run = block_exclusive_scan<kSelectThreads>(neq, S.scan_tmp, &eq_total);
+  int nsel = 0;
+  uint32_t selmask = 0u;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    if (c0 + j >= kept) break;
+    const uint32_t key = ckey[c0 + j];
+    bool sel = key > T;
+    if (key == T) {
+      sel = eq_run < need_eq;
+      ++eq_run;
+    }
+    if (sel) {
+      selmask |= 1u << j;
+      ++nsel;
+    }
+  }
+  int sel_total;
+  int pos = block_exclusive_scan<kSelectThreads>(nsel, S.scan_tmp, &sel_total);
+#pragma unroll
+  for (int j = 0; j < kPer; ++j)
+    if (selmask & (1u << j)) {
+      if (pos < k) out[pos] = (int32_t)cidx[c0 + j];
+      ++pos;
+    }
+  for (int i = k + threadIdx.x; i < k_max; i += kSelectThreads) out[i] = -1;
+  return true;
+}
+
 __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
@@ -208,11 +337,12 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
   int32_t* out = a.out_idx + (int64_t)th * a.k_max;
   if (a.out_count != nullptr && threadIdx.x == 0) a.out_count[th] = k;
 
-  if (k == L) {   // every visible token is kept (covers k == 0 with L == 0)
-    for (int i = threadIdx.x; i < a.k_max; i += kSelectThreads) out[i] = i < L ? i : -1;
+  if (k == L || k == 0) {   // every visible token is kept, or none
+    for (int i = threadIdx.x; i < a.k_max; i += kSelectThreads) out[i] = i < k ? i : -1;
     return;
   }
   const float* row = a.scores + (int64_t)th * a.score_stride;
+  if (L >= kFastMinL && select_fast(S, row, L, k, out, a.k_max)) return;
   const int tile_elems = kSelectThreads * kSelPerThread;
 
   // ---- pass 1: histogram of the top 11 key bits ----
