@@ -280,6 +280,15 @@ def time_cpu_oracle(w, k, budget_s=10.0):
 # ---------------------------------------------------------------------------
 # Native arm
 # ---------------------------------------------------------------------------
+def bench_k(cfg):
+    """k of the bench line: the configuration's k nearest the 50x sparsity the metric names
+    (None: the configuration's own per-token rule, ceil(frac * kv_len))."""
+    if not cfg.ks:
+        return None
+    target = cfg.max_seq_len / 50.0
+    return min(cfg.ks, key=lambda k: abs(k - target))
+
+
 def rank_seed(rank: int) -> int:
     """Seed of a rank's workload: every rank decodes its own batch of sequences (weak scaling)."""
     return rank
@@ -331,7 +340,7 @@ def run_native(args):
     tsd.load_library()
 
     cfg = W.CONFIGS[args.config]
-    k = cfg.ks[0] if cfg.ks else None
+    k = bench_k(cfg)
     w = W.make_workload(cfg, seed=rank_seed(rank))
     dw = W.to_device(w, dev)
     contiguous = cfg.layout == "contiguous"
@@ -560,7 +569,7 @@ def run_reference(args):
     except Exception:
         pass
     cfg = W.CONFIGS[args.config]
-    k = cfg.ks[0] if cfg.ks else None
+    k = bench_k(cfg)
     w = W.make_workload(cfg, seed=0)
     G = cfg.group
     scale = 1.0 / math.sqrt(128)
