@@ -460,6 +460,46 @@ def run_native(args):
                   "what": "label top-k (r channels per kv head, exact top-k of the approximate scores) and "
                           "exact top-k, each plus sparse decode, against dense decode on the same cache"}
 
+    # the decode step on the device as one CUDA graph: indexer (exact, or label channels) then
+    # sparse decode on the same workspace, replayed with L2 flushed before each replay; and the
+    # sparse leg alone as a graph (what its launch costs outside a graph)
+    out_g = torch.empty((T, Hq, 128), dtype=out_dtype, device=dev)
+    lse_g = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    kpt_g = kpt_dev
+
+    def step_exact():
+        tsd.topk_select(cache, queries, k_max, k_per_token=kpt_g, out_idx=idx_buf, out_count=cnt_buf, workspace=ws)
+        tsd.sparse_decode(cache, queries, idx_buf, out=out_g, lse=lse_g, workspace=ws)
+
+    def step_label():
+        tsd.topk_select_label(cache, label_index, queries, k_max, k_per_token=kpt_g, out_idx=idx_buf,
+                              out_count=cnt_buf, workspace=ws)
+        tsd.sparse_decode(cache, queries, idx_buf, out=out_g, lse=lse_g, workspace=ws)
+
+    def sparse_only():
+        tsd.sparse_decode(cache, queries, idx_buf, out=out_g, lse=lse_g, workspace=ws)
+
+    graph_us = {}
+    for name, fn in (("sparse_decode", sparse_only), ("step_exact_indexer", step_exact),
+                     ("step_label_indexer", step_label)):
+        fn()   # warm: buffers exist, launch attributes set
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        graph_us[name] = timed(g.replay, reps + 1)
+        del g
+    torch.cuda.synchronize()
+    if tsd.read_device_status(ws) != 0:
+        raise RuntimeError("device status bits set in the graph-captured steps")
+    gx = max_over_ranks([graph_us["sparse_decode"], graph_us["step_exact_indexer"], graph_us["step_label_indexer"]],
+                        dev)
+    graph_line = {"sparse_decode_us": round(gx[0] * 1e3, 2), "step_exact_indexer_us": round(gx[1] * 1e3, 2),
+                  "step_label_indexer_us": round(gx[2] * 1e3, 2),
+                  "net_speedup_exact": round(dense_ms / gx[1], 3), "net_speedup_label": round(dense_ms / gx[2], 3),
+                  "what": "one CUDA graph per decode step (indexer + sparse decode, k of this line), L2 flushed "
+                          "before each replay; dense decode by events as in legs_us"}
+
     # end to end through the public API with pinned host buffers
     q_host = dw.q.cpu().pin_memory()
     idx_host = idx_buf.cpu().pin_memory()
@@ -542,6 +582,7 @@ def run_native(args):
                              "d2h_bytes_per_step": o_bytes + T * Hq * 4,
                              "what": "host q in -> topk_select -> sparse_decode -> host out and lse"},
         "label_indexer": label_line,
+        "graph_step": graph_line,
         "gpu_launches": 4 * args.steps,
         "clocks": cl,
     }
