@@ -162,7 +162,9 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
                              const int32_t* idx, int32_t k_max, void* out, int32_t out_dtype,
                              float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream);
 
-/* Host: bytes of workspace tsd_dense_decode needs for these shapes (0 on invalid input). */
+/* Host: bytes of workspace tsd_dense_decode needs for these shapes on the current device
+ * (0 on invalid input).  As for sparse decode, the split into windows depends on the device's
+ * SM count (148 assumed when no device can be queried). */
 size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries);
 
 /*

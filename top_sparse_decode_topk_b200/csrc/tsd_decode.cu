@@ -315,7 +315,7 @@ __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id
   if (l == 0 && a.lse != nullptr) a.lse[list_id] = L > 0.f ? (mx + log2f(L)) * kLn2 : -CUDART_INF_F;
 }
 
-__global__ void __launch_bounds__(kSpThreads, 3) sparse_decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel(DecodeArgs a) {
   // task states of the CTA's 16 half-warps, combined per list before anything leaves the CTA
   __shared__ float2 s_ml[16];
   __shared__ __align__(16) float s_acc[16][kHeadDim];
@@ -472,7 +472,7 @@ static_assert(kDnStages * kDnStageBytes >= 16 * kDnConsumers * kCombFloats * 4, 
 static_assert(sizeof(DenseSmem) + 1024 <= 75 * 1024, "three dense CTAs per SM");
 
 template <bool QF32>
-__global__ void __launch_bounds__(kDnThreads, 3) dense_decode_kernel(DecodeArgs a, const __grid_constant__ KvMaps maps) {
+__global__ void __launch_bounds__(kDnThreads, kDnCtasPerSm) dense_decode_kernel(DecodeArgs a, const __grid_constant__ KvMaps maps) {
   extern __shared__ __align__(1024) unsigned char smem_dn[];
   DenseSmem& S = *reinterpret_cast<DenseSmem*>(smem_dn);
   const int split = blockIdx.x;

@@ -83,8 +83,10 @@ inline SparsePlan plan_sparse(const Shapes& s, int k_max, int num_sms) {
   return p;
 }
 
-// Dense decode: up to 16 lists per CTA (the mma M dimension) and a window of W tokens (a
-// multiple of the 64-token tile), sized for about four waves of 2 CTAs per SM.
+// Dense decode and top-k scoring: up to 16 lists per CTA (the mma M dimension) and a window
+// of W tokens (a multiple of the 64-token tile).  Every CTA streams the same number of tiles,
+// so the grid is sized to whole waves: `slots` CTAs (resident CTAs per SM x SMs x waves), cut
+// into as many windows per (sequence, kv head, list group) as fit.
 struct DensePlan {
   int lists_per_cta;
   int list_groups;
@@ -93,15 +95,17 @@ struct DensePlan {
 };
 
 constexpr int kDenseMaxLists = 16;
-constexpr int kDenseTargetCtas = 4 * 296;
+constexpr int kDnCtasPerSm = 3;    // resident dense-decode CTAs per SM (its launch bounds)
+constexpr int kScCtasPerSm = 5;    // resident top-k scoring CTAs per SM (its launch bounds)
+constexpr int kStreamWaves = 2;
 
-inline DensePlan plan_dense(const Shapes& s) {
+inline DensePlan plan_dense(const Shapes& s, int64_t slots) {
   DensePlan p;
   const int64_t m = s.group * s.max_tokens;
   p.lists_per_cta = (int)(m < kDenseMaxLists ? m : kDenseMaxLists);
   p.list_groups = (int)((m + p.lists_per_cta - 1) / p.lists_per_cta);
   const int64_t units = s.batch * s.hkv * p.list_groups;
-  int64_t ns = (kDenseTargetCtas + units - 1) / units;
+  int64_t ns = slots / units;
   const int64_t max_ns = (s.max_seq_len + 63) / 64;
   if (ns > max_ns) ns = max_ns;
   if (ns > kMaxSplits) ns = kMaxSplits;

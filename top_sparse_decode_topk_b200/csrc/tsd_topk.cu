@@ -36,28 +36,37 @@ constexpr int kSelPerThread = 16;                 // scores per thread per tile 
 // Scoring on tensor cores
 // ---------------------------------------------------------------------------
 // One CTA per (sequence b, kv head g, list group lg, window of W tokens).  A producer warp
-// streams 64-token K tiles through a 4-stage ring (TMA, tsd_kvtile.cuh); each of the 4
+// streams 64-token K tiles through a 2-stage ring (TMA, tsd_kvtile.cuh); each of the 4
 // consumer warps scores 16 tokens of every tile against the CTA's 16 query rows with
 // mma.m16n8k16 (bf16 inputs, fp32 accumulation; fp32 queries as bf16 hi + lo) and writes
-// the unscaled fp32 dots of tokens below each list's kv_len.
-constexpr int kScStages = 4;
+// the unscaled fp32 dots of tokens below each list's kv_len.  The streaming rate grows with
+// resident CTAs rather than ring depth, so the ring is short and 5 CTAs share an SM (the
+// fp32 remainder tile is only allocated for fp32 queries).
 constexpr int kScConsumers = 4;
 constexpr int kScThreads = 32 * (kScConsumers + 1);
 
-struct ScoreSmem {
-  alignas(1024) unsigned char stage[kScStages][kTileBytesKV];
-  alignas(1024) unsigned char qhi[kQTileBytes];
-  alignas(1024) unsigned char qlo[kQTileBytes];
-  uint64_t full[kScStages];
-  uint64_t empty[kScStages];
-  uint32_t abort;
+// shared-memory layout (offsets from a 1024-aligned base): stages, q hi, [q lo], barriers
+template <bool QF32, int NST>
+struct ScLayout {
+  static constexpr int kStages = NST;
+  static constexpr size_t qhi = (size_t)NST * kTileBytesKV;
+  static constexpr size_t qlo = qhi + kQTileBytes;
+  static constexpr size_t bars = qhi + (QF32 ? 2 : 1) * kQTileBytes;
+  static constexpr size_t bytes = bars + 2 * NST * sizeof(uint64_t) + 16;
 };
-static_assert(sizeof(ScoreSmem) + 1024 <= 75 * 1024, "three scoring CTAs per SM");
+constexpr int kScStages = 2;
+static_assert(ScLayout<true, kScStages>::bytes + 1024 <= 228 * 1024 / kScCtasPerSm, "scoring CTAs per SM");
 
 template <bool QF32>
-__global__ void __launch_bounds__(kScThreads, 3) topk_score_kernel(TopkArgs a, const __grid_constant__ KvMaps maps) {
+__global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(TopkArgs a, const __grid_constant__ KvMaps maps) {
+  using Lay = ScLayout<QF32, kScStages>;
   extern __shared__ __align__(1024) unsigned char smem_sc[];
-  ScoreSmem& S = *reinterpret_cast<ScoreSmem*>(smem_sc);
+  unsigned char* stages = smem_sc;
+  unsigned char* qhi = smem_sc + Lay::qhi;
+  unsigned char* qlo = smem_sc + Lay::qlo;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_sc + Lay::bars);
+  uint64_t* empty = full + kScStages;
+  uint32_t* abort_flag = reinterpret_cast<uint32_t*>(empty + kScStages);
   const int win = blockIdx.x;
   const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
   const int b = blockIdx.z;
@@ -72,25 +81,24 @@ __global__ void __launch_bounds__(kScThreads, 3) topk_score_kernel(TopkArgs a, c
   if (tok_end <= tok0) return;
   const int ntiles = (tok_end - tok0 + kTileTok - 1) / kTileTok;
   const bool use_tma = a.kv.page_table == nullptr || a.kv.page_shift >= 3;
-  // the swizzled tiles need 1024-byte alignment; refuse to run rather than mis-address them
-  if (smem_u32(S.stage[0]) & 1023u) {
+  if (smem_u32(stages) & 1023u) {
     if (threadIdx.x == 0) flag_status(a.status, TSD_DEV_TIMEOUT);
     return;
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kScStages; ++s) {
-      mbar_init(&S.full[s], use_tma ? 1 : 32);
-      mbar_init(&S.empty[s], kScConsumers);
+      mbar_init(&full[s], use_tma ? 1 : 32);
+      mbar_init(&empty[s], kScConsumers);
     }
     mbar_fence_init();
-    S.abort = 0;
+    *abort_flag = 0;
   }
-  store_q_tile(a.qv, si, g, G, lg * a.lists_per_cta, nlists, S.qhi, QF32 ? S.qlo : nullptr, threadIdx.x, kScThreads);
+  store_q_tile(a.qv, si, g, G, lg * a.lists_per_cta, nlists, qhi, QF32 ? qlo : nullptr, threadIdx.x, kScThreads);
   __syncthreads();
 
   if (warp == kScConsumers) {
-    produce_tiles<kScStages, kTileBytesKV, false>(a.kv, maps, b, g, tok0, tok_end, ntiles, &S.stage[0][0], S.full,
-                                                  S.empty, &S.abort, use_tma, lane, a.status);
+    produce_tiles<kScStages, kTileBytesKV, false>(a.kv, maps, b, g, tok0, tok_end, ntiles, stages, full,
+                                                  empty, abort_flag, use_tma, lane, a.status);
     return;
   }
   // this lane's query rows m = lane/4 and lane/4 + 8: visible length and score row
@@ -109,9 +117,9 @@ __global__ void __launch_bounds__(kScThreads, 3) topk_score_kernel(TopkArgs a, c
     }
   }
   for (int tile = 0; tile < ntiles; ++tile) {
-    if (!consume_wait<kScStages>(S.full, &S.abort, tile, lane, a.status)) break;
+    if (!consume_wait<kScStages>(full, abort_flag, tile, lane, a.status)) break;
     float sc[2][4];
-    qk_tile<QF32>(S.qhi, S.qlo, S.stage[tile % kScStages], warp, lane, sc);
+    qk_tile<QF32>(qhi, qlo, stages + (size_t)(tile % kScStages) * kTileBytesKV, warp, lane, sc);
     const int tbase = tok0 + tile * kTileTok + 16 * warp + 2 * (lane & 3);
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr)
@@ -126,7 +134,7 @@ __global__ void __launch_bounds__(kScThreads, 3) topk_score_kernel(TopkArgs a, c
       }
     // the stores consume every fragment read from the stage: release it to the producer
     __syncwarp();
-    if (lane == 0) mbar_arrive(&S.empty[tile % kScStages]);
+    if (lane == 0) mbar_arrive(&empty[tile % kScStages]);
   }
 }
 
@@ -475,10 +483,10 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(ScoreSmem));
+                                         (int)ScLayout<false, kScStages>::bytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(topk_score_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)sizeof(ScoreSmem));
+                               (int)ScLayout<true, kScStages>::bytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SelectSmem));
     if (e != cudaSuccess) return e;
@@ -486,9 +494,9 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
   }
   dim3 g1(nwin, hkv * a.list_groups, batch);
   if (a.qv.q_f32) {
-    topk_score_kernel<true><<<g1, kScThreads, sizeof(ScoreSmem), stream>>>(a, maps);
+    topk_score_kernel<true><<<g1, kScThreads, ScLayout<true, kScStages>::bytes, stream>>>(a, maps);
   } else {
-    topk_score_kernel<false><<<g1, kScThreads, sizeof(ScoreSmem), stream>>>(a, maps);
+    topk_score_kernel<false><<<g1, kScThreads, ScLayout<false, kScStages>::bytes, stream>>>(a, maps);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
