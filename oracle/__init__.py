@@ -21,6 +21,9 @@ Opportunity?" (gist.science technical summary, section 2 "Oracle Top-K" and
   Double-Sparsity-style approximate indexer the pages use to price indexing (section
   3.C): a few "label" channels per kv head chosen by magnitude, approximate scores over
   them; its selection is ``exact_topk`` of those scores.
+* ``floyd_sample``, ``stochastic_select``, ``weighted_attention`` (``vattention.py``): the
+  vAttention-style stochastic selection the pages evaluate (section 2): exact top-k plus a
+  uniform sample of the other tokens, each sample weighted by |rest| / m.
 * ``topk_sets_agree``: the acceptance rule for a GPU top-k set (exact set
   equality except for tokens whose score is within a relative band of the
   k-th score).
@@ -38,3 +41,4 @@ from .attention import (  # noqa: F401
 )
 from .compare import topk_sets_agree, output_errors  # noqa: F401
 from .label import channel_importance, choose_channels, label_scores  # noqa: F401
+from .vattention import floyd_sample, stochastic_select, weighted_attention  # noqa: F401

@@ -29,6 +29,7 @@ namespace tsd {
 
 constexpr int kLblSplits = 16;       // token splits per (sequence, kv head) for the |K| sums
 constexpr int kLblThreads = 256;
+constexpr int kLblUnroll = 4;        // tokens per thread in flight in the scoring kernel
 
 // ---------------------------------------------------------------------------
 // Channel choice (offline calibration)
@@ -176,24 +177,39 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
     qs[m][j] = v;
   }
   __syncthreads();
-  for (int tok = tok0 + threadIdx.x; tok < tok_end; tok += kLblThreads) {
-    const uint32_t row = kv_row(a.kv, b, g, tok);
-    if (row == kInvalidRow) {
-      flag_status(a.status, TSD_DEV_BAD_PAGE);
-      continue;
+  // kLblUnroll tokens per thread per step: their page-table lookups, then their label rows,
+  // are all in flight together
+  for (int base = tok0; base < tok_end; base += kLblThreads * kLblUnroll) {
+    uint32_t row[kLblUnroll];
+#pragma unroll
+    for (int u = 0; u < kLblUnroll; ++u) {
+      const int tok = base + u * kLblThreads + threadIdx.x;
+      row[u] = tok < tok_end ? kv_row(a.kv, b, g, tok) : kInvalidRow;
+      if (tok < tok_end && row[u] == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
     }
-    float kf[R];
-    const uint4* src = reinterpret_cast<const uint4*>(label + (int64_t)row * R);
+    uint4 raw[kLblUnroll][R / 8];
 #pragma unroll
-    for (int c = 0; c < R / 8; ++c) unpack8(__ldg(src + c), kf + 8 * c);
-    for (int m = 0; m < nlists; ++m) {
-      float s0 = 0.f, s1 = 0.f;
+    for (int u = 0; u < kLblUnroll; ++u) {
+      const uint4* src = reinterpret_cast<const uint4*>(label + (int64_t)row[u] * R);
 #pragma unroll
-      for (int j = 0; j < R; j += 2) {
-        s0 = fmaf(qs[m][j], kf[j], s0);
-        s1 = fmaf(qs[m][j + 1], kf[j + 1], s1);
+      for (int c = 0; c < R / 8; ++c) raw[u][c] = row[u] != kInvalidRow ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kLblUnroll; ++u) {
+      const int tok = base + u * kLblThreads + threadIdx.x;
+      if (row[u] == kInvalidRow) continue;
+      float kf[R];
+#pragma unroll
+      for (int c = 0; c < R / 8; ++c) unpack8(raw[u][c], kf + 8 * c);
+      for (int m = 0; m < nlists; ++m) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < R; j += 2) {
+          s0 = fmaf(qs[m][j], kf[j], s0);
+          s1 = fmaf(qs[m][j + 1], kf[j + 1], s1);
+        }
+        if (tok < kvl[m]) a.scores[srow[m] + tok] = s0 + s1;
       }
-      if (tok < kvl[m]) a.scores[srow[m] + tok] = s0 + s1;
     }
   }
 }
