@@ -479,9 +479,20 @@ def run_native(args):
     def sparse_only():
         tsd.sparse_decode(cache, queries, idx_buf, out=out_g, lse=lse_g, workspace=ws)
 
+    # vAttention-style: exact top-k plus m uniform samples of the rest, weighted decode
+    m_sto = 64
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234 + rank)
+    u_sto = torch.randint(-2**31, 2**31 - 1, (T, Hq, m_sto), dtype=torch.int32, device=dev, generator=gen)
+
+    def step_stochastic():
+        tsd.topk_select(cache, queries, k_max, k_per_token=kpt_g, out_idx=idx_buf, out_count=cnt_buf, workspace=ws)
+        sidx, slw = tsd.stochastic_select(cache, queries, idx_buf, u_sto)
+        tsd.sparse_decode(cache, queries, sidx, logw=slw, out=out_g, lse=lse_g, workspace=ws)
+
     graph_us = {}
     for name, fn in (("sparse_decode", sparse_only), ("step_exact_indexer", step_exact),
-                     ("step_label_indexer", step_label)):
+                     ("step_label_indexer", step_label), ("step_stochastic", step_stochastic)):
         fn()   # warm: buffers exist, launch attributes set
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
@@ -492,13 +503,17 @@ def run_native(args):
     torch.cuda.synchronize()
     if tsd.read_device_status(ws) != 0:
         raise RuntimeError("device status bits set in the graph-captured steps")
-    gx = max_over_ranks([graph_us["sparse_decode"], graph_us["step_exact_indexer"], graph_us["step_label_indexer"]],
-                        dev)
+    gx = max_over_ranks([graph_us["sparse_decode"], graph_us["step_exact_indexer"], graph_us["step_label_indexer"],
+                         graph_us["step_stochastic"]], dev)
     graph_line = {"sparse_decode_us": round(gx[0] * 1e3, 2), "step_exact_indexer_us": round(gx[1] * 1e3, 2),
                   "step_label_indexer_us": round(gx[2] * 1e3, 2),
+                  "step_stochastic_us": round(gx[3] * 1e3, 2), "stochastic_samples": m_sto,
                   "net_speedup_exact": round(dense_ms / gx[1], 3), "net_speedup_label": round(dense_ms / gx[2], 3),
-                  "what": "one CUDA graph per decode step (indexer + sparse decode, k of this line), L2 flushed "
-                          "before each replay; dense decode by events as in legs_us"}
+                  "net_speedup_stochastic": round(dense_ms / gx[3], 3),
+                  "what": "one CUDA graph per decode step (indexer + sparse decode, k of this line; the "
+                          "stochastic step adds m uniform samples of the other tokens with Horvitz-Thompson "
+                          "weights and decodes with them), L2 flushed before each replay; dense decode by "
+                          "events as in legs_us"}
 
     # end to end through the public API with pinned host buffers
     q_host = dw.q.cpu().pin_memory()

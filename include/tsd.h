@@ -162,6 +162,36 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
                              const int32_t* idx, int32_t k_max, void* out, int32_t out_dtype,
                              float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream);
 
+/*
+ * Weighted sparse decode: as tsd_sparse_decode, with entry i of list (t, h) weighted by
+ * w = exp(logw[t][h][i]): out = sum_i w_i e^{z_i} V_i / sum_i w_i e^{z_i} and
+ * lse = ln sum_i w_i e^{z_i}, z_i = sm_scale q.K_i.  logw: device fp32 [T][Hq][k_max], read
+ * only where idx >= 0.  Used with tsd_stochastic_select (the estimator of vAttention-style
+ * sampling); same workspace as tsd_sparse_decode.  Errors: as tsd_sparse_decode, plus
+ * INVALID_ARGUMENT for a NULL logw.
+ */
+tsd_status tsd_sparse_decode_weighted(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
+                                      const float* logw, int32_t k_max, void* out, int32_t out_dtype, float* lse,
+                                      void* ws, size_t ws_bytes, tsd_stream_t stream);
+
+/*
+ * vAttention-style stochastic selection ("Inference Time Context Sparsity: Illusion or
+ * Opportunity?", gist.science summary, section 2: stochastic index selection with vAttention,
+ * against deterministic top-k).  The pages give no sampling scheme; per (t, h) this keeps the
+ * top-k list S given in topk_idx (ascending, -1 padded, as tsd_topk_select writes it) and adds
+ * m' = min(m, |R|) tokens of R = [0, kv_len) minus S drawn uniformly without replacement by
+ * Floyd's algorithm: step j = |R| - m' .. |R| - 1 keeps rank u[t][h][j - |R| + m'] mod (j + 1),
+ * or j when that rank is already kept; rank r of R is its r-th smallest token.
+ * u: device uint32 [T][Hq][m], random words supplied by the caller.  Output (device, width
+ * k_max + m per list): out_idx int32 -- S and the sample merged ascending, then -1; out_logw
+ * fp32 -- 0 for S, ln(|R| / m') for sampled entries (the Horvitz-Thompson weight).  A topk_idx
+ * list that is not ascending or reaches kv_len is flagged in *status (TSD_DEV_BAD_INDEX, if
+ * status is not NULL) and treated as empty.  Errors: INVALID_ARGUMENT, UNSUPPORTED (m > 1024), CUDA.
+ */
+tsd_status tsd_stochastic_select(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* topk_idx,
+                                 int32_t k_max, const uint32_t* u, int32_t m, int32_t* out_idx, float* out_logw,
+                                 uint32_t* status, tsd_stream_t stream);
+
 /* Host: bytes of workspace tsd_dense_decode needs for these shapes on the current device
  * (0 on invalid input).  As for sparse decode, the split into windows depends on the device's
  * SM count (148 assumed when no device can be queried). */

@@ -28,7 +28,7 @@ from typing import Optional, Tuple
 
 __all__ = [
     "KVCache", "Queries", "Workspace", "TsdError", "topk_select", "sparse_decode", "dense_decode",
-    "LabelIndex", "label_channels", "label_cache_build", "topk_select_label",
+    "LabelIndex", "label_channels", "label_cache_build", "topk_select_label", "stochastic_select",
     "read_device_status", "library_path", "load_library", "DEV_BAD_INDEX", "DEV_UNSORTED",
     "DEV_BAD_PAGE", "DEV_BAD_SEQ",
 ]
@@ -87,6 +87,13 @@ EXPORTS = {
     "tsd_sparse_decode_static_ws": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
                                                    ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
                                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "tsd_sparse_decode_weighted": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
+                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                                  ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                                  ctypes.c_void_p]),
+    "tsd_stochastic_select": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_void_p,
+                                             ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "tsd_label_cache_bytes": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.c_int32]),
     "tsd_label_channels_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC)]),
     "tsd_label_channels": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
@@ -434,11 +441,13 @@ def _finish(out, host_out, lse, host_lse, stream):
 
 
 def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=None, lse=True,
-                  workspace: Optional[Workspace] = None, stream=None):
+                  workspace: Optional[Workspace] = None, stream=None, logw=None):
     """Attention of each (token, head) over the rows of its index list.
 
     idx: int32 [T, Hq, k_max], each list non-decreasing then -1 padded (as
-    topk_select writes it).  Returns (out [T, Hq, 128], lse [T, Hq] or None).
+    topk_select writes it).  logw: optional fp32 [T, Hq, k_max] natural-log weight of
+    each entry (tsd_sparse_decode_weighted; as stochastic_select writes it).
+    Returns (out [T, Hq, 128], lse [T, Hq] or None).
     Host (CPU) inputs are copied in and a host `out`/`lse` is filled on return
     (asynchronously from/to pinned memory, ordered on `stream`).
     """
@@ -458,11 +467,47 @@ def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=Non
     if nbytes == 0:
         raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_sparse_decode_workspace_size")
     ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, queries), sp)
-    _check(lib.tsd_sparse_decode(ctypes.byref(cs), ctypes.byref(qs), idx.data_ptr(), k_max, out.data_ptr(),
-                                 TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32,
-                                 None if lse is None else lse.data_ptr(), ws.data_ptr(), ws.numel(), sp),
-           "tsd_sparse_decode")
+    odt = TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32
+    lp = None if lse is None else lse.data_ptr()
+    if logw is None:
+        _check(lib.tsd_sparse_decode(ctypes.byref(cs), ctypes.byref(qs), idx.data_ptr(), k_max, out.data_ptr(), odt,
+                                     lp, ws.data_ptr(), ws.numel(), sp), "tsd_sparse_decode")
+    else:
+        logw = _to_device(logw, dev, s)
+        if logw.dtype != torch.float32 or tuple(logw.shape) != tuple(idx.shape) or not logw.is_contiguous():
+            raise ValueError("logw must be a contiguous float32 tensor shaped like idx")
+        _check(lib.tsd_sparse_decode_weighted(ctypes.byref(cs), ctypes.byref(qs), idx.data_ptr(), logw.data_ptr(),
+                                              k_max, out.data_ptr(), odt, lp, ws.data_ptr(), ws.numel(), sp),
+               "tsd_sparse_decode_weighted")
     return _finish(out, host_out, lse, host_lse, s)
+
+
+def stochastic_select(cache: KVCache, queries: Queries, topk_idx, u, status=None, stream=None):
+    """vAttention-style selection: the top-k lists plus m uniform samples of the other tokens.
+
+    topk_idx: int32 [T, Hq, k_max] (as topk_select writes it); u: uint32-valued int32 or
+    int64 [T, Hq, m] random words.  Returns (idx int32 [T, Hq, k_max + m] ascending, -1
+    padded; logw fp32 of the same shape: 0 for top-k entries, ln(|rest| / m') for samples)."""
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    queries = _on_device_queries(queries, dev, s)
+    topk_idx = _to_device(topk_idx, dev, s).contiguous()
+    u = _to_device(u, dev, s)
+    if u.dtype != torch.int32:
+        u = (u.to(torch.int64) & 0xFFFFFFFF).to(torch.int64)
+        u = torch.where(u >= 2**31, u - 2**32, u).to(torch.int32)   # same 32-bit words
+    u = u.contiguous()
+    T, Hq, k_max = (int(x) for x in topk_idx.shape)
+    m = int(u.shape[2])
+    idx = torch.empty((T, Hq, k_max + m), dtype=torch.int32, device=dev)
+    logw = torch.empty((T, Hq, k_max + m), dtype=torch.float32, device=dev)
+    cs, qs = cache.c_struct(), queries.c_struct()
+    _check(lib.tsd_stochastic_select(ctypes.byref(cs), ctypes.byref(qs), topk_idx.data_ptr(), k_max, u.data_ptr(), m,
+                                     idx.data_ptr(), logw.data_ptr(), None if status is None else status.data_ptr(),
+                                     sp), "tsd_stochastic_select")
+    return idx, logw
 
 
 def dense_decode(cache: KVCache, queries: Queries, out=None, out_dtype=None, lse=True,

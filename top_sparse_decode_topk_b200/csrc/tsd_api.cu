@@ -25,6 +25,9 @@ cudaError_t launch_label_channels(const KvView& kv, const QView& qv, int r, int3
                                   cudaStream_t stream);
 cudaError_t launch_label_build(const KvView& kv, const int32_t* channels, int r, int64_t rows, uint16_t* label,
                                uint32_t* status, cudaStream_t stream);
+cudaError_t launch_stochastic_select(const KvView& kv, const QView& qv, const int32_t* top, int k_max,
+                                     const uint32_t* u, int m, int32_t* out_idx, float* out_logw, uint32_t* status,
+                                     cudaStream_t stream);
 cudaError_t launch_label_topk(const TopkArgs& a, const uint16_t* label, const int32_t* channels, int r, int nwin,
                               int batch, int hkv, int num_lists, cudaStream_t stream);
 }  // namespace tsd
@@ -290,8 +293,8 @@ static tsd_status decode_common(const tsd_kv_cache* cache, const tsd_queries* qu
   return TSD_OK;
 }
 
-tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
-                             int32_t k_max, void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+static tsd_status sparse_decode_impl(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
+                                     const float* logw, int32_t k_max, void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
                              tsd_stream_t stream) {
   KvView kv; QView qv; Shapes sh;
   tsd_status st = decode_common(cache, queries, out, out_dtype, lse, ws, ws_bytes, &kv, &qv, &sh);
@@ -306,6 +309,7 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
   a.kv = kv;
   a.qv = qv;
   a.idx = idx;
+  a.logw = logw;
   a.k_max = k_max;
   a.span = p.entries;
   a.nsplit = p.nsplit;
@@ -318,8 +322,33 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
   a.counters = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_counters);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.off_ml);
   a.part_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_acc);
-  a.sched = static_cast<uint32_t*>(ws) + 1;
   return cuda_status(launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
+                             int32_t k_max, void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                             tsd_stream_t stream) {
+  return sparse_decode_impl(cache, queries, idx, nullptr, k_max, out, out_dtype, lse, ws, ws_bytes, stream);
+}
+
+tsd_status tsd_sparse_decode_weighted(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
+                                      const float* logw, int32_t k_max, void* out, int32_t out_dtype, float* lse,
+                                      void* ws, size_t ws_bytes, tsd_stream_t stream) {
+  if (logw == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  return sparse_decode_impl(cache, queries, idx, logw, k_max, out, out_dtype, lse, ws, ws_bytes, stream);
+}
+
+tsd_status tsd_stochastic_select(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* topk_idx,
+                                 int32_t k_max, const uint32_t* u, int32_t m, int32_t* out_idx, float* out_logw,
+                                 uint32_t* status, tsd_stream_t stream) {
+  KvView kv; QView qv; Shapes sh;
+  tsd_status st = check_inputs(cache, queries, &kv, &qv, &sh);
+  if (st != TSD_OK) return st;
+  if (topk_idx == nullptr || out_idx == nullptr || out_logw == nullptr || k_max < 1 || m < 0) return TSD_ERR_INVALID_ARGUMENT;
+  if (m > 1024) return TSD_ERR_UNSUPPORTED;
+  if (m > 0 && u == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_stochastic_select(kv, qv, topk_idx, k_max, u, m, out_idx, out_logw, status,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* queries, void* out, int32_t out_dtype,

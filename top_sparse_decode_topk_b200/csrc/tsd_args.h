@@ -11,6 +11,7 @@ struct DecodeArgs {
   KvView kv;
   QView qv;
   const int32_t* idx;   // sparse: [T][Hq][k_max]; dense: unused
+  const float* logw;    // sparse, optional: [T][Hq][k_max] natural-log weight of each entry
   int32_t k_max;
   int32_t span;         // sparse: entries per list per split (E); dense: tokens per window (W)
   int32_t nsplit;
@@ -20,7 +21,6 @@ struct DecodeArgs {
   int32_t out_f32;
   float* lse;
   uint32_t* status;
-  uint32_t* sched;      // sparse: [0] work-unit counter, [1] finished-CTA counter (zero region)
   uint32_t* counters;
   float2* part_ml;
   float* part_acc;

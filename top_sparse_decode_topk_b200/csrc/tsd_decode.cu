@@ -195,9 +195,9 @@ __device__ __forceinline__ void row_fetch(const DecodeArgs& a, uint32_t row, int
 // Online-softmax update of a half-warp's state with a batch of U rows at once: the U
 // scores are reduced together (independent shuffle chains), then one max, one rescale
 // and U independent exponentials -- the serial chain is per batch, not per row.
-template <int U>
-__device__ __forceinline__ void batch_update(const uint4* kq, const uint4* vq, const uint32_t* rr, const float* q,
-                                             float& m_run, float& l_run, float* acc, unsigned hmask) {
+template <int U, bool BIAS>
+__device__ __forceinline__ void batch_update(const uint4* kq, const uint4* vq, const uint32_t* rr, const float* bias,
+                                             const float* q, float& m_run, float& l_run, float* acc, unsigned hmask) {
   float s[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
@@ -215,6 +215,10 @@ __device__ __forceinline__ void batch_update(const uint4* kq, const uint4* vq, c
   for (int o = 1; o < 16; o <<= 1)
 #pragma unroll
     for (int u = 0; u < U; ++u) s[u] += __shfl_xor_sync(hmask, s[u], o);
+  if (BIAS) {   // entry weights: p_i = w_i exp(s_i), with ln w_i in base-2 units
+#pragma unroll
+    for (int u = 0; u < U; ++u) s[u] += bias[u];
+  }
   float mb = -CUDART_INF_F;
 #pragma unroll
   for (int u = 0; u < U; ++u)
@@ -315,6 +319,7 @@ __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id
   if (l == 0 && a.lse != nullptr) a.lse[list_id] = L > 0.f ? (mx + log2f(L)) * kLn2 : -CUDART_INF_F;
 }
 
+template <bool WEIGHTED>
 __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel(DecodeArgs a) {
   // task states of the CTA's 16 half-warps, combined per list before anything leaves the CTA
   __shared__ float2 s_ml[16];
@@ -382,19 +387,23 @@ __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel
         row = kv_row(a.kv, b, g, v);
         if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
       }
+      float lw = 0.f;
+      if (WEIGHTED && e < e1) lw = __ldg(a.logw + list_id * a.k_max + e) * kLog2e;
       // the 16 rows, U at a time
 #pragma unroll
       for (int j0 = 0; j0 < 16; j0 += kSpU) {
         uint32_t rr[kSpU];
+        float bias[kSpU];
         uint4 kq[kSpU], vq[kSpU];
 #pragma unroll
         for (int u = 0; u < kSpU; ++u) {
           rr[u] = __shfl_sync(hmask, row, j0 + u, 16);
+          bias[u] = WEIGHTED ? __shfl_sync(hmask, lw, j0 + u, 16) : 0.f;
           kq[u] = make_uint4(0, 0, 0, 0);
           vq[u] = make_uint4(0, 0, 0, 0);
           row_fetch(a, rr[u], l, kq[u], vq[u]);
         }
-        batch_update<kSpU>(kq, vq, rr, q, m_run, l_run, acc, hmask);
+        batch_update<kSpU, WEIGHTED>(kq, vq, rr, bias, q, m_run, l_run, acc, hmask);
       }
     }
     bad |= __shfl_xor_sync(hmask, bad, 1);
@@ -645,7 +654,11 @@ cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaSt
   const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
   const int64_t grid = (tasks + 15) / 16;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
-  sparse_decode_kernel<<<(unsigned)grid, kSpThreads, 0, stream>>>(a);
+  if (a.logw != nullptr) {
+    sparse_decode_kernel<true><<<(unsigned)grid, kSpThreads, 0, stream>>>(a);
+  } else {
+    sparse_decode_kernel<false><<<(unsigned)grid, kSpThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

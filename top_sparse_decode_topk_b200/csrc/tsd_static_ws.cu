@@ -77,7 +77,6 @@ extern "C" tsd_status tsd_sparse_decode_static_ws(const tsd_kv_cache* cache, con
   const DecodeLayout lay = decode_layout(sh, a.nsplit);
   char* ws = static_cast<char*>(base);
   a.status = status != nullptr ? status : reinterpret_cast<uint32_t*>(ws);
-  a.sched = reinterpret_cast<uint32_t*>(ws) + 1;
   a.counters = reinterpret_cast<uint32_t*>(ws + lay.off_counters);
   a.part_ml = reinterpret_cast<float2*>(ws + lay.off_ml);
   a.part_acc = reinterpret_cast<float*>(ws + lay.off_acc);

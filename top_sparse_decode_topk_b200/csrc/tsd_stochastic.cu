@@ -1,0 +1,164 @@
+// vAttention-style stochastic selection for sm_100a.
+//
+// Operation ("Inference Time Context Sparsity: Illusion or Opportunity?", gist.science
+// summary, section 2: vAttention's stochastic index selection, evaluated against
+// deterministic top-k).  The pages give no sampling scheme or estimator; here, per (query
+// token t, q head h): the exact top-k list S (from tsd_topk_select), plus m tokens drawn
+// uniformly without replacement from the rest R = [0, kv_len) minus S by Floyd's algorithm
+// (driven by caller-supplied random 32-bit words), each weighted by |R| / m -- the
+// Horvitz-Thompson estimate of the softmax sums over R.  The output is one ascending index
+// list with a natural-log weight per entry (0 for S), which the weighted sparse decode
+// consumes.
+//
+// One warp per list.  Floyd's m steps run in order (each step's membership test is a warp
+// scan of the ranks kept so far); the kept ranks are then sorted by counting, mapped to
+// tokens of R by a binary search over S (token = rank + #{s in S below it}), and merged with
+// S by each side's binary-search position.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "tsd_args.h"
+#include "tsd_common.cuh"
+
+namespace tsd {
+
+constexpr int kStoMaxM = 1024;
+constexpr int kStoWarps = 4;
+
+struct StochasticArgs {
+  KvView kv;
+  QView qv;
+  const int32_t* top;     // [T][Hq][k_max] ascending, -1 padded
+  int32_t k_max;
+  const uint32_t* u;      // [T][Hq][m] random words
+  int32_t m;
+  int32_t* out_idx;       // [T][Hq][k_max + m]
+  float* out_logw;        // [T][Hq][k_max + m]
+  uint32_t* status;       // nullable
+};
+
+// Number of entries of the ascending list a[0..n) that are < x.
+__device__ __forceinline__ int count_below(const int32_t* a, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(a + mid) < x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(StochasticArgs a) {
+  __shared__ uint32_t kept[kStoWarps][kStoMaxM];
+  __shared__ int32_t toks[kStoWarps][kStoMaxM];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t list = (int64_t)blockIdx.x * kStoWarps + warp;
+  const int64_t nlists = (int64_t)a.qv.num_tokens * a.qv.hq;
+  if (list >= nlists) return;
+  const int t = (int)(list / a.qv.hq);
+  // visible length of token t (sequence by binary search over q_indptr)
+  int b = t;
+  if (a.qv.q_indptr != nullptr) {
+    int lo = 0, hi = a.kv.batch;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(a.qv.q_indptr + mid) <= t) lo = mid; else hi = mid;
+    }
+    b = lo;
+  }
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, false);
+  const int L = (t >= si.t0 && t < si.t0 + si.n) ? kv_len_of(a.qv, si, t - si.t0) : 0;
+  const int32_t* top = a.top + list * a.k_max;
+  // valid prefix of the top-k list (entries >= 0, ascending, < L)
+  int ntop = 0;
+  bool bad = false;
+  for (int i = lane; i < a.k_max; i += 32) {
+    const int32_t v = __ldg(top + i);
+    if (v >= 0) {
+      ntop = i + 1;
+      bad |= v >= L || (i > 0 && __ldg(top + i - 1) >= v);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ntop = max(ntop, __shfl_xor_sync(0xFFFFFFFFu, ntop, o));
+  if (__any_sync(0xFFFFFFFFu, bad)) {   // not an ascending list of visible tokens: flag, keep nothing
+    if (lane == 0 && a.status != nullptr) flag_status(a.status, TSD_DEV_BAD_INDEX);
+    ntop = 0;
+  }
+  const int n = max(0, L - ntop);              // |R|
+  const int m = min(a.m, n);
+  const uint32_t* u = a.u + list * a.m;
+  uint32_t* kr = kept[warp];
+  // ---- Floyd: step j = n - m .. n - 1 keeps t = u mod (j + 1), or j on a collision ----
+  for (int s = 0; s < m; ++s) {
+    const uint32_t j = (uint32_t)(n - m + s);
+    const uint32_t tr = (uint32_t)(__ldg(u + s) % (j + 1u));
+    bool seen = false;
+    for (int i = lane; i < s; i += 32) seen |= kr[i] == tr;
+    seen = __any_sync(0xFFFFFFFFu, seen);
+    if (lane == 0) kr[s] = seen ? j : tr;
+    __syncwarp();
+  }
+  // ---- sort the kept ranks (distinct) by counting, and map each to its token of R ----
+  int32_t* tk = toks[warp];
+  for (int i = lane; i < m; i += 32) {
+    const uint32_t r = kr[i];
+    int pos = 0;
+    for (int j = 0; j < m; ++j) pos += kr[j] < r;
+    // token = r + jstar, jstar = first index with top[j] - j > r (top ascending and distinct)
+    int lo = 0, hi = ntop;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(top + mid) - mid > (int)r) hi = mid; else lo = mid + 1;
+    }
+    tk[pos] = (int32_t)r + lo;
+  }
+  __syncwarp();
+  // ---- merge S and the sample into one ascending list with log-weights ----
+  const int width = a.k_max + a.m;
+  int32_t* oi = a.out_idx + list * width;
+  float* ow = a.out_logw + list * width;
+  const float lw = m > 0 ? logf((float)n / (float)m) : 0.f;
+  for (int i = lane; i < ntop; i += 32) {
+    const int32_t v = __ldg(top + i);
+    int lo = 0, hi = m;   // sampled tokens below v
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (tk[mid] < v) lo = mid + 1; else hi = mid;
+    }
+    oi[i + lo] = v;
+    ow[i + lo] = 0.f;
+  }
+  for (int i = lane; i < m; i += 32) {
+    const int32_t v = tk[i];
+    const int below = count_below(top, ntop, v);
+    oi[i + below] = v;
+    ow[i + below] = lw;
+  }
+  for (int i = ntop + m + lane; i < width; i += 32) {
+    oi[i] = -1;
+    ow[i] = 0.f;
+  }
+}
+
+cudaError_t launch_stochastic_select(const KvView& kv, const QView& qv, const int32_t* top, int k_max,
+                                     const uint32_t* u, int m, int32_t* out_idx, float* out_logw, uint32_t* status,
+                                     cudaStream_t stream) {
+  StochasticArgs a;
+  a.kv = kv;
+  a.qv = qv;
+  a.top = top;
+  a.k_max = k_max;
+  a.u = u;
+  a.m = m;
+  a.out_idx = out_idx;
+  a.out_logw = out_logw;
+  a.status = status;
+  const int64_t nlists = (int64_t)qv.num_tokens * qv.hq;
+  const int64_t grid = (nlists + kStoWarps - 1) / kStoWarps;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  stochastic_select_kernel<<<(unsigned)grid, 32 * kStoWarps, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace tsd
