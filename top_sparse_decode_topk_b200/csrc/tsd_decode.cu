@@ -6,8 +6,9 @@
 // index list -- which may differ per token, per query and per head -- so that
 // the bytes read fall from O(N d) to O(k d).  Dense decode attends to every row.
 //
-// Sparse decode: one half-warp per task (16+ entries of one list); rows gathered into
-// registers; batched online softmax; per-list split-K merge by the last task to finish.
+// Sparse decode: one half-warp per task (16+ entries of one list); rows gathered through a
+// per-half-warp cp.async ring; batched online softmax; per-list split-K merge in the CTA,
+// then by the last CTA of the list to finish.
 // Dense decode: one CTA per (sequence, kv head, list group, window of W tokens); 64-token
 // K/V tiles arrive by TMA in a 2-stage shared-memory ring and q K^T and P V run on the
 // tensor cores; CTA-level partials are merged by the last CTA of the unit.
@@ -165,25 +166,30 @@ __device__ void finish_lists(const DecodeArgs& a, const SeqInfo& si, int b, int 
 // Sparse decode
 // ---------------------------------------------------------------------------
 // Design, from measurements on B200:
-//  * Scattered 256-byte rows are gathered with 16-byte loads straight into registers.
-//    For random 256-byte rows this reaches the copy bandwidth at large sizes; staging
-//    them in shared memory (cp.async, one bulk copy per row, or TMA gather4) is slower
-//    unless 4-6 CTAs per SM are resident.
-//  * What sets the gather rate is how many warps are issuing loads, so the work is cut
-//    into many small independent tasks: one half-warp (16 lanes x 16 bytes = one row)
-//    takes a chunk of E entries of one list (token x q head) and nothing else.  There is
-//    no block-level synchronisation and no shared memory.
+//  * Scattered 256-byte rows are gathered with 16-byte copies: lane l of a half-warp copies
+//    chunk l of each K and V row.  The copies go through a per-half-warp ring of kSpStages
+//    batches in shared memory (cp.async), so 12 rows are in flight per half-warp without
+//    spending registers on them.  Each lane reads back only what it copied itself, so the
+//    ring needs no synchronisation beyond each lane's own cp.async wait.  Against gathering
+//    into registers (4 rows in flight, 3 CTAs/SM) this measured 30.7 vs 32.8 us on
+//    llama3_8b.
+//  * What sets the gather rate is how many loads are in flight, so the work is cut into many
+//    small independent tasks: one half-warp (16 lanes x 16 bytes = one row) takes a chunk of
+//    E entries of one list (token x q head) and nothing else, and the plan sizes E so the
+//    grid fits one wave of resident CTAs.
 //  * Tasks are numbered (sequence, kv head, chunk, list) so that the lists of one kv head
 //    -- the q heads of a GQA group and the decode tokens of the sequence -- read the same
 //    token range in the same CTA at the same time: a row picked by several of them is
-//    read from DRAM once and served to the others from L1/L2.
+//    read from DRAM once and served to the others from L2.
 // Per row the half-warp computes a 128-dim dot (8 FMA per lane + a 4-step shuffle
 // reduction); its online softmax state (max, sum, 8 output dims per lane) is updated once
-// per batch of U rows in flight.  Each task writes its partial state; the last task of a list
-// to arrive (a per-list counter) merges them with log-sum-exp.  A list that fits one
-// task is written directly.
+// per batch of U rows.  The chunks of a list held by one CTA are combined in shared memory;
+// each CTA then writes one partial per list, and the last CTA of a list to arrive (a per-list
+// counter) merges them with log-sum-exp.  A list that fits one CTA is written directly.
 constexpr int kSpThreads = 256;   // 16 half-warps, one task each
-constexpr int kSpU = 4;           // rows in flight per half-warp
+constexpr int kSpU = 4;           // rows per softmax batch
+constexpr int kSpStages = 3;      // batches in flight per half-warp (cp.async ring)
+constexpr size_t kSpRingBytes = (size_t)16 * kSpStages * 2 * kSpU * 16 * sizeof(uint4);   // 96 KB
 
 __device__ __forceinline__ void row_fetch(const DecodeArgs& a, uint32_t row, int l, uint4& k, uint4& v) {
   if (row != kInvalidRow) {
@@ -321,6 +327,7 @@ __device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id
 
 template <bool WEIGHTED>
 __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel(DecodeArgs a) {
+  extern __shared__ __align__(16) uint4 sp_ring[];   // [16 half-warps][kSpStages][K, V][kSpU rows][16 lanes]
   // task states of the CTA's 16 half-warps, combined per list before anything leaves the CTA
   __shared__ float2 s_ml[16];
   __shared__ __align__(16) float s_acc[16][kHeadDim];
@@ -389,19 +396,38 @@ __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel
       }
       float lw = 0.f;
       if (WEIGHTED && e < e1) lw = __ldg(a.logw + list_id * a.k_max + e) * kLog2e;
-      // the 16 rows, U at a time
+      // the 16 rows, kSpU at a time, through this half-warp's ring of kSpStages stages in
+      // shared memory (cp.async): lane l copies, and later reads, chunk l of every row, so the
+      // ring needs no synchronisation beyond each lane's own cp.async wait
+      uint4* ring = sp_ring + (size_t)hw * kSpStages * 2 * kSpU * 16;
+      auto issue = [&](int bt) {
+        uint4* st = ring + (size_t)(bt % kSpStages) * 2 * kSpU * 16;
 #pragma unroll
-      for (int j0 = 0; j0 < 16; j0 += kSpU) {
+        for (int u = 0; u < kSpU; ++u) {
+          const uint32_t rr = __shfl_sync(hmask, row, bt * kSpU + u, 16);
+          if (rr != kInvalidRow) {
+            cp_async16(st + u * 16 + l, reinterpret_cast<const uint4*>(a.kv.k + (int64_t)rr * kHeadDim) + l);
+            cp_async16(st + (kSpU + u) * 16 + l, reinterpret_cast<const uint4*>(a.kv.v + (int64_t)rr * kHeadDim) + l);
+          }
+        }
+        cp_async_commit();
+      };
+#pragma unroll
+      for (int bt = 0; bt < kSpStages - 1; ++bt) issue(bt);
+#pragma unroll
+      for (int bt = 0; bt < 16 / kSpU; ++bt) {
+        if (bt + kSpStages - 1 < 16 / kSpU) issue(bt + kSpStages - 1); else cp_async_commit();
+        cp_async_wait<kSpStages - 1>();
+        const uint4* st = ring + (size_t)(bt % kSpStages) * 2 * kSpU * 16;
         uint32_t rr[kSpU];
         float bias[kSpU];
         uint4 kq[kSpU], vq[kSpU];
 #pragma unroll
         for (int u = 0; u < kSpU; ++u) {
-          rr[u] = __shfl_sync(hmask, row, j0 + u, 16);
-          bias[u] = WEIGHTED ? __shfl_sync(hmask, lw, j0 + u, 16) : 0.f;
-          kq[u] = make_uint4(0, 0, 0, 0);
-          vq[u] = make_uint4(0, 0, 0, 0);
-          row_fetch(a, rr[u], l, kq[u], vq[u]);
+          rr[u] = __shfl_sync(hmask, row, bt * kSpU + u, 16);
+          bias[u] = WEIGHTED ? __shfl_sync(hmask, lw, bt * kSpU + u, 16) : 0.f;
+          kq[u] = rr[u] != kInvalidRow ? st[u * 16 + l] : make_uint4(0, 0, 0, 0);
+          vq[u] = rr[u] != kInvalidRow ? st[(kSpU + u) * 16 + l] : make_uint4(0, 0, 0, 0);
         }
         batch_update<kSpU, WEIGHTED>(kq, vq, rr, bias, q, m_run, l_run, acc, hmask);
       }
@@ -654,10 +680,20 @@ cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaSt
   const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
   const int64_t grid = (tasks + 15) / 16;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSpRingBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(sparse_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSpRingBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
   if (a.logw != nullptr) {
-    sparse_decode_kernel<true><<<(unsigned)grid, kSpThreads, 0, stream>>>(a);
+    sparse_decode_kernel<true><<<(unsigned)grid, kSpThreads, kSpRingBytes, stream>>>(a);
   } else {
-    sparse_decode_kernel<false><<<(unsigned)grid, kSpThreads, 0, stream>>>(a);
+    sparse_decode_kernel<false><<<(unsigned)grid, kSpThreads, kSpRingBytes, stream>>>(a);
   }
   return cudaGetLastError();
 }

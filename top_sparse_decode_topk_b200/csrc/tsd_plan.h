@@ -55,7 +55,7 @@ struct SparsePlan {
   int nsplit;    // C
 };
 
-constexpr int kSpCtasPerSm = 3;   // resident sparse-decode CTAs per SM (its launch bounds)
+constexpr int kSpCtasPerSm = 2;   // resident sparse-decode CTAs per SM (launch bounds; 96 KB ring each)
 
 inline SparsePlan plan_sparse(const Shapes& s, int k_max, int num_sms) {
   SparsePlan p;
