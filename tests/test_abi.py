@@ -166,3 +166,34 @@ def test_multi_token_queries_need_bounds(lib):
     assert sparse(lib, c, q) == tsd.TSD_ERR_INVALID_ARGUMENT
     q = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=4)
     assert lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 2622) > 0
+
+
+@fake_pointer_call
+def test_label_and_stochastic_errors_before_launch(lib):
+    c, q = make_cache(), make_queries()
+    # label cache sizing is host arithmetic: rows x r x 2 bytes, 0 for an unsupported r
+    rows = c.num_pages * c.num_kv_heads * c.page_size
+    assert lib.tsd_label_cache_bytes(ctypes.byref(c), 16) == rows * 16 * 2
+    assert lib.tsd_label_cache_bytes(ctypes.byref(c), 12) == 0
+    assert lib.tsd_label_channels_workspace_size(ctypes.byref(c), ctypes.byref(q)) > 256
+    assert lib.tsd_label_channels(ctypes.byref(c), ctypes.byref(q), 12, FAKE, FAKE, 1 << 30, None) == \
+        tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_label_channels(ctypes.byref(c), ctypes.byref(q), 16, FAKE, FAKE, 16, None) == \
+        tsd.TSD_ERR_WORKSPACE_TOO_SMALL
+    assert lib.tsd_label_cache_build(ctypes.byref(c), FAKE, 24, FAKE, None, None) == tsd.TSD_ERR_UNSUPPORTED
+    assert lib.tsd_label_cache_build(ctypes.byref(c), None, 16, FAKE, None, None) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_label_cache_build(ctypes.byref(c), FAKE, 16, FAKE + 8, None, None) == \
+        tsd.TSD_ERR_INVALID_ARGUMENT   # misaligned label cache
+    assert lib.tsd_topk_select_label(ctypes.byref(c), FAKE, FAKE, 16, ctypes.byref(q), 655, None, FAKE, None,
+                                     FAKE, 16, None) == tsd.TSD_ERR_WORKSPACE_TOO_SMALL
+    assert lib.tsd_topk_select_label(ctypes.byref(c), FAKE, FAKE, 20, ctypes.byref(q), 655, None, FAKE, None,
+                                     FAKE, 1 << 40, None) == tsd.TSD_ERR_UNSUPPORTED
+    # stochastic selection and weighted decode
+    assert lib.tsd_stochastic_select(ctypes.byref(c), ctypes.byref(q), FAKE, 655, FAKE, 2048, FAKE, FAKE, None,
+                                     None) == tsd.TSD_ERR_UNSUPPORTED
+    assert lib.tsd_stochastic_select(ctypes.byref(c), ctypes.byref(q), FAKE, 655, None, 64, FAKE, FAKE, None,
+                                     None) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_stochastic_select(ctypes.byref(c), ctypes.byref(q), None, 655, FAKE, 64, FAKE, FAKE, None,
+                                     None) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_sparse_decode_weighted(ctypes.byref(c), ctypes.byref(q), FAKE, None, 655, FAKE, 0, None, FAKE,
+                                          1 << 40, None) == tsd.TSD_ERR_INVALID_ARGUMENT
