@@ -235,6 +235,52 @@ tsd_status tsd_sparse_decode_static_ws(const tsd_kv_cache* cache, const tsd_quer
  */
 tsd_status tsd_read_device_status(void* ws, tsd_stream_t stream, uint32_t* flags);
 
+/*
+ * tsd_topk_select, also returning the kept tokens' scores: out_scores device fp32
+ * [T][Hq][k_max], the unscaled q.K of each kept index (-inf in the padding; -0 as +0).
+ * Errors: as tsd_topk_select, plus INVALID_ARGUMENT for a NULL out_scores.
+ */
+tsd_status tsd_topk_select_scores(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                  const int32_t* k_per_token, int32_t* out_idx, float* out_scores,
+                                  int32_t* out_count, void* ws, size_t ws_bytes, tsd_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Context-parallel decode over a token-sharded cache.  Not on the pages: a way to run the
+ * path over contexts split across GPUs.  Rank r holds a token range of every sequence, the
+ * ranges in rank order.  Each rank:
+ *   1. runs tsd_topk_select_scores on its shard (single-token decode, or non-causal);
+ *   2. after the caller gathers every rank's (local index, score) candidates rank-major,
+ *      keeps the global top-k among them with tsd_cp_merge_select;
+ *   3. decodes its shard over the entries it keeps, with fp32 output and lse;
+ *   4. after the caller gathers the P (output, lse) pairs, merges them with
+ *      tsd_merge_partials.
+ * The global top-k lies in the union of the local top-k lists, so the result equals the
+ * single-GPU path's.
+ * --------------------------------------------------------------------------------------- */
+
+/*
+ * cand_idx, cand_scores: device [ranks][lists][k_cand]: each rank's shard-local token indices
+ * (ascending, -1 padding) and their scores, rank r's token range preceding rank r + 1's.
+ * Per list, keeps the k largest scores among all candidates (k = k_per_list[list] if not
+ * NULL, else k; ties to the lower global index) and writes the kept candidates of rank
+ * my_rank -- its local indices -- ascending, -1 padded, to out_idx [lists][k_out]; if more than
+ * k_out are kept there the rest are dropped and TSD_DEV_BAD_INDEX is set in *status (if not
+ * NULL).  ranks x k_cand <= 16384.  Errors: INVALID_ARGUMENT, UNSUPPORTED, CUDA.
+ */
+tsd_status tsd_cp_merge_select(const int32_t* cand_idx, const float* cand_scores, int32_t ranks, int64_t lists,
+                               int32_t k_cand, const int32_t* k_per_list, int32_t k, int32_t my_rank,
+                               int32_t* out_idx, int32_t k_out, uint32_t* status, tsd_stream_t stream);
+
+/*
+ * Merge P partial decode results of the same rows: out_parts device fp32 [parts][rows][128]
+ * (each normalised over its own entries), lse_parts [parts][rows].  out = sum_p w_p out_p /
+ * sum_p w_p with w_p = exp(lse_p - max_p lse_p); lse = max + ln sum_p w_p; rows whose parts
+ * are all -inf get out = 0 and lse = -inf.  out: device [rows][128] of out_dtype; lse: device
+ * fp32 [rows] or NULL.  16-byte aligned.  Errors: INVALID_ARGUMENT, UNSUPPORTED, CUDA.
+ */
+tsd_status tsd_merge_partials(int32_t parts, int64_t rows, const float* out_parts, const float* lse_parts, void* out,
+                              int32_t out_dtype, float* lse, tsd_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------
  * Label-channel approximate indexer (Double-Sparsity-style).
  *

@@ -197,3 +197,20 @@ def test_label_and_stochastic_errors_before_launch(lib):
                                      None) == tsd.TSD_ERR_INVALID_ARGUMENT
     assert lib.tsd_sparse_decode_weighted(ctypes.byref(c), ctypes.byref(q), FAKE, None, 655, FAKE, 0, None, FAKE,
                                           1 << 40, None) == tsd.TSD_ERR_INVALID_ARGUMENT
+
+
+@fake_pointer_call
+def test_context_parallel_errors_before_launch(lib):
+    c, q = make_cache(), make_queries()
+    assert lib.tsd_topk_select_scores(ctypes.byref(c), ctypes.byref(q), 655, None, FAKE, None, None, FAKE, 1 << 40,
+                                      None) == tsd.TSD_ERR_INVALID_ARGUMENT      # no score buffer
+    # ranks x candidates above what one CTA holds
+    assert lib.tsd_cp_merge_select(FAKE, FAKE, 8, 256, 4096, None, 655, 0, FAKE, 655, None, None) == \
+        tsd.TSD_ERR_UNSUPPORTED
+    assert lib.tsd_cp_merge_select(FAKE, FAKE, 4, 256, 655, None, 655, 4, FAKE, 655, None, None) == \
+        tsd.TSD_ERR_INVALID_ARGUMENT   # my_rank outside [0, ranks)
+    assert lib.tsd_cp_merge_select(None, FAKE, 4, 256, 655, None, 655, 0, FAKE, 655, None, None) == \
+        tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_merge_partials(4, 256, FAKE, FAKE, FAKE, 7, None, None) == tsd.TSD_ERR_UNSUPPORTED
+    assert lib.tsd_merge_partials(0, 256, FAKE, FAKE, FAKE, 0, None, None) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_merge_partials(4, 256, FAKE + 4, FAKE, FAKE, 0, None, None) == tsd.TSD_ERR_INVALID_ARGUMENT

@@ -69,3 +69,44 @@ def test_reference_arm_under_torchrun_prints_once():
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _cp_rank_main(rank: int, world: int, port: int, out_dir: str):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from top_sparse_decode_topk_b200 import context_parallel as CP
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # what a rank contributes to the candidate exchange: [T, Hq, k] indices and scores
+        idx = torch.arange(12, dtype=torch.int32).reshape(2, 2, 3) + 100 * rank
+        sc = torch.full((2, 2, 3), float(rank), dtype=torch.float32)
+        gi, gs = CP.gather_rank_major(idx), CP.gather_rank_major(sc)
+        with open(os.path.join(out_dir, f"cp{rank}.json"), "w") as f:
+            json.dump({"shape": list(gi.shape), "idx": gi.tolist(), "sc": gs[:, 0, 0, 0].tolist()}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_context_parallel_exchange_is_rank_major(tmp_path):
+    """The candidate and partial exchanges stack every rank's tensor in rank order, which the
+    merge kernels rely on (rank r's token range precedes rank r + 1's)."""
+    import torch.multiprocessing as mp
+    port = _free_port()
+    mp.start_processes(_cp_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True, start_method="spawn")
+    r0 = json.load(open(tmp_path / "cp0.json"))
+    r1 = json.load(open(tmp_path / "cp1.json"))
+    assert r0 == r1
+    assert r0["shape"] == [2, 2, 2, 3]
+    assert r0["sc"] == [0.0, 1.0]
+    assert r0["idx"][1][0][0] == [100, 101, 102]
+
+
+def test_shard_lengths_cover_the_context():
+    from top_sparse_decode_topk_b200 import context_parallel as CP
+    for n, world in ((32768, 4), (20001, 3), (131072, 8), (100, 7)):
+        S = CP.shard_length(n, world, 16)
+        assert S % 16 == 0 and S * world >= n and S * (world - 1) < n + 16 * world

@@ -94,6 +94,14 @@ EXPORTS = {
     "tsd_stochastic_select": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_void_p,
                                              ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "tsd_topk_select_scores": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
+                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tsd_cp_merge_select": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                           ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
+    "tsd_merge_partials": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
     "tsd_label_cache_bytes": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.c_int32]),
     "tsd_label_channels_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC)]),
     "tsd_label_channels": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
@@ -303,9 +311,11 @@ def _on_device_queries(queries: Queries, device, stream) -> Queries:
 # Operations
 # ---------------------------------------------------------------------------
 def topk_select(cache: KVCache, queries: Queries, k_max: int, k_per_token=None, out_idx=None, out_count=None,
-                workspace: Optional[Workspace] = None, stream=None) -> Tuple["object", "object"]:
+                workspace: Optional[Workspace] = None, stream=None, with_scores: bool = False, out_scores=None):
     """Exact top-k token indices per (query token, q head): int32 [T, Hq, k_max]
-    ascending, -1 padded, and the per-list counts int32 [T, Hq]."""
+    ascending, -1 padded, and the per-list counts int32 [T, Hq].  With `with_scores`, also
+    the kept tokens' unscaled scores fp32 [T, Hq, k_max] (-inf in the padding), returned
+    as (idx, scores, counts)."""
     import torch
     lib = load_library()
     dev = cache.device
@@ -324,10 +334,16 @@ def topk_select(cache: KVCache, queries: Queries, k_max: int, k_per_token=None, 
     if nbytes == 0:
         raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_topk_workspace_size")
     ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, queries), sp)
-    _check(lib.tsd_topk_select(ctypes.byref(cs), ctypes.byref(qs), int(k_max),
-                               None if k_per_token is None else k_per_token.data_ptr(),
-                               out_idx.data_ptr(), out_count.data_ptr(), ws.data_ptr(), ws.numel(), sp),
-           "tsd_topk_select")
+    kp = None if k_per_token is None else k_per_token.data_ptr()
+    if with_scores or out_scores is not None:
+        if out_scores is None:
+            out_scores = torch.empty((T, Hq, k_max), dtype=torch.float32, device=dev)
+        _check(lib.tsd_topk_select_scores(ctypes.byref(cs), ctypes.byref(qs), int(k_max), kp, out_idx.data_ptr(),
+                                          out_scores.data_ptr(), out_count.data_ptr(), ws.data_ptr(), ws.numel(),
+                                          sp), "tsd_topk_select_scores")
+        return out_idx, out_scores, out_count
+    _check(lib.tsd_topk_select(ctypes.byref(cs), ctypes.byref(qs), int(k_max), kp, out_idx.data_ptr(),
+                               out_count.data_ptr(), ws.data_ptr(), ws.numel(), sp), "tsd_topk_select")
     return out_idx, out_count
 
 

@@ -23,7 +23,7 @@ COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
           "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
 
 LIBS = {
-    "libtsd.so": ["tsd_api.cu", "tsd_decode.cu", "tsd_topk.cu", "tsd_label.cu", "tsd_stochastic.cu", "tsd_static_ws.cu"],
+    "libtsd.so": ["tsd_api.cu", "tsd_decode.cu", "tsd_topk.cu", "tsd_label.cu", "tsd_stochastic.cu", "tsd_cp.cu", "tsd_static_ws.cu"],
     "libtsd_workload.so": ["workload_fill.cu"],
 }
 HEADERS = ["tsd_common.cuh", "tsd_plan.h", "tsd_args.h", "tsd_kvtile.cuh"]

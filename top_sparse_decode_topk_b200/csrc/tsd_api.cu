@@ -28,6 +28,12 @@ cudaError_t launch_label_build(const KvView& kv, const int32_t* channels, int r,
 cudaError_t launch_stochastic_select(const KvView& kv, const QView& qv, const int32_t* top, int k_max,
                                      const uint32_t* u, int m, int32_t* out_idx, float* out_logw, uint32_t* status,
                                      cudaStream_t stream);
+cudaError_t launch_cp_merge_select(const int32_t* cand_idx, const float* cand_score, int P, int64_t lists, int kc,
+                                   const int32_t* k_per_list, int k, int my_rank, int32_t* out, int k_out,
+                                   uint32_t* status, cudaStream_t stream);
+int cp_max_candidates();
+cudaError_t launch_merge_partials(int P, int64_t rows, const float* out_parts, const float* lse_parts, void* out,
+                                  int out_f32, float* lse, cudaStream_t stream);
 cudaError_t launch_label_topk(const TopkArgs& a, const uint16_t* label, const int32_t* channels, int r, int nwin,
                               int batch, int hkv, int num_lists, cudaStream_t stream);
 }  // namespace tsd
@@ -247,9 +253,9 @@ size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_quer
   return decode_layout(sh, p.nsplit).total;
 }
 
-tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
-                           const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count, void* ws,
-                           size_t ws_bytes, tsd_stream_t stream) {
+static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                   const int32_t* k_per_token, int32_t* out_idx, float* out_scores,
+                                   int32_t* out_count, void* ws, size_t ws_bytes, tsd_stream_t stream) {
   KvView kv; QView qv; Shapes sh;
   tsd_status st = check_inputs(cache, queries, &kv, &qv, &sh);
   if (st != TSD_OK) return st;
@@ -265,6 +271,7 @@ tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries
   a.k_per_token = k_per_token;
   a.out_idx = out_idx;
   a.out_count = out_count;
+  a.out_scores = out_scores;
   a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
   a.score_stride = lay.score_stride;
   // scoring streams K in the dense path's tiles, with its own occupancy
@@ -278,6 +285,40 @@ tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries
   if (st != TSD_OK) return st;
   return cuda_status(launch_topk(a, maps, p.nsplit, (int)sh.batch, (int)sh.hkv, (int)(sh.tokens * sh.hq),
                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                           const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count, void* ws,
+                           size_t ws_bytes, tsd_stream_t stream) {
+  return topk_select_impl(cache, queries, k_max, k_per_token, out_idx, nullptr, out_count, ws, ws_bytes, stream);
+}
+
+tsd_status tsd_topk_select_scores(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                  const int32_t* k_per_token, int32_t* out_idx, float* out_scores,
+                                  int32_t* out_count, void* ws, size_t ws_bytes, tsd_stream_t stream) {
+  if (out_scores == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  return topk_select_impl(cache, queries, k_max, k_per_token, out_idx, out_scores, out_count, ws, ws_bytes, stream);
+}
+
+tsd_status tsd_cp_merge_select(const int32_t* cand_idx, const float* cand_scores, int32_t ranks, int64_t lists,
+                               int32_t k_cand, const int32_t* k_per_list, int32_t k, int32_t my_rank,
+                               int32_t* out_idx, int32_t k_out, uint32_t* status, tsd_stream_t stream) {
+  if (cand_idx == nullptr || cand_scores == nullptr || out_idx == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  if (ranks < 1 || lists < 1 || k_cand < 1 || k < 0 || k_out < 1 || my_rank < 0 || my_rank >= ranks)
+    return TSD_ERR_INVALID_ARGUMENT;
+  if ((int64_t)ranks * k_cand > cp_max_candidates()) return TSD_ERR_UNSUPPORTED;
+  return cuda_status(launch_cp_merge_select(cand_idx, cand_scores, ranks, lists, k_cand, k_per_list, k, my_rank,
+                                            out_idx, k_out, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tsd_status tsd_merge_partials(int32_t parts, int64_t rows, const float* out_parts, const float* lse_parts, void* out,
+                              int32_t out_dtype, float* lse, tsd_stream_t stream) {
+  if (parts < 1 || rows < 1 || out_parts == nullptr || lse_parts == nullptr || out == nullptr)
+    return TSD_ERR_INVALID_ARGUMENT;
+  if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return TSD_ERR_UNSUPPORTED;
+  if (((uintptr_t)out_parts & 15) != 0 || ((uintptr_t)out & 15) != 0) return TSD_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_merge_partials(parts, rows, out_parts, lse_parts, out, out_dtype == TSD_F32, lse,
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 static tsd_status decode_common(const tsd_kv_cache* cache, const tsd_queries* queries, void* out,

@@ -33,6 +33,7 @@ struct TopkArgs {
   const int32_t* k_per_token;
   int32_t* out_idx;
   int32_t* out_count;
+  float* out_scores;    // optional [T][Hq][k_max]: the kept tokens' scores (-inf in the padding)
   float* scores;
   int64_t score_stride;
   int32_t lists_per_cta;

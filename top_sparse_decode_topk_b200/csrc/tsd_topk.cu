@@ -18,6 +18,7 @@
 //    ordered pass keeps every key > T plus the lowest-index keys == T, writing
 //    them in ascending token order with block-wide prefix sums.
 #include <cuda_runtime.h>
+#include <math_constants.h>
 #include <stdint.h>
 
 #include "tsd_args.h"
@@ -193,11 +194,16 @@ __device__ __forceinline__ void load16(const float* row, int i0, int L, float* f
 // the exact radix select and the ordered output then run over those few thousand entries
 // only.  Returns false, having written nothing, when the sample says too many keys would be
 // kept or the pass kept more than fit or fewer than k: the caller then runs the full passes.
+// The score of an order-preserving key (inverse of score_key; -0 comes back as +0).
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 constexpr int kFastMinL = 4096;
 constexpr int kFastSample = 1024;
 constexpr int kFastCap = kCandMax / 2;   // kept entries: keys in cand[0, cap), indices in cand[cap, 2 cap)
 
-__device__ bool select_fast(SelectSmem& S, const float* row, int L, int k, int32_t* out, int k_max) {
+__device__ bool select_fast(SelectSmem& S, const float* row, int L, int k, int32_t* out, float* osc, int k_max) {
   uint32_t* ckey = S.cand;
   uint32_t* cidx = S.cand + kFastCap;
   // ---- the r_lo-th largest of a strided sample of keys ----
@@ -308,10 +314,16 @@ __device__ bool select_fast(SelectSmem& S, const float* row, int L, int k, int32
 #pragma unroll
   for (int j = 0; j < kPer; ++j)
     if (selmask & (1u << j)) {
-      if (pos < k) out[pos] = (int32_t)cidx[c0 + j];
+      if (pos < k) {
+        out[pos] = (int32_t)cidx[c0 + j];
+        if (osc != nullptr) osc[pos] = key_score(ckey[c0 + j]);
+      }
       ++pos;
     }
-  for (int i = k + threadIdx.x; i < k_max; i += kSelectThreads) out[i] = -1;
+  for (int i = k + threadIdx.x; i < k_max; i += kSelectThreads) {
+    out[i] = -1;
+    if (osc != nullptr) osc[i] = -CUDART_INF_F;
+  }
   return true;
 }
 
@@ -343,14 +355,18 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
   }
   const int k = kreq < L ? kreq : L;
   int32_t* out = a.out_idx + (int64_t)th * a.k_max;
+  float* osc = a.out_scores != nullptr ? a.out_scores + (int64_t)th * a.k_max : nullptr;
   if (a.out_count != nullptr && threadIdx.x == 0) a.out_count[th] = k;
+  const float* row = a.scores + (int64_t)th * a.score_stride;
 
   if (k == L || k == 0) {   // every visible token is kept, or none
-    for (int i = threadIdx.x; i < a.k_max; i += kSelectThreads) out[i] = i < k ? i : -1;
+    for (int i = threadIdx.x; i < a.k_max; i += kSelectThreads) {
+      out[i] = i < k ? i : -1;
+      if (osc != nullptr) osc[i] = i < k ? __ldcg(row + i) + 0.f : -CUDART_INF_F;
+    }
     return;
   }
-  const float* row = a.scores + (int64_t)th * a.score_stride;
-  if (L >= kFastMinL && select_fast(S, row, L, k, out, a.k_max)) return;
+  if (L >= kFastMinL && select_fast(S, row, L, k, out, osc, a.k_max)) return;
   const int tile_elems = kSelectThreads * kSelPerThread;
 
   // ---- pass 1: histogram of the top 11 key bits ----
@@ -466,13 +482,19 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
 #pragma unroll
     for (int j = 0; j < kSelPerThread; ++j)
       if (selmask & (1u << j)) {
-        if (pos < k) out[pos] = i0 + j;
+        if (pos < k) {
+          out[pos] = i0 + j;
+          if (osc != nullptr) osc[pos] = f[j] + 0.f;   // -0 as +0, like the key
+        }
         ++pos;
       }
     eq_before += eq_total;
     sel_before += sel_total;
   }
-  for (int i = k + threadIdx.x; i < a.k_max; i += kSelectThreads) out[i] = -1;
+  for (int i = k + threadIdx.x; i < a.k_max; i += kSelectThreads) {
+    out[i] = -1;
+    if (osc != nullptr) osc[i] = -CUDART_INF_F;
+  }
 }
 
 // ---------------------------------------------------------------------------
