@@ -275,7 +275,7 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
   a.score_stride = lay.score_stride;
   // scoring streams K in the dense path's tiles, with its own occupancy
-  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScCtasPerSm * kStreamWaves);
+  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScoreCtasPerSm * kStreamWaves);
   a.lists_per_cta = p.lists_per_cta;
   a.list_groups = p.list_groups;
   a.window = p.window;

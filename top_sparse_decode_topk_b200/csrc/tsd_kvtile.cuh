@@ -76,25 +76,26 @@ __device__ __forceinline__ int box_rows_get(BoxRows& br, const KvView& kv, int b
   return __shfl_sync(0xFFFFFFFFu, br.cur, box & 31);
 }
 
-// Issue the TMA loads of one 64-token tile (all 32 lanes call it; lane 0 issues) and
-// return the bytes issued (valid on lane 0).
+// Issue the TMA loads of one TT-token tile (all 32 lanes call it; lane 0 issues) and
+// return the bytes issued (valid on lane 0).  Each K/V half is a [TT rows][128 B] block.
+template <int TT = kTileTok>
 __device__ __forceinline__ uint32_t tile_issue_tma(const KvView& kv, const CUtensorMap* tmk, const CUtensorMap* tmv,
                                                    BoxRows& br, int b, int g, int tok0, int tok_end, int tile,
                                                    unsigned char* kdst, unsigned char* vdst, uint64_t* bar, int lane,
                                                    uint32_t* status) {
   const int bp = tma_box_rows(kv);
   uint32_t bytes = 0;
-  for (int r = 0; r < kTileTok; r += bp) {
-    const int box = (tile * kTileTok + r) / bp;
+  for (int r = 0; r < TT; r += bp) {
+    const int box = (tile * TT + r) / bp;
     const int y = box_rows_get(br, kv, b, g, tok0, tok_end, bp, lane, box, status);
     if (y == -1) break;
     if (y < 0) continue;
     if (lane == 0) {
       tma_load_2d(kdst + r * 128, tmk, 0, y, bar);
-      tma_load_2d(kdst + kHalfBytes + r * 128, tmk, 64, y, bar);
+      tma_load_2d(kdst + TT * 128 + r * 128, tmk, 64, y, bar);
       if (vdst != nullptr) {
         tma_load_2d(vdst + r * 128, tmv, 0, y, bar);
-        tma_load_2d(vdst + kHalfBytes + r * 128, tmv, 64, y, bar);
+        tma_load_2d(vdst + TT * 128 + r * 128, tmv, 64, y, bar);
       }
     }
     bytes += (vdst != nullptr ? 4 : 2) * bp * 128;
@@ -103,14 +104,15 @@ __device__ __forceinline__ uint32_t tile_issue_tma(const KvView& kv, const CUten
 }
 
 // cp.async path (pages < 8 tokens): called by all 32 lanes of the producer warp.
+template <int TT = kTileTok>
 __device__ __forceinline__ void tile_issue_cpasync(const KvView& kv, int b, int g, int tok, int tok_end,
                                                    unsigned char* kdst, unsigned char* vdst, int lane,
                                                    uint32_t* status) {
   const int ntensor = vdst != nullptr ? 2 : 1;
-  // 64 rows x 16 chunks per tensor; lane -> (row, chunk) pairs
-  for (int id = lane; id < kTileTok * 16 * ntensor; id += 32) {
-    const int which = id / (kTileTok * 16);
-    const int rc = id % (kTileTok * 16);
+  // TT rows x 16 chunks per tensor; lane -> (row, chunk) pairs
+  for (int id = lane; id < TT * 16 * ntensor; id += 32) {
+    const int which = id / (TT * 16);
+    const int rc = id % (TT * 16);
     const int r = rc >> 4, ch = rc & 15;
     const int t = tok + r;
     if (t >= tok_end) continue;
@@ -121,7 +123,7 @@ __device__ __forceinline__ void tile_issue_cpasync(const KvView& kv, int b, int 
     }
     const uint16_t* src = (which ? kv.v : kv.k) + (int64_t)row * kHeadDim + ch * 8;
     unsigned char* base = which ? vdst : kdst;
-    cp_async16(base + (ch >> 3) * kHalfBytes + sw128(r, ch & 7), src);
+    cp_async16(base + (ch >> 3) * (TT * 128) + sw128(r, ch & 7), src);
   }
 }
 
@@ -137,7 +139,7 @@ __device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) 
 // wait is bounded: on a timeout the producer flags TSD_DEV_TIMEOUT, raises `abort` and
 // stops.  Before returning it waits for its last fills to land, so that no copy into shared
 // memory is in flight when the CTA ends.
-template <int NST, int STAGE_BYTES, bool WITH_V>
+template <int NST, int STAGE_BYTES, bool WITH_V, int TT = kTileTok>
 __device__ __forceinline__ void produce_tiles(const KvView& kv, const KvMaps& maps, int b, int g, int tok0,
                                               int tok_end, int ntiles, unsigned char* stages, uint64_t* full,
                                               uint64_t* empty, uint32_t* abort, bool use_tma, int lane,
@@ -162,20 +164,20 @@ __device__ __forceinline__ void produce_tiles(const KvView& kv, const KvMaps& ma
       }
     }
     unsigned char* kd = stages + (size_t)s * STAGE_BYTES;
-    unsigned char* vd = WITH_V ? kd + kTileBytesKV : nullptr;
-    const int tok = tok0 + tile * kTileTok;
+    unsigned char* vd = WITH_V ? kd + 2 * TT * 128 : nullptr;
+    const int tok = tok0 + tile * TT;
     if (use_tma) {
       // the expected bytes must be registered before the loads can complete the phase
-      const int rows = min(kTileTok, tok_end - tok);
+      const int rows = min(TT, tok_end - tok);
       const uint32_t want = (uint32_t)((rows + bp - 1) / bp) * kLoadsPerBox * bp * 128;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], want);
       __syncwarp();
-      const uint32_t got = tile_issue_tma(kv, &maps.k, &maps.v, br, b, g, tok0, tok_end, tile, kd, vd, &full[s], lane,
-                                          status);
+      const uint32_t got = tile_issue_tma<TT>(kv, &maps.k, &maps.v, br, b, g, tok0, tok_end, tile, kd, vd, &full[s],
+                                              lane, status);
       // boxes skipped for a bad page never arrive: complete their bytes so the phase ends
       if (lane == 0 && got < want) mbar_complete_tx(&full[s], want - got);
     } else {
-      tile_issue_cpasync(kv, b, g, tok, tok_end, kd, vd, lane, status);
+      tile_issue_cpasync<TT>(kv, b, g, tok, tok_end, kd, vd, lane, status);
       cp_async_mbar_arrive(&full[s]);
     }
     issued = tile + 1;

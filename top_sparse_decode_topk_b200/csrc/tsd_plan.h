@@ -96,7 +96,10 @@ struct DensePlan {
 
 constexpr int kDenseMaxLists = 16;
 constexpr int kDnCtasPerSm = 3;    // resident dense-decode CTAs per SM (its launch bounds)
-constexpr int kScCtasPerSm = 5;    // resident top-k scoring CTAs per SM (its launch bounds)
+constexpr int kScCtasPerSm = 5;    // resident top-k scoring CTAs per SM, warp-MMA kernel (its launch bounds)
+constexpr int kScTcCtasPerSm = 5;  // the same for the tcgen05 scoring kernel
+constexpr int kScoreCtasPerSm = kScCtasPerSm;
+static_assert(kScTcCtasPerSm == kScCtasPerSm, "both scoring kernels share one window plan");
 constexpr int kStreamWaves = 2;
 
 inline DensePlan plan_dense(const Shapes& s, int64_t slots) {

@@ -20,10 +20,13 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 #include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "tsd_args.h"
 #include "tsd_common.cuh"
 #include "tsd_kvtile.cuh"
+#include "tsd_umma.cuh"
 
 namespace tsd {
 
@@ -136,6 +139,189 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
     // the stores consume every fragment read from the stage: release it to the producer
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[tile % kScStages]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Scoring on the fifth-generation tensor cores (tcgen05)
+// ---------------------------------------------------------------------------
+// The same work as topk_score_kernel with the MMA transposed: D[64 tokens x 16 lists] =
+// K_tile[64 x 128] x Q[16 x 128]^T, one tcgen05.mma (M = 64, N = 16, K = 16) per k-step,
+// issued by a single thread with both operands read from shared memory -- the K tile exactly
+// as the TMA load wrote it (K-major, 128-byte swizzle) and the query tile in the same
+// layout -- and the fp32 accumulator in tensor memory.
+//   warp 0     : TMA producer, 64-token K tiles into a 2-stage ring;
+//   warp 1     : allocates 32 tensor-memory columns (two 16-column accumulators) and, from one
+//                lane, issues the MMAs of each tile and commits them to the stage's "empty"
+//                barrier and the accumulator's "full" barrier;
+//   warps 2..5 : epilogue: with M = 64, rows 16 q .. 16 q + 15 of the accumulator sit in
+//                tensor-memory lanes 32 q .. 32 q + 15, so the warp reading lane quarter q
+//                gets 16 tokens x 16 lists with tcgen05.ld, releases the accumulator and stores
+//                the lists' scores.
+// Every wait is bounded; on a timeout the CTA flags TSD_DEV_TIMEOUT, drains the MMAs it issued
+// and frees its tensor memory before returning.
+// Measured against topk_score_kernel on llama3_8b (top-k leg, CUDA events): 155.6 vs 144.4 us
+// at 5 CTAs per SM (M = 128 tiles at 3 CTAs per SM: 171.0 us).  The kernel is bound by the K
+// stream, and the extra hop through the MMA issuer and tensor memory costs more than the
+// warp-level MMAs it replaces, so it is selected only with TSD_SCORE_KERNEL=tcgen05.
+constexpr int kTcTile = 64;                        // tokens per tile = the MMA's M (64 or 128)
+constexpr int kTcStages = 2;
+constexpr int kTcStageBytes = 2 * kTcTile * 128;   // two 128-byte halves of kTcTile rows
+constexpr int kTcThreads = 192;
+constexpr int kTcCtasPerSm = kScTcCtasPerSm;
+// Accumulator rows per tensor-memory lane quarter: with M = 128 row r is lane r; with M = 64
+// rows 16 q .. 16 q + 15 sit in lanes 32 q .. 32 q + 15 (the single-CTA M = 64 layout).
+constexpr int kTcRowsPerQuarter = kTcTile / 4;
+constexpr uint32_t kTcCols = 32;
+
+template <bool QF32>
+struct TcLayout {
+  static constexpr size_t qhi = (size_t)kTcStages * kTcStageBytes;
+  static constexpr size_t qlo = qhi + kQTileBytes;
+  static constexpr size_t bars = qhi + (QF32 ? 2 : 1) * kQTileBytes;
+  static constexpr size_t lists = bars + (2 * kTcStages + 4) * sizeof(uint64_t) + 16;   // score rows, lengths
+  static constexpr size_t bytes = lists + 16 * sizeof(int64_t) + 16 * sizeof(int);
+};
+static_assert(TcLayout<true>::bytes + 1024 <= 228 * 1024 / kTcCtasPerSm, "tensor-core scoring CTAs per SM");
+
+template <bool QF32>
+__global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
+    topk_score_tc_kernel(TopkArgs a, const __grid_constant__ KvMaps maps) {
+  using Lay = TcLayout<QF32>;
+  extern __shared__ __align__(1024) unsigned char smem_tc[];
+  unsigned char* stages = smem_tc;
+  unsigned char* qhi = smem_tc + Lay::qhi;
+  unsigned char* qlo = smem_tc + Lay::qlo;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_tc + Lay::bars);
+  uint64_t* empty = full + kTcStages;
+  uint64_t* accf = empty + kTcStages;
+  uint64_t* acce = accf + 2;
+  uint32_t* abort_flag = reinterpret_cast<uint32_t*>(acce + 2);
+  uint32_t* tmem_slot = abort_flag + 1;
+  int64_t* s_srow = reinterpret_cast<int64_t*>(smem_tc + Lay::lists);
+  int* s_kvl = reinterpret_cast<int*>(s_srow + 16);
+  const int win = blockIdx.x;
+  const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, win == 0 && g == 0 && lg == 0 && threadIdx.x == 0);
+  const int G = a.qv.hq / a.kv.hkv;
+  int nlists = si.n * G - lg * a.lists_per_cta;
+  if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
+  if (nlists <= 0) return;
+  const int tok0 = win * a.window;
+  const int tok_end = min(tok0 + a.window, si.len);
+  if (tok_end <= tok0) return;
+  const int ntiles = (tok_end - tok0 + kTcTile - 1) / kTcTile;
+  const bool use_tma = a.kv.page_table == nullptr || a.kv.page_shift >= 3;
+  if (smem_u32(stages) & 1023u) {   // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) flag_status(a.status, TSD_DEV_TIMEOUT);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full[s], use_tma ? 1 : 32);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&accf[s], 1);
+      mbar_init(&acce[s], 4);
+    }
+    mbar_fence_init();
+    *abort_flag = 0;
+  }
+  if (threadIdx.x < 16) {
+    const int m = threadIdx.x;
+    s_kvl[m] = 0;
+    s_srow[m] = 0;
+    if (m < nlists) {
+      const int mg = lg * a.lists_per_cta + m;
+      const int j = mg / G;
+      s_kvl[m] = min(kv_len_of(a.qv, si, j), tok_end);
+      s_srow[m] = ((int64_t)(si.t0 + j) * a.qv.hq + g * G + (mg - j * G)) * a.score_stride;
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTcCols);
+    tmem_relinquish();
+  }
+  store_q_tile(a.qv, si, g, G, lg * a.lists_per_cta, nlists, qhi, QF32 ? qlo : nullptr, threadIdx.x, kTcThreads);
+  // the query tile is read by the tensor cores (async proxy): order the generic stores first
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    produce_tiles<kTcStages, kTcStageBytes, false, kTcTile>(a.kv, maps, b, g, tok0, tok_end, ntiles, stages, full,
+                                                            empty, abort_flag, use_tma, lane, a.status);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(kTcTile, 16);
+      const uint32_t qh = smem_u32(qhi), ql = smem_u32(qlo);
+      int issued = 0;
+      for (int tile = 0; tile < ntiles; ++tile) {
+        const int s = tile % kTcStages, acc = tile & 1;
+        bool ok = mbar_wait(&full[s], (tile / kTcStages) & 1);
+        if (ok && tile >= 2) ok = mbar_wait(&acce[acc], ((tile >> 1) - 1) & 1);
+        if (!ok || *reinterpret_cast<volatile uint32_t*>(abort_flag)) {
+          if (!ok) {
+            flag_status(a.status, TSD_DEV_TIMEOUT);
+            atomicOr(abort_flag, 1u);
+          }
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t kb = smem_u32(stages + (size_t)s * kTcStageBytes);
+        const uint32_t d = tmem + (uint32_t)(acc * 16);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t oa = (uint32_t)((ks >> 2) * (kTcTile * 128) + (ks & 3) * 32);
+          const uint32_t ob = (uint32_t)((ks >> 2) * kQHalfBytes + (ks & 3) * 32);
+          umma_bf16(d, sw128_desc(kb + oa, 1024), sw128_desc(qh + ob, 1024), idesc, ks > 0);
+          if (QF32) umma_bf16(d, sw128_desc(kb + oa, 1024), sw128_desc(ql + ob, 1024), idesc, true);
+        }
+        umma_commit(&empty[s]);   // the stage may be refilled once these MMAs have read it
+        umma_commit(&accf[acc]);  // the accumulator is ready
+        issued = tile + 1;
+      }
+      // no MMA may be in flight when tensor memory is freed
+      if (issued > 0 && !mbar_wait(&accf[(issued - 1) & 1], ((issued - 1) >> 1) & 1))
+        flag_status(a.status, TSD_DEV_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3;   // this warp's 32 tensor-memory lanes: tokens 32 q .. 32 q + 31
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int acc = tile & 1;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&accf[acc], (tile >> 1) & 1);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) {
+        if (lane == 0) flag_status(a.status, TSD_DEV_TIMEOUT);
+        break;
+      }
+      tc_fence_after_sync();
+      uint32_t r[16];
+      tmem_ld16(tmem + (uint32_t)(acc * 16) + ((uint32_t)(32 * quarter) << 16), r);
+      tmem_wait_ld();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[acc]);
+      const int tok = tok0 + tile * kTcTile + kTcRowsPerQuarter * quarter + lane;
+      if (lane < kTcRowsPerQuarter) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          if (m < nlists && tok < s_kvl[m]) a.scores[s_srow[m] + tok] = __uint_as_float(r[m]);
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTcCols);
   }
 }
 
@@ -500,6 +686,14 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
+// Which scoring kernel runs: the warp-level mma.sync kernel (default, the faster one on the
+// measured workloads), or with TSD_SCORE_KERNEL=tcgen05 in the environment the tcgen05
+// kernel.  Both use 5 CTAs per SM, so the window plan is the same.
+static bool score_on_tcgen05() {
+  const char* e = getenv("TSD_SCORE_KERNEL");
+  return e != nullptr && strcmp(e, "tcgen05") == 0;
+}
+
 cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int batch, int hkv, int num_lists,
                         cudaStream_t stream) {
   static bool configured = false;
@@ -510,12 +704,24 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
       e = cudaFuncSetAttribute(topk_score_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)ScLayout<true, kScStages>::bytes);
     if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)TcLayout<false>::bytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topk_score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)TcLayout<true>::bytes);
+    if (e == cudaSuccess)
       e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SelectSmem));
     if (e != cudaSuccess) return e;
     configured = true;
   }
   dim3 g1(nwin, hkv * a.list_groups, batch);
-  if (a.qv.q_f32) {
+  if (score_on_tcgen05()) {
+    if (a.qv.q_f32) {
+      topk_score_tc_kernel<true><<<g1, kTcThreads, TcLayout<true>::bytes, stream>>>(a, maps);
+    } else {
+      topk_score_tc_kernel<false><<<g1, kTcThreads, TcLayout<false>::bytes, stream>>>(a, maps);
+    }
+  } else if (a.qv.q_f32) {
     topk_score_kernel<true><<<g1, kScThreads, ScLayout<true, kScStages>::bytes, stream>>>(a, maps);
   } else {
     topk_score_kernel<false><<<g1, kScThreads, ScLayout<false, kScStages>::bytes, stream>>>(a, maps);
