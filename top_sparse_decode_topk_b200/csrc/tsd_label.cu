@@ -140,7 +140,7 @@ __global__ void label_build_kernel(KvView kv, const int32_t* channels, int r, in
 template <int R>
 __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, const uint16_t* label,
                                                                   const int32_t* channels) {
-  __shared__ float qs[16][R];
+  __shared__ __align__(16) float qs[16][R];
   __shared__ int kvl[16];
   __shared__ int64_t srow[16];
   const int win = blockIdx.x;
@@ -203,10 +203,14 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
       for (int c = 0; c < R / 8; ++c) unpack8(raw[u][c], kf + 8 * c);
       for (int m = 0; m < nlists; ++m) {
         float s0 = 0.f, s1 = 0.f;
+        const float4* qm = reinterpret_cast<const float4*>(qs[m]);   // 16-byte shared loads
 #pragma unroll
-        for (int j = 0; j < R; j += 2) {
-          s0 = fmaf(qs[m][j], kf[j], s0);
-          s1 = fmaf(qs[m][j + 1], kf[j + 1], s1);
+        for (int j = 0; j < R; j += 4) {
+          const float4 qv = qm[j / 4];
+          s0 = fmaf(qv.x, kf[j], s0);
+          s1 = fmaf(qv.y, kf[j + 1], s1);
+          s0 = fmaf(qv.z, kf[j + 2], s0);
+          s1 = fmaf(qv.w, kf[j + 3], s1);
         }
         if (tok < kvl[m]) a.scores[srow[m] + tok] = s0 + s1;
       }
