@@ -25,6 +25,7 @@ namespace tsd {
 
 constexpr int kStoMaxM = 1024;
 constexpr int kStoWarps = 4;
+constexpr int kStoTopCache = 2048;   // top-k lists up to this long are searched in shared memory
 
 struct StochasticArgs {
   KvView kv;
@@ -38,19 +39,27 @@ struct StochasticArgs {
   uint32_t* status;       // nullable
 };
 
-// Number of entries of the ascending list a[0..n) that are < x.
+// Number of entries of the ascending list a[0..n) that are < x (a in shared or global memory).
 __device__ __forceinline__ int count_below(const int32_t* a, int n, int x) {
   int lo = 0, hi = n;
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    if (__ldg(a + mid) < x) lo = mid + 1; else hi = mid;
+    if (a[mid] < x) lo = mid + 1; else hi = mid;
   }
   return lo;
 }
 
+struct StoSmem {
+  uint32_t kept[kStoWarps][kStoMaxM];
+  int32_t toks[kStoWarps][kStoMaxM];
+  int32_t top[kStoWarps][kStoTopCache];
+};
+
 __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(StochasticArgs a) {
-  __shared__ uint32_t kept[kStoWarps][kStoMaxM];
-  __shared__ int32_t toks[kStoWarps][kStoMaxM];
+  extern __shared__ __align__(16) unsigned char sto_smem[];
+  StoSmem& SM = *reinterpret_cast<StoSmem*>(sto_smem);
+  auto& kept = SM.kept;
+  auto& toks = SM.toks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t list = (int64_t)blockIdx.x * kStoWarps + warp;
   const int64_t nlists = (int64_t)a.qv.num_tokens * a.qv.hq;
@@ -69,14 +78,22 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
   const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, false);
   const int L = (t >= si.t0 && t < si.t0 + si.n) ? kv_len_of(a.qv, si, t - si.t0) : 0;
   const int32_t* top = a.top + list * a.k_max;
-  // valid prefix of the top-k list (entries >= 0, ascending, < L)
+  // the top list, searched many times below, is read once into shared memory when it fits;
+  // its valid prefix (entries >= 0, ascending, < L) is then checked there
+  const int32_t* topc = top;
+  if (a.k_max <= kStoTopCache) {
+#pragma unroll 4
+    for (int i = lane; i < a.k_max; i += 32) SM.top[warp][i] = __ldg(top + i);
+    __syncwarp();
+    topc = SM.top[warp];
+  }
   int ntop = 0;
   bool bad = false;
   for (int i = lane; i < a.k_max; i += 32) {
-    const int32_t v = __ldg(top + i);
+    const int32_t v = topc[i];
     if (v >= 0) {
       ntop = i + 1;
-      bad |= v >= L || (i > 0 && __ldg(top + i - 1) >= v);
+      bad |= v >= L || (i > 0 && topc[i - 1] >= v);
     }
   }
 #pragma unroll
@@ -89,10 +106,15 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
   const int m = min(a.m, n);
   const uint32_t* u = a.u + list * a.m;
   uint32_t* kr = kept[warp];
+  // the random words go to shared memory first (the token array is free until the mapping),
+  // so that Floyd's sequential steps do not wait on global loads
+  uint32_t* us = reinterpret_cast<uint32_t*>(toks[warp]);
+  for (int s = lane; s < m; s += 32) us[s] = __ldg(u + s);
+  __syncwarp();
   // ---- Floyd: step j = n - m .. n - 1 keeps t = u mod (j + 1), or j on a collision ----
   for (int s = 0; s < m; ++s) {
     const uint32_t j = (uint32_t)(n - m + s);
-    const uint32_t tr = (uint32_t)(__ldg(u + s) % (j + 1u));
+    const uint32_t tr = us[s] % (j + 1u);
     bool seen = false;
     for (int i = lane; i < s; i += 32) seen |= kr[i] == tr;
     seen = __any_sync(0xFFFFFFFFu, seen);
@@ -109,7 +131,7 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
     int lo = 0, hi = ntop;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (__ldg(top + mid) - mid > (int)r) hi = mid; else lo = mid + 1;
+      if (topc[mid] - mid > (int)r) hi = mid; else lo = mid + 1;
     }
     tk[pos] = (int32_t)r + lo;
   }
@@ -120,7 +142,7 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
   float* ow = a.out_logw + list * width;
   const float lw = m > 0 ? logf((float)n / (float)m) : 0.f;
   for (int i = lane; i < ntop; i += 32) {
-    const int32_t v = __ldg(top + i);
+    const int32_t v = topc[i];
     int lo = 0, hi = m;   // sampled tokens below v
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
@@ -131,7 +153,7 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
   }
   for (int i = lane; i < m; i += 32) {
     const int32_t v = tk[i];
-    const int below = count_below(top, ntop, v);
+    const int below = count_below(topc, ntop, v);
     oi[i + below] = v;
     ow[i + below] = lw;
   }
@@ -157,7 +179,14 @@ cudaError_t launch_stochastic_select(const KvView& kv, const QView& qv, const in
   const int64_t nlists = (int64_t)qv.num_tokens * qv.hq;
   const int64_t grid = (nlists + kStoWarps - 1) / kStoWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
-  stochastic_select_kernel<<<(unsigned)grid, 32 * kStoWarps, 0, stream>>>(a);
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(stochastic_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(StoSmem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  stochastic_select_kernel<<<(unsigned)grid, 32 * kStoWarps, sizeof(StoSmem), stream>>>(a);
   return cudaGetLastError();
 }
 
