@@ -249,7 +249,7 @@ size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_que
 size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries) {
   Shapes sh;
   if (sizes_for(cache, queries, &sh) != TSD_OK) return 0;
-  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm * kStreamWaves);
+  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm);
   return decode_layout(sh, p.nsplit).total;
 }
 
@@ -275,7 +275,7 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
   a.score_stride = lay.score_stride;
   // scoring streams K in the dense path's tiles, with its own occupancy
-  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScoreCtasPerSm * kStreamWaves);
+  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScoreCtasPerSm);
   a.lists_per_cta = p.lists_per_cta;
   a.list_groups = p.list_groups;
   a.window = p.window;
@@ -397,7 +397,7 @@ tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* querie
   KvView kv; QView qv; Shapes sh;
   tsd_status st = decode_common(cache, queries, out, out_dtype, lse, ws, ws_bytes, &kv, &qv, &sh);
   if (st != TSD_OK) return st;
-  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm * kStreamWaves);
+  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm);
   const DecodeLayout lay = decode_layout(sh, p.nsplit);
   if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
   DecodeArgs a;
@@ -513,7 +513,7 @@ tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k,
   a.out_count = out_count;
   a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
   a.score_stride = lay.score_stride;
-  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm * kStreamWaves);
+  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm);
   a.lists_per_cta = p.lists_per_cta;
   a.list_groups = p.list_groups;
   a.window = p.window;

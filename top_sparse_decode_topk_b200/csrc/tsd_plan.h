@@ -84,9 +84,8 @@ inline SparsePlan plan_sparse(const Shapes& s, int k_max, int num_sms) {
 }
 
 // Dense decode and top-k scoring: up to 16 lists per CTA (the mma M dimension) and a window
-// of W tokens (a multiple of the 64-token tile).  Every CTA streams the same number of tiles,
-// so the grid is sized to whole waves: `slots` CTAs (resident CTAs per SM x SMs x waves), cut
-// into as many windows per (sequence, kv head, list group) as fit.
+// of W tokens (a multiple of the 64-token tile) per (sequence, kv head, list group).  `wave`
+// is the number of resident CTAs (CTAs per SM x SMs).
 struct DensePlan {
   int lists_per_cta;
   int list_groups;
@@ -100,21 +99,48 @@ constexpr int kScCtasPerSm = 5;    // resident top-k scoring CTAs per SM, warp-M
 constexpr int kScTcCtasPerSm = 5;  // the same for the tcgen05 scoring kernel
 constexpr int kScoreCtasPerSm = kScCtasPerSm;
 static_assert(kScTcCtasPerSm == kScCtasPerSm, "both scoring kernels share one window plan");
-constexpr int kStreamWaves = 2;
+constexpr int64_t kMaxWindow = 8192;   // tokens per dense / scoring CTA at most
 
-inline DensePlan plan_dense(const Shapes& s, int64_t slots) {
+// Window of `ns` windows over max_seq_len, rounded up to whole 64-token tiles.
+inline int64_t dense_window(int64_t max_seq_len, int64_t ns) {
+  const int64_t w = (max_seq_len + ns - 1) / ns;
+  return (w + 63) / 64 * 64;
+}
+
+inline DensePlan plan_dense(const Shapes& s, int64_t wave) {
   DensePlan p;
   const int64_t m = s.group * s.max_tokens;
   p.lists_per_cta = (int)(m < kDenseMaxLists ? m : kDenseMaxLists);
   p.list_groups = (int)((m + p.lists_per_cta - 1) / p.lists_per_cta);
   const int64_t units = s.batch * s.hkv * p.list_groups;
-  int64_t ns = slots / units;
-  const int64_t max_ns = (s.max_seq_len + 63) / 64;
+  int64_t max_ns = (s.max_seq_len + 63) / 64;
+  if (max_ns > kMaxSplits) max_ns = kMaxSplits;
+  if (max_ns < 1) max_ns = 1;
+  // Every CTA streams about the same number of tiles: size the grid to two whole waves of
+  // `wave` resident CTAs.
+  int64_t ns = 2 * wave / units;
   if (ns > max_ns) ns = max_ns;
-  if (ns > kMaxSplits) ns = kMaxSplits;
   if (ns < 1) ns = 1;
-  int64_t w = (s.max_seq_len + ns - 1) / ns;
-  w = (w + 63) / 64 * 64;
+  if (dense_window(s.max_seq_len, ns) > kMaxWindow) {
+    // Few units over a long max_seq_len (a large or ragged batch).  Windows are sized on
+    // max_seq_len while sequences may be much shorter (windows past a sequence's end exit at
+    // once), and a long sequence cut into few windows leaves its CTAs running alone at the
+    // end: cap the window at kMaxWindow and, above that floor, take the split count whose
+    // whole waves x (window + one tile of merge and prologue) is least.
+    int64_t lo = (s.max_seq_len + kMaxWindow - 1) / kMaxWindow;
+    if (lo > max_ns) lo = max_ns;
+    int64_t hi = 4 * wave / units + 1;
+    if (hi > max_ns) hi = max_ns;
+    if (hi < lo) hi = lo;
+    int64_t best = -1;
+    for (int64_t n = lo; n <= hi; ++n) {
+      const int64_t w = dense_window(s.max_seq_len, n);
+      const int64_t nse = (s.max_seq_len + w - 1) / w;
+      const int64_t cost = ((units * nse + wave - 1) / wave) * (w + 64);
+      if (best < 0 || cost < best) { best = cost; ns = n; }
+    }
+  }
+  const int64_t w = dense_window(s.max_seq_len, ns);
   p.window = (int)w;
   p.nsplit = (int)((s.max_seq_len + w - 1) / w);
   return p;
