@@ -69,8 +69,26 @@ def workload_desc(cfg, k):
         "workload": f"{cfg.name}: {cfg.description}",
         "batch": cfg.batch, "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": 128,
         "context": cfg.max_seq_len, "k": k, "tokens_per_seq": cfg.tokens_per_seq,
-        "l2": "flushed before every timed leg (256 MiB device write)",
+        "l2": "flushed before every timed leg: 256 MiB device write, then a 256 MiB read (no input, and "
+              "none of the flush's dirty lines, left in L2)",
     }
+
+
+class L2Flush:
+    """Evict L2 (126 MB on B200) before a timed leg: write a 256 MiB buffer, then read another
+    256 MiB one.  The read pushes the write's dirty lines out of L2 too, so the timed kernel
+    neither finds its inputs in L2 nor pays for writing back lines the flush left dirty."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(32 << 20, dtype=torch.int64, device=dev)
+        self.sink = torch.zeros((), dtype=torch.int64, device=dev)
+
+    def __call__(self):
+        import torch
+        self.w.fill_(1)
+        torch.sum(self.r, dim=0, out=self.sink)
 
 
 # ---------------------------------------------------------------------------
@@ -356,7 +374,7 @@ def run_native(args):
     out_dtype = torch.float32 if cfg.out_dtype == "f32" else torch.bfloat16
     ws = tsd.Workspace(dev)
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     idx_buf = torch.empty((len(w.kv_len), cfg.num_q_heads, k_max), dtype=torch.int32, device=dev)
     cnt_buf = torch.empty((len(w.kv_len), cfg.num_q_heads), dtype=torch.int32, device=dev)
 
@@ -372,7 +390,7 @@ def run_native(args):
     legs = [leg_topk, leg_sparse, leg_dense]
     for _ in range(max(3, args.warmup)):
         for leg in legs:
-            flush.fill_(1)
+            flush()
             leg()
     torch.cuda.synchronize()
     if tsd.read_device_status(ws) != 0:
@@ -385,7 +403,7 @@ def run_native(args):
     with ClockSampler(local) as clocks:
         for s in range(args.steps):
             for j, leg in enumerate(legs):
-                flush.fill_(1)
+                flush()
                 ev[s][2 * j].record(stream)
                 leg()
                 ev[s][2 * j + 1].record(stream)
@@ -423,7 +441,7 @@ def run_native(args):
     def timed(fn, reps):
         out = []
         for _ in range(reps):
-            flush.fill_(1)
+            flush()
             a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a_.record(stream)
             fn()
@@ -524,12 +542,12 @@ def run_native(args):
                      causal=cfg.causal, sm_scale=scale)
     e2e_ms, e2e_idx_ms = [], []
     for s in range(args.warmup + args.steps):
-        flush.fill_(1)
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         tsd.sparse_decode(cache, hq, idx_host, out=out_host, lse=lse_host, workspace=ws)
         b.record(stream)
-        flush.fill_(1)
+        flush()
         c, d = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         c.record(stream)
         idx_d, _ = tsd.topk_select(cache, hq, k_max, k_per_token=kpt_dev, out_idx=idx_buf, out_count=cnt_buf,

@@ -166,314 +166,414 @@ __device__ void finish_lists(const DecodeArgs& a, const SeqInfo& si, int b, int 
 // Sparse decode
 // ---------------------------------------------------------------------------
 // Design, from measurements on B200:
-//  * Scattered 256-byte rows are gathered with 16-byte copies: lane l of a half-warp copies
-//    chunk l of each K and V row.  The copies go through a per-half-warp ring of kSpStages
-//    batches in shared memory (cp.async), so 12 rows are in flight per half-warp without
-//    spending registers on them.  Each lane reads back only what it copied itself, so the
-//    ring needs no synchronisation beyond each lane's own cp.async wait.  Against gathering
-//    into registers (4 rows in flight, 3 CTAs/SM) this measured 30.7 vs 32.8 us on
-//    llama3_8b.
-//  * What sets the gather rate is how many loads are in flight, so the work is cut into many
-//    small independent tasks: one half-warp (16 lanes x 16 bytes = one row) takes a chunk of
-//    E entries of one list (token x q head) and nothing else, and the plan sizes E so the
-//    grid fits one wave of resident CTAs.
-//  * Tasks are numbered (sequence, kv head, chunk, list) so that the lists of one kv head
-//    -- the q heads of a GQA group and the decode tokens of the sequence -- read the same
-//    token range in the same CTA at the same time: a row picked by several of them is
-//    read from DRAM once and served to the others from L2.
-// Per row the half-warp computes a 128-dim dot (8 FMA per lane + a 4-step shuffle
-// reduction); its online softmax state (max, sum, 8 output dims per lane) is updated once
-// per batch of U rows.  The chunks of a list held by one CTA are combined in shared memory;
-// each CTA then writes one partial per list, and the last CTA of a list to arrive (a per-list
-// counter) merges them with log-sum-exp.  A list that fits one CTA is written directly.
-constexpr int kSpThreads = 256;   // 16 half-warps, one task each
-constexpr int kSpU = 4;           // rows per softmax batch
-constexpr int kSpStages = 3;      // batches in flight per half-warp (cp.async ring)
-constexpr size_t kSpRingBytes = (size_t)16 * kSpStages * 2 * kSpU * 16 * sizeof(uint4);   // 96 KB
+//  * One warp per task: a chunk of E entries of one list (token x q head).  The plan sizes E
+//    so that the grid fits one wave of resident CTAs; the CTA's warps take consecutive
+//    chunks of a list, which are combined in shared memory before anything leaves the CTA.
+//  * The task's rows are gathered 16 at a time (a tile: 16 K rows then 16 V rows, 256 bytes
+//    each) into a per-warp ring of kSpStages tiles in shared memory with 16-byte cp.async
+//    copies; rows that are not there (padding, -1 entries, bad pages) are zero-filled by the
+//    same copies.  Entries are resolved a window of 32 (one per lane) at a time, and two
+//    windows ahead: the page-table rows of window w + 2 and the raw indices of window w + 3
+//    are in flight while window w's tiles are consumed, so a tile's rows are known a whole
+//    window before its copies are issued.
+//  * Both contractions of a tile run on the tensor cores (mma.m16n8k16, bf16 in, fp32
+//    accumulate), with the unused columns of the n = 8 operand carrying a second bf16 part:
+//      scores  S(16 rows x 8) = K(16 x 128) . [q_hi, q_lo, 0 ...]    (columns 0 and 1 summed)
+//      output  O^T(128 x 8) += V^T(128 x 16) . [P_hi, P_lo, 0 ...]   (columns 0 and 1 summed)
+//    where x_hi = bf16(x) and x_lo = bf16(x - x_hi), so an fp32 q and the fp32 softmax
+//    weights enter with about 16 significant bits.  Against one CUDA-core dot product per
+//    row and half-warp this cuts the instructions per gathered row about fivefold.
+//  * Online softmax in base-2 units with a lazily moved reference: the running maximum is
+//    only raised (and the state rescaled) when a tile exceeds it by more than 2^8, so most
+//    tiles skip the rescale; weights then stay below 2^8.
+// The CTA's per-task states of a list are combined in shared memory; each CTA then writes one
+// partial per list, and the last CTA of a list to arrive (a per-list counter) merges them with
+// log-sum-exp.  A list held by one CTA alone is written directly.
+constexpr int kSpWarps = kSpTasksPerCta;
+constexpr int kSpThreads = 32 * kSpWarps;
+constexpr int kSpTileRows = 16;
+constexpr int kSpHalfBytes = kSpTileRows * kHeadDim * 2;   // 16 rows of K (or V): 4 KB
+constexpr int kSpTileBytes = 2 * kSpHalfBytes;
+constexpr size_t kSpRingBytes = (size_t)kSpWarps * kSpStages * kSpTileBytes;
+constexpr float kSpLazyMax = 8.f;   // base-2 units the running maximum may lag behind
+static_assert(kSpStages >= 2 && kSpStages <= 3, "the ring looks at most one window (two tiles) ahead");
+static_assert(kSpCtasPerSm * (kSpRingBytes + 2048) <= 228 * 1024, "resident sparse CTAs per SM");
 
-__device__ __forceinline__ void row_fetch(const DecodeArgs& a, uint32_t row, int l, uint4& k, uint4& v) {
-  if (row != kInvalidRow) {
-    k = __ldg(reinterpret_cast<const uint4*>(a.kv.k + (int64_t)row * kHeadDim) + l);
-    v = __ldg(reinterpret_cast<const uint4*>(a.kv.v + (int64_t)row * kHeadDim) + l);
+// Byte offset of 16-byte chunk c of row r in a tile of 256-byte rows, the chunk index XOR-ed
+// with (r mod 8): the 8 rows one ldmatrix phase reads fall in 8 different bank groups.
+__device__ __forceinline__ uint32_t sp_off(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 7)) << 4)); }
+
+// 16-byte cp.async that writes zeros (and reads nothing) when !valid.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t smem, const void* gmem, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem), "l"(gmem), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+// Four consecutive output dims [d, d + 4) of (token t, q head h).
+__device__ __forceinline__ void store_out4(const DecodeArgs& a, int t, int h, int d, float4 v) {
+  const int64_t o = ((int64_t)t * a.qv.hq + h) * kHeadDim + d;
+  if (a.out_f32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + o) = v;
+  } else {
+    uint2 w;
+    w.x = (uint32_t)f32_to_bf16_rne(v.x) | ((uint32_t)f32_to_bf16_rne(v.y) << 16);
+    w.y = (uint32_t)f32_to_bf16_rne(v.z) | ((uint32_t)f32_to_bf16_rne(v.w) << 16);
+    *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + o) = w;
   }
 }
 
-// Online-softmax update of a half-warp's state with a batch of U rows at once: the U
-// scores are reduced together (independent shuffle chains), then one max, one rescale
-// and U independent exponentials -- the serial chain is per batch, not per row.
-template <int U, bool BIAS>
-__device__ __forceinline__ void batch_update(const uint4* kq, const uint4* vq, const uint32_t* rr, const float* bias,
-                                             const float* q, float& m_run, float& l_run, float* acc, unsigned hmask) {
-  float s[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    float kf[8];
-    unpack8(kq[u], kf);
-    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      s0 = fmaf(q[j], kf[j], s0);
-      s1 = fmaf(q[j + 1], kf[j + 1], s1);
-    }
-    s[u] = s0 + s1;
-  }
-#pragma unroll
-  for (int o = 1; o < 16; o <<= 1)
-#pragma unroll
-    for (int u = 0; u < U; ++u) s[u] += __shfl_xor_sync(hmask, s[u], o);
-  if (BIAS) {   // entry weights: p_i = w_i exp(s_i), with ln w_i in base-2 units
-#pragma unroll
-    for (int u = 0; u < U; ++u) s[u] += bias[u];
-  }
-  float mb = -CUDART_INF_F;
-#pragma unroll
-  for (int u = 0; u < U; ++u)
-    if (rr[u] != kInvalidRow) mb = fmaxf(mb, s[u]);
-  if (mb == -CUDART_INF_F) return;   // no valid row in the batch (uniform over the half-warp)
-  const float m_new = fmaxf(m_run, mb);
-  const float alpha = fast_exp2(m_run - m_new);   // 0 on the first batch (m_run = -inf)
-  l_run *= alpha;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] *= alpha;
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const float p = rr[u] != kInvalidRow ? fast_exp2(s[u] - m_new) : 0.f;
-    l_run += p;
-    float vf[8];
-    unpack8(vq[u], vf);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = fmaf(p, vf[j], acc[j]);
-  }
-  m_run = m_new;
-}
-
-// End of a list's work in one CTA: a list whose tasks all ran in this CTA is written
-// directly; otherwise this CTA's partial state (partial c of C) is stored, and the last CTA
-// of the list to arrive (per-list counter) merges the C partials with log-sum-exp.  Called
-// by the 16 lanes of one half-warp (hmask), lane l holding output dims [8l, 8l+8).
-__device__ __forceinline__ void finish_task(const DecodeArgs& a, int64_t list_id, int t, int h, int C, int c,
-                                            float m_run, float l_run, const float* acc, int l, unsigned hmask) {
-  if (C == 1) {   // the whole list in one CTA
+// End of a list's work in one CTA, by one warp (lane l holding output dims [4l, 4l + 4)): a
+// list whose chunks all ran in this CTA is written directly; otherwise this CTA's partial
+// state (partial c of C) is stored, and the last CTA of the list to arrive (per-list counter)
+// merges the C partials with log-sum-exp.
+__device__ __forceinline__ void finish_list(const DecodeArgs& a, int64_t list_id, int t, int h, int C, int c,
+                                            float m_run, float l_run, float4 acc, int l) {
+  if (C == 1) {
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, acc[i] * inv);
+    store_out4(a, t, h, 4 * l, make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
     if (l == 0 && a.lse != nullptr) a.lse[list_id] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -CUDART_INF_F;
     return;
   }
-  // partial of this task, then the per-list arrival count
   const int64_t pidx = list_id * a.nsplit + c;
   if (l == 0) a.part_ml[pidx] = make_float2(m_run, l_run);
-  float4* pa = reinterpret_cast<float4*>(a.part_acc + pidx * kHeadDim + 8 * l);
-  pa[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  pa[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  reinterpret_cast<float4*>(a.part_acc + pidx * kHeadDim)[l] = acc;
   __threadfence();
-  __syncwarp(hmask);
+  __syncwarp();
   uint32_t prev = 0;
   if (l == 0) {
     prev = atomicAdd(a.counters + list_id, 1u);
     if (prev == (uint32_t)(C - 1)) atomicExch(a.counters + list_id, 0u);   // leave it zero for the next call
   }
-  prev = __shfl_sync(hmask, prev, 0, 16);
+  prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
   if (prev != (uint32_t)(C - 1)) return;
   __threadfence();
-  // last task of the list: merge its C partials (lanes over splits for the max and sum,
-  // then 8 output dims per lane with independent loads)
+  // last CTA of the list: max and sum over the C partials (lanes over partials), then 4 dims
+  // per lane with 8 independent loads in flight
   const float2* ml = a.part_ml + list_id * a.nsplit;
   float mx = -CUDART_INF_F;
-  for (int i = l; i < C; i += 16) mx = fmaxf(mx, __ldcg(&ml[i]).x);
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 2));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 8));
-  float L = 0.f;
-  float o[8];
+  for (int i = l; i < C; i += 32) mx = fmaxf(mx, __ldcg(&ml[i]).x);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  float L = 0.f;
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
   if (mx != -CUDART_INF_F) {
-    for (int i = l; i < C; i += 16) {
+    for (int i = l; i < C; i += 32) {
       const float2 x = __ldcg(&ml[i]);
       L = fmaf(fast_exp2(x.x - mx), x.y, L);
     }
-    L += __shfl_xor_sync(hmask, L, 1);
-    L += __shfl_xor_sync(hmask, L, 2);
-    L += __shfl_xor_sync(hmask, L, 4);
-    L += __shfl_xor_sync(hmask, L, 8);
-    for (int c0 = 0; c0 < C; c0 += 4) {
-      float w[4];
-      float4 x0[4], x1[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int cc = c0 + u;
-        w[u] = cc < C ? fast_exp2(__ldcg(&ml[cc]).x - mx) : 0.f;
-        const float4* src =
-            reinterpret_cast<const float4*>(a.part_acc + (list_id * a.nsplit + (cc < C ? cc : 0)) * kHeadDim + 8 * l);
-        x0[u] = __ldcg(src);
-        x1[u] = __ldcg(src + 1);
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+    const float4* src = reinterpret_cast<const float4*>(a.part_acc + list_id * a.nsplit * kHeadDim) + l;
+    for (int c0 = 0; c0 < C; c0 += 8) {
+      float w[8];
+      float4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int cc = c0 + u < C ? c0 + u : C - 1;
+        w[u] = c0 + u < C ? fast_exp2(__ldcg(&ml[cc]).x - mx) : 0.f;
+        x[u] = __ldcg(src + (int64_t)cc * (kHeadDim / 4));
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        o[0] = fmaf(w[u], x0[u].x, o[0]); o[1] = fmaf(w[u], x0[u].y, o[1]);
-        o[2] = fmaf(w[u], x0[u].z, o[2]); o[3] = fmaf(w[u], x0[u].w, o[3]);
-        o[4] = fmaf(w[u], x1[u].x, o[4]); o[5] = fmaf(w[u], x1[u].y, o[5]);
-        o[6] = fmaf(w[u], x1[u].z, o[6]); o[7] = fmaf(w[u], x1[u].w, o[7]);
+      for (int u = 0; u < 8; ++u) {
+        r.x = fmaf(w[u], x[u].x, r.x); r.y = fmaf(w[u], x[u].y, r.y);
+        r.z = fmaf(w[u], x[u].z, r.z); r.w = fmaf(w[u], x[u].w, r.w);
       }
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) store_out(a, t, h, 8 * l + i, o[i] * inv);
+  store_out4(a, t, h, 4 * l, make_float4(r.x * inv, r.y * inv, r.z * inv, r.w * inv));
   if (l == 0 && a.lse != nullptr) a.lse[list_id] = L > 0.f ? (mx + log2f(L)) * kLn2 : -CUDART_INF_F;
 }
 
 template <bool WEIGHTED>
 __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel(DecodeArgs a) {
-  extern __shared__ __align__(16) uint4 sp_ring[];   // [16 half-warps][kSpStages][K, V][kSpU rows][16 lanes]
-  // task states of the CTA's 16 half-warps, combined per list before anything leaves the CTA
-  __shared__ float2 s_ml[16];
-  __shared__ __align__(16) float s_acc[16][kHeadDim];
-  __shared__ int64_t s_list[16];
+  extern __shared__ __align__(128) unsigned char sp_ring[];   // [warp][kSpStages][K rows, V rows]
+  // task states of the CTA's warps, combined per list before anything leaves the CTA
+  __shared__ float2 s_ml[kSpWarps];
+  __shared__ __align__(16) float s_acc[kSpWarps][kHeadDim];
+  __shared__ int64_t s_list[kSpWarps];
+  constexpr unsigned FULL = 0xFFFFFFFFu;
   const int lane = threadIdx.x & 31;
-  const int l = threadIdx.x & 15;
-  const int hw = threadIdx.x >> 4;
-  const unsigned hmask = 0xFFFFu << (lane & 16);
+  const int warp = threadIdx.x >> 5;
   const int G = a.qv.hq / a.kv.hkv;
   const int M = a.lists_per_cta;   // list slots per (sequence, kv head): G x max tokens per sequence
   const int C = a.nsplit;          // tasks (chunks) per list
   const int E = a.span;            // entries per task
-  const int64_t task = (int64_t)blockIdx.x * 16 + hw;
-  const int64_t total = (int64_t)a.kv.batch * a.kv.hkv * C * M;
+  // tasks are numbered (sequence, kv head, list, chunk): a CTA's warps hold consecutive
+  // chunks of a list
+  const int64_t task = (int64_t)blockIdx.x * kSpWarps + warp;
+  const int64_t total = (int64_t)a.kv.batch * a.kv.hkv * M * C;
   const int64_t tk = task < total ? task : total - 1;
-  const int m = (int)(tk % M);
-  int64_t rest = tk / M;
-  const int c = (int)(rest % C);
-  rest /= C;
+  const int c = (int)(tk % C);
+  int64_t rest = tk / C;
+  const int m = (int)(rest % M);
+  rest /= M;
   const int g = (int)(rest % a.kv.hkv);
   const int b = (int)(rest / a.kv.hkv);
 
-  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, task == tk && c == 0 && g == 0 && m == 0 && l == 0);
+  // The gather's first rows wait on a chain of dependent reads (sequence -> index -> page ->
+  // row).  Without q_indptr a sequence has the single query token t = b, so the list is known
+  // before the sequence descriptor arrives: the first four windows of raw indices are loaded
+  // alongside it.
+  const int e0 = c * E;
+  const int e1 = min(e0 + E, a.k_max);
+  const int nwin = (e1 - e0 + 31) >> 5;   // windows of 32 entries (two tiles), one per lane
+  const bool early = a.qv.q_indptr == nullptr && task < total && m < G && b < a.qv.num_tokens;
+  int32_t raw0[4];
+  int32_t prev0 = -1;
+  if (early) {
+    const int32_t* lst = a.idx + ((int64_t)b * a.qv.hq + g * G + m) * a.k_max;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int e = e0 + 32 * w + lane;
+      raw0[w] = (w < nwin && e < e1) ? __ldg(lst + e) : -1;
+    }
+    if (lane == 0 && e0 > 0) prev0 = __ldg(lst + e0 - 1);
+  }
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, task == tk && c == 0 && g == 0 && m == 0 && lane == 0);
   const int j = m / G;
   const bool valid = task < total && j < si.n;   // no list for slots past this sequence's tokens
   const int t = si.t0 + j, h = g * G + (m - j * G);
   const int64_t list_id = valid ? (int64_t)t * a.qv.hq + h : -1;
-  float m_run = -CUDART_INF_F, l_run = 0.f, acc[8];
+  float m_run = -CUDART_INF_F, l_run = 0.f;   // l_run: this lane's share of the sum
+  float o[8][4];                              // O^T accumulators, m-tile i = dims [16i, 16i + 16)
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
   if (valid) {
     const int kvlen = kv_len_of(a.qv, si, j);
-    const float scale = a.qv.sm_scale * kLog2e;
-    // this lane's 8 query dims [8l, 8l+8), scaled so that dots are base-2 softmax units
-    float q[8];
+    const float scale = a.qv.sm_scale * kLog2e;   // dots -> base-2 softmax units
+    // q as the B operand of the score MMA (k = dims, n = columns): lane 4n + i holds column n,
+    // dims 16ks + 2i, +1 and 16ks + 2i + 8, +9; column 0 = bf16(q), column 1 = q - bf16(q)
+    uint32_t qb[8][2];
     {
-      const int64_t qb = list_id * kHeadDim + 8 * l;
-      if (a.qv.q_f32) {
-        const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.qv.q) + qb);
-        const float4 x = __ldg(p), y = __ldg(p + 1);
-        q[0] = x.x; q[1] = x.y; q[2] = x.z; q[3] = x.w; q[4] = y.x; q[5] = y.y; q[6] = y.z; q[7] = y.w;
-      } else {
-        unpack8(__ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.qv.q) + qb)), q);
-      }
+      const int col = lane >> 2, i2 = 2 * (lane & 3);
+      const int64_t qb0 = list_id * kHeadDim;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] *= scale;
+      for (int ks = 0; ks < 8; ++ks) {
+        qb[ks][0] = qb[ks][1] = 0u;
+        if (col < 2) {
+          const int d0 = 16 * ks + i2;
+          float x0, x1, y0, y1;
+          if (a.qv.q_f32) {
+            const float* qp = reinterpret_cast<const float*>(a.qv.q) + qb0;
+            const float2 u = __ldg(reinterpret_cast<const float2*>(qp + d0));
+            const float2 v = __ldg(reinterpret_cast<const float2*>(qp + d0 + 8));
+            x0 = u.x; x1 = u.y; y0 = v.x; y1 = v.y;
+          } else {
+            const uint16_t* qp = reinterpret_cast<const uint16_t*>(a.qv.q) + qb0;
+            const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(qp + d0));
+            const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(qp + d0 + 8));
+            x0 = bf16lo(u); x1 = bf16hi(u); y0 = bf16lo(v); y1 = bf16hi(v);
+          }
+          uint32_t h0, l0, h1, l1;
+          split_bf16(x0, x1, h0, l0);
+          split_bf16(y0, y1, h1, l1);
+          qb[ks][0] = col == 0 ? h0 : l0;
+          qb[ks][1] = col == 0 ? h1 : l1;
+        }
+      }
     }
 
     const int32_t* lst = a.idx + list_id * a.k_max;
-    const int e0 = c * E;
-    const int e1 = min(e0 + E, a.k_max);
+    const int ntile = (e1 - e0 + kSpTileRows - 1) / kSpTileRows;
     uint32_t bad = 0;
-    for (int base = e0; base < e1; base += 16) {
-      // this lane's entry: index, predecessor check, validity, physical row
-      const int e = base + l;
-      const int32_t v = e < e1 ? __ldg(lst + e) : -1;
-      uint32_t before = __shfl_up_sync(hmask, (uint32_t)v, 1, 16);
-      if (l == 0 && e > 0 && e < e1) before = (uint32_t)__ldg(lst + e - 1);
-      if (e < e1 && e > 0 && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
-      if (e < e1 && (v < -1 || v >= kvlen)) bad |= TSD_DEV_BAD_INDEX;
+    auto load_raw = [&](int wi) -> int32_t {   // raw index of entry e0 + 32 wi + lane, -1 past the end
+      const int e = e0 + 32 * wi + lane;
+      return (wi < nwin && e < e1) ? __ldg(lst + e) : -1;
+    };
+    auto load_lw = [&](int wi) -> float {      // its weight, base-2 units
+      const int e = e0 + 32 * wi + lane;
+      return (WEIGHTED && wi < nwin && e < e1) ? __ldg(a.logw + list_id * a.k_max + e) * kLog2e : 0.f;
+    };
+    // window wi's raw indices -> physical rows, with the order / range / page checks; `prev`
+    // is (in lane 0) the raw index of the entry before the window
+    auto resolve = [&](int wi, int32_t v, int32_t prev) -> uint32_t {
+      const int e = e0 + 32 * wi + lane;
+      uint32_t before = __shfl_up_sync(FULL, (uint32_t)v, 1);
+      if (lane == 0) before = (uint32_t)prev;
+      const bool in = wi < nwin && e < e1;
+      if (in && e > 0 && (uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
+      if (in && (v < -1 || v >= kvlen)) bad |= TSD_DEV_BAD_INDEX;
       uint32_t row = kInvalidRow;
-      if (e < e1 && v >= 0 && v < kvlen) {
+      if (in && v >= 0 && v < kvlen) {
         row = kv_row(a.kv, b, g, v);
         if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
       }
-      float lw = 0.f;
-      if (WEIGHTED && e < e1) lw = __ldg(a.logw + list_id * a.k_max + e) * kLog2e;
-      // the 16 rows, kSpU at a time, through this half-warp's ring of kSpStages stages in
-      // shared memory (cp.async): lane l copies, and later reads, chunk l of every row, so the
-      // ring needs no synchronisation beyond each lane's own cp.async wait
-      uint4* ring = sp_ring + (size_t)hw * kSpStages * 2 * kSpU * 16;
-      auto issue = [&](int bt) {
-        uint4* st = ring + (size_t)(bt % kSpStages) * 2 * kSpU * 16;
+      return row;
+    };
+    // tile p (0 or 1) of the window whose rows are `rows` -> ring stage `stage`: lane l copies
+    // chunk l mod 16 of rows 2i + l / 16
+    const uint32_t ring = smem_u32(sp_ring) + (uint32_t)(warp * kSpStages * kSpTileBytes);
+    auto issue = [&](uint32_t rows, int p, int stage) {
+      const uint32_t st = ring + (uint32_t)(stage * kSpTileBytes);
+      const int cc = lane & 15;
 #pragma unroll
-        for (int u = 0; u < kSpU; ++u) {
-          const uint32_t rr = __shfl_sync(hmask, row, bt * kSpU + u, 16);
-          if (rr != kInvalidRow) {
-            cp_async16(st + u * 16 + l, reinterpret_cast<const uint4*>(a.kv.k + (int64_t)rr * kHeadDim) + l);
-            cp_async16(st + (kSpU + u) * 16 + l, reinterpret_cast<const uint4*>(a.kv.v + (int64_t)rr * kHeadDim) + l);
+      for (int i = 0; i < kSpTileRows / 2; ++i) {
+        const int r = 2 * i + (lane >> 4);
+        const uint32_t rr = __shfl_sync(FULL, rows, 16 * p + r);
+        const bool ok = rr != kInvalidRow;
+        const int64_t off = ok ? (int64_t)rr * kHeadDim : 0;
+        const uint32_t so = sp_off(r, cc);
+        cp_async16_zfill(st + so, reinterpret_cast<const uint4*>(a.kv.k + off) + cc, ok);
+        cp_async16_zfill(st + kSpHalfBytes + so, reinterpret_cast<const uint4*>(a.kv.v + off) + cc, ok);
+      }
+      cp_async_commit();
+    };
+
+    // rows of windows wi, wi + 1 and wi + 2 resolved, raw indices of window wi + 3 loaded: a
+    // window's page-table reads are issued a whole window before its first tile is issued
+    if (!early) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) raw0[w] = load_raw(w);
+      if (lane == 0 && e0 > 0) prev0 = __ldg(lst + e0 - 1);
+    }
+    const int32_t v0 = raw0[0], v1 = raw0[1], v2 = raw0[2];
+    int32_t v3 = raw0[3];
+    float lw_cur = load_lw(0), lw_nxt = load_lw(1), lw_n2 = load_lw(2), lw_n3 = load_lw(3);
+    uint32_t row_cur = resolve(0, v0, prev0);
+    int32_t last = __shfl_sync(FULL, v0, 31);
+    uint32_t row_nxt = resolve(1, v1, last);
+    last = __shfl_sync(FULL, v1, 31);
+    uint32_t row_n2 = resolve(2, v2, last);
+    last = __shfl_sync(FULL, v2, 31);
+#pragma unroll
+    for (int ta = 0; ta < kSpStages - 1; ++ta) {   // tiles 0 .. kSpStages - 2, all in window 0
+      if (ta < ntile) issue(row_cur, ta, ta); else cp_async_commit();
+    }
+    // lanes 4i hold the scores of tile rows i and i + 8
+    const int gi = lane >> 2;
+    const bool scol = (lane & 3) == 0;
+    // P^T as the B operand of the output MMA: lane 4n + i needs rows 2i, 2i + 1 (from lanes
+    // 8i, 8i + 4, first score) and 2i + 8, 2i + 9 (second score); n = 0 takes bf16(P), n = 1 the rest
+    const int psrc = 8 * (lane & 3);
+    // ldmatrix lane addresses: K (non-transposed) rows l mod 16, chunk half l / 16; V
+    // (transposed) rows (l mod 8) + 8 (l / 16), chunk half (l / 8) mod 2
+    const int kr = lane & 15, kh = lane >> 4;
+    const int vr = (lane & 7) + 8 * (lane >> 4), vh = (lane >> 3) & 1;
+    int stage = 0;
+    for (int wi = 0; wi < nwin; ++wi) {
+      const uint32_t vmask = __ballot_sync(FULL, row_cur != kInvalidRow);
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const int tt = 2 * wi + p;
+        if (tt >= ntile) break;
+        // keep kSpStages - 1 tiles ahead of the one consumed
+        {
+          const int ta = tt + kSpStages - 1;
+          const int ap = (p + kSpStages - 1) & 1;
+          const bool next_win = ((p + kSpStages - 1) >> 1) != 0;
+          const int ast = stage == 0 ? kSpStages - 1 : stage - 1;
+          __syncwarp();
+          if (ta < ntile) issue(next_win ? row_nxt : row_cur, ap, ast); else cp_async_commit();
+        }
+        cp_async_wait<kSpStages - 1>();
+        __syncwarp();   // every lane's copies of this tile have landed
+        const uint32_t st = ring + (uint32_t)(stage * kSpTileBytes);
+        const uint32_t tmask = (vmask >> (16 * p)) & 0xFFFFu;
+        // scores: two accumulator chains over the 8 k-steps
+        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t af[4];
+          ldsm_x4(st + sp_off(kr, 2 * ks + kh), af[0], af[1], af[2], af[3]);
+          mma_bf16((ks & 1) ? d1 : d0, af, qb[ks][0], qb[ks][1]);
+        }
+        float s0 = ((d0[0] + d1[0]) + (d0[1] + d1[1])) * scale;
+        float s1 = ((d0[2] + d1[2]) + (d0[3] + d1[3])) * scale;
+        if (WEIGHTED) {   // entry weights: p_i = w_i exp(s_i), with ln w_i in base-2 units
+          s0 += __shfl_sync(FULL, lw_cur, 16 * p + gi);
+          s1 += __shfl_sync(FULL, lw_cur, 16 * p + gi + 8);
+        }
+        s0 = (scol && ((tmask >> gi) & 1u)) ? s0 : -CUDART_INF_F;
+        s1 = (scol && ((tmask >> (gi + 8)) & 1u)) ? s1 : -CUDART_INF_F;
+        float mt = fmaxf(s0, s1);
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 4));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
+        mt = __shfl_sync(FULL, mt, 0);
+        if (mt != -CUDART_INF_F) {   // uniform over the warp
+          if (mt > m_run + kSpLazyMax) {   // move the reference (always on the first valid tile)
+            const float alpha = fast_exp2(m_run - mt);
+            l_run *= alpha;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              o[i][0] *= alpha; o[i][1] *= alpha; o[i][2] *= alpha; o[i][3] *= alpha;
+            }
+            m_run = mt;
+          }
+          const float p0 = fast_exp2(s0 - m_run), p1 = fast_exp2(s1 - m_run);   // 0 for masked rows
+          l_run += p0 + p1;
+          const float x0 = __shfl_sync(FULL, p0, psrc), x1 = __shfl_sync(FULL, p0, psrc + 4);
+          const float y0 = __shfl_sync(FULL, p1, psrc), y1 = __shfl_sync(FULL, p1, psrc + 4);
+          uint32_t h0, l0, h1, l1;
+          split_bf16(x0, x1, h0, l0);
+          split_bf16(y0, y1, h1, l1);
+          const uint32_t pb0 = lane < 4 ? h0 : (lane < 8 ? l0 : 0u);
+          const uint32_t pb1 = lane < 4 ? h1 : (lane < 8 ? l1 : 0u);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint32_t af[4];
+            ldsm_x4_t(st + kSpHalfBytes + sp_off(vr, 2 * i + vh), af[0], af[1], af[2], af[3]);
+            mma_bf16(o[i], af, pb0, pb1);
           }
         }
-        cp_async_commit();
-      };
-#pragma unroll
-      for (int bt = 0; bt < kSpStages - 1; ++bt) issue(bt);
-#pragma unroll
-      for (int bt = 0; bt < 16 / kSpU; ++bt) {
-        if (bt + kSpStages - 1 < 16 / kSpU) issue(bt + kSpStages - 1); else cp_async_commit();
-        cp_async_wait<kSpStages - 1>();
-        const uint4* st = ring + (size_t)(bt % kSpStages) * 2 * kSpU * 16;
-        uint32_t rr[kSpU];
-        float bias[kSpU];
-        uint4 kq[kSpU], vq[kSpU];
-#pragma unroll
-        for (int u = 0; u < kSpU; ++u) {
-          rr[u] = __shfl_sync(hmask, row, bt * kSpU + u, 16);
-          bias[u] = WEIGHTED ? __shfl_sync(hmask, lw, bt * kSpU + u, 16) : 0.f;
-          kq[u] = rr[u] != kInvalidRow ? st[u * 16 + l] : make_uint4(0, 0, 0, 0);
-          vq[u] = rr[u] != kInvalidRow ? st[(kSpU + u) * 16 + l] : make_uint4(0, 0, 0, 0);
-        }
-        batch_update<kSpU, WEIGHTED>(kq, vq, rr, bias, q, m_run, l_run, acc, hmask);
+        stage = stage + 1 == kSpStages ? 0 : stage + 1;
+      }
+      // rotate: window wi + 1 becomes current, resolve window wi + 3, load window wi + 4
+      row_cur = row_nxt;
+      row_nxt = row_n2;
+      row_n2 = resolve(wi + 3, v3, last);
+      last = __shfl_sync(FULL, v3, 31);
+      v3 = load_raw(wi + 4);
+      if (WEIGHTED) {
+        lw_cur = lw_nxt;
+        lw_nxt = lw_n2;
+        lw_n2 = lw_n3;
+        lw_n3 = load_lw(wi + 4);
       }
     }
-    bad |= __shfl_xor_sync(hmask, bad, 1);
-    bad |= __shfl_xor_sync(hmask, bad, 2);
-    bad |= __shfl_xor_sync(hmask, bad, 4);
-    bad |= __shfl_xor_sync(hmask, bad, 8);
-    if (l == 0 && bad) flag_status(a.status, bad);
+    cp_async_wait<0>();
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) bad |= __shfl_xor_sync(FULL, bad, o2);
+    if (lane == 0 && bad) flag_status(a.status, bad);
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) l_run += __shfl_xor_sync(FULL, l_run, o2);
+    l_run = __shfl_sync(FULL, l_run, 0);
   }
 
-  if (C == 1) {   // every list is one task (uniform over the grid)
-    if (valid) finish_task(a, list_id, t, h, 1, 0, m_run, l_run, acc, l, hmask);
-    return;
+  // task states -> shared memory (lanes 4i hold dims 16k + i and 16k + i + 8, columns 0 + 1)
+  if (lane == 0) {
+    s_ml[warp] = make_float2(m_run, l_run);
+    s_list[warp] = list_id;
   }
-  // Chunks c, c+1, ... of a list are M tasks apart, so a CTA holds up to 16/M consecutive
-  // chunks of each of its lists.  Their states are combined here, and each list leaves the
-  // CTA as a single partial: the cross-CTA merge reads (16/M)x fewer partials.
-  if (l == 0) {
-    s_ml[hw] = make_float2(m_run, l_run);
-    s_list[hw] = list_id;
-  }
-  *reinterpret_cast<float4*>(&s_acc[hw][8 * l]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  *reinterpret_cast<float4*>(&s_acc[hw][8 * l + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  __syncthreads();
-  if (!valid || (hw >= M && s_list[hw - M] == list_id)) return;   // not the first chunk of its list here
-  for (int o = hw + M; o < 16 && s_list[o] == list_id; o += M) {
-    const float2 x = s_ml[o];
-    const float mn = fmaxf(m_run, x.x);
-    if (mn == -CUDART_INF_F) continue;
-    const float wa = fast_exp2(m_run - mn), wb = fast_exp2(x.x - mn);
-    l_run = l_run * wa + x.y * wb;
+  if ((lane & 3) == 0) {
+    const int i = lane >> 2;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = acc[i] * wa + s_acc[o][8 * l + i] * wb;
-    m_run = mn;
+    for (int k = 0; k < 8; ++k) {
+      s_acc[warp][16 * k + i] = o[k][0] + o[k][1];
+      s_acc[warp][16 * k + i + 8] = o[k][2] + o[k][3];
+    }
   }
-  // partials of the list = CTAs that hold one of its chunks (with M <= 16 every CTA from the
-  // first chunk's to the last chunk's holds one); this CTA's partial index
-  int parts = C, part = c;
-  if (M <= 16) {
-    const int64_t first = (((int64_t)b * a.kv.hkv + g) * C) * M + m;
-    const int64_t last = first + (int64_t)(C - 1) * M;
-    parts = (int)((last >> 4) - (first >> 4) + 1);
-    part = (int)((int64_t)blockIdx.x - (first >> 4));
+  __syncthreads();
+  if (!valid || (warp > 0 && s_list[warp - 1] == list_id)) return;   // not the first chunk of its list here
+  float mm = m_run, ll = l_run;
+  float4 acc = *reinterpret_cast<const float4*>(&s_acc[warp][4 * lane]);
+  for (int w2 = warp + 1; w2 < kSpWarps && s_list[w2] == list_id; ++w2) {
+    const float2 x = s_ml[w2];
+    const float mn = fmaxf(mm, x.x);
+    if (mn == -CUDART_INF_F) continue;
+    const float wa = fast_exp2(mm - mn), wb = fast_exp2(x.x - mn);
+    const float4 y = *reinterpret_cast<const float4*>(&s_acc[w2][4 * lane]);
+    ll = ll * wa + x.y * wb;
+    acc.x = acc.x * wa + y.x * wb; acc.y = acc.y * wa + y.y * wb;
+    acc.z = acc.z * wa + y.z * wb; acc.w = acc.w * wa + y.w * wb;
+    mm = mn;
   }
-  finish_task(a, list_id, t, h, parts, part, m_run, l_run, acc, l, hmask);
+  // partials of the list = CTAs that hold one of its chunks; this CTA's partial index
+  const int64_t first = (((int64_t)b * a.kv.hkv + g) * M + m) * C;
+  const int64_t fc = first / kSpWarps, lc = (first + C - 1) / kSpWarps;
+  finish_list(a, list_id, t, h, (int)(lc - fc + 1), (int)((int64_t)blockIdx.x - fc), mm, ll, acc, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -678,7 +778,7 @@ __global__ void __launch_bounds__(kDnThreads, kDnCtasPerSm) dense_decode_kernel(
 // ---------------------------------------------------------------------------
 cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
   const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
-  const int64_t grid = (tasks + 15) / 16;
+  const int64_t grid = (tasks + kSpWarps - 1) / kSpWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
   static bool configured = false;
   if (!configured) {

@@ -42,20 +42,22 @@ inline size_t zero_region_bytes(const Shapes& s) {
 constexpr int kMaxSparseK = kMaxSplits * kMaxEntriesPerSplit;
 
 // Sparse decode: every list (token x q head) is cut into C tasks of E entries (E a
-// multiple of 16); a task is one half-warp and a CTA runs 16 tasks.  Every task takes about
-// the same time, so a grid that spills a little into a second wave of resident CTAs costs
-// nearly a whole extra wave.  The plan therefore takes the smallest E whose tasks fit one
-// wave (kSpCtasPerSm CTAs on each SM).  When even one task per list leaves that wave well
-// under-filled (many lists, as with several decode tokens per sequence), it cuts the lists
-// finer instead, about two tasks per resident half-warp, and lets the lists of unequal
-// length even out.  C stays <= kMaxSplits either way.
+// multiple of 16, the row tile); a task is one warp and a CTA runs kSpTasksPerCta tasks.
+// Every task takes about the same time, so a grid that spills a little into a second wave
+// of resident CTAs costs nearly a whole extra wave.  The plan therefore takes the smallest
+// E whose tasks fit one wave (kSpCtasPerSm CTAs on each SM).  When even one task per list
+// leaves that wave well under-filled (many lists, as with several decode tokens per
+// sequence), it cuts the lists finer instead, about two tasks per resident warp, and lets
+// the lists of unequal length even out.  C stays <= kMaxSplits either way.
 struct SparsePlan {
   int lists;     // list slots per (sequence, kv head): G x max tokens per sequence
   int entries;   // E
   int nsplit;    // C
 };
 
-constexpr int kSpCtasPerSm = 2;   // resident sparse-decode CTAs per SM (launch bounds; 96 KB ring each)
+constexpr int kSpTasksPerCta = 4;   // warps per sparse-decode CTA, one task each
+constexpr int kSpStages = 3;        // 16-row tiles in each warp's shared-memory ring (8 KB each)
+constexpr int kSpCtasPerSm = 2;     // resident sparse-decode CTAs per SM (its launch bounds)
 
 inline SparsePlan plan_sparse(const Shapes& s, int k_max, int num_sms) {
   SparsePlan p;
@@ -63,18 +65,19 @@ inline SparsePlan plan_sparse(const Shapes& s, int k_max, int num_sms) {
   const int64_t slots = (int64_t)num_sms * kSpCtasPerSm;
   const int64_t units = s.batch * s.hkv * p.lists;
   const int kr = (k_max + 15) / 16 * 16;
+  constexpr int NW = kSpTasksPerCta;
   int e = 16;
   for (; e < kr; e += 16) {
     const int64_t ns = (k_max + e - 1) / e;
-    if (ns <= kMaxSplits && (units * ns + 15) / 16 <= slots) break;
+    if (ns <= kMaxSplits && (units * ns + NW - 1) / NW <= slots) break;
   }
-  const int64_t ctas = (units * ((k_max + e - 1) / e) + 15) / 16;
-  if (4 * ctas < 3 * slots) {   // one wave would be under-filled: about two tasks per half-warp
+  const int64_t ctas = (units * ((k_max + e - 1) / e) + NW - 1) / NW;
+  if (4 * ctas < 3 * slots) {   // one wave would be under-filled: about two tasks per warp
     const double total = (double)s.tokens * s.hq * k_max;
-    e = (int)(total / (2.0 * 16.0 * (double)slots));
+    e = (int)(total / (2.0 * NW * (double)slots));
     e = (e + 15) / 16 * 16;
     if (e < 16) e = 16;
-    if (e > 1024) e = 1024;
+    if (e > kMaxEntriesPerSplit) e = kMaxEntriesPerSplit;
     if (e > kr) e = kr;
     if ((k_max + e - 1) / e > kMaxSplits) e = ((k_max + kMaxSplits - 1) / kMaxSplits + 15) / 16 * 16;
   }
