@@ -533,6 +533,53 @@ def run_native(args):
                           "weights and decodes with them), L2 flushed before each replay; dense decode by "
                           "events as in legs_us"}
 
+    # A second figure: 20 sparse-decode steps back to back in one CUDA graph, each over its own
+    # index set (the top-k lists of a different seeded random query batch), L2 flushed once before
+    # each replay.  Launches are pipelined here, so this is the per-step time without the
+    # launch-and-event overhead of a single timed call.
+    n_rot = 20
+    gq = torch.Generator(device=dev)
+    gq.manual_seed(4321 + rank)
+    rot = []
+    rot_bytes = 0
+    for _ in range(n_rot):
+        qi = torch.randn(dw.q.shape, device=dev, generator=gq).to(dw.q.dtype)
+        qsi = tsd.Queries(qi, q_indptr=dw.q_indptr if multi else None, max_tokens_per_seq=cfg.tokens_per_seq,
+                          causal=cfg.causal, sm_scale=scale)
+        ii = torch.empty_like(idx_buf)
+        tsd.topk_select(cache, qsi, k_max, k_per_token=kpt_dev, out_idx=ii, out_count=torch.empty_like(cnt_buf),
+                        workspace=ws)
+        rot.append((qsi, ii))
+        rot_bytes += unique_rows(ii, torch.from_numpy(w.token_seq).to(dev), Hkv, G, cfg.max_seq_len) * 512
+    rot_bytes += n_rot * (q_bytes + o_bytes)
+
+    def rot_steps():
+        for qsi, ii in rot:
+            tsd.sparse_decode(cache, qsi, ii, out=out_g, lse=lse_g, workspace=ws)
+
+    rot_steps()
+    torch.cuda.synchronize()
+    g20 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g20):
+        rot_steps()
+    t20 = timed(g20.replay, reps + 1)
+    del g20
+    torch.cuda.synchronize()
+    if tsd.read_device_status(ws) != 0:
+        raise RuntimeError("device status bits set in the rotating-index graph")
+    t20 = max_over_ranks([t20], dev)[0]
+    rot_us = t20 * 1e3 / n_rot
+    rot_gbs = gbs(rot_bytes / n_rot, t20 / n_rot)
+    graph20_line = {"sparse_decode_us_per_step": round(rot_us, 3), "steps": n_rot,
+                    "achieved_gbs": round(rot_gbs, 1), "frac": round(rot_gbs / hbm, 4),
+                    "what": "20 sparse-decode steps back to back in one CUDA graph, each over the top-k lists of a "
+                            "different seeded random query batch; L2 flushed once before each replay; bytes are "
+                            "each step's own unique rows + q + out"}
+    sp_samples = ms[:, 1] * 1e3
+    sparse_stats = dict(zip(("median", "min", "p90"), max_over_ranks(
+        [float(np.median(sp_samples)), float(np.min(sp_samples)), float(np.percentile(sp_samples, 90))], dev)))
+    sparse_stats = {k_: round(v_, 3) for k_, v_ in sparse_stats.items()}
+
     # end to end through the public API with pinned host buffers
     q_host = dw.q.cpu().pin_memory()
     idx_host = idx_buf.cpu().pin_memory()
@@ -616,6 +663,8 @@ def run_native(args):
                              "what": "host q in -> topk_select -> sparse_decode -> host out and lse"},
         "label_indexer": label_line,
         "graph_step": graph_line,
+        "graph20_rotating": graph20_line,
+        "sparse_leg_us_stats": sparse_stats,
         "gpu_launches": 4 * args.steps,
         "clocks": cl,
     }

@@ -208,15 +208,32 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 // ---------------------------------------------------------------------------
 // TMA tensor loads and warp-level bf16 tensor-core MMA
 // ---------------------------------------------------------------------------
-// 2-D tiled TMA load (box given by the tensor map) into shared memory, completion
-// counted on `bar`.  x is the innermost (element) coordinate and must be a multiple of
-// 8 for bf16 (16 bytes); y is the row.
-__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar) {
+// L2 policy for streams that are read once (the K/V tiles of dense decode and top-k scoring):
+// their lines are the first to be evicted, so the stream does not push out data that the next
+// kernel reads from L2 (the score workspace between scoring and selection).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+  return p;
+}
+
+// 2-D tiled TMA load (box given by the tensor map) into shared memory under an L2 cache
+// policy, completion counted on `bar`.  x is the innermost (element) coordinate and must be a
+// multiple of 8 for bf16 (16 bytes); y is the row.
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* tmap, int x, int y, uint64_t* bar,
+                                                 uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
-          smem_u32(dst)),
-      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;\n" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// cp_async16 with an L2 cache policy.
+__device__ __forceinline__ void cp_async16_hint(void* smem, const void* gmem, uint64_t policy) {
+  uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "l"(policy)
+               : "memory");
 }
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-row tile written by TMA

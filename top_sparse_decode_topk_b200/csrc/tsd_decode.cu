@@ -195,9 +195,11 @@ constexpr int kSpTileRows = 16;
 constexpr int kSpHalfBytes = kSpTileRows * kHeadDim * 2;   // 16 rows of K (or V): 4 KB
 constexpr int kSpTileBytes = 2 * kSpHalfBytes;
 constexpr size_t kSpRingBytes = (size_t)kSpWarps * kSpStages * kSpTileBytes;
+constexpr int kSpPtEntries = 2048;                     // page-table row cached in shared memory up to this length
+constexpr size_t kSpSmemBytes = kSpRingBytes + kSpPtEntries * sizeof(int32_t);
 constexpr float kSpLazyMax = 8.f;   // base-2 units the running maximum may lag behind
 static_assert(kSpStages >= 2 && kSpStages <= 3, "the ring looks at most one window (two tiles) ahead");
-static_assert(kSpCtasPerSm * (kSpRingBytes + 2048) <= 228 * 1024, "resident sparse CTAs per SM");
+static_assert(kSpCtasPerSm * (kSpSmemBytes + 4096) <= 228 * 1024, "resident sparse CTAs per SM");
 
 // Byte offset of 16-byte chunk c of row r in a tile of 256-byte rows, the chunk index XOR-ed
 // with (r mod 8): the 8 rows one ldmatrix phase reads fall in 8 different bank groups.
@@ -330,6 +332,19 @@ __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel
     }
     if (lane == 0 && e0 > 0) prev0 = __ldg(lst + e0 - 1);
   }
+  // When the CTA's tasks all belong to one sequence and its page-table row is short, the row
+  // is copied into shared memory alongside the index loads: the page lookups of the gather then
+  // cost no global round trip.
+  const int64_t per_seq = (int64_t)a.kv.hkv * M * C;
+  const int64_t t_first = (int64_t)blockIdx.x * kSpWarps;
+  const int64_t t_last = (t_first + kSpWarps < total ? t_first + kSpWarps : total) - 1;
+  const bool pt_smem = a.kv.page_table != nullptr && a.kv.max_pages <= kSpPtEntries && t_first / per_seq == t_last / per_seq;
+  int32_t* s_pt = reinterpret_cast<int32_t*>(sp_ring + kSpRingBytes);
+  if (pt_smem) {
+    const int32_t* src = a.kv.page_table + (t_first / per_seq) * a.kv.max_pages;
+    for (int i = threadIdx.x; i < a.kv.max_pages; i += kSpThreads) s_pt[i] = __ldg(src + i);
+    __syncthreads();
+  }
   const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, task == tk && c == 0 && g == 0 && m == 0 && lane == 0);
   const int j = m / G;
   const bool valid = task < total && j < si.n;   // no list for slots past this sequence's tokens
@@ -397,7 +412,13 @@ __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel
       if (in && (v < -1 || v >= kvlen)) bad |= TSD_DEV_BAD_INDEX;
       uint32_t row = kInvalidRow;
       if (in && v >= 0 && v < kvlen) {
-        row = kv_row(a.kv, b, g, v);
+        if (pt_smem) {   // the same mapping as kv_row, from the shared-memory copy
+          const int32_t page = s_pt[v >> a.kv.page_shift];
+          if (page >= 0 && (int64_t)page < a.kv.num_pages)
+            row = (uint32_t)((((int64_t)page * a.kv.hkv + g) << a.kv.page_shift) | (v & ((1 << a.kv.page_shift) - 1)));
+        } else {
+          row = kv_row(a.kv, b, g, v);
+        }
         if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
       }
       return row;
@@ -783,17 +804,17 @@ cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaSt
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSpRingBytes);
+                                         (int)kSpSmemBytes);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(sparse_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kSpRingBytes);
+                               (int)kSpSmemBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   if (a.logw != nullptr) {
-    sparse_decode_kernel<true><<<(unsigned)grid, kSpThreads, kSpRingBytes, stream>>>(a);
+    sparse_decode_kernel<true><<<(unsigned)grid, kSpThreads, kSpSmemBytes, stream>>>(a);
   } else {
-    sparse_decode_kernel<false><<<(unsigned)grid, kSpThreads, kSpRingBytes, stream>>>(a);
+    sparse_decode_kernel<false><<<(unsigned)grid, kSpThreads, kSpSmemBytes, stream>>>(a);
   }
   return cudaGetLastError();
 }

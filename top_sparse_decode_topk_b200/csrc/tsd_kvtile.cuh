@@ -91,11 +91,12 @@ __device__ __forceinline__ uint32_t tile_issue_tma(const KvView& kv, const CUten
     if (y == -1) break;
     if (y < 0) continue;
     if (lane == 0) {
-      tma_load_2d(kdst + r * 128, tmk, 0, y, bar);
-      tma_load_2d(kdst + TT * 128 + r * 128, tmk, 64, y, bar);
+      const uint64_t pol = l2_evict_first();
+      tma_load_2d_hint(kdst + r * 128, tmk, 0, y, bar, pol);
+      tma_load_2d_hint(kdst + TT * 128 + r * 128, tmk, 64, y, bar, pol);
       if (vdst != nullptr) {
-        tma_load_2d(vdst + r * 128, tmv, 0, y, bar);
-        tma_load_2d(vdst + TT * 128 + r * 128, tmv, 64, y, bar);
+        tma_load_2d_hint(vdst + r * 128, tmv, 0, y, bar, pol);
+        tma_load_2d_hint(vdst + TT * 128 + r * 128, tmv, 64, y, bar, pol);
       }
     }
     bytes += (vdst != nullptr ? 4 : 2) * bp * 128;
@@ -123,7 +124,7 @@ __device__ __forceinline__ void tile_issue_cpasync(const KvView& kv, int b, int 
     }
     const uint16_t* src = (which ? kv.v : kv.k) + (int64_t)row * kHeadDim + ch * 8;
     unsigned char* base = which ? vdst : kdst;
-    cp_async16(base + (ch >> 3) * (TT * 128) + sw128(r, ch & 7), src);
+    cp_async16_hint(base + (ch >> 3) * (TT * 128) + sw128(r, ch & 7), src, l2_evict_first());
   }
 }
 
