@@ -374,39 +374,46 @@ __device__ __forceinline__ void load16(const float* row, int i0, int L, float* f
 }
 
 // Fast path for lists much longer than k: a threshold from a sample, then ONE pass over the
-// scores.  The r-th largest key lo of a 1024-score strided sample, with r the sample's expected
-// count above the k-th score plus 4 standard deviations, has at least k scores at or above it;
-// one ordered pass copies every (index, key) with key >= lo into shared memory in index order;
-// the exact radix select and the ordered output then run over those few thousand entries
-// only.  Returns false, having written nothing, when the sample says too many keys would be
-// kept or the pass kept more than fit or fewer than k: the caller then runs the full passes.
+// scores.  Take a strided sample of the list (1024 scores, or 4096 from 64K scores on) and r,
+// its expected count above the k-th score plus 4 standard deviations plus 4.  The sample's
+// r-th largest key with its low 10 bits cleared (lo) has, with overwhelming probability, at
+// least k scores at or above it.  One ordered pass copies every (index, key) with key >= lo
+// into shared memory in index order; the exact radix select and the ordered output then run
+// over those few thousand entries only.  Returns false, having written nothing, when the
+// sample says too many keys would be kept or the pass kept more than fit or fewer than k: the
+// caller then runs the full passes.
 // The score of an order-preserving key (inverse of score_key; -0 comes back as +0).
 __device__ __forceinline__ float key_score(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 constexpr int kFastMinL = 4096;
-constexpr int kFastSample = 1024;
+constexpr int kFastSample = 1024;        // sampled scores, lists shorter than kFastLongL
+constexpr int kFastSampleLong = 4096;    // the same from kFastLongL on: a tighter threshold
+constexpr int kFastLongL = 65536;
 constexpr int kFastCap = kCandMax / 2;   // kept entries: keys in cand[0, cap), indices in cand[cap, 2 cap)
 
 __device__ bool select_fast(SelectSmem& S, const float* row, int L, int k, int32_t* out, float* osc, int k_max) {
   uint32_t* ckey = S.cand;
   uint32_t* cidx = S.cand + kFastCap;
   // ---- the r_lo-th largest of a strided sample of keys ----
-  const float mean = (float)kFastSample * (float)k / (float)L;
-  const int r_lo = (int)ceilf(mean + 4.f * sqrtf(mean) + 8.f);
-  if (r_lo >= kFastSample || (int64_t)r_lo * L > (int64_t)kFastCap * kFastSample * 3 / 4) return false;
-  for (int s = threadIdx.x; s < kFastSample; s += kSelectThreads)
-    ckey[s] = score_key(__ldcg(row + (int)(((int64_t)s * L) / kFastSample)));
+  const int ns = L >= kFastLongL ? kFastSampleLong : kFastSample;
+  const float mean = (float)ns * (float)k / (float)L;
+  const int r_lo = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
+  if (r_lo >= ns || (int64_t)r_lo * L > (int64_t)kFastCap * ns * 3 / 4) return false;
+  for (int s = threadIdx.x; s < ns; s += kSelectThreads)
+    ckey[s] = score_key(__ldcg(row + (int)(((int64_t)s * L) / ns)));
+  // two 11-bit rounds: lo is the r_lo-th largest sampled key with its low 10 bits cleared,
+  // which keeps a little more than the exact sample key would
   uint32_t prefix = 0u;
   int need = r_lo, shift = 32;
-  while (shift > 0) {
-    const int nb = shift >= 11 ? 11 : shift;
+  while (shift > 10) {
+    const int nb = 11;
     shift -= nb;
     const bool first = shift + nb == 32;
     for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[i] = 0u;
     __syncthreads();
-    for (int c = threadIdx.x; c < kFastSample; c += kSelectThreads) {
+    for (int c = threadIdx.x; c < ns; c += kSelectThreads) {
       const uint32_t key = ckey[c];
       if (first || (key >> (shift + nb)) == prefix) atomicAdd(&S.hist[(key >> shift) & ((1u << nb) - 1u)], 1u);
     }
@@ -416,33 +423,39 @@ __device__ bool select_fast(SelectSmem& S, const float* row, int L, int k, int32
     need -= S.found_above;
     __syncthreads();
   }
-  const uint32_t lo_key = prefix;
+  const uint32_t lo_key = prefix << shift;
 
   // ---- one ordered pass: every key >= lo, in index order ----
+  // The key map is monotone, so key >= lo is score >= lo_f, the score whose key is lo: the
+  // pass compares floats and forms keys only for the entries it keeps.
+  const float lo_f = key_score(lo_key);
   const int tile_elems = kSelectThreads * kSelPerThread;
   int kept = 0;
   for (int base = 0; base < L; base += tile_elems) {
     const int i0 = base + threadIdx.x * kSelPerThread;
     float f[kSelPerThread];
     load16(row, i0, L, f);
-    uint32_t keys[kSelPerThread];
-    int n = 0;
+    uint32_t keep = 0u;
+    if (base + tile_elems <= L) {   // a full tile (uniform over the block)
 #pragma unroll
-    for (int j = 0; j < kSelPerThread; ++j) {
-      keys[j] = score_key(f[j]);
-      n += (i0 + j < L && keys[j] >= lo_key);
+      for (int j = 0; j < kSelPerThread; ++j) keep |= (f[j] >= lo_f ? 1u : 0u) << j;
+    } else {
+#pragma unroll
+      for (int j = 0; j < kSelPerThread; ++j) keep |= (i0 + j < L && f[j] >= lo_f ? 1u : 0u) << j;
     }
     int tot;
-    int pos = kept + block_exclusive_scan<kSelectThreads>(n, S.scan_tmp, &tot);
+    int pos = kept + block_exclusive_scan<kSelectThreads>(__popc(keep), S.scan_tmp, &tot);
+    if (keep != 0u) {
 #pragma unroll
-    for (int j = 0; j < kSelPerThread; ++j)
-      if (i0 + j < L && keys[j] >= lo_key) {
-        if (pos < kFastCap) {
-          ckey[pos] = keys[j];
-          cidx[pos] = (uint32_t)(i0 + j);
+      for (int j = 0; j < kSelPerThread; ++j)
+        if ((keep >> j) & 1u) {
+          if (pos < kFastCap) {
+            ckey[pos] = score_key(f[j]);
+            cidx[pos] = (uint32_t)(i0 + j);
+          }
+          ++pos;
         }
-        ++pos;
-      }
+    }
     kept += tot;
   }
   __syncthreads();
@@ -638,18 +651,17 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
   const int need_eq = need;    // how many keys == T are kept (the lowest indices)
 
   // ---- output pass: ordered compaction of (key > T) or (key == T and among the first need_eq) ----
+  // (compared as floats: key > T is score > T_f and key == T is score == T_f, -0 == +0 included)
+  const float T_f = key_score(T);
   int eq_before = 0, sel_before = 0;
   for (int base = 0; base < L; base += tile_elems) {
     const int i0 = base + threadIdx.x * kSelPerThread;
     float f[kSelPerThread];
     load16(row, i0, L, f);
-    uint32_t keys[kSelPerThread];
     int neq = 0;
 #pragma unroll
-    for (int j = 0; j < kSelPerThread; ++j) {
-      keys[j] = score_key(f[j]);
-      if (i0 + j < L && keys[j] == T) ++neq;
-    }
+    for (int j = 0; j < kSelPerThread; ++j)
+      if (i0 + j < L && f[j] == T_f) ++neq;
     int eq_total;
     int eq_run = eq_before + block_exclusive_scan<kSelectThreads>(neq, S.scan_tmp, &eq_total);
     int nsel = 0;
@@ -658,8 +670,8 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
     for (int j = 0; j < kSelPerThread; ++j) {
       bool sel = false;
       if (i0 + j < L) {
-        if (keys[j] > T) sel = true;
-        else if (keys[j] == T) { sel = eq_run < need_eq; ++eq_run; }
+        if (f[j] > T_f) sel = true;
+        else if (f[j] == T_f) { sel = eq_run < need_eq; ++eq_run; }
       }
       if (sel) { selmask |= 1u << j; ++nsel; }
     }
