@@ -281,6 +281,30 @@ def test_page_sizes(page_size):
                     out_is_bf16=False, dense=True)
 
 
+def test_ctas_spanning_two_sequences():
+    """A shape whose tasks per sequence (kv heads x lists x chunks = 1 x 2 x 19) are not a
+    multiple of a sparse-decode CTA's 4 warps: some CTAs hold the end of one sequence and the
+    start of the next.  Those look pages up in global memory, the others in the page-table row
+    they cached in shared memory; every list must match the oracle either way."""
+    T = torch()
+    cfg = W.DecodeConfig(name="straddle", batch=5, num_q_heads=2, num_kv_heads=1, seq_len=4096, ks=(300,),
+                         planted=True, causal=True)
+    w = W.make_workload(cfg, seed=5, seq_lens=[3000, 700, 4096, 1500, 2222])
+    dw, cache, queries = setup(w)
+    inp = PT.OracleInputs(w)
+    idx, cnt = tsd.topk_select(cache, queries, 300)
+    T.cuda.synchronize()
+    PT.check_topk(inp, idx.cpu().numpy(), cnt.cpu().numpy(), w.k_per_token(300), all_pairs(w))
+    lists = oracle_lists(inp, w, 300, w.k_per_token(300), all_pairs(w))
+    out, lse = run_sparse(cache, queries, lists, out_f32=True)
+    PT.check_decode(inp, lists, out, lse, all_pairs(w), SM_SCALE, out_is_bf16=False)
+    for maker in (W.uniform_indices, W.zipf_page_run_indices):
+        lists = maker(w, 300)
+        out, lse = run_sparse(cache, queries, lists, out_f32=False)
+        PT.check_decode(inp, lists, out, lse, all_pairs(w), SM_SCALE, out_is_bf16=True)
+    assert tsd.read_device_status() == 0
+
+
 def test_deterministic(small):
     T = torch()
     w, dw, cache, queries, inp = small
