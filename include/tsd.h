@@ -162,6 +162,28 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
                              const int32_t* idx, int32_t k_max, void* out, int32_t out_dtype,
                              float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream);
 
+/* Host: bytes of workspace tsd_sparse_decode_host needs: the tsd_sparse_decode workspace
+ * followed by device staging for q, the index lists, out and lse (0 on invalid input). */
+size_t tsd_sparse_decode_host_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries,
+                                             int32_t k_max, int32_t out_dtype);
+
+/*
+ * tsd_sparse_decode for per-step inputs and outputs that live in host memory, in one call:
+ * queries->q, idx, out and lse may be host pointers (page-locked memory lets the copies run
+ * asynchronously; pageable memory works but each copy then waits for the host).  On `stream`
+ * the call enqueues the copies of q and idx into device staging inside `ws`, the sparse decode,
+ * and the copies of out (and lse, when non-NULL) back, and returns before they finish:
+ * synchronise the stream before reading out or lse, or before reusing q or idx.  The copy
+ * direction follows from the pointers (unified addressing), so device pointers work too.  The
+ * cache (k, v, page_table, seq_lens) and queries->q_indptr stay device pointers.
+ * ws: at least tsd_sparse_decode_host_workspace_size bytes; its leading region follows the
+ * tsd_sparse_decode rules.  Errors: as tsd_sparse_decode (nothing is enqueued on a
+ * host-checkable error); CUDA if a copy cannot be enqueued.
+ */
+tsd_status tsd_sparse_decode_host(const tsd_kv_cache* cache, const tsd_queries* queries,
+                                  const int32_t* idx, int32_t k_max, void* out, int32_t out_dtype,
+                                  float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream);
+
 /*
  * Weighted sparse decode: as tsd_sparse_decode, with entry i of list (t, h) weighted by
  * w = exp(logw[t][h][i]): out = sum_i w_i e^{z_i} V_i / sum_i w_i e^{z_i} and

@@ -160,6 +160,30 @@ def test_other_errors_before_launch(lib):
 
 
 @fake_pointer_call
+def test_host_buffer_decode_errors_before_any_copy(lib):
+    """tsd_sparse_decode_host rejects what tsd_sparse_decode rejects, before it enqueues a copy."""
+    c, q = make_cache(), make_queries()
+    sz = lib.tsd_sparse_decode_host_workspace_size(ctypes.byref(c), ctypes.byref(q), 655, 0)
+    base = lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 655)
+    # the decode workspace, then staging for q (bf16), the lists, out (bf16) and lse
+    assert sz >= base + 8 * 32 * (128 * 2 + 655 * 4 + 128 * 2 + 4)
+    assert lib.tsd_sparse_decode_host_workspace_size(ctypes.byref(c), ctypes.byref(q), 655, 5) == 0
+    assert lib.tsd_sparse_decode_host_workspace_size(ctypes.byref(c), ctypes.byref(q), 0, 0) == 0
+
+    def host(cc=c, qq=q, k_max=655, out_dtype=0, idx=FAKE + 0x500000, ws_bytes=1 << 40):
+        return lib.tsd_sparse_decode_host(ctypes.byref(cc), ctypes.byref(qq), idx, k_max, FAKE + 0x600000, out_dtype,
+                                          None, FAKE + 0x700000, ws_bytes, None)
+    assert host(ws_bytes=base) == tsd.TSD_ERR_WORKSPACE_TOO_SMALL
+    assert host(k_max=0) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert host(idx=None) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert host(out_dtype=5) == tsd.TSD_ERR_UNSUPPORTED
+    assert host(cc=make_cache(head_dim=64)) == tsd.TSD_ERR_UNSUPPORTED
+    assert host(qq=make_queries(sm_scale=0.0)) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_sparse_decode_host(None, ctypes.byref(q), FAKE, 8, FAKE, 0, None, FAKE, 1 << 40, None) == \
+        tsd.TSD_ERR_INVALID_ARGUMENT
+
+
+@fake_pointer_call
 def test_multi_token_queries_need_bounds(lib):
     c = make_cache(batch=32)
     q = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=0)

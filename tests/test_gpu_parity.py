@@ -281,6 +281,32 @@ def test_page_sizes(page_size):
                     out_is_bf16=False, dense=True)
 
 
+@pytest.mark.parametrize("out_f32,with_lse", [(False, True), (True, True), (False, False)])
+def test_host_buffers_match_the_device_path(small, out_f32, with_lse):
+    """sparse_decode on pinned host q, lists, out and lse (one tsd_sparse_decode_host call:
+    copies in, decode, copies back) gives exactly the device path's result, and the oracle's."""
+    T = torch()
+    w, dw, cache, queries, inp = small
+    lists = W.uniform_indices(w, 250)
+    odt = T.float32 if out_f32 else T.bfloat16
+    out_d, lse_d = tsd.sparse_decode(cache, queries, T.from_numpy(lists).cuda(), out_dtype=odt)
+    qh = tsd.Queries(dw.q.cpu().pin_memory(), q_indptr=dw.q_indptr, max_tokens_per_seq=SMALL.tokens_per_seq,
+                     causal=True, sm_scale=SM_SCALE)
+    out_h = T.empty(tuple(out_d.shape), dtype=odt).pin_memory()
+    lse_h = T.empty(tuple(lse_d.shape), dtype=T.float32).pin_memory() if with_lse else None
+    o, l = tsd.sparse_decode(cache, qh, T.from_numpy(lists).pin_memory(), out=out_h, lse=lse_h)
+    T.cuda.synchronize()
+    assert o.data_ptr() == out_h.data_ptr()
+    assert T.equal(out_h, out_d.cpu())
+    if with_lse:
+        assert T.equal(lse_h, lse_d.cpu())
+    else:
+        assert l is None
+    PT.check_decode(inp, lists, PT.bf16_to_np(out_h), lse_d.cpu().numpy(), all_pairs(w), SM_SCALE,
+                    out_is_bf16=not out_f32)
+    assert tsd.read_device_status() == 0
+
+
 def test_ctas_spanning_two_sequences():
     """A shape whose tasks per sequence (kv heads x lists x chunks = 1 x 2 x 19) are not a
     multiple of a sparse-decode CTA's 4 warps: some CTAs hold the end of one sequence and the

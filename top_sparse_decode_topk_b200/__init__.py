@@ -79,6 +79,11 @@ EXPORTS = {
     "tsd_sparse_decode": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_void_p,
                                          ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "tsd_sparse_decode_host_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
+                                                                ctypes.c_int32, ctypes.c_int32]),
+    "tsd_sparse_decode_host": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_void_p,
+                                              ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "tsd_dense_decode_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC)]),
     "tsd_dense_decode": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_void_p,
                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
@@ -471,6 +476,9 @@ def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=Non
     lib = load_library()
     dev = cache.device
     s, sp = _stream_ptr(stream, dev)
+    host = lambda x: x is not None and x is not True and x is not False and x.device.type == "cpu"
+    if logw is None and host(queries.q) and host(idx) and host(out) and (lse is None or lse is False or host(lse)):
+        return _sparse_decode_host(lib, cache, queries, idx, out, None if lse is False else lse, workspace, s, sp)
     queries = _on_device_queries(queries, dev, s)
     idx = _to_device(idx, dev, s)
     if idx.dtype != torch.int32 or idx.dim() != 3 or not idx.is_contiguous():
@@ -496,6 +504,38 @@ def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=Non
                                               k_max, out.data_ptr(), odt, lp, ws.data_ptr(), ws.numel(), sp),
                "tsd_sparse_decode_weighted")
     return _finish(out, host_out, lse, host_lse, s)
+
+
+def _sparse_decode_host(lib, cache: KVCache, queries: Queries, idx, out, lse, workspace, s, sp):
+    """sparse_decode with q, idx, out and lse in host memory: one tsd_sparse_decode_host call
+    enqueues the copies in, the decode and the copies back on `s` (asynchronous: synchronise
+    the stream before reading out/lse)."""
+    import torch
+    dev = cache.device
+    if idx.dtype != torch.int32 or idx.dim() != 3 or not idx.is_contiguous():
+        raise ValueError("idx must be a contiguous int32 [T, Hq, k_max] tensor")
+    if out.dtype not in (torch.bfloat16, torch.float32) or not out.is_contiguous():
+        raise TypeError("out must be a contiguous bfloat16 or float32 tensor")
+    if not queries.q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    T, Hq = int(queries.q.shape[0]), int(queries.q.shape[1])
+    if tuple(out.shape) != (T, Hq, 128) or int(idx.shape[0]) != T or int(idx.shape[1]) != Hq:
+        raise ValueError("q, idx and out shapes disagree")
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (T, Hq) or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 [T, Hq] tensor")
+    qd = Queries(q=queries.q, q_indptr=_to_device(queries.q_indptr, dev, s), max_tokens_per_seq=queries.max_tokens_per_seq,
+                 causal=queries.causal, sm_scale=queries.sm_scale)
+    cs, qs = cache.c_struct(), qd.c_struct()
+    k_max = int(idx.shape[2])
+    odt = TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32
+    nbytes = lib.tsd_sparse_decode_host_workspace_size(ctypes.byref(cs), ctypes.byref(qs), k_max, odt)
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_sparse_decode_host_workspace_size")
+    ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, qd), sp)
+    _check(lib.tsd_sparse_decode_host(ctypes.byref(cs), ctypes.byref(qs), idx.data_ptr(), k_max, out.data_ptr(), odt,
+                                      None if lse is None else lse.data_ptr(), ws.data_ptr(), ws.numel(), sp),
+           "tsd_sparse_decode_host")
+    return out, lse
 
 
 def stochastic_select(cache: KVCache, queries: Queries, topk_idx, u, status=None, stream=None):

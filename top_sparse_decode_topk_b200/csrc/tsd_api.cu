@@ -372,6 +372,81 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
   return sparse_decode_impl(cache, queries, idx, nullptr, k_max, out, out_dtype, lse, ws, ws_bytes, stream);
 }
 
+// Device staging of tsd_sparse_decode_host, after the sparse-decode workspace.
+struct HostStaging {
+  size_t off_q, off_idx, off_out, off_lse, total;
+};
+
+static bool host_staging(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max, int32_t out_dtype,
+                         HostStaging* hs, size_t* decode_bytes) {
+  Shapes sh;
+  if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return false;
+  if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return false;
+  const SparsePlan p = plan_sparse(sh, k_max, current_sm_count());
+  *decode_bytes = decode_layout(sh, p.nsplit).total;
+  const size_t lists = (size_t)queries->num_tokens * queries->num_q_heads;
+  size_t off = align256(*decode_bytes);
+  hs->off_q = off;
+  off += align256(lists * kHeadDim * (queries->q_dtype == TSD_F32 ? 4 : 2));
+  hs->off_idx = off;
+  off += align256(lists * (size_t)k_max * sizeof(int32_t));
+  hs->off_out = off;
+  off += align256(lists * kHeadDim * (out_dtype == TSD_F32 ? 4 : 2));
+  hs->off_lse = off;
+  off += align256(lists * sizeof(float));
+  hs->total = off;
+  return true;
+}
+
+size_t tsd_sparse_decode_host_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                             int32_t out_dtype) {
+  HostStaging hs;
+  size_t dec;
+  return host_staging(cache, queries, k_max, out_dtype, &hs, &dec) ? hs.total : 0;
+}
+
+tsd_status tsd_sparse_decode_host(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
+                                  int32_t k_max, void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                                  tsd_stream_t stream) {
+  if (cache == nullptr || queries == nullptr || queries->q == nullptr || idx == nullptr || out == nullptr ||
+      ws == nullptr)
+    return TSD_ERR_INVALID_ARGUMENT;
+  HostStaging hs;
+  size_t dec;
+  if (!host_staging(cache, queries, k_max, out_dtype, &hs, &dec)) {
+    // report the same status tsd_sparse_decode would
+    KvView kv; QView qv; Shapes sh;
+    const tsd_status st = check_inputs(cache, queries, &kv, &qv, &sh);
+    if (st != TSD_OK) return st;
+    if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return TSD_ERR_UNSUPPORTED;
+    return k_max > kMaxSparseK ? TSD_ERR_UNSUPPORTED : TSD_ERR_INVALID_ARGUMENT;
+  }
+  if (ws_bytes < hs.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
+  char* base = static_cast<char*>(ws);
+  tsd_queries qd = *queries;
+  qd.q = base + hs.off_q;
+  int32_t* idx_d = reinterpret_cast<int32_t*>(base + hs.off_idx);
+  void* out_d = base + hs.off_out;
+  float* lse_d = lse != nullptr ? reinterpret_cast<float*>(base + hs.off_lse) : nullptr;
+  // validate everything the decode checks before enqueueing any copy
+  {
+    KvView kv; QView qv; Shapes sh;
+    const tsd_status st = decode_common(cache, &qd, out_d, out_dtype, lse_d, ws, dec, &kv, &qv, &sh);
+    if (st != TSD_OK) return st;
+  }
+  const size_t lists = (size_t)queries->num_tokens * queries->num_q_heads;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(base + hs.off_q, queries->q, lists * kHeadDim * (queries->q_dtype == TSD_F32 ? 4 : 2),
+                                  cudaMemcpyDefault, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(idx_d, idx, lists * (size_t)k_max * sizeof(int32_t), cudaMemcpyDefault, s);
+  if (e != cudaSuccess) return TSD_ERR_CUDA;
+  const tsd_status st = sparse_decode_impl(cache, &qd, idx_d, nullptr, k_max, out_d, out_dtype, lse_d, ws, dec, stream);
+  if (st != TSD_OK) return st;
+  e = cudaMemcpyAsync(out, out_d, lists * kHeadDim * (out_dtype == TSD_F32 ? 4 : 2), cudaMemcpyDefault, s);
+  if (e == cudaSuccess && lse != nullptr) e = cudaMemcpyAsync(lse, lse_d, lists * sizeof(float), cudaMemcpyDefault, s);
+  return e == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+}
+
 tsd_status tsd_sparse_decode_weighted(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
                                       const float* logw, int32_t k_max, void* out, int32_t out_dtype, float* lse,
                                       void* ws, size_t ws_bytes, tsd_stream_t stream) {
