@@ -198,6 +198,12 @@ class KVCache:
         return int(self.k.shape[1])
 
     def c_struct(self) -> _KvCacheC:
+        key = (self.k.data_ptr(), self.v.data_ptr(), tuple(self.k.shape), self.seq_lens.data_ptr(),
+               int(self.seq_lens.shape[0]), int(self.max_seq_len),
+               None if self.page_table is None else (self.page_table.data_ptr(), tuple(self.page_table.shape)))
+        cached = self.__dict__.get("_c_struct")
+        if cached is not None and cached[0] == key:   # the same tensors: the struct is unchanged
+            return cached[1]
         c = _KvCacheC()
         c.k = self.k.data_ptr()
         c.v = self.v.data_ptr()
@@ -218,6 +224,7 @@ class KVCache:
             c.page_table = self.page_table.data_ptr()
             c.max_pages_per_seq = int(self.page_table.shape[1])
             c.num_pages = int(self.k.shape[0])
+        self.__dict__["_c_struct"] = (key, c)
         return c
 
 
@@ -506,6 +513,9 @@ def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=Non
     return _finish(out, host_out, lse, host_lse, s)
 
 
+_HOST_WS_BYTES = {}
+
+
 def _sparse_decode_host(lib, cache: KVCache, queries: Queries, idx, out, lse, workspace, s, sp):
     """sparse_decode with q, idx, out and lse in host memory: one tsd_sparse_decode_host call
     enqueues the copies in, the decode and the copies back on `s` (asynchronous: synchronise
@@ -523,15 +533,21 @@ def _sparse_decode_host(lib, cache: KVCache, queries: Queries, idx, out, lse, wo
         raise ValueError("q, idx and out shapes disagree")
     if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (T, Hq) or not lse.is_contiguous()):
         raise ValueError("lse must be a contiguous float32 [T, Hq] tensor")
-    qd = Queries(q=queries.q, q_indptr=_to_device(queries.q_indptr, dev, s), max_tokens_per_seq=queries.max_tokens_per_seq,
-                 causal=queries.causal, sm_scale=queries.sm_scale)
+    qd = queries if queries.q_indptr is None or queries.q_indptr.device == dev else Queries(
+        q=queries.q, q_indptr=_to_device(queries.q_indptr, dev, s), max_tokens_per_seq=queries.max_tokens_per_seq,
+        causal=queries.causal, sm_scale=queries.sm_scale)
     cs, qs = cache.c_struct(), qd.c_struct()
     k_max = int(idx.shape[2])
     odt = TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32
-    nbytes = lib.tsd_sparse_decode_host_workspace_size(ctypes.byref(cs), ctypes.byref(qs), k_max, odt)
-    if nbytes == 0:
-        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_sparse_decode_host_workspace_size")
-    ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, qd), sp)
+    skey = _shape_key(cache, qd)
+    size_key = (skey, k_max, odt, qs.q_dtype)
+    nbytes = _HOST_WS_BYTES.get(size_key)
+    if nbytes is None:   # the size depends only on the shapes: asked once per shape
+        nbytes = lib.tsd_sparse_decode_host_workspace_size(ctypes.byref(cs), ctypes.byref(qs), k_max, odt)
+        if nbytes == 0:
+            raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_sparse_decode_host_workspace_size")
+        _HOST_WS_BYTES[size_key] = nbytes
+    ws = _ws(workspace, dev).get(nbytes, skey, sp)
     _check(lib.tsd_sparse_decode_host(ctypes.byref(cs), ctypes.byref(qs), idx.data_ptr(), k_max, out.data_ptr(), odt,
                                       None if lse is None else lse.data_ptr(), ws.data_ptr(), ws.numel(), sp),
            "tsd_sparse_decode_host")
