@@ -10,10 +10,11 @@
 // list with a natural-log weight per entry (0 for S), which the weighted sparse decode
 // consumes.
 //
-// One warp per list.  Floyd's m steps run in order (each step's membership test is a warp
-// scan of the ranks kept so far); the kept ranks are then sorted by counting, mapped to
-// tokens of R by a binary search over S (token = rank + #{s in S below it}), and merged with
-// S by each side's binary-search position.
+// One warp per list.  Floyd's m draws are computed in parallel; collisions are then resolved
+// in step order by parallel searches for the first repeated value, one search per collision.  The kept ranks are then sorted by
+// counting, mapped to tokens of R by a binary search over S (token = rank + #{s in S below it}),
+// and merged with S: each sample by a binary search over S, each lane's contiguous chunk of S by
+// one binary search and a forward scan of the samples.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -111,15 +112,30 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
   uint32_t* us = reinterpret_cast<uint32_t*>(toks[warp]);
   for (int s = lane; s < m; s += 32) us[s] = __ldg(u + s);
   __syncwarp();
-  // ---- Floyd: step j = n - m .. n - 1 keeps t = u mod (j + 1), or j on a collision ----
-  for (int s = 0; s < m; ++s) {
-    const uint32_t j = (uint32_t)(n - m + s);
-    const uint32_t tr = us[s] % (j + 1u);
-    bool seen = false;
-    for (int i = lane; i < s; i += 32) seen |= kr[i] == tr;
-    seen = __any_sync(0xFFFFFFFFu, seen);
-    if (lane == 0) kr[s] = seen ? j : tr;
+  // ---- Floyd: step s (j_s = n - m + s) keeps t_s = u_s mod (j_s + 1), or j_s if t_s was
+  // kept before ----
+  // All draws t_s are computed in parallel.  Then, repeatedly: steps before `from` are final;
+  // the first step s >= from whose current value repeats an earlier kept value is a collision
+  // of the sequential algorithm (the steps between keep their draws), so it keeps j_s, which
+  // exceeds every earlier kept value and so never collides itself; the search resumes at s + 1.
+  // With m << n collisions are rare and this is one or two parallel passes.
+  for (int s = lane; s < m; s += 32) kr[s] = us[s] % ((uint32_t)(n - m + s) + 1u);
+  __syncwarp();
+  for (int from = 0;;) {
+    int first = m;   // the first step >= from whose value repeats an earlier one (branch-free scans)
+    for (int s = lane; s < m; s += 32) {
+      const uint32_t v = kr[s];
+      bool rep = false;
+      for (int i = 0; i < s; ++i) rep |= kr[i] == v;
+      if (rep && s >= from && s < first) first = s;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xFFFFFFFFu, first, o));
+    if (first == m) break;
     __syncwarp();
+    if (lane == 0) kr[first] = (uint32_t)(n - m + first);
+    __syncwarp();
+    from = first + 1;
   }
   // ---- sort the kept ranks (distinct) by counting, and map each to its token of R ----
   int32_t* tk = toks[warp];
@@ -141,15 +157,27 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
   int32_t* oi = a.out_idx + list * width;
   float* ow = a.out_logw + list * width;
   const float lw = m > 0 ? logf((float)n / (float)m) : 0.f;
-  for (int i = lane; i < ntop; i += 32) {
-    const int32_t v = topc[i];
-    int lo = 0, hi = m;   // sampled tokens below v
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (tk[mid] < v) lo = mid + 1; else hi = mid;
+  // top entries: lane l walks its contiguous chunk, one binary search for the chunk start
+  // then a forward scan of the (ascending) samples
+  {
+    const int chunk = (ntop + 31) >> 5;
+    const int i0 = lane * chunk, i1 = min(ntop, i0 + chunk);
+    int pos = 0;   // sampled tokens below the current top entry
+    if (i0 < i1) {
+      const int32_t v0 = topc[i0];
+      int lo = 0, hi = m;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (tk[mid] < v0) lo = mid + 1; else hi = mid;
+      }
+      pos = lo;
     }
-    oi[i + lo] = v;
-    ow[i + lo] = 0.f;
+    for (int i = i0; i < i1; ++i) {
+      const int32_t v = topc[i];
+      while (pos < m && tk[pos] < v) ++pos;
+      oi[i + pos] = v;
+      ow[i + pos] = 0.f;
+    }
   }
   for (int i = lane; i < m; i += 32) {
     const int32_t v = tk[i];
