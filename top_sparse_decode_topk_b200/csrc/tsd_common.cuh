@@ -66,27 +66,42 @@ __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {
   atomicOr(status, bits);
 }
 
-__device__ __forceinline__ SeqInfo seq_info(const KvView& kv, const QView& qv, int b, uint32_t* status,
-                                            bool report) {
-  SeqInfo s;
-  int len = __ldg(kv.seq_lens + b);
-  int t0, t1;
+// The raw descriptor of sequence b (seq_lens[b] and its q_indptr range), loaded but not yet
+// checked, so that a kernel can put other loads in flight before it waits on these.
+struct SeqRaw {
+  int len, t0, t1;
+};
+
+__device__ __forceinline__ SeqRaw seq_load(const KvView& kv, const QView& qv, int b) {
+  SeqRaw r;
+  r.len = __ldg(kv.seq_lens + b);
   if (qv.q_indptr != nullptr) {
-    t0 = __ldg(qv.q_indptr + b);
-    t1 = __ldg(qv.q_indptr + b + 1);
+    r.t0 = __ldg(qv.q_indptr + b);
+    r.t1 = __ldg(qv.q_indptr + b + 1);
   } else {
-    t0 = b;
-    t1 = b + 1;
+    r.t0 = b;
+    r.t1 = b + 1;
   }
-  bool bad = len < 0 || len > kv.max_seq_len || t0 < 0 || t1 < t0 || t1 > qv.num_tokens ||
-             (t1 - t0) > qv.max_tokens;
+  return r;
+}
+
+__device__ __forceinline__ SeqInfo seq_check(const KvView& kv, const QView& qv, const SeqRaw& r, uint32_t* status,
+                                             bool report) {
+  SeqInfo s;
+  const bool bad = r.len < 0 || r.len > kv.max_seq_len || r.t0 < 0 || r.t1 < r.t0 || r.t1 > qv.num_tokens ||
+                   (r.t1 - r.t0) > qv.max_tokens;
   if (bad) {
     if (report) flag_status(status, TSD_DEV_BAD_SEQ_BIT);
     s.t0 = 0; s.n = 0; s.len = 0;
     return s;
   }
-  s.t0 = t0; s.n = t1 - t0; s.len = len;
+  s.t0 = r.t0; s.n = r.t1 - r.t0; s.len = r.len;
   return s;
+}
+
+__device__ __forceinline__ SeqInfo seq_info(const KvView& kv, const QView& qv, int b, uint32_t* status,
+                                            bool report) {
+  return seq_check(kv, qv, seq_load(kv, qv, b), status, report);
 }
 
 // Tokens visible to query j (0-based) of the n tokens of a sequence with len cached tokens.

@@ -1,8 +1,7 @@
 // Work decomposition and workspace layout of libtsd (host and device).
 //
 // Workspace layout (bytes from the start; every region 256-byte aligned):
-//   [0, 256)              header: device status word (uint32) at offset 0; sparse-decode
-//                         work-unit counter at byte 4 and finished-CTA counter at byte 8
+//   [0, 256)              header: device status word (uint32) at offset 0, the rest reserved
 //   counters              uint32, one per list (token x q head): arrival counters of the
 //                         split-K merge (zero between calls)
 //   -- everything above is the "zero region": it must be zero when a call starts and every
