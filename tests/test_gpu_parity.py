@@ -307,6 +307,26 @@ def test_host_buffers_match_the_device_path(small, out_f32, with_lse):
     assert tsd.read_device_status() == 0
 
 
+def test_host_buffers_with_fp32_queries(small):
+    """The host-buffer call stages an fp32 q (4 bytes per element) the same way: it matches the
+    device path on the same fp32 queries exactly."""
+    T = torch()
+    w, dw, cache, queries, inp = small
+    lists = W.zipf_page_run_indices(w, 180)
+    qf = dw.q.float()
+    qd = tsd.Queries(qf, q_indptr=dw.q_indptr, max_tokens_per_seq=SMALL.tokens_per_seq, causal=True,
+                     sm_scale=SM_SCALE)
+    out_d, lse_d = tsd.sparse_decode(cache, qd, T.from_numpy(lists).cuda(), out_dtype=T.float32)
+    qh = tsd.Queries(qf.cpu().pin_memory(), q_indptr=dw.q_indptr, max_tokens_per_seq=SMALL.tokens_per_seq,
+                     causal=True, sm_scale=SM_SCALE)
+    out_h = T.empty(tuple(out_d.shape), dtype=T.float32).pin_memory()
+    lse_h = T.empty(tuple(lse_d.shape), dtype=T.float32).pin_memory()
+    tsd.sparse_decode(cache, qh, T.from_numpy(lists).pin_memory(), out=out_h, lse=lse_h)
+    T.cuda.synchronize()
+    assert T.equal(out_h, out_d.cpu()) and T.equal(lse_h, lse_d.cpu())
+    assert tsd.read_device_status() == 0
+
+
 def test_ctas_spanning_two_sequences():
     """A shape whose tasks per sequence (kv heads x lists x chunks = 1 x 2 x 19) are not a
     multiple of a sparse-decode CTA's 4 warps: some CTAs hold the end of one sequence and the

@@ -118,10 +118,24 @@ __global__ void __launch_bounds__(32 * kStoWarps) stochastic_select_kernel(Stoch
   // the first step s >= from whose current value repeats an earlier kept value is a collision
   // of the sequential algorithm (the steps between keep their draws), so it keeps j_s, which
   // exceeds every earlier kept value and so never collides itself; the search resumes at s + 1.
-  // With m << n collisions are rare and this is one or two parallel passes.
+  // With m << n collisions are rare and this is one or two parallel passes; after four passes
+  // the remaining steps run in order (a warp scan per membership test), which bounds the cost
+  // when m is not small against n.
   for (int s = lane; s < m; s += 32) kr[s] = us[s] % ((uint32_t)(n - m + s) + 1u);
   __syncwarp();
-  for (int from = 0;;) {
+  for (int from = 0, passes = 0;; ++passes) {
+    if (passes == 4) {   // many collisions (m not << n): the remaining steps in order
+      for (int s = from; s < m; ++s) {
+        const uint32_t v = kr[s];   // still the draw t_s: only steps before `from` were changed
+        bool seen = false;
+        for (int i = lane; i < s; i += 32) seen |= kr[i] == v;
+        seen = __any_sync(0xFFFFFFFFu, seen);
+        __syncwarp();
+        if (seen && lane == 0) kr[s] = (uint32_t)(n - m + s);
+        __syncwarp();
+      }
+      break;
+    }
     int first = m;   // the first step >= from whose value repeats an earlier one (branch-free scans)
     for (int s = lane; s < m; s += 32) {
       const uint32_t v = kr[s];
