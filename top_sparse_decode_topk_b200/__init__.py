@@ -540,7 +540,7 @@ def _sparse_decode_host(lib, cache: KVCache, queries: Queries, idx, out, lse, wo
     k_max = int(idx.shape[2])
     odt = TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32
     skey = _shape_key(cache, qd)
-    size_key = (skey, k_max, odt, qs.q_dtype)
+    size_key = (str(dev), skey, k_max, odt, qs.q_dtype)   # the work split depends on the device's SM count
     nbytes = _HOST_WS_BYTES.get(size_key)
     if nbytes is None:   # the size depends only on the shapes: asked once per shape
         nbytes = lib.tsd_sparse_decode_host_workspace_size(ctypes.byref(cs), ctypes.byref(qs), k_max, odt)
