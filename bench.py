@@ -677,9 +677,12 @@ def run_native(args):
         flush()
         c, d = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         c.record(stream)
-        idx_d, _ = tsd.topk_select(cache, hq, k_max, k_per_token=kpt_dev, out_idx=idx_buf, out_count=cnt_buf,
+        # q crosses to the device once (inside the timed region) and serves both calls
+        qdev = tsd.Queries(hq.q.to(dev, non_blocking=True), q_indptr=hq.q_indptr,
+                           max_tokens_per_seq=hq.max_tokens_per_seq, causal=hq.causal, sm_scale=hq.sm_scale)
+        idx_d, _ = tsd.topk_select(cache, qdev, k_max, k_per_token=kpt_dev, out_idx=idx_buf, out_count=cnt_buf,
                                    workspace=ws)
-        tsd.sparse_decode(cache, hq, idx_d, out=out_host, lse=lse_host, workspace=ws)
+        tsd.sparse_decode(cache, qdev, idx_d, out=out_host, lse=lse_host, workspace=ws)
         d.record(stream)
         torch.cuda.synchronize()
         if s >= args.warmup:
