@@ -16,6 +16,11 @@ beside it.  Multi-GPU runs are weak scaling: every rank decodes its own batch
 (no data-path collective), the timings are the max over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference] [--config NAME]
+                  [--also NAME,NAME]
+
+The default workload is the ragged batch (32 sequences of 8K-128K tokens, 4 decode queries
+each, k = ceil(0.02 kv_len)): the largest that fits one GPU.  The three legs of the
+Llama-3-8B- and Qwen2.5-72B-shaped workloads are timed too and reported beside it.
 """
 
 from __future__ import annotations
@@ -46,7 +51,11 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["native", "reference"], default="native")
-    p.add_argument("--config", default="llama3_8b")
+    p.add_argument("--config", default="ragged",
+                   help="workload of the line (default: the ragged batch, the largest single-GPU one)")
+    p.add_argument("--also", default="llama3_8b,qwen25_72b",
+                   help="comma-separated workloads whose three legs are timed too and reported under "
+                        "other_workloads ('' for none)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--record-traffic", metavar="NCU_CSV",
                    help="write profiles/dram_traffic.json for --config from an ncu --csv log of "
@@ -324,7 +333,7 @@ def time_cpu_oracle(w, k, budget_s=10.0):
     rng = np.random.default_rng(0)
     groups = [(int(rng.integers(cfg.batch)), int(rng.integers(cfg.num_kv_heads))) for _ in range(2)]
     data = []
-    groups_kv, where = [], []
+    groups_kv, where, toks = [], [], []
     for b, g in groups:
         K = oracle.from_bf16_bits(w.logical_kv_bits(b, g, "k"))
         V = oracle.from_bf16_bits(w.logical_kv_bits(b, g, "v"))
@@ -334,16 +343,17 @@ def time_cpu_oracle(w, k, budget_s=10.0):
             for h in range(g * G, (g + 1) * G):
                 data.append((oracle.from_bf16_bits(w.q_bits[t, h]), K[:L], V[:L]))
                 where.append((len(groups_kv) - 1, L))
+                toks.append(t)
     nlists = len(data)
     total_lists = len(w.kv_len) * cfg.num_q_heads
     kk = w.k_per_token(k)
-    idxs = [oracle.exact_topk(oracle.attention_scores(q, Kb), int(kk[0])) for q, Kb, _ in data]
+    idxs = [oracle.exact_topk(oracle.attention_scores(q, Kb), int(kk[t])) for (q, Kb, _), t in zip(data, toks)]
     # top-k
     t0 = time.perf_counter()
     reps_topk = 0
     while True:
-        for q, Kb, _ in data:
-            oracle.exact_topk(oracle.attention_scores(q, Kb), int(kk[0]))
+        for (q, Kb, _), t in zip(data, toks):
+            oracle.exact_topk(oracle.attention_scores(q, Kb), int(kk[t]))
         reps_topk += 1
         if time.perf_counter() - t0 > budget_s / 2:
             break
@@ -411,6 +421,61 @@ def sum_over_ranks(values, device):
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
         dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return t.tolist()
+
+
+def time_legs(tsd, W, name, rank, dev, steps, warmup, flush):
+    """The three legs (exact top-k, sparse decode at the workload's 50x k, dense decode) of one more
+    workload, timed like the line's own legs (CUDA events, L2 flushed before each), with the
+    algorithmic bytes of each.  Every rank runs it on its own batch; the caller reduces."""
+    import numpy as np
+    import torch
+    cfg = W.CONFIGS[name]
+    k = bench_k(cfg)
+    w = W.make_workload(cfg, seed=rank_seed(rank))
+    dw = W.to_device(w, dev)
+    cache = tsd.KVCache(dw.k, dw.v, dw.seq_lens, max_seq_len=cfg.max_seq_len,
+                        page_table=None if cfg.layout == "contiguous" else dw.page_table)
+    multi = cfg.tokens_per_seq > 1
+    queries = tsd.Queries(dw.q, q_indptr=dw.q_indptr if multi else None, max_tokens_per_seq=cfg.tokens_per_seq,
+                          causal=cfg.causal, sm_scale=1.0 / math.sqrt(128))
+    kpt = w.k_per_token(k)
+    k_max = int(kpt.max())
+    kpt_dev = None if k is not None else torch.from_numpy(kpt).to(dev)
+    odt = torch.float32 if cfg.out_dtype == "f32" else torch.bfloat16
+    ws = tsd.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+    T, Hq = len(w.kv_len), cfg.num_q_heads
+    idx = torch.empty((T, Hq, k_max), dtype=torch.int32, device=dev)
+    cnt = torch.empty((T, Hq), dtype=torch.int32, device=dev)
+    legs = [lambda: tsd.topk_select(cache, queries, k_max, k_per_token=kpt_dev, out_idx=idx, out_count=cnt,
+                                    workspace=ws),
+            lambda: tsd.sparse_decode(cache, queries, idx, out_dtype=odt, workspace=ws),
+            lambda: tsd.dense_decode(cache, queries, out_dtype=odt, workspace=ws)]
+    for _ in range(max(3, warmup)):
+        for leg in legs:
+            flush()
+            leg()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for s_ in range(steps):
+        for j, leg in enumerate(legs):
+            flush()
+            ev[s_][2 * j].record(stream)
+            leg()
+            ev[s_][2 * j + 1].record(stream)
+    torch.cuda.synchronize()
+    if tsd.read_device_status(ws) != 0:
+        raise RuntimeError(f"device status bits set on {name}")
+    ms = np.array([[ev[s_][2 * j].elapsed_time(ev[s_][2 * j + 1]) for j in range(3)] for s_ in range(steps)])
+    U = unique_rows(idx, torch.from_numpy(w.token_seq).to(dev), cfg.num_kv_heads, cfg.group, cfg.max_seq_len)
+    ob = 4 if odt == torch.float32 else 2
+    q_bytes, o_bytes = T * Hq * 128 * 2, T * Hq * 128 * ob
+    ctx_rows = int(sum(int(L) for L in w.seq_lens)) * cfg.num_kv_heads
+    nbytes = [ctx_rows * 256 + q_bytes + T * Hq * k_max * 4, U * 512 + q_bytes + o_bytes,
+              ctx_rows * 512 + q_bytes + o_bytes]
+    del cache, queries, dw, ws, idx, cnt
+    torch.cuda.empty_cache()
+    return ms.mean(axis=0).tolist(), nbytes, k_max, U
 
 
 def run_native(args):
@@ -692,6 +757,25 @@ def run_native(args):
     if tsd.read_device_status(ws) != 0:
         raise RuntimeError("device status bits set during the timed run")
 
+    # the three legs of the other workloads named by --also (every rank, same order)
+    others = {}
+    for name in [x for x in args.also.split(",") if x and x != cfg.name]:
+        o_ms, o_bytes, o_k, o_u = time_legs(tsd, W, name, rank, dev, max(3, args.steps // 2), args.warmup, flush)
+        o_ms = max_over_ranks(o_ms, dev)
+        o_gbs = [gbs(b_, m_) for b_, m_ in zip(o_bytes, o_ms)]
+        others[name] = {
+            "k": o_k, "unique_rows": o_u,
+            "legs_us": {"topk_select": round(o_ms[0] * 1e3, 3), "sparse_decode": round(o_ms[1] * 1e3, 3),
+                        "dense_decode": round(o_ms[2] * 1e3, 3)},
+            "achieved_gbs": {"topk_select": round(o_gbs[0], 1), "sparse_decode": round(o_gbs[1], 1),
+                             "dense_decode": round(o_gbs[2], 1)},
+            "frac_of_peak": {"topk_select": round(o_gbs[0] / hbm, 4), "sparse_decode": round(o_gbs[1] / hbm, 4),
+                             "dense_decode": round(o_gbs[2] / hbm, 4)},
+            "speedup_vs_dense": round(o_ms[2] / o_ms[1], 3),
+            "speedup_vs_dense_with_indexer": round(o_ms[2] / (o_ms[0] + o_ms[1]), 3),
+            "algorithmic_bytes": {"topk_select": o_bytes[0], "sparse_decode": o_bytes[1],
+                                  "dense_decode": o_bytes[2]}}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_cpu_oracle(w, k)
@@ -715,8 +799,11 @@ def run_native(args):
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
-        "storage_dtype": "bf16",
+        "dtype": "bf16",
+        "dtype_detail": "bf16 K/V/q storage; q.K and P.V on bf16 tensor-core MMAs (mma.sync m16n8k16) with fp32 "
+                        "accumulation; the softmax weights enter P.V as a bf16 hi + lo pair (about 16 significant "
+                        "bits); softmax, split merge and normalisation in fp32; "
+                        + ("fp32 output" if out_dtype == torch.float32 else "bf16 output"),
         "data": "synthetic (seeded Philox N(0,1) bf16 K/V/q with planted needles/sink/window)"
                 if cfg.planted else "synthetic (seeded Philox N(0,1) bf16 K/V/q)",
         "config": workload_desc(cfg, k_max),
@@ -748,6 +835,7 @@ def run_native(args):
         "graph_step": graph_line,
         "graph20_rotating": graph20_line,
         "sparse_leg_us_stats": sparse_stats,
+        "other_workloads": others,
         "gpu_launches": 4 * args.steps,
         "clocks": cl,
     }

@@ -239,7 +239,9 @@ tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* querie
  *  - Shapes whose scratch exceeds 16 MiB return TSD_ERR_WORKSPACE_TOO_SMALL without
  *    launching (16 MiB covers e.g. 8 sequences x 32 q heads at k = 655).
  *  - The first call on each device looks up the array's device address with that device
- *    current; make that first call before any stream capture.
+ *    current and keeps it for later calls; make that first call before any stream capture.
+ *    A cudaDeviceReset destroys the array with the context: the kept address is then stale,
+ *    so do not call this entry point on a device after resetting it in the same process.
  *  - Every call shares the one array and clears its status word and merge counters on
  *    `stream` before launching: calls that overlap on the GPU (other streams, other host
  *    threads) race and must be serialized by the caller.

@@ -39,6 +39,12 @@ from .attention import (  # noqa: F401
     from_bf16_bits,
     sparse_attention,
 )
-from .compare import topk_sets_agree, output_errors  # noqa: F401
+from .compare import (  # noqa: F401
+    bf16_half_ulp,
+    elementwise_bar,
+    output_errors,
+    output_within,
+    topk_sets_agree,
+)
 from .label import channel_importance, choose_channels, label_scores  # noqa: F401
 from .vattention import floyd_sample, stochastic_select, weighted_attention  # noqa: F401

@@ -17,11 +17,10 @@ import numpy as np
 import oracle
 from top_sparse_decode_topk_b200 import workload as W
 
-# Acceptance bars.  bf16 outputs: max-abs 5e-3 and rel-L2 2e-3 (task statement); the
-# max-abs bar is applied on top of the output format's own rounding (half a bf16 ulp
-# of the exact value), since above |o| = 1.28 that rounding alone exceeds 5e-3.
-# fp32 outputs: derived from the arithmetic (fp32 accumulation and ex2.approx give
-# relative errors ~1e-6 on outputs of size ~1).
+# Acceptance bars.  bf16 outputs: max-abs 5e-3 and rel-L2 2e-3; where bf16 rounding alone
+# exceeds 5e-3 (|o| >= 2) the per-element bar is half a bf16 ulp plus 1e-4 |o|
+# (oracle.elementwise_bar).  fp32 outputs: derived from the arithmetic (fp32
+# accumulation and ex2.approx give relative errors ~1e-6 on outputs of size ~1).
 BF16_MAX_ABS, BF16_REL_L2 = 5e-3, 2e-3
 F32_MAX_ABS, F32_REL_L2 = 1e-4, 2e-5
 LSE_ABS = 1e-3
@@ -107,13 +106,6 @@ def check_topk(inp: OracleInputs, gpu_idx: np.ndarray, gpu_count: np.ndarray, k_
     return stats
 
 
-def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
-    """Half the spacing of bf16 numbers at |x| (8 significant bits)."""
-    a = np.abs(np.asarray(x, dtype=np.float64))
-    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
-    return np.exp2(e - 8)
-
-
 def check_decode(inp: OracleInputs, idx: np.ndarray, out: np.ndarray, lse: np.ndarray, pairs, sm_scale: float,
                  out_is_bf16: bool, dense: bool = False) -> Tuple[float, float]:
     """Compare GPU rows with the oracle; returns the worst (max_abs, rel_l2)."""
@@ -126,12 +118,10 @@ def check_decode(inp: OracleInputs, idx: np.ndarray, out: np.ndarray, lse: np.nd
         else:
             o_ref, lse_ref = inp.attend(t, h, idx[t, h], sm_scale)
         o = out[t, h].astype(np.float64)
-        ma, rl = oracle.output_errors(o, o_ref)
+        ma, _ = oracle.output_errors(o, o_ref)
         worst_abs = max(worst_abs, ma)
-        allowed = tol_abs + (bf16_half_ulp(o_ref) if out_is_bf16 else 0.0)
-        excess = np.abs(o - o_ref) - allowed
-        assert np.all(excess <= 0), (f"(t={t}, h={h}) error {ma:.3g} exceeds {tol_abs}"
-                                     f"{' + half a bf16 ulp' if out_is_bf16 else ''}")
+        ok, why = oracle.output_within(o, o_ref, tol_abs, math.inf, out_is_bf16)
+        assert ok, f"(t={t}, h={h}): {why}"
         refs.append(o_ref)
         gots.append(o)
         if lse is not None:

@@ -238,3 +238,21 @@ def test_context_parallel_errors_before_launch(lib):
     assert lib.tsd_merge_partials(4, 256, FAKE, FAKE, FAKE, 7, None, None) == tsd.TSD_ERR_UNSUPPORTED
     assert lib.tsd_merge_partials(0, 256, FAKE, FAKE, FAKE, 0, None, None) == tsd.TSD_ERR_INVALID_ARGUMENT
     assert lib.tsd_merge_partials(4, 256, FAKE + 4, FAKE, FAKE, 0, None, None) == tsd.TSD_ERR_INVALID_ARGUMENT
+
+
+@fake_pointer_call
+def test_static_scratch_refuses_oversize_shapes(lib):
+    """tsd_sparse_decode_static_ws refuses, on the host, a shape whose scratch exceeds its
+    16 MiB array: 2048 tokens x 32 heads of split-K rows alone are over 34 MB."""
+    c = make_cache(batch=512, max_pages=8192, num_pages=512 * 8192, max_seq_len=131072)
+    q = make_queries(tokens=2048, q_indptr=FAKE + 0x800000, max_tokens=4)
+    need = lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 2622)
+    assert need > 2 * (16 << 20)
+    rc = lib.tsd_sparse_decode_static_ws(ctypes.byref(c), ctypes.byref(q), FAKE + 0x500000, 2622, FAKE + 0x600000,
+                                         tsd.TSD_BF16, None, None, None)
+    assert rc == tsd.TSD_ERR_WORKSPACE_TOO_SMALL
+    # and rejects bad arguments the way tsd_sparse_decode does
+    assert lib.tsd_sparse_decode_static_ws(ctypes.byref(make_cache(head_dim=64)), ctypes.byref(make_queries()),
+                                           FAKE, 8, FAKE, 0, None, None, None) == tsd.TSD_ERR_UNSUPPORTED
+    assert lib.tsd_sparse_decode_static_ws(ctypes.byref(make_cache()), ctypes.byref(make_queries()), None, 8, FAKE,
+                                           0, None, None, None) == tsd.TSD_ERR_INVALID_ARGUMENT

@@ -412,7 +412,7 @@ def test_full_qwen25_72b():
 
 
 def test_full_ragged():
-    _full_topk_and_decode("ragged", ks=(None,), n_random=6, check_dense=False)
+    _full_topk_and_decode("ragged", ks=(None,), n_random=6)
 
 
 def test_full_sweep():

@@ -12,7 +12,9 @@
 // GPU that loads this library holds that much memory until the process exits.
 // Host code cannot use the array's name as an address: the first call on each
 // device asks the runtime for the array's device address (cudaGetSymbolAddress)
-// with that device current, checks the result and keeps it for later calls.
+// with that device current, checks the result and keeps it for later calls.  The kept
+// address belongs to the device's primary context: after a cudaDeviceReset it is stale, and
+// the entry point must not be called on that device again in the same process.
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
