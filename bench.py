@@ -630,9 +630,9 @@ def run_native(args):
     lse_g = torch.empty((T, Hq), dtype=torch.float32, device=dev)
     kpt_g = kpt_dev
 
-    def step_exact():
-        tsd.topk_select(cache, queries, k_max, k_per_token=kpt_g, out_idx=idx_buf, out_count=cnt_buf, workspace=ws)
-        tsd.sparse_decode(cache, queries, idx_buf, out=out_g, lse=lse_g, workspace=ws)
+    def step_exact():   # the library's one-call step (tsd_decode_step)
+        tsd.decode_step(cache, queries, k_max, k_per_token=kpt_g, out_idx=idx_buf, out_count=cnt_buf, out=out_g,
+                        lse=lse_g, workspace=ws)
 
     def step_label():
         tsd.topk_select_label(cache, label_index, queries, k_max, k_per_token=kpt_g, out_idx=idx_buf,
@@ -673,7 +673,8 @@ def run_native(args):
                   "step_stochastic_us": round(gx[3] * 1e3, 2), "stochastic_samples": m_sto,
                   "net_speedup_exact": round(dense_ms / gx[1], 3), "net_speedup_label": round(dense_ms / gx[2], 3),
                   "net_speedup_stochastic": round(dense_ms / gx[3], 3),
-                  "what": "one CUDA graph per decode step (indexer + sparse decode, k of this line; the "
+                  "what": "one CUDA graph per decode step (indexer + sparse decode, k of this line; the exact "
+                          "step is one tsd_decode_step call; the "
                           "stochastic step adds m uniform samples of the other tokens with Horvitz-Thompson "
                           "weights and decodes with them), L2 flushed before each replay; dense decode by "
                           "events as in legs_us"}
@@ -760,21 +761,21 @@ def run_native(args):
     # the three legs of the other workloads named by --also (every rank, same order)
     others = {}
     for name in [x for x in args.also.split(",") if x and x != cfg.name]:
-        o_ms, o_bytes, o_k, o_u = time_legs(tsd, W, name, rank, dev, max(3, args.steps // 2), args.warmup, flush)
-        o_ms = max_over_ranks(o_ms, dev)
-        o_gbs = [gbs(b_, m_) for b_, m_ in zip(o_bytes, o_ms)]
+        x_ms, x_bytes, x_k, x_u = time_legs(tsd, W, name, rank, dev, max(3, args.steps // 2), args.warmup, flush)
+        x_ms = max_over_ranks(x_ms, dev)
+        x_gbs = [gbs(b_, m_) for b_, m_ in zip(x_bytes, x_ms)]
         others[name] = {
-            "k": o_k, "unique_rows": o_u,
-            "legs_us": {"topk_select": round(o_ms[0] * 1e3, 3), "sparse_decode": round(o_ms[1] * 1e3, 3),
-                        "dense_decode": round(o_ms[2] * 1e3, 3)},
-            "achieved_gbs": {"topk_select": round(o_gbs[0], 1), "sparse_decode": round(o_gbs[1], 1),
-                             "dense_decode": round(o_gbs[2], 1)},
-            "frac_of_peak": {"topk_select": round(o_gbs[0] / hbm, 4), "sparse_decode": round(o_gbs[1] / hbm, 4),
-                             "dense_decode": round(o_gbs[2] / hbm, 4)},
-            "speedup_vs_dense": round(o_ms[2] / o_ms[1], 3),
-            "speedup_vs_dense_with_indexer": round(o_ms[2] / (o_ms[0] + o_ms[1]), 3),
-            "algorithmic_bytes": {"topk_select": o_bytes[0], "sparse_decode": o_bytes[1],
-                                  "dense_decode": o_bytes[2]}}
+            "k": x_k, "unique_rows": x_u,
+            "legs_us": {"topk_select": round(x_ms[0] * 1e3, 3), "sparse_decode": round(x_ms[1] * 1e3, 3),
+                        "dense_decode": round(x_ms[2] * 1e3, 3)},
+            "achieved_gbs": {"topk_select": round(x_gbs[0], 1), "sparse_decode": round(x_gbs[1], 1),
+                             "dense_decode": round(x_gbs[2], 1)},
+            "frac_of_peak": {"topk_select": round(x_gbs[0] / hbm, 4), "sparse_decode": round(x_gbs[1] / hbm, 4),
+                             "dense_decode": round(x_gbs[2] / hbm, 4)},
+            "speedup_vs_dense": round(x_ms[2] / x_ms[1], 3),
+            "speedup_vs_dense_with_indexer": round(x_ms[2] / (x_ms[0] + x_ms[1]), 3),
+            "algorithmic_bytes": {"topk_select": x_bytes[0], "sparse_decode": x_bytes[1],
+                                  "dense_decode": x_bytes[2]}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

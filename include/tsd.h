@@ -151,10 +151,11 @@ size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_que
  *   lse[t,h] = M + ln sum_i exp(z_i - M)       (natural log of the scaled scores)
  * idx: device int32 [T][Hq][k_max].  Each list holds token indices in non-decreasing order
  *   (as tsd_topk_select writes them), followed by -1 padding; every entry is one term, so a
- *   repeated token counts once per occurrence.  Entries >= kv_len(t) or < -1 are skipped and
- *   set TSD_DEV_BAD_INDEX; an observed descending pair sets TSD_DEV_UNSORTED (the result for
- *   such a list is unspecified).  Rows shared by several lists of one kv head (the q heads of a
- *   GQA group and the query tokens of one sequence) are loaded from memory once.
+ *   repeated token counts once per occurrence.  A list ends at its first -1: the entries after
+ *   it are padding and may be left unread.  Entries >= kv_len(t) or < -1 are skipped and set
+ *   TSD_DEV_BAD_INDEX; an observed descending pair sets TSD_DEV_UNSORTED (the result for such a
+ *   list is unspecified).  Rows shared by several lists of one kv head (the q heads of a GQA
+ *   group and the query tokens of one sequence) are loaded from memory once.
  * out: device [T][Hq][128] of out_dtype (TSD_BF16 or TSD_F32).  An empty list gives zeros.
  * lse: device f32 [T][Hq] or NULL; -inf for an empty list.
  */
@@ -227,6 +228,34 @@ size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_quer
 tsd_status tsd_dense_decode(const tsd_kv_cache* cache, const tsd_queries* queries, void* out,
                             int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
                             tsd_stream_t stream);
+
+/* Host: bytes of workspace tsd_decode_step needs for these shapes on the current device: the
+ * larger of the top-k and sparse-decode workspaces (they share one region, used one after the
+ * other), plus room for the index lists when the caller passes no out_idx (0 on invalid input). */
+size_t tsd_decode_step_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max);
+
+/*
+ * One decode step of the method: the exact top-k indexer followed by sparse decode over the
+ * rows it selected ("Inference Time Context Sparsity: Illusion or Opportunity?", section 3.C,
+ * "Indexing overhead": the indexer's cost is part of the end-to-end step).  It computes
+ *   idx = tsd_topk_select(cache, queries, k_max, k_per_token)
+ *   out, lse = tsd_sparse_decode(cache, queries, idx)
+ * with both calls on one workspace and on `stream`: the fp32 score rows of the first are read
+ * by its own selection kernel (the K stream is loaded evict-first, so they stay in L2), and
+ * the second reuses the same bytes for its split-K partials.  Nothing is allocated and the
+ * host never waits, so the step can be captured into one CUDA graph and replayed.
+ * out_idx  : device int32 [T][Hq][k_max] receiving the selected lists, or NULL to keep them
+ *            inside `ws`.
+ * out_count: device int32 [T][Hq] or NULL; receives min(k_t, kv_len(t)).
+ * out, out_dtype, lse: as tsd_sparse_decode.
+ * ws: at least tsd_decode_step_workspace_size bytes, 256-byte aligned, zeroed once
+ *   (tsd_workspace_init); every call leaves its leading region zero again.
+ * Errors: as tsd_topk_select and tsd_sparse_decode (nothing is launched on a host-checkable
+ * error); device-detected problems set bits in the status word at the start of `ws`.
+ */
+tsd_status tsd_decode_step(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                           const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count, void* out,
+                           int32_t out_dtype, float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream);
 
 /*
  * Sparse decode for callers that cannot allocate device memory.  The pages have no

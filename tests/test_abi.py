@@ -256,3 +256,28 @@ def test_static_scratch_refuses_oversize_shapes(lib):
                                            FAKE, 8, FAKE, 0, None, None, None) == tsd.TSD_ERR_UNSUPPORTED
     assert lib.tsd_sparse_decode_static_ws(ctypes.byref(make_cache()), ctypes.byref(make_queries()), None, 8, FAKE,
                                            0, None, None, None) == tsd.TSD_ERR_INVALID_ARGUMENT
+
+
+@fake_pointer_call
+def test_decode_step_errors_before_launch(lib):
+    """tsd_decode_step checks what both of its calls check before it enqueues anything, and
+    sizes one region for the two workspaces (plus the lists when the caller keeps none)."""
+    c, q = make_cache(), make_queries()
+    step = lib.tsd_decode_step_workspace_size(ctypes.byref(c), ctypes.byref(q), 655)
+    topk = lib.tsd_topk_workspace_size(ctypes.byref(c), ctypes.byref(q), 655)
+    dec = lib.tsd_sparse_decode_workspace_size(ctypes.byref(c), ctypes.byref(q), 655)
+    assert step >= max(topk, dec) + 8 * 32 * 655 * 4
+    assert step < topk + dec + 8 * 32 * 655 * 4 + 1024   # one shared region, not two
+    assert lib.tsd_decode_step_workspace_size(ctypes.byref(c), ctypes.byref(q), 0) == 0
+
+    def call(cc=c, qq=q, k_max=655, out=FAKE + 0x600000, out_dtype=0, ws=FAKE + 0x700000, ws_bytes=1 << 40,
+             out_idx=None):
+        return lib.tsd_decode_step(ctypes.byref(cc), ctypes.byref(qq), k_max, None, out_idx, None, out, out_dtype,
+                                   None, ws, ws_bytes, None)
+    assert call(ws_bytes=max(topk, dec)) == tsd.TSD_ERR_WORKSPACE_TOO_SMALL   # no room for the lists
+    assert call(k_max=0) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert call(out=None) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert call(out_dtype=5) == tsd.TSD_ERR_UNSUPPORTED
+    assert call(ws=FAKE + 0x700010) == tsd.TSD_ERR_INVALID_ARGUMENT        # workspace not 256-byte aligned
+    assert call(cc=make_cache(head_dim=64)) == tsd.TSD_ERR_UNSUPPORTED
+    assert call(k_max=1 << 20) == tsd.TSD_ERR_UNSUPPORTED

@@ -89,6 +89,12 @@ EXPORTS = {
                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.c_void_p]),
     "tsd_read_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "tsd_decode_step_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
+                                                         ctypes.c_int32]),
+    "tsd_decode_step": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                       ctypes.c_void_p]),
     "tsd_sparse_decode_static_ws": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
                                                    ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
                                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
@@ -511,6 +517,37 @@ def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=Non
                                               k_max, out.data_ptr(), odt, lp, ws.data_ptr(), ws.numel(), sp),
                "tsd_sparse_decode_weighted")
     return _finish(out, host_out, lse, host_lse, s)
+
+
+def decode_step(cache: KVCache, queries: Queries, k_max: int, k_per_token=None, out_idx=None, out_count=None,
+                out=None, out_dtype=None, lse=True, workspace: Optional[Workspace] = None, stream=None):
+    """One decode step (tsd_decode_step): exact top-k, then sparse decode over the selected
+    rows, on one workspace and with no host synchronisation, so that it can be captured in a
+    CUDA graph.  Device tensors only.  out_idx: int32 [T, Hq, k_max] to receive the lists, or
+    None to keep them in the workspace.  Returns (out, lse or None, out_idx or None)."""
+    import torch
+    lib = load_library()
+    dev = cache.device
+    s, sp = _stream_ptr(stream, dev)
+    for name, t in (("q", queries.q), ("k_per_token", k_per_token), ("out_idx", out_idx), ("out_count", out_count),
+                    ("out", out)):
+        if t is not None and t.device != dev:
+            raise ValueError(f"decode_step takes device tensors only ({name} is on {t.device})")
+    if k_per_token is not None and (k_per_token.dtype != torch.int32 or k_per_token.numel() != queries.q.shape[0]):
+        raise ValueError("k_per_token must be int32 [T]")
+    out_dtype = out_dtype or (out.dtype if out is not None else torch.bfloat16)
+    out, _, lse, _ = _out_buffers(queries, out, out_dtype, lse, dev)
+    cs, qs = cache.c_struct(), queries.c_struct()
+    nbytes = lib.tsd_decode_step_workspace_size(ctypes.byref(cs), ctypes.byref(qs), int(k_max))
+    if nbytes == 0:
+        raise TsdError(TSD_ERR_INVALID_ARGUMENT, "tsd_decode_step_workspace_size")
+    ws = _ws(workspace, dev).get(nbytes, _shape_key(cache, queries), sp)
+    odt = TSD_BF16 if out.dtype == torch.bfloat16 else TSD_F32
+    ptr = lambda t: None if t is None else t.data_ptr()
+    _check(lib.tsd_decode_step(ctypes.byref(cs), ctypes.byref(qs), int(k_max), ptr(k_per_token), ptr(out_idx),
+                               ptr(out_count), out.data_ptr(), odt, ptr(lse), ws.data_ptr(), ws.numel(), sp),
+           "tsd_decode_step")
+    return out, lse, out_idx
 
 
 _HOST_WS_BYTES = {}

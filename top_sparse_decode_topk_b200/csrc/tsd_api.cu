@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -225,6 +226,29 @@ static int current_sm_count() {
   return cache[dev];
 }
 
+// Work decomposition of tsd_sparse_decode.  The one-task-per-warp kernel fits its grid to one
+// wave of resident CTAs; when its tasks need more than one wave, the persistent kernel takes
+// the call instead.  TSD_SPARSE_KERNEL=wave|stream forces either form and TSD_SPARSE_CHUNK
+// sets the persistent form's entries per task (both for measurements; read at every call, so
+// size the workspace under the same setting as the call).
+static SparsePlan sparse_plan(const Shapes& sh, int k_max) {
+  const int sms = current_sm_count();
+  const char* kind = getenv("TSD_SPARSE_KERNEL");
+  const char* chunk = getenv("TSD_SPARSE_CHUNK");
+  const int e_override = chunk != nullptr ? atoi(chunk) : 0;
+  const SparsePlan wave = plan_sparse(sh, k_max, sms);
+  bool stream;
+  if (kind != nullptr && strcmp(kind, "stream") == 0) {
+    stream = true;
+  } else if (kind != nullptr && strcmp(kind, "wave") == 0) {
+    stream = false;
+  } else {
+    const int64_t ctas = (sh.batch * sh.hkv * wave.lists * (int64_t)wave.nsplit + kSpTasksPerCta - 1) / kSpTasksPerCta;
+    stream = ctas > (int64_t)sms * kSpCtasPerSm;
+  }
+  return stream ? plan_sparse_stream(sh, k_max, sms, e_override) : wave;
+}
+
 static tsd_status sizes_for(const tsd_kv_cache* cache, const tsd_queries* queries, Shapes* sh) {
   if (cache == nullptr || queries == nullptr) return TSD_ERR_INVALID_ARGUMENT;
   KvView kv; QView qv;
@@ -242,7 +266,7 @@ static tsd_status sizes_for(const tsd_kv_cache* cache, const tsd_queries* querie
 size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max) {
   Shapes sh;
   if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return 0;
-  const SparsePlan p = plan_sparse(sh, k_max, current_sm_count());
+  const SparsePlan p = sparse_plan(sh, k_max);
   return decode_layout(sh, p.nsplit).total;
 }
 
@@ -342,7 +366,7 @@ static tsd_status sparse_decode_impl(const tsd_kv_cache* cache, const tsd_querie
   if (st != TSD_OK) return st;
   if (idx == nullptr || k_max < 1) return TSD_ERR_INVALID_ARGUMENT;
   if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
-  const SparsePlan p = plan_sparse(sh, k_max, current_sm_count());
+  const SparsePlan p = sparse_plan(sh, k_max);
   const DecodeLayout lay = decode_layout(sh, p.nsplit);
   if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
   DecodeArgs a;
@@ -363,6 +387,8 @@ static tsd_status sparse_decode_impl(const tsd_kv_cache* cache, const tsd_querie
   a.counters = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_counters);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + lay.off_ml);
   a.part_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_acc);
+  a.sched = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 4);
+  a.persistent = p.stream;
   return cuda_status(launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -370,6 +396,49 @@ tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queri
                              int32_t k_max, void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
                              tsd_stream_t stream) {
   return sparse_decode_impl(cache, queries, idx, nullptr, k_max, out, out_dtype, lse, ws, ws_bytes, stream);
+}
+
+// tsd_decode_step: the top-k and sparse-decode workspaces overlaid on one region (the score
+// rows are dead once the selection has run), then the index lists when the caller keeps none.
+struct StepLayout {
+  size_t shared, off_idx, total;
+};
+
+static bool step_layout(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max, bool own_idx,
+                        StepLayout* L) {
+  Shapes sh;
+  if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return false;
+  const size_t topk = topk_layout(sh).total;
+  const size_t dec = decode_layout(sh, sparse_plan(sh, k_max).nsplit).total;
+  L->shared = align256(topk > dec ? topk : dec);
+  L->off_idx = L->shared;
+  L->total = L->shared + (own_idx ? align256((size_t)sh.tokens * sh.hq * k_max * sizeof(int32_t)) : 0);
+  return true;
+}
+
+size_t tsd_decode_step_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max) {
+  StepLayout L;
+  return step_layout(cache, queries, k_max, true, &L) ? L.total : 0;
+}
+
+tsd_status tsd_decode_step(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                           const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count, void* out,
+                           int32_t out_dtype, float* lse, void* ws, size_t ws_bytes, tsd_stream_t stream) {
+  // every host check of both calls runs before anything is enqueued
+  {
+    KvView kv; QView qv; Shapes sh;
+    tsd_status st = decode_common(cache, queries, out, out_dtype, lse, ws, ws_bytes, &kv, &qv, &sh);
+    if (st != TSD_OK) return st;
+    if (k_max < 1) return TSD_ERR_INVALID_ARGUMENT;
+    if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
+  }
+  StepLayout L;
+  if (!step_layout(cache, queries, k_max, out_idx == nullptr, &L)) return TSD_ERR_INVALID_ARGUMENT;
+  if (ws_bytes < L.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
+  int32_t* idx = out_idx != nullptr ? out_idx : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.off_idx);
+  tsd_status st = topk_select_impl(cache, queries, k_max, k_per_token, idx, nullptr, out_count, ws, L.shared, stream);
+  if (st != TSD_OK) return st;
+  return sparse_decode_impl(cache, queries, idx, nullptr, k_max, out, out_dtype, lse, ws, L.shared, stream);
 }
 
 // Device staging of tsd_sparse_decode_host, after the sparse-decode workspace.
@@ -382,7 +451,7 @@ static bool host_staging(const tsd_kv_cache* cache, const tsd_queries* queries, 
   Shapes sh;
   if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return false;
   if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return false;
-  const SparsePlan p = plan_sparse(sh, k_max, current_sm_count());
+  const SparsePlan p = sparse_plan(sh, k_max);
   *decode_bytes = decode_layout(sh, p.nsplit).total;
   const size_t lists = (size_t)queries->num_tokens * queries->num_q_heads;
   size_t off = align256(*decode_bytes);
@@ -626,9 +695,10 @@ tsd_status prepare_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* q
   if (out == nullptr || idx == nullptr || k_max < 1) return TSD_ERR_INVALID_ARGUMENT;
   if (out_dtype != TSD_BF16 && out_dtype != TSD_F32) return TSD_ERR_UNSUPPORTED;
   if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
-  const SparsePlan p = plan_sparse(*sh, k_max, current_sm_count());
+  const SparsePlan p = sparse_plan(*sh, k_max);
   const DecodeLayout lay = decode_layout(*sh, p.nsplit);
   memset(a, 0, sizeof(*a));
+  a->persistent = p.stream;
   a->kv = kv;
   a->qv = qv;
   a->idx = idx;

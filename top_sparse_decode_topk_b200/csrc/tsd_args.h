@@ -24,6 +24,8 @@ struct DecodeArgs {
   uint32_t* counters;
   float2* part_ml;
   float* part_acc;
+  uint32_t* sched;      // sparse, persistent kernel: [0] next task to hand out, [1] warps done (zero region)
+  int32_t persistent;   // sparse: 1 runs the persistent kernel (span = E, a multiple of 32)
 };
 
 struct TopkArgs {

@@ -601,6 +601,442 @@ __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel
 }
 
 // ---------------------------------------------------------------------------
+// Sparse decode, persistent form
+// ---------------------------------------------------------------------------
+// The one-task-per-warp kernel above fits its grid to one wave of resident CTAs.  When the
+// lists outnumber that wave (many decode tokens, long and unequal lists), it runs several
+// waves whose CTAs each pay the dependent start (sequence -> index -> page -> row) again, and
+// its last wave runs with idle SMs.  This form keeps kSsCtasPerSm CTAs on every SM for the
+// whole call instead.  Every warp takes (list, chunk) tasks from a counter in the workspace
+// until none is left, and its pipeline runs straight across task boundaries:
+//   S3  raw indices of a window (32 entries, one per lane) -- a new task is fetched here;
+//   S2  the window resolved to physical rows (order / range / page checks);
+//   S1  the window whose two 16-row tiles are being copied into the ring;
+//   S0  the window whose tiles are consumed (q K^T, online softmax, P V on the tensor cores).
+// A task's descriptor (list, chunk, bounds) and its q row sit in a per-warp shared-memory slot
+// from the fetch until the task finishes.  A chunk whose first entry is -1 lies past the end
+// of its list and is skipped at the fetch; a window whose entries are all -1 ends its task.
+// Split-K partials: a list of C > 1 chunks has its non-empty chunks write partials and arrive
+// on the list's counter; the chunk that holds the list's last entry adds its chunk count in
+// the counter's upper half, so the arrival that completes the count -- whichever it is --
+// merges the partials.  The last warp of the grid to finish clears the counters.
+constexpr int kSsWarps = kSsWarpsPerCta;
+constexpr int kSsThreads = 32 * kSsWarps;
+constexpr int kSsSlots = 4;                                   // task slots per warp
+constexpr uint32_t kTagSlot = 3u;                            // slot bits of a window tag
+constexpr uint32_t kTagFirst = 1u << 8;                      // first window of its task
+constexpr uint32_t kTagLast = 1u << 9;                       // last window of its task
+constexpr uint32_t kTagBubble = 1u << 10;                    // a window with no entries
+constexpr uint32_t kTagEnd = 1u << 11;                       // the warp has no task left
+static_assert(kSsSlots - 1 == (int)kTagSlot, "slot bits");
+
+struct SsDesc {
+  int list, c, e1, kvlen, b, g, pad0, pad1;
+};
+constexpr size_t kSsRingBytes = (size_t)kSsWarps * kSpStages * kSpTileBytes;
+constexpr size_t kSsQBytes = (size_t)kSsWarps * kSsSlots * 512;   // fp32 q rows at most
+constexpr size_t kSsDescBytes = (size_t)kSsWarps * kSsSlots * sizeof(SsDesc);
+constexpr size_t kSsAccBytes = (size_t)kSsWarps * kHeadDim * sizeof(float);
+constexpr size_t kSsSmemBytes = kSsRingBytes + kSsQBytes + kSsDescBytes + kSsAccBytes;
+static_assert(kSsCtasPerSm * (kSsSmemBytes + 2048) <= 228 * 1024, "resident persistent CTAs per SM");
+
+// One 16-row tile of a list (ring stage `st`: K rows then V rows, chunk-swizzled): scores on
+// the tensor cores, the lazily moved online softmax, and O^T += V^T P^T.  `tmask` holds the
+// tile's valid rows; lw (weighted form) is this lane's entry weight of the tile's window.
+template <bool WEIGHTED>
+__device__ __forceinline__ void sp_tile(uint32_t st, uint32_t tmask, const uint32_t (&qb)[8][2], float scale,
+                                        float lw, int p, float& m_run, float& l_run, float (&o)[8][4]) {
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  const int lane = threadIdx.x & 31;
+  const int gi = lane >> 2;
+  const bool scol = (lane & 3) == 0;
+  const int psrc = 8 * (lane & 3);
+  const int kr = lane & 15, kh = lane >> 4;
+  const int vr = (lane & 7) + 8 * (lane >> 4), vh = (lane >> 3) & 1;
+  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    uint32_t af[4];
+    ldsm_x4(st + sp_off(kr, 2 * ks + kh), af[0], af[1], af[2], af[3]);
+    mma_bf16((ks & 1) ? d1 : d0, af, qb[ks][0], qb[ks][1]);
+  }
+  float s0 = ((d0[0] + d1[0]) + (d0[1] + d1[1])) * scale;
+  float s1 = ((d0[2] + d1[2]) + (d0[3] + d1[3])) * scale;
+  if (WEIGHTED) {
+    s0 += __shfl_sync(FULL, lw, 16 * p + gi);
+    s1 += __shfl_sync(FULL, lw, 16 * p + gi + 8);
+  }
+  s0 = (scol && ((tmask >> gi) & 1u)) ? s0 : -CUDART_INF_F;
+  s1 = (scol && ((tmask >> (gi + 8)) & 1u)) ? s1 : -CUDART_INF_F;
+  float mt = fmaxf(s0, s1);
+  mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 4));
+  mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 8));
+  mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 16));
+  mt = __shfl_sync(FULL, mt, 0);
+  if (mt == -CUDART_INF_F) return;   // uniform over the warp
+  if (mt > m_run + kSpLazyMax) {
+    const float alpha = fast_exp2(m_run - mt);
+    l_run *= alpha;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      o[i][0] *= alpha; o[i][1] *= alpha; o[i][2] *= alpha; o[i][3] *= alpha;
+    }
+    m_run = mt;
+  }
+  const float p0 = fast_exp2(s0 - m_run), p1 = fast_exp2(s1 - m_run);
+  l_run += p0 + p1;
+  const float x0 = __shfl_sync(FULL, p0, psrc), x1 = __shfl_sync(FULL, p0, psrc + 4);
+  const float y0 = __shfl_sync(FULL, p1, psrc), y1 = __shfl_sync(FULL, p1, psrc + 4);
+  uint32_t h0, l0, h1, l1;
+  split_bf16(x0, x1, h0, l0);
+  split_bf16(y0, y1, h1, l1);
+  const uint32_t pb0 = lane < 4 ? h0 : (lane < 8 ? l0 : 0u);
+  const uint32_t pb1 = lane < 4 ? h1 : (lane < 8 ? l1 : 0u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t af[4];
+    ldsm_x4_t(st + kSpHalfBytes + sp_off(vr, 2 * i + vh), af[0], af[1], af[2], af[3]);
+    mma_bf16(o[i], af, pb0, pb1);
+  }
+}
+
+// Merge the `ce` split partials of list `list_id` (lane l: output dims [4l, 4l + 4)) and write
+// out and lse.
+__device__ __forceinline__ void merge_partials_of_list(const DecodeArgs& a, int64_t list_id, int ce, int l) {
+  const float2* ml = a.part_ml + list_id * a.nsplit;
+  float mx = -CUDART_INF_F;
+  for (int i = l; i < ce; i += 32) mx = fmaxf(mx, __ldcg(&ml[i]).x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  float L = 0.f;
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx != -CUDART_INF_F) {
+    for (int i = l; i < ce; i += 32) {
+      const float2 x = __ldcg(&ml[i]);
+      L = fmaf(fast_exp2(x.x - mx), x.y, L);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+    const float4* src = reinterpret_cast<const float4*>(a.part_acc + list_id * a.nsplit * kHeadDim) + l;
+    for (int c0 = 0; c0 < ce; c0 += 8) {
+      float w[8];
+      float4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int cc = c0 + u < ce ? c0 + u : ce - 1;
+        const float m = __ldcg(&ml[cc]).x;
+        w[u] = (c0 + u < ce && m != -CUDART_INF_F) ? fast_exp2(m - mx) : 0.f;
+        x[u] = __ldcg(src + (int64_t)cc * (kHeadDim / 4));
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (w[u] == 0.f) continue;   // an empty partial's row is never read into the sum
+        r.x = fmaf(w[u], x[u].x, r.x); r.y = fmaf(w[u], x[u].y, r.y);
+        r.z = fmaf(w[u], x[u].z, r.z); r.w = fmaf(w[u], x[u].w, r.w);
+      }
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const int t = (int)(list_id / a.qv.hq), h = (int)(list_id % a.qv.hq);
+  store_out4(a, t, h, 4 * l, make_float4(r.x * inv, r.y * inv, r.z * inv, r.w * inv));
+  if (l == 0 && a.lse != nullptr) a.lse[list_id] = L > 0.f ? (mx + log2f(L)) * kLn2 : -CUDART_INF_F;
+}
+
+template <bool WEIGHTED>
+__global__ void __launch_bounds__(kSsThreads, kSsCtasPerSm) sparse_stream_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char ss_smem[];
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int G = a.qv.hq / a.kv.hkv;
+  const int M = a.lists_per_cta;   // list slots per (sequence, kv head)
+  const int C = a.nsplit;          // chunks per list
+  const int E = a.span;            // entries per chunk, a multiple of 32
+  const int64_t total = (int64_t)a.kv.batch * a.kv.hkv * M * C;
+  const uint32_t ring = smem_u32(ss_smem) + (uint32_t)(warp * kSpStages * kSpTileBytes);
+  unsigned char* qslot = ss_smem + kSsRingBytes + (size_t)warp * kSsSlots * 512;
+  SsDesc* desc = reinterpret_cast<SsDesc*>(ss_smem + kSsRingBytes + kSsQBytes) + warp * kSsSlots;
+  float* accbuf = reinterpret_cast<float*>(ss_smem + kSsRingBytes + kSsQBytes + kSsDescBytes) + warp * kHeadDim;
+  const float scale = a.qv.sm_scale * kLog2e;
+  const int qbytes = a.qv.q_f32 ? 512 : 256;
+  uint32_t bad = 0;
+
+  // ---- S3: task fetch and raw index loads.  The next task number is taken one task ahead.
+  uint32_t tau_next = 0;
+  if (lane == 0) tau_next = atomicAdd(a.sched, 1u);
+  tau_next = __shfl_sync(FULL, tau_next, 0);
+  int p_slot = 0, p_w = 0, p_nwin = 0, p_e0 = 0, p_e1 = 0;
+  int64_t p_base = 0;
+  uint32_t p_seq = 0;
+  bool p_end = false;
+  int32_t v3 = -1, prev3 = 0;
+  float lw3 = 0.f;
+  uint32_t tag3 = kTagBubble;
+
+  auto produce = [&]() {
+    const int32_t last_raw = __shfl_sync(FULL, v3, 31);
+    if (!p_end && p_w + 1 < p_nwin) {   // the next window of the current task
+      ++p_w;
+      const int e = p_e0 + 32 * p_w + lane;
+      v3 = e < p_e1 ? __ldg(a.idx + p_base + e) : -1;
+      lw3 = (WEIGHTED && e < p_e1) ? __ldg(a.logw + p_base + e) * kLog2e : 0.f;
+      prev3 = last_raw;
+      tag3 = (uint32_t)p_slot | (p_w + 1 == p_nwin ? kTagLast : 0u);
+      return;
+    }
+    for (;;) {   // the next task that has entries
+      const int64_t tau = (int64_t)tau_next;
+      if (p_end || tau >= total) {
+        p_end = true;
+        v3 = -1; prev3 = 0; lw3 = 0.f;
+        tag3 = kTagEnd;
+        return;
+      }
+      uint32_t nx = 0;
+      if (lane == 0) nx = atomicAdd(a.sched, 1u);
+      tau_next = __shfl_sync(FULL, nx, 0);
+      const int c = (int)(tau % C);
+      int64_t r = tau / C;
+      const int m = (int)(r % M);
+      r /= M;
+      const int g = (int)(r % a.kv.hkv);
+      const int b = (int)(r / a.kv.hkv);
+      const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, c == 0 && g == 0 && m == 0 && lane == 0);
+      const int j = m / G;
+      if (j >= si.n) continue;   // no list in this slot (fewer query tokens than the bound)
+      const int list = (si.t0 + j) * a.qv.hq + g * G + (m - j * G);
+      const int64_t base = (int64_t)list * a.k_max;
+      const int e0 = c * E;
+      const int e1 = min(e0 + E, a.k_max);
+      const int e = e0 + lane;
+      const int32_t v = e < e1 ? __ldg(a.idx + base + e) : -1;
+      if (c > 0 && __shfl_sync(FULL, v, 0) == -1) continue;   // past the end of its list
+      const int slot = (int)(p_seq++ % kSsSlots);
+      if (lane == 0) {
+        SsDesc d;
+        d.list = list; d.c = c; d.e1 = e1; d.kvlen = kv_len_of(a.qv, si, j); d.b = b; d.g = g;
+        d.pad0 = d.pad1 = 0;
+        desc[slot] = d;
+      }
+      // the task's q row -> its slot; the copy joins the next tile's commit group, several groups
+      // before the task's first tile is consumed
+      if (lane * 16 < qbytes)
+        cp_async16(qslot + slot * 512 + lane * 16, static_cast<const char*>(a.qv.q) + (int64_t)list * qbytes + lane * 16);
+      __syncwarp();
+      p_slot = slot; p_base = base; p_e0 = e0; p_e1 = e1; p_w = 0;
+      p_nwin = (e1 - e0 + 31) >> 5;
+      v3 = v;
+      lw3 = (WEIGHTED && e < e1) ? __ldg(a.logw + base + e) * kLog2e : 0.f;
+      prev3 = c > 0 ? __ldg(a.idx + base + e0 - 1) : 0;
+      tag3 = (uint32_t)slot | kTagFirst | (p_nwin == 1 ? kTagLast : 0u);
+      return;
+    }
+  };
+
+  // ---- S2: a window's raw indices -> physical rows (checks as in the one-task kernel)
+  auto resolve = [&](int32_t v, int32_t prev, uint32_t tag) -> uint32_t {
+    uint32_t row = kInvalidRow;
+    if (tag & (kTagBubble | kTagEnd)) return row;
+    const SsDesc& d = desc[tag & kTagSlot];
+    const int b = d.b, g = d.g, kvlen = d.kvlen;
+    uint32_t before = __shfl_up_sync(FULL, (uint32_t)v, 1);
+    if (lane == 0) before = (uint32_t)prev;
+    if ((uint32_t)v < before) bad |= TSD_DEV_UNSORTED;
+    if (v < -1 || v >= kvlen) bad |= TSD_DEV_BAD_INDEX;
+    if (v >= 0 && v < kvlen) {
+      row = kv_row(a.kv, b, g, v);
+      if (row == kInvalidRow) bad |= TSD_DEV_BAD_PAGE;
+    }
+    return row;
+  };
+
+  // tile p (0 or 1) of a window whose rows are `rows` -> ring stage `stage` (an empty commit
+  // group when the tile has no valid row)
+  auto issue = [&](uint32_t rows, uint32_t vmask, int p, int stage) {
+    if (((vmask >> (16 * p)) & 0xFFFFu) != 0u) {
+      const uint32_t st = ring + (uint32_t)(stage * kSpTileBytes);
+      const int cc = lane & 15;
+#pragma unroll
+      for (int i = 0; i < kSpTileRows / 2; ++i) {
+        const int r = 2 * i + (lane >> 4);
+        const uint32_t rr = __shfl_sync(FULL, rows, 16 * p + r);
+        const bool ok = rr != kInvalidRow;
+        const int64_t off = ok ? (int64_t)rr * kHeadDim : 0;
+        const uint32_t so = sp_off(r, cc);
+        cp_async16_zfill(st + so, reinterpret_cast<const uint4*>(a.kv.k + off) + cc, ok);
+        cp_async16_zfill(st + kSpHalfBytes + so, reinterpret_cast<const uint4*>(a.kv.v + off) + cc, ok);
+      }
+    }
+    cp_async_commit();
+  };
+
+  // ---- pipeline fill: S3 -> S2 -> S1 -> S0
+  uint32_t tag0 = kTagBubble, tag1 = kTagBubble, tag2 = kTagBubble;
+  uint32_t row1 = kInvalidRow, row2 = kInvalidRow;
+  uint32_t vm0 = 0, vm1 = 0, vm2 = 0;
+  float lw0 = 0.f, lw1 = 0.f, lw2 = 0.f;
+  // one step: S0 <- S1 <- S2 <- resolve(S3) <- produce()
+  auto shift = [&]() {
+    tag0 = tag1; vm0 = vm1; lw0 = lw1;
+    tag1 = tag2; row1 = row2; vm1 = vm2; lw1 = lw2;
+    if (!(tag3 & (kTagBubble | kTagEnd | kTagFirst)) && __ballot_sync(FULL, v3 != -1) == 0u) {
+      // a later window with no entries: its task ended with the window now in S1
+      tag1 |= kTagLast;
+      p_nwin = p_w;
+      tag2 = kTagBubble; row2 = kInvalidRow; vm2 = 0u; lw2 = 0.f;
+    } else {
+      row2 = resolve(v3, prev3, tag3);
+      vm2 = __ballot_sync(FULL, row2 != kInvalidRow);
+      tag2 = tag3;
+      lw2 = lw3;
+    }
+    produce();
+  };
+  // after the first window is produced and shifted twice it is in S1: its two tiles go into
+  // stages 0 and 1, and one more shift makes it S0
+  produce();
+  shift();
+  shift();
+  issue(row1, vm1, 0, 0);
+  issue(row1, vm1, 1, 1);
+  shift();
+
+  float m_run = -CUDART_INF_F, l_run = 0.f;
+  float o[8][4];
+  uint32_t qb[8][2];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    qb[i][0] = qb[i][1] = 0u;
+  }
+  int stage = 0;
+  while (!(tag0 & kTagEnd)) {
+    const bool real = !(tag0 & kTagBubble);
+    int32_t nf = -1;   // first entry after the task's chunk (its list's end when -1)
+    if (real && (tag0 & kTagFirst)) {
+      // a new task: reset the state and read q from its slot.  The q copy was issued when the
+      // window was produced, before its tiles: it is in the group of the window's first tile or
+      // an older one, so all groups but the newest (the window's second tile) must be complete.
+      m_run = -CUDART_INF_F;
+      l_run = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+      cp_async_wait<1>();
+      __syncwarp();
+      const int col = lane >> 2, i2 = 2 * (lane & 3);
+      const unsigned char* qs = qslot + (tag0 & kTagSlot) * 512;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        qb[ks][0] = qb[ks][1] = 0u;
+        if (col < 2) {
+          const int d0 = 16 * ks + i2;
+          float x0, x1, y0, y1;
+          if (a.qv.q_f32) {
+            const float2 u = *reinterpret_cast<const float2*>(qs + 4 * d0);
+            const float2 v = *reinterpret_cast<const float2*>(qs + 4 * (d0 + 8));
+            x0 = u.x; x1 = u.y; y0 = v.x; y1 = v.y;
+          } else {
+            const uint32_t u = *reinterpret_cast<const uint32_t*>(qs + 2 * d0);
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(qs + 2 * (d0 + 8));
+            x0 = bf16lo(u); x1 = bf16hi(u); y0 = bf16lo(v); y1 = bf16hi(v);
+          }
+          uint32_t h0, l0, h1, l1;
+          split_bf16(x0, x1, h0, l0);
+          split_bf16(y0, y1, h1, l1);
+          qb[ks][0] = col == 0 ? h0 : l0;
+          qb[ks][1] = col == 0 ? h1 : l1;
+        }
+      }
+    }
+    if (real && (tag0 & kTagLast)) {
+      const SsDesc& d = desc[tag0 & kTagSlot];
+      if (d.e1 < a.k_max) nf = __ldg(a.idx + (int64_t)d.list * a.k_max + d.e1);
+    }
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      // the same tile of the next window (S1) goes into the stage consumed last
+      __syncwarp();
+      issue(row1, vm1, p, stage == 0 ? kSpStages - 1 : stage - 1);
+      cp_async_wait<kSpStages - 1>();
+      __syncwarp();
+      const uint32_t tmask = (vm0 >> (16 * p)) & 0xFFFFu;
+      if (tmask != 0u)
+        sp_tile<WEIGHTED>(ring + (uint32_t)(stage * kSpTileBytes), tmask, qb, scale, lw0, p, m_run, l_run, o);
+      stage = stage + 1 == kSpStages ? 0 : stage + 1;
+    }
+    if (real && (tag0 & kTagLast)) {
+      // finish the task: the lane sums of l, the O^T fragments -> 4 dims per lane
+      const SsDesc d = desc[tag0 & kTagSlot];
+      float l = l_run;
+#pragma unroll
+      for (int o2 = 4; o2 < 32; o2 <<= 1) l += __shfl_xor_sync(FULL, l, o2);
+      l = __shfl_sync(FULL, l, 0);
+      if ((lane & 3) == 0) {
+        const int i = lane >> 2;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          accbuf[16 * k + i] = o[k][0] + o[k][1];
+          accbuf[16 * k + i + 8] = o[k][2] + o[k][3];
+        }
+      }
+      __syncwarp();
+      const float4 acc = *reinterpret_cast<const float4*>(accbuf + 4 * lane);
+      __syncwarp();
+      const int64_t list_id = d.list;
+      const bool last_chunk = d.e1 >= a.k_max || __shfl_sync(FULL, nf, 0) == -1;
+      if (C == 1 || (d.c == 0 && last_chunk)) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const int t = d.list / a.qv.hq, h = d.list % a.qv.hq;
+        store_out4(a, t, h, 4 * lane, make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
+        if (lane == 0 && a.lse != nullptr) a.lse[list_id] = l > 0.f ? (m_run + log2f(l)) * kLn2 : -CUDART_INF_F;
+      } else {
+        const int64_t pidx = list_id * a.nsplit + d.c;
+        if (lane == 0) a.part_ml[pidx] = make_float2(l > 0.f ? m_run : -CUDART_INF_F, l);
+        reinterpret_cast<float4*>(a.part_acc + pidx * kHeadDim)[lane] = acc;
+        __threadfence();
+        __syncwarp();
+        uint32_t now = 0;
+        if (lane == 0) {
+          const uint32_t add = 1u + (last_chunk ? ((uint32_t)(d.c + 1) << 16) : 0u);
+          now = atomicAdd(a.counters + list_id, add) + add;
+        }
+        now = __shfl_sync(FULL, now, 0);
+        const uint32_t need = now >> 16;
+        if (need != 0u && (now & 0xFFFFu) == need) {   // this arrival completed the list
+          __threadfence();
+          // a malformed list (entries after its -1 padding) can claim more chunks than it has:
+          // the merge never reads past the list's own C partials
+          merge_partials_of_list(a, list_id, (int)min(need, (uint32_t)C), lane);
+          if (lane == 0) atomicExch(a.counters + list_id, 0u);
+        }
+      }
+    }
+    shift();
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) bad |= __shfl_xor_sync(FULL, bad, o2);
+  if (lane == 0 && bad) flag_status(a.status, bad);
+
+  // the last warp of the grid to finish leaves the counters zero for the next call
+  uint32_t done = 0;
+  if (lane == 0) {
+    __threadfence();
+    done = atomicAdd(a.sched + 1, 1u);
+  }
+  done = __shfl_sync(FULL, done, 0);
+  if (done + 1 == gridDim.x * (uint32_t)kSsWarps) {
+    __threadfence();
+    const int64_t lists = (int64_t)a.qv.num_tokens * a.qv.hq;
+    for (int64_t i = lane; i < lists; i += 32) a.counters[i] = 0u;
+    if (lane == 0) {
+      a.sched[0] = 0u;
+      a.sched[1] = 0u;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Dense decode on tensor cores
 // ---------------------------------------------------------------------------
 // One CTA per (sequence b, kv head g, list group lg, window of W tokens): up to 16 lists
@@ -800,7 +1236,38 @@ __global__ void __launch_bounds__(kDnThreads, kDnCtasPerSm) dense_decode_kernel(
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
+// The persistent form: kSsCtasPerSm CTAs per SM (fewer when there are fewer tasks).
+static cudaError_t launch_sparse_stream(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
+  const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
+  if (tasks >= ((int64_t)1 << 31) || a.sched == nullptr) return cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  int64_t grid = (int64_t)sms * kSsCtasPerSm;
+  const int64_t need = (tasks + kSsWarps - 1) / kSsWarps;
+  if (grid > need) grid = need;
+  if (grid < 1) grid = 1;
+  static bool configured = false;
+  if (!configured) {
+    e = cudaFuncSetAttribute(sparse_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSsSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(sparse_stream_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSsSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  if (a.logw != nullptr) {
+    sparse_stream_kernel<true><<<(unsigned)grid, kSsThreads, kSsSmemBytes, stream>>>(a);
+  } else {
+    sparse_stream_kernel<false><<<(unsigned)grid, kSsThreads, kSsSmemBytes, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
+  if (a.persistent) return launch_sparse_stream(a, batch, hkv, stream);
   const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
   const int64_t grid = (tasks + kSpWarps - 1) / kSpWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;

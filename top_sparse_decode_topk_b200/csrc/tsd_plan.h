@@ -1,7 +1,9 @@
 // Work decomposition and workspace layout of libtsd (host and device).
 //
 // Workspace layout (bytes from the start; every region 256-byte aligned):
-//   [0, 256)              header: device status word (uint32) at offset 0, the rest reserved
+//   [0, 256)              header: device status word (uint32) at offset 0; the persistent
+//                         sparse kernel's task and done counters (uint32) at offsets 4 and 8;
+//                         the rest reserved
 //   counters              uint32, one per list (token x q head): arrival counters of the
 //                         split-K merge (zero between calls)
 //   -- everything above is the "zero region": it must be zero when a call starts and every
@@ -52,6 +54,7 @@ struct SparsePlan {
   int lists;     // list slots per (sequence, kv head): G x max tokens per sequence
   int entries;   // E
   int nsplit;    // C
+  int stream;    // 1: the persistent kernel (tasks handed out through a counter), 0: one task per warp
 };
 
 constexpr int kSpTasksPerCta = 4;   // warps per sparse-decode CTA, one task each
@@ -82,6 +85,37 @@ inline SparsePlan plan_sparse(const Shapes& s, int k_max, int num_sms) {
   }
   p.entries = e;
   p.nsplit = (k_max + e - 1) / e;
+  p.stream = 0;
+  return p;
+}
+
+// Persistent sparse decode: kSsCtasPerSm CTAs of kSsWarpsPerCta warps on every SM, each warp
+// taking (list, chunk) tasks from a counter until none is left, with the next task's first
+// windows prefetched while the current one drains.  Lists are cut into chunks of E entries (a
+// multiple of the 32-entry window): E is sized for about six tasks per warp, so that the warps
+// finish together, within [64, 512] so that a task is long enough to hide its start and the
+// split-K partials stay a few percent of the traffic.
+constexpr int kSsWarpsPerCta = 4;
+constexpr int kSsCtasPerSm = 2;
+
+inline SparsePlan plan_sparse_stream(const Shapes& s, int k_max, int num_sms, int entries_override) {
+  SparsePlan p;
+  p.lists = (int)(s.group * s.max_tokens);
+  const double warps = (double)num_sms * kSsCtasPerSm * kSsWarpsPerCta;
+  const double work = (double)s.tokens * s.hq * k_max;
+  const int kr = (k_max + 31) / 32 * 32;
+  int e = entries_override > 0 ? entries_override : (int)(work / (warps * 6.0));
+  e = (e + 31) / 32 * 32;
+  if (entries_override <= 0) {
+    if (e < 64) e = 64;
+    if (e > 512) e = 512;
+  }
+  if (e < 32) e = 32;
+  if (e > kr) e = kr;
+  if ((k_max + e - 1) / e > kMaxSplits) e = ((k_max + kMaxSplits - 1) / kMaxSplits + 31) / 32 * 32;
+  p.entries = e;
+  p.nsplit = (k_max + e - 1) / e;
+  p.stream = 1;
   return p;
 }
 

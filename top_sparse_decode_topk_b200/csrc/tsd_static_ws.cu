@@ -82,5 +82,6 @@ extern "C" tsd_status tsd_sparse_decode_static_ws(const tsd_kv_cache* cache, con
   a.counters = reinterpret_cast<uint32_t*>(ws + lay.off_counters);
   a.part_ml = reinterpret_cast<float2*>(ws + lay.off_ml);
   a.part_acc = reinterpret_cast<float*>(ws + lay.off_acc);
+  a.sched = reinterpret_cast<uint32_t*>(ws + 4);
   return launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, s) == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }

@@ -218,9 +218,21 @@ CONFIGS: Dict[str, DecodeConfig] = {
         ks=tuple(k_for_sparsity(65536, x) for x in (1, 4, 10, 25, 50, 100, 200)),
         index_mode="uniform", planted=False,
         description="batch 16, 32/8 heads, N=65536, k in {N..N/200}, uniform or Zipf page-run indices"),
+    # reduced copies of two shapes above, small enough for detailed profiler captures (a few GB
+    # on the device) while the rows the sparse kernel reads still exceed the 126 MB L2
+    "qwen25_72b_b2": DecodeConfig(
+        name="qwen25_72b_b2", batch=2, num_q_heads=64, num_kv_heads=8, seq_len=131072,
+        ks=(2621,), planted=True,
+        description="the Qwen2.5-72B shape with batch 2: 64/8 heads, N=131072, k=2621, paged (16)"),
+    "ragged_8": DecodeConfig(
+        name="ragged_8", batch=8, num_q_heads=32, num_kv_heads=8, seq_len_range=(8192, 131072),
+        tokens_per_seq=4, k_frac_ceil=0.02, planted=True,
+        description="the ragged batch with 8 seqs: len U[8192,131072], 4 causal decode queries each, "
+                    "32/8 heads, k=ceil(0.02*kv_len), paged (16)"),
 }
 
-CONFIG_IDS = {"tiny": 1, "llama3_8b": 2, "qwen25_72b": 3, "ragged": 4, "sweep": 5}
+CONFIG_IDS = {"tiny": 1, "llama3_8b": 2, "qwen25_72b": 3, "ragged": 4, "sweep": 5, "qwen25_72b_b2": 6,
+              "ragged_8": 7}
 
 
 # --------------------------------------------------------------------------
