@@ -60,6 +60,10 @@ def parse():
     p.add_argument("--record-traffic", metavar="NCU_CSV",
                    help="write profiles/dram_traffic.json for --config from an ncu --csv log of "
                         "dram__bytes_read.sum, dram__bytes_write.sum and gpu__time_duration.sum (no GPU work)")
+    p.add_argument("--plain-line", metavar="JSON",
+                   help="with --record-traffic: the bench line of the same command run without ncu; its "
+                        "sparse-decode algorithmic bytes are stored beside the captured traffic, so that the "
+                        "figure can be scaled to a larger copy of the workload")
     return p.parse_args()
 
 
@@ -170,32 +174,55 @@ def source_sha(names):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, workload: str, source):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+# workloads whose traffic is captured on a reduced copy (the full size is beyond a detailed
+# profiler capture): the copy's DRAM bytes per algorithmic byte, times the full launch's
+# algorithmic bytes
+TRAFFIC_SCALED_FROM = {"ragged": "ragged_8", "qwen25_72b": "qwen25_72b_b2"}
+
+
+def ncu_traffic(kernel: str, workload: str, source, algorithmic_bytes=None):
+    """(DRAM bytes per launch, how) from the committed ncu summary, if it was taken on the
+    current kernel source (else (None, reason)).  A workload captured only as a reduced copy
+    gets the copy's DRAM/algorithmic ratio times its own algorithmic bytes."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        e = d[kernel][workload]
-        if e.get("source_sha") != source_sha(source):
-            return None
-        return float(e["bytes_per_launch"])
     except Exception:
-        return None
+        return None, "no capture recorded"
+    rec = d.get(kernel, {})
+    for name, scaled in ((workload, False), (TRAFFIC_SCALED_FROM.get(workload), True)):
+        e = rec.get(name) if name else None
+        if e is None:
+            continue
+        if e.get("source_sha") != source_sha(source):
+            return None, f"the {name} capture predates the current kernel source"
+        if not scaled:
+            return float(e["bytes_per_launch"]), f"ncu capture of {name}"
+        if algorithmic_bytes is None or not e.get("algorithmic_bytes"):
+            return None, f"the {name} capture has no algorithmic bytes to scale by"
+        ratio = float(e["bytes_per_launch"]) / float(e["algorithmic_bytes"])
+        return ratio * algorithmic_bytes, (f"ncu capture of {name} (DRAM/algorithmic = {ratio:.4f}), scaled "
+                                           f"to this launch's algorithmic bytes")
+    return None, "no capture of this kernel on this workload"
 
 
 # kernel -> the csrc files that decide its code and launch shape
 KERNEL_SOURCES = {
     "sparse_decode_kernel": SPARSE_SOURCES,
+    "sparse_stream_kernel": SPARSE_SOURCES,
     "dense_decode_kernel": ["tsd_decode.cu", "tsd_plan.h", "tsd_common.cuh", "tsd_kvtile.cuh"],
     "topk_score_kernel": ["tsd_topk.cu", "tsd_plan.h", "tsd_common.cuh", "tsd_kvtile.cuh"],
     "topk_select_kernel": ["tsd_topk.cu", "tsd_plan.h", "tsd_common.cuh"],
 }
 
 
-def record_traffic(csv_path: str, workload: str):
+def record_traffic(csv_path: str, workload: str, plain_line: str = None):
     """Fold one ncu --csv metric log into profiles/dram_traffic.json (first launch of each kernel)."""
+    alg = None
+    if plain_line:
+        with open(plain_line) as f:
+            alg = json.loads(f.read().strip().splitlines()[-1])["roofline"]["algorithmic_bytes"]
     import csv
     with open(csv_path) as f:
         rows = list(csv.reader(f))
@@ -229,6 +256,8 @@ def record_traffic(csv_path: str, workload: str):
             "bytes_per_launch": rd + wr, "read": rd, "write": wr,
             "duration_us": round(e.get("gpu__time_duration.sum", float("nan")) / 1e3, 3),
             "sources": KERNEL_SOURCES[kern], "source_sha": source_sha(KERNEL_SOURCES[kern])}
+        if alg is not None and kern.startswith("sparse_"):
+            out[kern][workload]["algorithmic_bytes"] = alg
     with open(path, "w") as f:
         json.dump(out, f, indent=1)
     print(json.dumps({k: v for k, v in out.items() if k != "_about"}, indent=1))
@@ -788,7 +817,8 @@ def run_native(args):
         return
 
     cl = clocks.summary()
-    traffic = ncu_traffic("sparse_decode_kernel", cfg.name, SPARSE_SOURCES)
+    plan = tsd.sparse_decode_plan(cache, queries, k_max)
+    traffic, traffic_how = ncu_traffic(plan["kernel"], cfg.name, SPARSE_SOURCES, sparse_bytes)
     line = {
         "metric": METRIC,
         "value": round(sparse_ms * 1e3, 3),
@@ -815,8 +845,9 @@ def run_native(args):
         "speedup_vs_dense": round(dense_ms / sparse_ms, 3),
         "speedup_vs_dense_with_indexer": round(dense_ms / (sparse_ms + topk_ms), 3),
         "roofline": {"bound": "hbm", "achieved": round(sparse_gbs, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(sparse_gbs / hbm, 4), "traffic": traffic,
-                     "kernel": "sparse_decode_kernel", "peak_source": f"{peak_kind} copy bandwidth",
+                     "frac": round(sparse_gbs / hbm, 4),
+                     "traffic": None if traffic is None else round(traffic), "traffic_source": traffic_how,
+                     "kernel": plan["kernel"], "plan": plan, "peak_source": f"{peak_kind} copy bandwidth",
                      "frac_of_nominal_8tbs": round(sparse_gbs / NOMINAL_HBM_GBS, 4),
                      "algorithmic_bytes": sparse_bytes, "unique_rows": U, "entries": entries,
                      "index_bytes_not_counted": index_bytes},
@@ -913,7 +944,7 @@ def run_reference(args):
 def main():
     args = parse()
     if args.record_traffic:
-        record_traffic(args.record_traffic, args.config)
+        record_traffic(args.record_traffic, args.config, args.plain_line)
     elif args.impl == "reference":
         run_reference(args)
     else:

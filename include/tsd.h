@@ -143,6 +143,16 @@ tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries
 size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries,
                                         int32_t k_max);
 
+/* Host: the work decomposition tsd_sparse_decode would use for these shapes on the current
+ * device, for diagnostics and benchmarks: *persistent = 1 for the persistent kernel
+ * (sparse_stream_kernel: every warp takes (list, chunk) tasks from a counter until none is
+ * left), 0 for the one-task-per-warp kernel (sparse_decode_kernel: one wave of CTAs);
+ * *entries_per_task = index entries per task; *tasks_per_list = tasks (split-K partials) per
+ * list.  Device pointers may be NULL.  Errors: INVALID_ARGUMENT, UNSUPPORTED (as
+ * tsd_sparse_decode's host checks). */
+tsd_status tsd_sparse_decode_plan(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                  int32_t* persistent, int32_t* entries_per_task, int32_t* tasks_per_list);
+
 /*
  * Sparse decode attention over per-(token, head) index lists (pages section 2,
  * "Hardware implementation"; section 3.C).  For each query token t and q head h:

@@ -281,3 +281,30 @@ def test_decode_step_errors_before_launch(lib):
     assert call(ws=FAKE + 0x700010) == tsd.TSD_ERR_INVALID_ARGUMENT        # workspace not 256-byte aligned
     assert call(cc=make_cache(head_dim=64)) == tsd.TSD_ERR_UNSUPPORTED
     assert call(k_max=1 << 20) == tsd.TSD_ERR_UNSUPPORTED
+
+
+def test_sparse_decode_plan_choice(lib):
+    """The work decomposition query (host arithmetic only).  One decode token per sequence and
+    k = 655 over 8 sequences x 8 kv heads x 4 q heads fits one wave as 4 chunks of 176 entries;
+    the ragged shape (128 tokens, 32 heads, k up to 2622) needs more than one wave and takes the
+    persistent kernel with 512-entry chunks (148 SMs assumed without a device)."""
+    c, q = make_cache(), make_queries()
+    p, e, n = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    args = (ctypes.byref(p), ctypes.byref(e), ctypes.byref(n))
+    try:
+        import torch
+        if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
+            pytest.skip("the expected splits assume 148 SMs")
+    except ImportError:
+        pass
+    assert lib.tsd_sparse_decode_plan(ctypes.byref(c), ctypes.byref(q), 655, *args) == tsd.TSD_OK
+    assert (p.value, e.value, n.value) == (0, 176, 4)
+    rc = make_cache(batch=32, max_pages=8192, num_pages=32 * 8192, max_seq_len=131072)
+    rq = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=4)
+    assert lib.tsd_sparse_decode_plan(ctypes.byref(rc), ctypes.byref(rq), 2622, *args) == tsd.TSD_OK
+    assert (p.value, e.value, n.value) == (1, 512, 6)
+    assert lib.tsd_sparse_decode_plan(ctypes.byref(c), ctypes.byref(q), 0, *args) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_sparse_decode_plan(ctypes.byref(c), ctypes.byref(q), 655, None, ctypes.byref(e),
+                                      ctypes.byref(n)) == tsd.TSD_ERR_INVALID_ARGUMENT
+    bad = make_cache(head_dim=64)
+    assert lib.tsd_sparse_decode_plan(ctypes.byref(bad), ctypes.byref(q), 655, *args) == tsd.TSD_ERR_UNSUPPORTED

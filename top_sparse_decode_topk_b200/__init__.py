@@ -89,6 +89,9 @@ EXPORTS = {
                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.c_void_p]),
     "tsd_read_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "tsd_sparse_decode_plan": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
+                                              ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
+                                              ctypes.POINTER(ctypes.c_int32)]),
     "tsd_decode_step_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC),
                                                          ctypes.c_int32]),
     "tsd_decode_step": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
@@ -517,6 +520,18 @@ def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=Non
                                               k_max, out.data_ptr(), odt, lp, ws.data_ptr(), ws.numel(), sp),
                "tsd_sparse_decode_weighted")
     return _finish(out, host_out, lse, host_lse, s)
+
+
+def sparse_decode_plan(cache: KVCache, queries: Queries, k_max: int) -> dict:
+    """The work decomposition sparse_decode would use (tsd_sparse_decode_plan): the kernel's
+    name, entries per task and tasks (split-K partials) per list."""
+    lib = load_library()
+    cs, qs = cache.c_struct(), queries.c_struct()
+    p, e, c = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib.tsd_sparse_decode_plan(ctypes.byref(cs), ctypes.byref(qs), int(k_max), ctypes.byref(p),
+                                      ctypes.byref(e), ctypes.byref(c)), "tsd_sparse_decode_plan")
+    return {"kernel": "sparse_stream_kernel" if p.value else "sparse_decode_kernel",
+            "entries_per_task": e.value, "tasks_per_list": c.value}
 
 
 def decode_step(cache: KVCache, queries: Queries, k_max: int, k_per_token=None, out_idx=None, out_count=None,

@@ -227,10 +227,13 @@ static int current_sm_count() {
 }
 
 // Work decomposition of tsd_sparse_decode.  The one-task-per-warp kernel fits its grid to one
-// wave of resident CTAs; when its tasks need more than one wave, the persistent kernel takes
-// the call instead.  TSD_SPARSE_KERNEL=wave|stream forces either form and TSD_SPARSE_CHUNK
-// sets the persistent form's entries per task (both for measurements; read at every call, so
-// size the workspace under the same setting as the call).
+// wave of resident CTAs.  The persistent kernel takes the call instead when that plan needs
+// more than one wave, or when it fits one wave only by giving every warp a whole list of 256
+// entries or more: lists of unequal length then leave the wave waiting on its longest list,
+// while the persistent kernel cuts lists into chunks and balances them over all warps.
+// TSD_SPARSE_KERNEL=wave|stream forces either form and TSD_SPARSE_CHUNK sets the persistent
+// form's entries per task (both for measurements; read at every call, so size the workspace
+// under the same setting as the call).
 static SparsePlan sparse_plan(const Shapes& sh, int k_max) {
   const int sms = current_sm_count();
   const char* kind = getenv("TSD_SPARSE_KERNEL");
@@ -244,7 +247,7 @@ static SparsePlan sparse_plan(const Shapes& sh, int k_max) {
     stream = false;
   } else {
     const int64_t ctas = (sh.batch * sh.hkv * wave.lists * (int64_t)wave.nsplit + kSpTasksPerCta - 1) / kSpTasksPerCta;
-    stream = ctas > (int64_t)sms * kSpCtasPerSm;
+    stream = ctas > (int64_t)sms * kSpCtasPerSm || (wave.nsplit == 1 && k_max >= 256);
   }
   return stream ? plan_sparse_stream(sh, k_max, sms, e_override) : wave;
 }
@@ -268,6 +271,21 @@ size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_que
   if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return 0;
   const SparsePlan p = sparse_plan(sh, k_max);
   return decode_layout(sh, p.nsplit).total;
+}
+
+tsd_status tsd_sparse_decode_plan(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                  int32_t* persistent, int32_t* entries_per_task, int32_t* tasks_per_list) {
+  Shapes sh;
+  if (k_max < 1 || persistent == nullptr || entries_per_task == nullptr || tasks_per_list == nullptr)
+    return TSD_ERR_INVALID_ARGUMENT;
+  if (k_max > kMaxSparseK) return TSD_ERR_UNSUPPORTED;
+  const tsd_status st = sizes_for(cache, queries, &sh);
+  if (st != TSD_OK) return st;
+  const SparsePlan p = sparse_plan(sh, k_max);
+  *persistent = p.stream;
+  *entries_per_task = p.entries;
+  *tasks_per_list = p.nsplit;
+  return TSD_OK;
 }
 
 size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries) {
@@ -298,6 +316,9 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   a.out_scores = out_scores;
   a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
   a.score_stride = lay.score_stride;
+  a.samples = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_samples);
+  a.sample_stride = lay.sample_stride;
+  a.sample_shift = lay.sample_shift;
   // scoring streams K in the dense path's tiles, with its own occupancy
   const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScoreCtasPerSm);
   a.lists_per_cta = p.lists_per_cta;
@@ -657,6 +678,9 @@ tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k,
   a.out_count = out_count;
   a.scores = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_scores);
   a.score_stride = lay.score_stride;
+  a.samples = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_samples);
+  a.sample_stride = lay.sample_stride;
+  a.sample_shift = lay.sample_shift;
   const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm);
   a.lists_per_cta = p.lists_per_cta;
   a.list_groups = p.list_groups;

@@ -38,6 +38,9 @@ struct TopkArgs {
   float* out_scores;    // optional [T][Hq][k_max]: the kept tokens' scores (-inf in the padding)
   float* scores;
   int64_t score_stride;
+  float* samples;         // [T][Hq][sample_stride]: score of every 2^sample_shift-th token
+  int64_t sample_stride;
+  int32_t sample_shift;
   int32_t lists_per_cta;
   int32_t list_groups;
   int32_t window;

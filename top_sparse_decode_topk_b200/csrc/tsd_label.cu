@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
   __shared__ __align__(16) float qs[16][R];
   __shared__ int kvl[16];
   __shared__ int64_t srow[16];
+  __shared__ int64_t prow[16];   // the list's sample row (every 2^sample_shift-th token's score)
   const int win = blockIdx.x;
   const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
   const int b = blockIdx.z;
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
       if (j == 0) {
         kvl[m] = min(kv_len_of(a.qv, si, jt), tok_end);
         srow[m] = ((int64_t)(si.t0 + jt) * a.qv.hq + h) * a.score_stride;
+        prow[m] = ((int64_t)(si.t0 + jt) * a.qv.hq + h) * a.sample_stride;
       }
     }
     qs[m][j] = v;
@@ -212,7 +214,10 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
           s0 = fmaf(qv.z, kf[j + 2], s0);
           s1 = fmaf(qv.w, kf[j + 3], s1);
         }
-        if (tok < kvl[m]) a.scores[srow[m] + tok] = s0 + s1;
+        if (tok < kvl[m]) {
+          a.scores[srow[m] + tok] = s0 + s1;
+          if ((tok & ((1 << a.sample_shift) - 1)) == 0) a.samples[prow[m] + (tok >> a.sample_shift)] = s0 + s1;
+        }
       }
     }
   }

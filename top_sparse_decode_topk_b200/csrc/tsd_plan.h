@@ -11,6 +11,8 @@
 //   decode partials       float2 [T][Hq][nsplit] (running max, running sum; base-2 units)
 //                         float  [T][Hq][nsplit][128] (unnormalised output rows)
 //   top-k scores          float  [T][Hq][score_stride] (fp32 q.K of every visible token)
+//   top-k score samples   float  [T][Hq][sample_stride]: every 2^sample_shift-th token's score
+//                         (its strided sample for the selection's threshold)
 #pragma once
 
 #include <stddef.h>
@@ -198,9 +200,17 @@ inline DecodeLayout decode_layout(const Shapes& s, int nsplit) {
   return l;
 }
 
+// The scoring kernels also write every 2^sample_shift-th token's score into a compact sample
+// row, so that the selection reads its sample contiguously.  The stride is 32 tokens, doubled
+// while the sample would exceed kMaxSample scores.
+constexpr int64_t kMaxSample = 4096;
+
 struct TopkLayout {
   size_t off_scores;
   int64_t score_stride;
+  size_t off_samples;
+  int32_t sample_shift;
+  int64_t sample_stride;
   size_t total;
 };
 
@@ -208,7 +218,11 @@ inline TopkLayout topk_layout(const Shapes& s) {
   TopkLayout l;
   l.score_stride = (s.max_seq_len + 3) / 4 * 4;
   l.off_scores = zero_region_bytes(s);
-  l.total = l.off_scores + align256((size_t)s.tokens * s.hq * l.score_stride * sizeof(float));
+  l.sample_shift = 5;
+  while (((s.max_seq_len + (1LL << l.sample_shift) - 1) >> l.sample_shift) > kMaxSample) ++l.sample_shift;
+  l.sample_stride = (((s.max_seq_len + (1LL << l.sample_shift) - 1) >> l.sample_shift) + 3) / 4 * 4;
+  l.off_samples = l.off_scores + align256((size_t)s.tokens * s.hq * l.score_stride * sizeof(float));
+  l.total = l.off_samples + align256((size_t)s.tokens * s.hq * l.sample_stride * sizeof(float));
   return l;
 }
 

@@ -108,18 +108,23 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
   // this lane's query rows m = lane/4 and lane/4 + 8: visible length and score row
   int kvl[2];
   float* srow[2];
+  float* prow[2];   // the list's sample row: the score of every 2^sample_shift-th token
 #pragma unroll
   for (int hr = 0; hr < 2; ++hr) {
     const int m = (lane >> 2) + 8 * hr;
     kvl[hr] = 0;
     srow[hr] = a.scores;
+    prow[hr] = a.samples;
     if (m < nlists) {
       const int mg = lg * a.lists_per_cta + m;
       const int j = mg / G;
       kvl[hr] = min(kv_len_of(a.qv, si, j), tok_end);
-      srow[hr] = a.scores + ((int64_t)(si.t0 + j) * a.qv.hq + g * G + (mg - j * G)) * a.score_stride;
+      const int64_t list = (int64_t)(si.t0 + j) * a.qv.hq + g * G + (mg - j * G);
+      srow[hr] = a.scores + list * a.score_stride;
+      prow[hr] = a.samples + list * a.sample_stride;
     }
   }
+  const int smask = (1 << a.sample_shift) - 1;
   for (int tile = 0; tile < ntiles; ++tile) {
     if (!consume_wait<kScStages>(full, abort_flag, tile, lane, a.status)) break;
     float sc[2][4];
@@ -135,6 +140,7 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
         } else if (tk < kvl[hr]) {
           srow[hr][tk] = sc[nt][2 * hr];
         }
+        if ((tk & smask) == 0 && tk < kvl[hr]) prow[hr][tk >> a.sample_shift] = sc[nt][2 * hr];
       }
     // the stores consume every fragment read from the stage: release it to the producer
     __syncwarp();
@@ -313,7 +319,11 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
       if (lane < kTcRowsPerQuarter) {
 #pragma unroll
         for (int m = 0; m < 16; ++m)
-          if (m < nlists && tok < s_kvl[m]) a.scores[s_srow[m] + tok] = __uint_as_float(r[m]);
+          if (m < nlists && tok < s_kvl[m]) {
+            a.scores[s_srow[m] + tok] = __uint_as_float(r[m]);
+            if ((tok & ((1 << a.sample_shift) - 1)) == 0)
+              a.samples[s_srow[m] / a.score_stride * a.sample_stride + (tok >> a.sample_shift)] = __uint_as_float(r[m]);
+          }
       }
     }
   }
@@ -328,11 +338,17 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
 // ---------------------------------------------------------------------------
 // Selection
 // ---------------------------------------------------------------------------
+constexpr int kSelWarps = kSelectThreads / 32;
+
+constexpr int kSelMaskIters = 16;   // segment steps whose keep masks the fast path keeps (L <= 128K)
+
 struct SelectSmem {
-  uint32_t hist[kSelBins];
+  uint32_t hist[2][kSelBins];   // the fast path alternates; the multi-pass path uses hist[0]
   uint32_t cand[kCandMax];
-  int scan_tmp[kSelectThreads / 32 + 1];
+  uint16_t keep[kSelWarps][kSelMaskIters][32];   // fast path: each lane's keep bits of each step
+  int scan_tmp[kSelWarps + 1];
   int found_bin, found_above, ncand;
+  int wcount[kSelWarps];
 };
 
 // hist[0..nbins): find d with count(> d) < need <= count(>= d).  Results in S.found_*.
@@ -346,14 +362,14 @@ __device__ void select_bin(SelectSmem& S, int nbins, int need) {
   int local = 0;
   for (int j = 0; j < per; ++j) {
     const int bin = hi - 1 - j;
-    if (bin >= 0) local += (int)S.hist[bin];
+    if (bin >= 0) local += (int)S.hist[0][bin];
   }
   int total;
   int run = block_exclusive_scan<kSelectThreads>(local, S.scan_tmp, &total);
   for (int j = 0; j < per; ++j) {
     const int bin = hi - 1 - j;
     if (bin < 0) break;
-    const int c = (int)S.hist[bin];
+    const int c = (int)S.hist[0][bin];
     if (run < need && run + c >= need) {
       S.found_bin = bin;
       S.found_above = run;
@@ -373,152 +389,287 @@ __device__ __forceinline__ void load16(const float* row, int i0, int L, float* f
   }
 }
 
-// Fast path for lists much longer than k: a threshold from a sample, then ONE pass over the
-// scores.  Take a strided sample of the list (1024 scores, or 4096 from 64K scores on) and r,
-// its expected count above the k-th score plus 4 standard deviations plus 4.  The sample's
-// r-th largest key with its low 10 bits cleared (lo) has, with overwhelming probability, at
-// least k scores at or above it.  One ordered pass copies every (index, key) with key >= lo
-// into shared memory in index order; the exact radix select and the ordered output then run
-// over those few thousand entries only.  Returns false, having written nothing, when the
-// sample says too many keys would be kept or the pass kept more than fit or fewer than k: the
-// caller then runs the full passes.
 // The score of an order-preserving key (inverse of score_key; -0 comes back as +0).
 __device__ __forceinline__ float key_score(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-constexpr int kFastMinL = 4096;
-constexpr int kFastSample = 1024;        // sampled scores, lists shorter than kFastLongL
-constexpr int kFastSampleLong = 4096;    // the same from kFastLongL on: a tighter threshold
-constexpr int kFastLongL = 65536;
-constexpr int kFastCap = kCandMax / 2;   // kept entries: keys in cand[0, cap), indices in cand[cap, 2 cap)
-
-__device__ bool select_fast(SelectSmem& S, const float* row, int L, int k, int32_t* out, float* osc, int k_max) {
-  uint32_t* ckey = S.cand;
-  uint32_t* cidx = S.cand + kFastCap;
-  // ---- the r_lo-th largest of a strided sample of keys ----
-  const int ns = L >= kFastLongL ? kFastSampleLong : kFastSample;
-  const float mean = (float)ns * (float)k / (float)L;
-  const int r_lo = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
-  if (r_lo >= ns || (int64_t)r_lo * L > (int64_t)kFastCap * ns * 3 / 4) return false;
-  for (int s = threadIdx.x; s < ns; s += kSelectThreads)
-    ckey[s] = score_key(__ldcg(row + (int)(((int64_t)s * L) / ns)));
-  // two 11-bit rounds: lo is the r_lo-th largest sampled key with its low 10 bits cleared,
-  // which keeps a little more than the exact sample key would
-  uint32_t prefix = 0u;
-  int need = r_lo, shift = 32;
-  while (shift > 10) {
-    const int nb = 11;
-    shift -= nb;
-    const bool first = shift + nb == 32;
-    for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[i] = 0u;
-    __syncthreads();
-    for (int c = threadIdx.x; c < ns; c += kSelectThreads) {
-      const uint32_t key = ckey[c];
-      if (first || (key >> (shift + nb)) == prefix) atomicAdd(&S.hist[(key >> shift) & ((1u << nb) - 1u)], 1u);
-    }
-    __syncthreads();
-    select_bin(S, 1 << nb, need);
-    prefix = (prefix << nb) | (uint32_t)S.found_bin;
-    need -= S.found_above;
-    __syncthreads();
+// Warp 0 only: in hist[0, nb) find the bin d (scanning from the top) with count(bins above d)
+// < need <= count(bins >= d); lane 0 writes S.found_bin and S.found_above.  Lane l first sums
+// the contiguous bins [nb - (l + 1) per, nb - l per), read in a rotated order so that the 32
+// lanes hit 32 different banks; a lane scan finds the lane whose range crosses `need`, and
+// the 32 lanes then split that range (per / 32 bins each) for a second scan.
+__device__ __forceinline__ void warp_find_bin(SelectSmem& S, const uint32_t* hist, int nb, int need) {
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  const int lane = threadIdx.x & 31;
+  const int per = nb >> 5;
+  int sum = 0;
+  {
+    const int hi = nb - lane * per;
+    for (int j = 0; j < per; ++j) sum += (int)hist[hi - 1 - ((j + lane) & (per - 1))];
   }
-  const uint32_t lo_key = prefix << shift;
+  int inc = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(FULL, inc, o);
+    if (lane >= o) inc += y;
+  }
+  const unsigned cross = __ballot_sync(FULL, inc - sum < need && need <= inc);
+  if (cross == 0u) {   // only for inconsistent counts
+    if (lane == 0) {
+      S.found_bin = 0;
+      S.found_above = 0;
+    }
+    return;
+  }
+  const int cl = __ffs(cross) - 1;
+  const int base_above = __shfl_sync(FULL, inc - sum, cl);
+  const int top = nb - cl * per;        // the crossing lane's bins are [top - per, top)
+  const int q = per >> 5;               // bins per lane in the second step (1 or 2)
+  int s2 = 0;
+  for (int t = 0; t < q; ++t) s2 += (int)hist[top - 1 - (lane * q + t)];
+  int inc2 = s2;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(FULL, inc2, o);
+    if (lane >= o) inc2 += y;
+  }
+  const int ex2 = base_above + inc2 - s2;
+  const unsigned c2 = __ballot_sync(FULL, ex2 < need && need <= base_above + inc2);
+  const int l2 = c2 ? __ffs(c2) - 1 : 0;
+  if (lane == l2) {
+    int run = ex2, bin = top - 1 - lane * q;
+    for (int t = 0; t < q; ++t) {
+      const int b = top - 1 - (lane * q + t);
+      const int c = (int)hist[b];
+      bin = b;
+      if (run + c >= need) break;
+      run += c;
+    }
+    S.found_bin = bin;
+    S.found_above = run;
+  }
+}
 
-  // ---- one ordered pass: every key >= lo, in index order ----
-  // The key map is monotone, so key >= lo is score >= lo_f, the score whose key is lo: the
-  // pass compares floats and forms keys only for the entries it keeps.
-  const float lo_f = key_score(lo_key);
-  const int tile_elems = kSelectThreads * kSelPerThread;
-  int kept = 0;
-  for (int base = 0; base < L; base += tile_elems) {
-    const int i0 = base + threadIdx.x * kSelPerThread;
-    float f[kSelPerThread];
-    load16(row, i0, L, f);
-    uint32_t keep = 0u;
-    if (base + tile_elems <= L) {   // a full tile (uniform over the block)
-#pragma unroll
-      for (int j = 0; j < kSelPerThread; ++j) keep |= (f[j] >= lo_f ? 1u : 0u) << j;
-    } else {
-#pragma unroll
-      for (int j = 0; j < kSelPerThread; ++j) keep |= (i0 + j < L && f[j] >= lo_f ? 1u : 0u) << j;
-    }
-    int tot;
-    int pos = kept + block_exclusive_scan<kSelectThreads>(__popc(keep), S.scan_tmp, &tot);
-    if (keep != 0u) {
-#pragma unroll
-      for (int j = 0; j < kSelPerThread; ++j)
-        if ((keep >> j) & 1u) {
-          if (pos < kFastCap) {
-            ckey[pos] = score_key(f[j]);
-            cidx[pos] = (uint32_t)(i0 + j);
-          }
-          ++pos;
-        }
-    }
-    kept += tot;
+// One radix round over keys[0, n) in shared memory: histogram of the nb-bit digit at `shift`
+// of the keys whose higher bits equal `prefix` (every key when `first`) into hist[cur], while
+// hist[cur ^ 1] is zeroed for the next round; then warp 0 finds the digit holding the
+// need-th largest key.  hist[cur] must be zero on entry.  Two block barriers.
+__device__ __forceinline__ void radix_round(SelectSmem& S, const uint32_t* keys, int n, int nb, int shift, bool first,
+                                            uint32_t prefix, int need, int cur) {
+  uint32_t* h = S.hist[cur];
+  uint32_t* z = S.hist[cur ^ 1];
+  for (int i = threadIdx.x; i < kSelBins; i += kSelectThreads) z[i] = 0u;
+  const uint32_t mask = (1u << nb) - 1u;
+  for (int c = threadIdx.x; c < n; c += kSelectThreads) {
+    const uint32_t key = keys[c];
+    if (first || (key >> (shift + nb)) == prefix) atomicAdd(&h[(key >> shift) & mask], 1u);
   }
   __syncthreads();
-  if (kept > kFastCap || kept < k) return false;
+  if (threadIdx.x < 32) warp_find_bin(S, h, 1 << nb, need);
+  __syncthreads();
+}
 
-  // ---- exact k-th key among the kept entries ----
-  prefix = 0u;
-  need = k;
-  shift = 32;
-  while (shift > 0) {
-    const int nb = shift >= 11 ? 11 : shift;
-    shift -= nb;
-    const bool first = shift + nb == 32;
-    for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[i] = 0u;
-    __syncthreads();
-    for (int c = threadIdx.x; c < kept; c += kSelectThreads) {
-      const uint32_t key = ckey[c];
-      if (first || (key >> (shift + nb)) == prefix) atomicAdd(&S.hist[(key >> shift) & ((1u << nb) - 1u)], 1u);
-    }
-    __syncthreads();
-    select_bin(S, 1 << nb, need);
-    prefix = (prefix << nb) | (uint32_t)S.found_bin;
-    need -= S.found_above;
-    __syncthreads();
-  }
-  const uint32_t T = prefix;
-  const int need_eq = need;
+constexpr int kFastMinL = 4096;
+constexpr int kFastCap = kCandMax / 2;   // kept entries: keys in cand[0, cap), indices in cand[cap, 2 cap)
+constexpr int kFastUnroll = 4;           // float4 loads in flight per lane in the segment passes
 
-  // ---- ordered output over the kept entries ----
-  constexpr int kPer = (kFastCap + kSelectThreads - 1) / kSelectThreads;
-  const int c0 = threadIdx.x * kPer;
-  int neq = 0;
+// Fast path for lists much longer than k: a threshold from a sample, then the scores at or
+// above it, then the exact selection among those few.
+//  1. The list's strided sample -- every 2^sample_shift-th score (every 32nd up to 128K tokens),
+//     written by the scoring kernel into a compact row and read here contiguously -- and r,
+//     its expected count above the k-th score plus 4 standard deviations plus 4.  Two radix
+//     rounds give the sample's r-th largest key with its low 10 bits cleared (lo), which has,
+//     with overwhelming probability, at least k scores at or above it.  The result does not
+//     depend on the sample: whatever lo is, at least k kept scores means every top-k score is
+//     kept, and fewer means the fallback below.
+//  2. Every warp owns a contiguous segment of the list: it counts its scores >= lo, the
+//     counts give every warp its output offset, and it copies its (key, index) pairs in index
+//     order (ballot and lane scan) -- a second read of the segment, from L2.  One barrier
+//     orders the whole list, where a block-wide scan per tile took three.
+//  3. Three radix rounds among the kept keys give the exact k-th key T and how many keys equal
+//     to T are kept; keys > T and the lowest-index keys == T are written in index order.
+// Each radix digit is found by one warp, on histograms that alternate between two buffers.
+// Returns false, having written nothing, when the sample says too many keys would be kept or
+// the segments hold more than fit or fewer than k: the caller then runs the multi-pass path.
+__device__ bool select_fast(SelectSmem& S, const float* row, const float* samp, int sample_shift, int L, int k,
+                            int32_t* out, float* osc, int k_max) {
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t* ckey = S.cand;
+  uint32_t* cidx = S.cand + kFastCap;
+  // ---- 1. the threshold lo from a strided sample ----
+  // the scoring kernel wrote every 2^sample_shift-th score of the list to its sample row
+  const int ns = (L + (1 << sample_shift) - 1) >> sample_shift;
+  const float mean = (float)ns * (float)k / (float)L;
+  const int r_lo = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
+  if (ns > kFastCap || r_lo >= ns || (int64_t)r_lo * L > (int64_t)kFastCap * ns * 3 / 4) return false;
+  for (int i = threadIdx.x; i < kSelBins; i += kSelectThreads) S.hist[0][i] = 0u;
+  for (int s = threadIdx.x; s < ns; s += kSelectThreads) ckey[s] = score_key(__ldcg(samp + s));
+  __syncthreads();
+  radix_round(S, ckey, ns, 11, 21, true, 0u, r_lo, 0);
+  uint32_t prefix = (uint32_t)S.found_bin;
+  int need = r_lo - S.found_above;
+  radix_round(S, ckey, ns, 11, 10, false, prefix, need, 1);
+  prefix = (prefix << 11) | (uint32_t)S.found_bin;
+  const float lo_f = key_score(prefix << 10);   // key >= lo  <=>  score >= lo_f (the map is monotone)
+
+  // ---- 2. the scores >= lo, in index order ----
+  // Each step a warp reads kRow * kFastUnroll scores: lane l the float4s at base + kRow u + 4 l.
+  // The counting pass keeps every lane's keep bits of every step (16 bits: float4 u, element j
+  // at bit 4 u + j) when the segment has at most kSelMaskIters steps, so that the copying pass
+  // skips the steps where the warp keeps nothing and visits only the kept elements.
+  constexpr int kRow = 128;
+  constexpr int kStep = kRow * kFastUnroll;
+  const int seg = ((L + kSelWarps - 1) / kSelWarps + kRow - 1) / kRow * kRow;
+  const int s0 = min(warp * seg, L), s1 = min(s0 + seg, L);
+  const bool masks = (seg + kStep - 1) / kStep <= kSelMaskIters;
+  auto keep_bits = [&](const float4* v, int base) -> uint32_t {
+    uint32_t m = 0u;
+    if (base + kStep <= s1) {   // a whole step inside the segment (uniform over the warp)
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) neq += (c0 + j < kept && ckey[c0 + j] == T);
-  int eq_total;
-  int eq_run = block_exclusive_scan<kSelectThreads>(neq, S.scan_tmp, &eq_total);
-  int nsel = 0;
-  uint32_t selmask = 0u;
+      for (int u = 0; u < kFastUnroll; ++u)
+        m |= ((uint32_t)(v[u].x >= lo_f) | ((uint32_t)(v[u].y >= lo_f) << 1) | ((uint32_t)(v[u].z >= lo_f) << 2) |
+              ((uint32_t)(v[u].w >= lo_f) << 3)) << (4 * u);
+    } else {
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    if (c0 + j >= kept) break;
-    const uint32_t key = ckey[c0 + j];
-    bool sel = key > T;
-    if (key == T) {
-      sel = eq_run < need_eq;
-      ++eq_run;
-    }
-    if (sel) {
-      selmask |= 1u << j;
-      ++nsel;
-    }
-  }
-  int sel_total;
-  int pos = block_exclusive_scan<kSelectThreads>(nsel, S.scan_tmp, &sel_total);
-#pragma unroll
-  for (int j = 0; j < kPer; ++j)
-    if (selmask & (1u << j)) {
-      if (pos < k) {
-        out[pos] = (int32_t)cidx[c0 + j];
-        if (osc != nullptr) osc[pos] = key_score(ckey[c0 + j]);
+      for (int u = 0; u < kFastUnroll; ++u) {
+        const int i = base + kRow * u + 4 * lane;
+        m |= ((uint32_t)(i < s1 && v[u].x >= lo_f) | ((uint32_t)(i + 1 < s1 && v[u].y >= lo_f) << 1) |
+              ((uint32_t)(i + 2 < s1 && v[u].z >= lo_f) << 2) | ((uint32_t)(i + 3 < s1 && v[u].w >= lo_f) << 3))
+             << (4 * u);
       }
-      ++pos;
     }
+    return m;
+  };
+  auto load_step = [&](float4* v, int base) {
+#pragma unroll
+    for (int u = 0; u < kFastUnroll; ++u) {
+      const int i = base + kRow * u + 4 * lane;
+      v[u] = i < s1 ? __ldcg(reinterpret_cast<const float4*>(row + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  int cnt = 0;
+  for (int base = s0, it = 0; base < s1; base += kStep, ++it) {
+    float4 v[kFastUnroll];
+    load_step(v, base);
+    const uint32_t m = keep_bits(v, base);
+    cnt += __popc(m);
+    if (masks) S.keep[warp][it][lane] = (uint16_t)m;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(FULL, cnt, o);
+  if (lane == 0) S.wcount[warp] = cnt;
+  __syncthreads();
+  int off = 0, kept = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) {
+    const int c = S.wcount[w];
+    off += w < warp ? c : 0;
+    kept += c;
+  }
+  if (kept > kFastCap || kept < k) return false;   // the same decision in every thread
+  static_assert(kFastUnroll <= 4, "one 8-bit count field per float4 in a 32-bit word");
+  for (int base = s0, it = 0; base < s1; base += kStep, ++it) {
+    uint32_t m;
+    float4 v[kFastUnroll];
+    if (masks) {
+      m = S.keep[warp][it][lane];
+      if (__ballot_sync(FULL, m != 0u) == 0u) continue;   // nothing kept in this step
+      load_step(v, base);
+    } else {
+      load_step(v, base);
+      m = keep_bits(v, base);
+    }
+    // the kept counts of the lane's float4s (each <= 4) packed 8 bits apart: one lane scan gives
+    // every float4's output offset (a field's warp total is at most 128)
+    uint32_t packed = 0u;
+#pragma unroll
+    for (int u = 0; u < kFastUnroll; ++u) packed |= (uint32_t)__popc((m >> (4 * u)) & 0xFu) << (8 * u);
+    uint32_t inc = packed;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(FULL, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const uint32_t excl = inc - packed, tot = __shfl_sync(FULL, inc, 31);
+#pragma unroll
+    for (int u = 0; u < kFastUnroll; ++u) {
+      int pos = off + (int)((excl >> (8 * u)) & 0xFFu);
+      uint32_t nib = (m >> (4 * u)) & 0xFu;
+      const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      while (nib != 0u) {
+        const int j = __ffs(nib) - 1;
+        nib &= nib - 1u;
+        float x = f[0];
+        x = j == 1 ? f[1] : x;
+        x = j == 2 ? f[2] : x;
+        x = j == 3 ? f[3] : x;
+        ckey[pos] = score_key(x);
+        cidx[pos] = (uint32_t)(base + kRow * u + 4 * lane + j);
+        ++pos;
+      }
+      off += (int)((tot >> (8 * u)) & 0xFFu);
+    }
+  }
+  __syncthreads();
+
+  // ---- 3. the exact k-th key among the kept ones, then the ordered output ----
+  radix_round(S, ckey, kept, 11, 21, true, 0u, k, 0);
+  prefix = (uint32_t)S.found_bin;
+  need = k - S.found_above;
+  radix_round(S, ckey, kept, 11, 10, false, prefix, need, 1);
+  prefix = (prefix << 11) | (uint32_t)S.found_bin;
+  need -= S.found_above;
+  radix_round(S, ckey, kept, 10, 0, false, prefix, need, 0);
+  const uint32_t T = (prefix << 10) | (uint32_t)S.found_bin;
+  const int need_eq = need - S.found_above;   // keys == T to keep: the lowest-index ones
+
+  // warp w takes the kept entries [r0, r1); its lanes walk them 32 at a time
+  const int R = (kept + kSelWarps - 1) / kSelWarps;
+  const int r0 = min(warp * R, kept), r1 = min(r0 + R, kept);
+  int neq = 0;
+  for (int c = r0 + lane; c < r1; c += 32) neq += ckey[c] == T;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) neq += __shfl_xor_sync(FULL, neq, o);
+  if (lane == 0) S.wcount[warp] = neq;
+  __syncthreads();
+  int eq_before = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) eq_before += w < warp ? S.wcount[w] : 0;
+  const unsigned below = (1u << lane) - 1u;
+  int nsel = 0, eq_run = eq_before;
+  for (int c0 = r0; c0 < r1; c0 += 32) {
+    const int c = c0 + lane;
+    const uint32_t key = c < r1 ? ckey[c] : 0u;
+    const bool eq = c < r1 && key == T;
+    const unsigned eqm = __ballot_sync(FULL, eq);
+    const bool sel = c < r1 && (key > T || (eq && eq_run + __popc(eqm & below) < need_eq));
+    nsel += __popc(__ballot_sync(FULL, sel));
+    eq_run += __popc(eqm);
+  }
+  __syncthreads();   // every warp has read the equal-key counts
+  if (lane == 0) S.wcount[warp] = nsel;
+  __syncthreads();
+  int pos = 0;
+#pragma unroll
+  for (int w = 0; w < kSelWarps; ++w) pos += w < warp ? S.wcount[w] : 0;
+  eq_run = eq_before;
+  for (int c0 = r0; c0 < r1; c0 += 32) {
+    const int c = c0 + lane;
+    const uint32_t key = c < r1 ? ckey[c] : 0u;
+    const bool eq = c < r1 && key == T;
+    const unsigned eqm = __ballot_sync(FULL, eq);
+    const bool sel = c < r1 && (key > T || (eq && eq_run + __popc(eqm & below) < need_eq));
+    const unsigned selm = __ballot_sync(FULL, sel);
+    const int p = pos + __popc(selm & below);
+    if (sel && p < k) {
+      out[p] = (int32_t)cidx[c];
+      if (osc != nullptr) osc[p] = key_score(key);
+    }
+    pos += __popc(selm);
+    eq_run += __popc(eqm);
+  }
   for (int i = k + threadIdx.x; i < k_max; i += kSelectThreads) {
     out[i] = -1;
     if (osc != nullptr) osc[i] = -CUDART_INF_F;
@@ -565,11 +716,13 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
     }
     return;
   }
-  if (L >= kFastMinL && select_fast(S, row, L, k, out, osc, a.k_max)) return;
+  if (L >= kFastMinL &&
+      select_fast(S, row, a.samples + (int64_t)th * a.sample_stride, a.sample_shift, L, k, out, osc, a.k_max))
+    return;
   const int tile_elems = kSelectThreads * kSelPerThread;
 
   // ---- pass 1: histogram of the top 11 key bits ----
-  for (int i = threadIdx.x; i < kSelBins; i += kSelectThreads) S.hist[i] = 0u;
+  for (int i = threadIdx.x; i < kSelBins; i += kSelectThreads) S.hist[0][i] = 0u;
   __syncthreads();
   for (int base = 0; base < L; base += tile_elems) {
     const int i0 = base + threadIdx.x * kSelPerThread;
@@ -577,13 +730,13 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
     load16(row, i0, L, f);
 #pragma unroll
     for (int j = 0; j < kSelPerThread; ++j)
-      if (i0 + j < L) atomicAdd(&S.hist[score_key(f[j]) >> 21], 1u);
+      if (i0 + j < L) atomicAdd(&S.hist[0][score_key(f[j]) >> 21], 1u);
   }
   __syncthreads();
   select_bin(S, kSelBins, k);
   uint32_t prefix = (uint32_t)S.found_bin & (kSelBins - 1);
   int need = k - S.found_above;
-  int ccount = (int)S.hist[prefix];
+  int ccount = (int)S.hist[0][prefix];
   int shift = 21;
   __syncthreads();
 
@@ -591,7 +744,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
   while (ccount > kCandMax && shift > 0) {
     const int nb = shift >= 11 ? 11 : shift;
     shift -= nb;
-    for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[i] = 0u;
+    for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[0][i] = 0u;
     __syncthreads();
     for (int base = 0; base < L; base += tile_elems) {
       const int i0 = base + threadIdx.x * kSelPerThread;
@@ -600,7 +753,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
 #pragma unroll
       for (int j = 0; j < kSelPerThread; ++j) {
         const uint32_t key = score_key(f[j]);
-        if (i0 + j < L && (key >> (shift + nb)) == prefix) atomicAdd(&S.hist[(key >> shift) & ((1u << nb) - 1)], 1u);
+        if (i0 + j < L && (key >> (shift + nb)) == prefix) atomicAdd(&S.hist[0][(key >> shift) & ((1u << nb) - 1)], 1u);
       }
     }
     __syncthreads();
@@ -608,7 +761,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
     const uint32_t d = (uint32_t)S.found_bin & ((1u << nb) - 1);
     prefix = (prefix << nb) | d;
     need -= S.found_above;
-    ccount = (int)S.hist[d];
+    ccount = (int)S.hist[0][d];
     __syncthreads();
   }
 
@@ -634,11 +787,11 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
     while (shift > 0) {
       const int nb = shift >= 8 ? 8 : shift;
       shift -= nb;
-      for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[i] = 0u;
+      for (int i = threadIdx.x; i < (1 << nb); i += kSelectThreads) S.hist[0][i] = 0u;
       __syncthreads();
       for (int c = threadIdx.x; c < nc; c += kSelectThreads) {
         const uint32_t key = S.cand[c];
-        if ((key >> (shift + nb)) == prefix) atomicAdd(&S.hist[(key >> shift) & ((1u << nb) - 1)], 1u);
+        if ((key >> (shift + nb)) == prefix) atomicAdd(&S.hist[0][(key >> shift) & ((1u << nb) - 1)], 1u);
       }
       __syncthreads();
       select_bin(S, 1 << nb, need);
