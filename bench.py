@@ -9,8 +9,9 @@ traffic O(k d) instead of O(N d)).
 One step runs the whole path on one batch of the workload:
   exact top-k indexer (score + select) -> sparse decode on the selected rows
   -> dense decode on the same cache (the comparator),
-each leg bracketed by CUDA events on the launching stream, with a 256 MiB
-write (twice the 126 MB L2) before each leg so every leg reads from HBM.
+each leg captured once into a CUDA graph and replayed between two CUDA events on
+the launching stream, with a 256 MiB write and a 256 MiB read (twice the 126 MB
+L2) before each leg so every leg reads from HBM.
 `value` is the sparse-decode leg (the metric); the other legs are reported
 beside it.  Multi-GPU runs are weak scaling: every rank decodes its own batch
 (no data-path collective), the timings are the max over ranks.
@@ -84,6 +85,8 @@ def workload_desc(cfg, k):
         "context": cfg.max_seq_len, "k": k, "tokens_per_seq": cfg.tokens_per_seq,
         "l2": "flushed before every timed leg: 256 MiB device write, then a 256 MiB read (no input, and "
               "none of the flush's dirty lines, left in L2)",
+        "timing": "each leg (its library call) captured once into a CUDA graph; CUDA events around every "
+                  "replay on the launching stream",
     }
 
 
@@ -452,6 +455,20 @@ def sum_over_ranks(values, device):
     return t.tolist()
 
 
+def leg_graph(fn):
+    """`fn` (one leg: its library calls, buffers already sized by an eager run) captured once
+    into a CUDA graph.  The timed region then replays it: the whole leg is enqueued in one call,
+    so host-side launch overhead never leaves the GPU idle inside the events."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def time_legs(tsd, W, name, rank, dev, steps, warmup, flush):
     """The three legs (exact top-k, sparse decode at the workload's 50x k, dense decode) of one more
     workload, timed like the line's own legs (CUDA events, L2 flushed before each), with the
@@ -484,15 +501,17 @@ def time_legs(tsd, W, name, rank, dev, steps, warmup, flush):
         for leg in legs:
             flush()
             leg()
+    graphs = [leg_graph(leg) for leg in legs]
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
     torch.cuda.synchronize()
     for s_ in range(steps):
-        for j, leg in enumerate(legs):
+        for j, g in enumerate(graphs):
             flush()
             ev[s_][2 * j].record(stream)
-            leg()
+            g.replay()
             ev[s_][2 * j + 1].record(stream)
     torch.cuda.synchronize()
+    del graphs
     if tsd.read_device_status(ws) != 0:
         raise RuntimeError(f"device status bits set on {name}")
     ms = np.array([[ev[s_][2 * j].elapsed_time(ev[s_][2 * j + 1]) for j in range(3)] for s_ in range(steps)])
@@ -569,6 +588,7 @@ def run_native(args):
     torch.cuda.synchronize()
     if tsd.read_device_status(ws) != 0:
         raise RuntimeError("device status bits set during warm-up")
+    leg_graphs = [leg_graph(leg) for leg in legs]
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     if world > 1:
@@ -576,12 +596,13 @@ def run_native(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         for s in range(args.steps):
-            for j, leg in enumerate(legs):
+            for j, g in enumerate(leg_graphs):
                 flush()
                 ev[s][2 * j].record(stream)
-                leg()
+                g.replay()
                 ev[s][2 * j + 1].record(stream)
         torch.cuda.synchronize()
+    del leg_graphs
     if world > 1:
         dist.barrier()
     ms = np.array([[ev[s][2 * j].elapsed_time(ev[s][2 * j + 1]) for j in range(3)] for s in range(args.steps)])

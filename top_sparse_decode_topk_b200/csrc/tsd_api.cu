@@ -17,7 +17,7 @@
 #include "tsd_kvtile.cuh"
 
 namespace tsd {
-cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream);
+cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream, bool dependent);
 cudaError_t launch_dense_decode(const DecodeArgs& a, const KvMaps& maps, int batch, int hkv, cudaStream_t stream);
 cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int batch, int hkv, int num_lists,
                         cudaStream_t stream);
@@ -379,9 +379,12 @@ static tsd_status decode_common(const tsd_kv_cache* cache, const tsd_queries* qu
   return TSD_OK;
 }
 
+// `dependent`: launched right after the selection that wrote idx (tsd_decode_step), as its
+// programmatic dependent: the decode kernel starts while the selection drains and waits for it
+// before its first read.
 static tsd_status sparse_decode_impl(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
-                                     const float* logw, int32_t k_max, void* out, int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
-                             tsd_stream_t stream) {
+                                     const float* logw, int32_t k_max, void* out, int32_t out_dtype, float* lse,
+                                     void* ws, size_t ws_bytes, tsd_stream_t stream, bool dependent = false) {
   KvView kv; QView qv; Shapes sh;
   tsd_status st = decode_common(cache, queries, out, out_dtype, lse, ws, ws_bytes, &kv, &qv, &sh);
   if (st != TSD_OK) return st;
@@ -410,7 +413,8 @@ static tsd_status sparse_decode_impl(const tsd_kv_cache* cache, const tsd_querie
   a.part_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_acc);
   a.sched = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 4);
   a.persistent = p.stream;
-  return cuda_status(launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, reinterpret_cast<cudaStream_t>(stream), dependent));
 }
 
 tsd_status tsd_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
@@ -459,7 +463,7 @@ tsd_status tsd_decode_step(const tsd_kv_cache* cache, const tsd_queries* queries
   int32_t* idx = out_idx != nullptr ? out_idx : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.off_idx);
   tsd_status st = topk_select_impl(cache, queries, k_max, k_per_token, idx, nullptr, out_count, ws, L.shared, stream);
   if (st != TSD_OK) return st;
-  return sparse_decode_impl(cache, queries, idx, nullptr, k_max, out, out_dtype, lse, ws, L.shared, stream);
+  return sparse_decode_impl(cache, queries, idx, nullptr, k_max, out, out_dtype, lse, ws, L.shared, stream, true);
 }
 
 // Device staging of tsd_sparse_decode_host, after the sparse-decode workspace.

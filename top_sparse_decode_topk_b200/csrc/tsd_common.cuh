@@ -111,6 +111,17 @@ __device__ __forceinline__ int kv_len_of(const QView& qv, const SeqInfo& s, int 
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch (a kernel launched with the programmatic stream serialization
+// attribute may start while the previous kernel of the stream drains)
+// ---------------------------------------------------------------------------
+// In the dependent kernel: wait until the previous kernel has completed and its writes are
+// visible.  A no-op when the kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+// In the previous kernel: this CTA no longer holds back the dependent kernel's launch (which
+// starts once every CTA has done so or exited; it still waits in pdl_wait for completion).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Numerics
 // ---------------------------------------------------------------------------
 // 2^x via the hardware approximation (ex2.approx, documented PTX instruction).
@@ -118,6 +129,21 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Two fp32 lanes of one 64-bit register (Blackwell's packed fp32x2 arithmetic): d = a * b + c
+// lane by lane, each lane rounded as a scalar fmaf.
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// A bf16 pair (low half = first element) -> the fp32 pair in one 64-bit register (exact).
+__device__ __forceinline__ unsigned long long bf16x2_to_f32x2(uint32_t w) {
+  return ((unsigned long long)(w & 0xFFFF0000u) << 32) | (unsigned long long)(w << 16);
+}
+__device__ __forceinline__ float f32x2_sum(unsigned long long v) {
+  return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
 }
 
 // Two bf16 packed in a 32-bit word -> two fp32 (exact: bf16 is the top half of fp32).
@@ -313,6 +339,24 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tmp /* >= N
   *total = warp_tmp[NT / 32];
   __syncthreads();
   return excl;
+}
+
+// Launch `kernel` on `stream` as a programmatic dependent of the kernel before it: it may start
+// while that kernel drains, and must call pdl_wait() before it reads anything that kernel writes.
+template <typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 }  // namespace tsd

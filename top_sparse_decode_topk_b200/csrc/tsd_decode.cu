@@ -290,6 +290,7 @@ __device__ __forceinline__ void finish_list(const DecodeArgs& a, int64_t list_id
 template <bool WEIGHTED>
 __global__ void __launch_bounds__(kSpThreads, kSpCtasPerSm) sparse_decode_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char sp_ring[];   // [warp][kSpStages][K rows, V rows]
+  pdl_wait();   // a dependent launch (after the selection that wrote idx) starts here
   // task states of the CTA's warps, combined per list before anything leaves the CTA
   __shared__ float2 s_ml[kSpWarps];
   __shared__ __align__(16) float s_acc[kSpWarps][kHeadDim];
@@ -745,6 +746,7 @@ __device__ __forceinline__ void merge_partials_of_list(const DecodeArgs& a, int6
 template <bool WEIGHTED>
 __global__ void __launch_bounds__(kSsThreads, kSsCtasPerSm) sparse_stream_kernel(DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char ss_smem[];
+  pdl_wait();   // a dependent launch (after the selection that wrote idx) starts here
   constexpr unsigned FULL = 0xFFFFFFFFu;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -795,8 +797,14 @@ __global__ void __launch_bounds__(kSsThreads, kSsCtasPerSm) sparse_stream_kernel
       uint32_t nx = 0;
       if (lane == 0) nx = atomicAdd(a.sched, 1u);
       tau_next = __shfl_sync(FULL, nx, 0);
-      const int c = (int)(tau % C);
-      int64_t r = tau / C;
+      // tasks are numbered chunk-major: (chunk, sequence, kv head, list).  Every list's chunk 0 is
+      // handed out first, then every list's chunk 1, and so on, so all lists advance through
+      // their entries together, as in a single wave: a row that several lists of a kv head
+      // select (at similar ranks of their ascending lists) is read again while the first read is
+      // still in L2.  Chunks past the end of short lists come last and are skipped at the fetch.
+      const int64_t slots = (int64_t)a.kv.batch * a.kv.hkv * M;
+      const int c = (int)(tau / slots);
+      int64_t r = tau - (int64_t)c * slots;
       const int m = (int)(r % M);
       r /= M;
       const int g = (int)(r % a.kv.hkv);
@@ -1237,7 +1245,8 @@ __global__ void __launch_bounds__(kDnThreads, kDnCtasPerSm) dense_decode_kernel(
 // Host launchers
 // ---------------------------------------------------------------------------
 // The persistent form: kSsCtasPerSm CTAs per SM (fewer when there are fewer tasks).
-static cudaError_t launch_sparse_stream(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
+static cudaError_t launch_sparse_stream(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream,
+                                        bool dependent) {
   const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
   if (tasks >= ((int64_t)1 << 31) || a.sched == nullptr) return cudaErrorInvalidValue;
   int dev = 0, sms = 0;
@@ -1258,16 +1267,14 @@ static cudaError_t launch_sparse_stream(const DecodeArgs& a, int batch, int hkv,
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  if (a.logw != nullptr) {
-    sparse_stream_kernel<true><<<(unsigned)grid, kSsThreads, kSsSmemBytes, stream>>>(a);
-  } else {
-    sparse_stream_kernel<false><<<(unsigned)grid, kSsThreads, kSsSmemBytes, stream>>>(a);
-  }
+  auto kernel = a.logw != nullptr ? sparse_stream_kernel<true> : sparse_stream_kernel<false>;
+  if (dependent) return launch_dependent(kernel, dim3((unsigned)grid), dim3(kSsThreads), kSsSmemBytes, stream, a);
+  kernel<<<(unsigned)grid, kSsThreads, kSsSmemBytes, stream>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream) {
-  if (a.persistent) return launch_sparse_stream(a, batch, hkv, stream);
+cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream, bool dependent) {
+  if (a.persistent) return launch_sparse_stream(a, batch, hkv, stream, dependent);
   const int64_t tasks = (int64_t)batch * hkv * a.nsplit * a.lists_per_cta;
   const int64_t grid = (tasks + kSpWarps - 1) / kSpWarps;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
@@ -1281,11 +1288,9 @@ cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaSt
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  if (a.logw != nullptr) {
-    sparse_decode_kernel<true><<<(unsigned)grid, kSpThreads, kSpSmemBytes, stream>>>(a);
-  } else {
-    sparse_decode_kernel<false><<<(unsigned)grid, kSpThreads, kSpSmemBytes, stream>>>(a);
-  }
+  auto kernel = a.logw != nullptr ? sparse_decode_kernel<true> : sparse_decode_kernel<false>;
+  if (dependent) return launch_dependent(kernel, dim3((unsigned)grid), dim3(kSpThreads), kSpSmemBytes, stream, a);
+  kernel<<<(unsigned)grid, kSpThreads, kSpSmemBytes, stream>>>(a);
   return cudaGetLastError();
 }
 

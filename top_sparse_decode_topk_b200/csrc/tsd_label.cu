@@ -179,15 +179,49 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
     qs[m][j] = v;
   }
   __syncthreads();
-  // kLblUnroll tokens per thread per step: their page-table lookups, then their label rows,
-  // are all in flight together
-  for (int base = tok0; base < tok_end; base += kLblThreads * kLblUnroll) {
+  pdl_launch_dependents();   // the selection may launch; it waits for this kernel's scores
+  // Each warp walks steps of kLblStep consecutive tokens (lane l takes tokens 32 u + l of the
+  // step), the CTA's warps taking consecutive steps.  With pages of 4 tokens or more, a step's
+  // tokens lie in at most 32 pages: lane l holds the page-table entry of the step's l-th page,
+  // loaded one step ahead, and every token finds its row with a shuffle, so that only the
+  // label-row loads wait on memory inside a step.
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  constexpr int kWarps = kLblThreads / 32;
+  constexpr int kLblStep = 32 * kLblUnroll;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool paged = a.kv.page_table != nullptr;
+  const int shift = a.kv.page_shift;
+  const int pmask = (1 << shift) - 1;
+  const bool shfl_pages = paged && shift >= 2;   // a step then spans at most 32 pages
+  const int32_t* pt = paged ? a.kv.page_table + (int64_t)b * a.kv.max_pages : nullptr;
+  auto step_pages = [&](int st0) -> int32_t {    // lane l: the page entry of the step's l-th page
+    if (!shfl_pages || st0 >= tok_end) return -1;
+    const int p = (st0 >> shift) + lane;
+    return p <= ((min(st0 + kLblStep, tok_end) - 1) >> shift) ? __ldg(pt + p) : -1;
+  };
+  int st0 = tok0 + warp * kLblStep;
+  int32_t pg = step_pages(st0);
+  for (; st0 < tok_end; st0 += kWarps * kLblStep) {
+    const int32_t pg_next = step_pages(st0 + kWarps * kLblStep);
     uint32_t row[kLblUnroll];
 #pragma unroll
     for (int u = 0; u < kLblUnroll; ++u) {
-      const int tok = base + u * kLblThreads + threadIdx.x;
-      row[u] = tok < tok_end ? kv_row(a.kv, b, g, tok) : kInvalidRow;
-      if (tok < tok_end && row[u] == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
+      const int tok = st0 + 32 * u + lane;
+      if (shfl_pages) {
+        // tokens of a step start on a multiple of min(page, 64), so rel < 32
+        const int rel = ((st0 & pmask) + 32 * u + lane) >> shift;
+        const int32_t page = __shfl_sync(FULL, pg, rel & 31);
+        row[u] = kInvalidRow;
+        if (tok < tok_end) {
+          if (page >= 0 && (int64_t)page < a.kv.num_pages)
+            row[u] = (uint32_t)((((int64_t)page * a.kv.hkv + g) << shift) | (tok & pmask));
+          else
+            flag_status(a.status, TSD_DEV_BAD_PAGE);
+        }
+      } else {
+        row[u] = tok < tok_end ? kv_row(a.kv, b, g, tok) : kInvalidRow;
+        if (tok < tok_end && row[u] == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
+      }
     }
     uint4 raw[kLblUnroll][R / 8];
 #pragma unroll
@@ -198,28 +232,35 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
     }
 #pragma unroll
     for (int u = 0; u < kLblUnroll; ++u) {
-      const int tok = base + u * kLblThreads + threadIdx.x;
+      const int tok = st0 + 32 * u + lane;
       if (row[u] == kInvalidRow) continue;
-      float kf[R];
+      // channel pairs (2i, 2i + 1) as packed fp32x2: one fma.rn.f32x2 per pair, the even
+      // channels summed in the low lane and the odd ones in the high lane
+      unsigned long long k2[R / 2];
 #pragma unroll
-      for (int c = 0; c < R / 8; ++c) unpack8(raw[u][c], kf + 8 * c);
+      for (int c = 0; c < R / 8; ++c) {
+        k2[4 * c] = bf16x2_to_f32x2(raw[u][c].x);
+        k2[4 * c + 1] = bf16x2_to_f32x2(raw[u][c].y);
+        k2[4 * c + 2] = bf16x2_to_f32x2(raw[u][c].z);
+        k2[4 * c + 3] = bf16x2_to_f32x2(raw[u][c].w);
+      }
       for (int m = 0; m < nlists; ++m) {
-        float s0 = 0.f, s1 = 0.f;
-        const float4* qm = reinterpret_cast<const float4*>(qs[m]);   // 16-byte shared loads
+        const ulonglong2* qm = reinterpret_cast<const ulonglong2*>(qs[m]);   // 16-byte shared loads
+        unsigned long long acc = 0ull;
 #pragma unroll
-        for (int j = 0; j < R; j += 4) {
-          const float4 qv = qm[j / 4];
-          s0 = fmaf(qv.x, kf[j], s0);
-          s1 = fmaf(qv.y, kf[j + 1], s1);
-          s0 = fmaf(qv.z, kf[j + 2], s0);
-          s1 = fmaf(qv.w, kf[j + 3], s1);
+        for (int j = 0; j < R / 4; ++j) {
+          const ulonglong2 qq = qm[j];
+          acc = ffma2(qq.x, k2[2 * j], acc);
+          acc = ffma2(qq.y, k2[2 * j + 1], acc);
         }
+        const float sc = f32x2_sum(acc);
         if (tok < kvl[m]) {
-          a.scores[srow[m] + tok] = s0 + s1;
-          if ((tok & ((1 << a.sample_shift) - 1)) == 0) a.samples[prow[m] + (tok >> a.sample_shift)] = s0 + s1;
+          a.scores[srow[m] + tok] = sc;
+          if ((tok & ((1 << a.sample_shift) - 1)) == 0) a.samples[prow[m] + (tok >> a.sample_shift)] = sc;
         }
       }
     }
+    pg = pg_next;
   }
 }
 

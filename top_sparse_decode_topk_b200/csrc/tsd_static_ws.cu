@@ -26,7 +26,7 @@
 #include "tsd_plan.h"
 
 namespace tsd {
-cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream);
+cudaError_t launch_sparse_decode(const DecodeArgs& a, int batch, int hkv, cudaStream_t stream, bool dependent);
 tsd_status prepare_sparse_decode(const tsd_kv_cache* cache, const tsd_queries* queries, const int32_t* idx,
                                  int32_t k_max, void* out, int32_t out_dtype, float* lse, DecodeArgs* a,
                                  Shapes* sh, size_t* ws_needed, size_t* zero_bytes);
@@ -83,5 +83,5 @@ extern "C" tsd_status tsd_sparse_decode_static_ws(const tsd_kv_cache* cache, con
   a.part_ml = reinterpret_cast<float2*>(ws + lay.off_ml);
   a.part_acc = reinterpret_cast<float*>(ws + lay.off_acc);
   a.sched = reinterpret_cast<uint32_t*>(ws + 4);
-  return launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, s) == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
+  return launch_sparse_decode(a, (int)sh.batch, (int)sh.hkv, s, false) == cudaSuccess ? TSD_OK : TSD_ERR_CUDA;
 }

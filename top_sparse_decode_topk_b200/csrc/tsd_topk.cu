@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
   }
   store_q_tile(a.qv, si, g, G, lg * a.lists_per_cta, nlists, qhi, QF32 ? qlo : nullptr, threadIdx.x, kScThreads);
   __syncthreads();
+  pdl_launch_dependents();   // the selection may launch; it waits for this kernel's scores
 
   if (warp == kScConsumers) {
     produce_tiles<kScStages, kTileBytesKV, false>(a.kv, maps, b, g, tok0, tok_end, ntiles, stages, full,
@@ -708,6 +709,10 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
   float* osc = a.out_scores != nullptr ? a.out_scores + (int64_t)th * a.k_max : nullptr;
   if (a.out_count != nullptr && threadIdx.x == 0) a.out_count[th] = k;
   const float* row = a.scores + (int64_t)th * a.score_stride;
+  // launched as a dependent of the scoring kernel: everything above read only the call's
+  // inputs; the scores are read only once that kernel has completed
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (k == L || k == 0) {   // every visible token is kept, or none
     for (int i = threadIdx.x; i < a.k_max; i += kSelectThreads) {
@@ -893,8 +898,7 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  topk_select_kernel<<<num_lists, kSelectThreads, sizeof(SelectSmem), stream>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(topk_select_kernel, dim3(num_lists), dim3(kSelectThreads), sizeof(SelectSmem), stream, a);
 }
 
 // The selection alone, over scores another kernel wrote into the workspace (the label indexer).
@@ -906,8 +910,7 @@ cudaError_t launch_topk_select_only(const TopkArgs& a, int num_lists, cudaStream
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  topk_select_kernel<<<num_lists, kSelectThreads, sizeof(SelectSmem), stream>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(topk_select_kernel, dim3(num_lists), dim3(kSelectThreads), sizeof(SelectSmem), stream, a);
 }
 
 }  // namespace tsd
