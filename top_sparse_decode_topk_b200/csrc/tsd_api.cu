@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <math.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -295,6 +296,38 @@ size_t tsd_dense_decode_workspace_size(const tsd_kv_cache* cache, const tsd_quer
   return decode_layout(sh, p.nsplit).total;
 }
 
+// The exact indexer's candidate filter.  TSD_TOPK_FILTER unset: on when the score rows would not
+// stay in L2 (see topk_select_impl); "1": on wherever it can serve the call; "0": off;
+// "rescore": on with every threshold disabled, so that every list takes the selection's row
+// recomputation (a test hook for that path).
+enum { kFilterAuto = -1, kFilterOff = 0, kFilterOn = 1, kFilterRescore = 2 };
+static int filter_mode() {
+  const char* e = getenv("TSD_TOPK_FILTER");
+  if (e == nullptr) return kFilterAuto;
+  if (strcmp(e, "0") == 0) return kFilterOff;
+  if (strcmp(e, "rescore") == 0) return kFilterRescore;
+  return kFilterOn;
+}
+
+// Score rows above this many bytes leave L2 between the scoring kernel and the selection, so
+// the unfiltered form writes them to DRAM and reads them back; below it they stay in the 126 MB
+// L2 and the filter's pre-pass costs more than it saves.
+constexpr double kFilterMinRowBytes = 64.0 * 1024 * 1024;
+
+// Whether a list of any length with k <= k_max passes the threshold kernel's size test when its
+// sample takes every 2^shift-th token: with m = k_max / 2^shift the expected sample count above
+// the k-th score is at most m + 1, and r = ceil(m + 1 + 4 sqrt(m + 1) + 4) samples at stride
+// 2^shift stand for at most r 2^shift candidates, which must stay within 3/4 of the buffer.
+static bool filter_fits(int32_t k_max, int shift) {
+  const double m = (double)k_max / (double)(1LL << shift) + 1.0;
+  const double r = ceil(m + 4.0 * sqrt(m) + 4.0);
+  return r * (double)(1LL << shift) <= (double)kTopkCandCap * 3.0 / 4.0;
+}
+static bool score_on_tcgen05_host() {
+  const char* e = getenv("TSD_SCORE_KERNEL");
+  return e != nullptr && strcmp(e, "tcgen05") == 0;
+}
+
 static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
                                    const int32_t* k_per_token, int32_t* out_idx, float* out_scores,
                                    int32_t* out_count, void* ws, size_t ws_bytes, tsd_stream_t stream) {
@@ -319,8 +352,25 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   a.samples = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_samples);
   a.sample_stride = lay.sample_stride;
   a.sample_shift = lay.sample_shift;
+  // The candidate filter (sample pre-pass, per-list threshold, candidate appends while scoring,
+  // no score rows) serves bf16 queries with the warp-MMA scoring kernel when k_max is small
+  // enough for the candidates to fit; the kept scores' output (tsd_topk_select_scores), fp32
+  // queries and larger k take the paths over the full score rows.
+  const int fm = filter_mode();
+  const double row_bytes = (double)sh.tokens * sh.hq * (double)lay.score_stride * sizeof(float);
+  const bool can = !qv.q_f32 && out_scores == nullptr && !score_on_tcgen05_host();
+  if (fm == kFilterRescore) a.filter = can ? 2 : 0;
+  else if (fm == kFilterOn) a.filter = can && filter_fits(k_max, lay.sample_shift + 1) ? 1 : 0;
+  else if (fm == kFilterAuto)
+    a.filter = can && filter_fits(k_max, lay.sample_shift + 1) && row_bytes > kFilterMinRowBytes ? 1 : 0;
+  else a.filter = 0;
+  if (a.filter) a.sample_shift = lay.sample_shift + 1;   // the pre-pass samples every other sample slot
+  a.lo_key = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_lo);
+  a.cand = reinterpret_cast<uint2*>(static_cast<char*>(ws) + lay.off_cand);
+  a.meta = reinterpret_cast<int2*>(static_cast<char*>(ws) + lay.off_meta);
+  a.cand_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 256);
   // scoring streams K in the dense path's tiles, with its own occupancy
-  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScoreCtasPerSm);
+  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScoreCtasPerSm, kMaxWindowScore);
   a.lists_per_cta = p.lists_per_cta;
   a.list_groups = p.list_groups;
   a.window = p.window;
@@ -685,7 +735,9 @@ tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k,
   a.samples = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_samples);
   a.sample_stride = lay.sample_stride;
   a.sample_shift = lay.sample_shift;
-  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm);
+  a.filter = 0;
+  a.cand_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 256);
+  const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm, kMaxWindowScore);
   a.lists_per_cta = p.lists_per_cta;
   a.list_groups = p.list_groups;
   a.window = p.window;

@@ -41,6 +41,11 @@ struct TopkArgs {
   float* samples;         // [T][Hq][sample_stride]: score of every 2^sample_shift-th token
   int64_t sample_stride;
   int32_t sample_shift;
+  int32_t filter;         // 1: the sample pre-pass, thresholds and candidate appends run (exact indexer)
+  uint32_t* lo_key;       // [T][Hq] candidate threshold keys (filter)
+  uint2* cand;            // [T][Hq][kTopkCandCap] (key, index) candidates (filter)
+  uint32_t* cand_cnt;     // [T][Hq] candidate slots reserved (zero region; the selection clears it)
+  int2* meta;             // [T][Hq] (kv_len, k) of each list (filter: threshold kernel -> selection)
   int32_t lists_per_cta;
   int32_t list_groups;
   int32_t window;

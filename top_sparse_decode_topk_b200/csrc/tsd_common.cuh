@@ -172,6 +172,11 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The score of an order-preserving key (inverse of score_key; -0 comes back as +0).
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 // ---------------------------------------------------------------------------
 // Asynchronous global->shared copies (cp.async, 16 bytes, L2-only caching)
 // ---------------------------------------------------------------------------

@@ -137,7 +137,11 @@ __global__ void label_build_kernel(KvView kv, const int32_t* channels, int r, in
 // One CTA per (window, kv head x list group, sequence); each thread scores tokens
 // tok0 + threadIdx.x, + 256, ... against up to 16 lists whose label queries sit in shared
 // memory.  Unscaled fp32 dots; bf16 x bf16 products are exact, only the R-term sum rounds.
-template <int R>
+// NL = 0: any number of lists (at most 16), their queries, bounds and score rows read from shared
+// memory per list.  NL = 4: at most 4 lists (one decode token of a GQA group of 4, as in the
+// Llama-3-8B shape), whose query pairs, bounds and score rows live in registers, the list loop
+// unrolled; 2 tokens per lane per step keep the registers within two CTAs per SM.
+template <int R, int NL>
 __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, const uint16_t* label,
                                                                   const int32_t* channels) {
   __shared__ __align__(16) float qs[16][R];
@@ -187,8 +191,28 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
   // label-row loads wait on memory inside a step.
   constexpr unsigned FULL = 0xFFFFFFFFu;
   constexpr int kWarps = kLblThreads / 32;
-  constexpr int kLblStep = 32 * kLblUnroll;
+  constexpr int U = NL > 0 ? 2 : kLblUnroll;   // tokens per lane per step
+  constexpr int kLblStep = 32 * U;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NR = NL > 0 ? NL : 1;
+  unsigned long long qr[NR][R / 2];   // NL > 0: list m's query channel pairs
+  int kvr[NR];
+  int64_t srr[NR], prr[NR];
+  if constexpr (NL > 0) {
+#pragma unroll
+    for (int m = 0; m < NL; ++m) {
+      const ulonglong2* qm = reinterpret_cast<const ulonglong2*>(qs[m]);
+#pragma unroll
+      for (int j = 0; j < R / 4; ++j) {
+        const ulonglong2 qq = qm[j];
+        qr[m][2 * j] = qq.x;
+        qr[m][2 * j + 1] = qq.y;
+      }
+      kvr[m] = m < nlists ? kvl[m] : 0;
+      srr[m] = m < nlists ? srow[m] : 0;
+      prr[m] = m < nlists ? prow[m] : 0;
+    }
+  }
   const bool paged = a.kv.page_table != nullptr;
   const int shift = a.kv.page_shift;
   const int pmask = (1 << shift) - 1;
@@ -203,9 +227,9 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
   int32_t pg = step_pages(st0);
   for (; st0 < tok_end; st0 += kWarps * kLblStep) {
     const int32_t pg_next = step_pages(st0 + kWarps * kLblStep);
-    uint32_t row[kLblUnroll];
+    uint32_t row[U];
 #pragma unroll
-    for (int u = 0; u < kLblUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int tok = st0 + 32 * u + lane;
       if (shfl_pages) {
         // tokens of a step start on a multiple of min(page, 64), so rel < 32
@@ -223,15 +247,15 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
         if (tok < tok_end && row[u] == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
       }
     }
-    uint4 raw[kLblUnroll][R / 8];
+    uint4 raw[U][R / 8];
 #pragma unroll
-    for (int u = 0; u < kLblUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const uint4* src = reinterpret_cast<const uint4*>(label + (int64_t)row[u] * R);
 #pragma unroll
       for (int c = 0; c < R / 8; ++c) raw[u][c] = row[u] != kInvalidRow ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < kLblUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int tok = st0 + 32 * u + lane;
       if (row[u] == kInvalidRow) continue;
       // channel pairs (2i, 2i + 1) as packed fp32x2: one fma.rn.f32x2 per pair, the even
@@ -244,19 +268,34 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
         k2[4 * c + 2] = bf16x2_to_f32x2(raw[u][c].z);
         k2[4 * c + 3] = bf16x2_to_f32x2(raw[u][c].w);
       }
-      for (int m = 0; m < nlists; ++m) {
-        const ulonglong2* qm = reinterpret_cast<const ulonglong2*>(qs[m]);   // 16-byte shared loads
-        unsigned long long acc = 0ull;
+      const bool sampled = (tok & ((1 << a.sample_shift) - 1)) == 0;
+      if constexpr (NL > 0) {
 #pragma unroll
-        for (int j = 0; j < R / 4; ++j) {
-          const ulonglong2 qq = qm[j];
-          acc = ffma2(qq.x, k2[2 * j], acc);
-          acc = ffma2(qq.y, k2[2 * j + 1], acc);
+        for (int m = 0; m < NL; ++m) {
+          unsigned long long acc = 0ull;
+#pragma unroll
+          for (int j = 0; j < R / 2; ++j) acc = ffma2(qr[m][j], k2[j], acc);
+          const float sc = f32x2_sum(acc);
+          if (tok < kvr[m]) {
+            a.scores[srr[m] + tok] = sc;
+            if (sampled) a.samples[prr[m] + (tok >> a.sample_shift)] = sc;
+          }
         }
-        const float sc = f32x2_sum(acc);
-        if (tok < kvl[m]) {
-          a.scores[srow[m] + tok] = sc;
-          if ((tok & ((1 << a.sample_shift) - 1)) == 0) a.samples[prow[m] + (tok >> a.sample_shift)] = sc;
+      } else {
+        for (int m = 0; m < nlists; ++m) {
+          const ulonglong2* qm = reinterpret_cast<const ulonglong2*>(qs[m]);   // 16-byte shared loads
+          unsigned long long acc = 0ull;
+#pragma unroll
+          for (int j = 0; j < R / 4; ++j) {
+            const ulonglong2 qq = qm[j];
+            acc = ffma2(qq.x, k2[2 * j], acc);
+            acc = ffma2(qq.y, k2[2 * j + 1], acc);
+          }
+          const float sc = f32x2_sum(acc);
+          if (tok < kvl[m]) {
+            a.scores[srow[m] + tok] = sc;
+            if (sampled) a.samples[prow[m] + (tok >> a.sample_shift)] = sc;
+          }
         }
       }
     }
@@ -297,10 +336,17 @@ cudaError_t launch_topk_select_only(const TopkArgs& a, int num_lists, cudaStream
 cudaError_t launch_label_topk(const TopkArgs& a, const uint16_t* label, const int32_t* channels, int r, int nwin,
                               int batch, int hkv, int num_lists, cudaStream_t stream) {
   dim3 grid(nwin, hkv * a.list_groups, batch);
+  const bool few = a.lists_per_cta <= 4;   // the lists' queries fit in registers (r <= 16)
   switch (r) {
-    case 8: label_score_kernel<8><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
-    case 16: label_score_kernel<16><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
-    case 32: label_score_kernel<32><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
+    case 8:
+      if (few) label_score_kernel<8, 4><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
+      else label_score_kernel<8, 0><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
+      break;
+    case 16:
+      if (few) label_score_kernel<16, 4><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
+      else label_score_kernel<16, 0><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
+      break;
+    case 32: label_score_kernel<32, 0><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
     default: return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaGetLastError();

@@ -137,7 +137,15 @@ constexpr int kScCtasPerSm = 5;    // resident top-k scoring CTAs per SM, warp-M
 constexpr int kScTcCtasPerSm = 5;  // the same for the tcgen05 scoring kernel
 constexpr int kScoreCtasPerSm = kScCtasPerSm;
 static_assert(kScTcCtasPerSm == kScCtasPerSm, "both scoring kernels share one window plan");
-constexpr int64_t kMaxWindow = 8192;   // tokens per dense / scoring CTA at most
+// Tokens per CTA at most.  Windows are sized on max_seq_len, so on a ragged batch (lengths
+// 8K-128K against a 128K bound) about half the windows lie past their sequence's end and exit at
+// once, and the live ones run in coarse waves.  Measured on the ragged batch (CUDA graphs, L2
+// flushed): the top-k leg took 1677 us with 8192-token windows and 1585 us with 4096 (2048: 1589);
+// dense decode took 2006 us with 8192 and 1979 us with 4096, but on the Qwen2.5-72B shape 4096
+// forced a third wave of dense CTAs (392 -> 405 us).  So the scoring kernels cap at 4096 tokens and
+// dense decode at 8192.
+constexpr int64_t kMaxWindowDense = 8192;
+constexpr int64_t kMaxWindowScore = 4096;
 
 // Window of `ns` windows over max_seq_len, rounded up to whole 64-token tiles.
 inline int64_t dense_window(int64_t max_seq_len, int64_t ns) {
@@ -145,7 +153,7 @@ inline int64_t dense_window(int64_t max_seq_len, int64_t ns) {
   return (w + 63) / 64 * 64;
 }
 
-inline DensePlan plan_dense(const Shapes& s, int64_t wave) {
+inline DensePlan plan_dense(const Shapes& s, int64_t wave, int64_t kMaxWindow = kMaxWindowDense) {
   DensePlan p;
   const int64_t m = s.group * s.max_tokens;
   p.lists_per_cta = (int)(m < kDenseMaxLists ? m : kDenseMaxLists);
@@ -205,12 +213,19 @@ inline DecodeLayout decode_layout(const Shapes& s, int nsplit) {
 // while the sample would exceed kMaxSample scores.
 constexpr int64_t kMaxSample = 4096;
 
+// Candidates of the exact indexer (tsd_topk_select): the scoring kernel also appends every
+// (key, index) at or above a list's sampled threshold, at most kTopkCandCap per list.
+constexpr int kTopkCandCap = 8192;
+
 struct TopkLayout {
   size_t off_scores;
   int64_t score_stride;
   size_t off_samples;
   int32_t sample_shift;
   int64_t sample_stride;
+  size_t off_lo;      // uint32 [T][Hq]: each list's candidate threshold key
+  size_t off_cand;    // uint2 [T][Hq][kTopkCandCap]: (key, index) candidates
+  size_t off_meta;    // int2 [T][Hq]: each list's (kv_len, k), written by the threshold kernel
   size_t total;
 };
 
@@ -222,7 +237,10 @@ inline TopkLayout topk_layout(const Shapes& s) {
   while (((s.max_seq_len + (1LL << l.sample_shift) - 1) >> l.sample_shift) > kMaxSample) ++l.sample_shift;
   l.sample_stride = (((s.max_seq_len + (1LL << l.sample_shift) - 1) >> l.sample_shift) + 3) / 4 * 4;
   l.off_samples = l.off_scores + align256((size_t)s.tokens * s.hq * l.score_stride * sizeof(float));
-  l.total = l.off_samples + align256((size_t)s.tokens * s.hq * l.sample_stride * sizeof(float));
+  l.off_lo = l.off_samples + align256((size_t)s.tokens * s.hq * l.sample_stride * sizeof(float));
+  l.off_cand = l.off_lo + align256((size_t)s.tokens * s.hq * sizeof(uint32_t));
+  l.off_meta = l.off_cand + align256((size_t)s.tokens * s.hq * kTopkCandCap * 2 * sizeof(uint32_t));
+  l.total = l.off_meta + align256((size_t)s.tokens * s.hq * 2 * sizeof(int32_t));
   return l;
 }
 

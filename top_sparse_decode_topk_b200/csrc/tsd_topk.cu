@@ -61,6 +61,10 @@ struct ScLayout {
 constexpr int kScStages = 2;
 static_assert(ScLayout<true, kScStages>::bytes + 1024 <= 228 * 1024 / kScCtasPerSm, "scoring CTAs per SM");
 
+// Candidate slots a quad reserves at a time, and the index that marks a reserved slot left unused.
+constexpr uint32_t kCandChunk = 8;
+constexpr uint32_t kCandHole = 0xFFFFFFFFu;
+
 template <bool QF32>
 __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(TopkArgs a, const __grid_constant__ KvMaps maps) {
   using Lay = ScLayout<QF32, kScStages>;
@@ -126,26 +130,102 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
     }
   }
   const int smask = (1 << a.sample_shift) - 1;
+  // candidate filter: this lane's lists' threshold keys and candidate buffers (the test is on
+  // the order-preserving key, so that every score the full-row selection ranks above lo is kept)
+  uint32_t lo_k[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+  uint32_t* ccnt[2] = {nullptr, nullptr};
+  uint2* cbuf[2] = {nullptr, nullptr};
+  uint32_t pool_next[2] = {0u, 0u}, pool_end[2] = {0u, 0u};   // the quad's reserved, unused slots
+  if (a.filter) {
+    pdl_wait();   // the threshold kernel wrote lo
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int m = (lane >> 2) + 8 * hr;
+      if (m < nlists) {
+        const int mg = lg * a.lists_per_cta + m;
+        const int j = mg / G;
+        const int64_t list = (int64_t)(si.t0 + j) * a.qv.hq + g * G + (mg - j * G);
+        lo_k[hr] = __ldcg(a.lo_key + list);
+        ccnt[hr] = a.cand_cnt + list;
+        cbuf[hr] = a.cand + list * kTopkCandCap;
+      }
+    }
+  }
   for (int tile = 0; tile < ntiles; ++tile) {
     if (!consume_wait<kScStages>(full, abort_flag, tile, lane, a.status)) break;
     float sc[2][4];
     qk_tile<QF32>(qhi, qlo, stages + (size_t)(tile % kScStages) * kTileBytesKV, warp, lane, sc);
-    const int tbase = tok0 + tile * kTileTok + 16 * warp + 2 * (lane & 3);
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int tk = tbase + 8 * nt;   // even: the pair (tk, tk + 1) is 8-byte aligned
-        if (tk + 1 < kvl[hr]) {
-          *reinterpret_cast<float2*>(srow[hr] + tk) = make_float2(sc[nt][2 * hr], sc[nt][2 * hr + 1]);
-        } else if (tk < kvl[hr]) {
-          srow[hr][tk] = sc[nt][2 * hr];
-        }
-        if ((tk & smask) == 0 && tk < kvl[hr]) prow[hr][tk >> a.sample_shift] = sc[nt][2 * hr];
-      }
-    // the stores consume every fragment read from the stage: release it to the producer
+    // the fragments are in registers: release the stage to the producer before the stores
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[tile % kScStages]);
+    const int tbase = tok0 + tile * kTileTok + 16 * warp + 2 * (lane & 3);
+    if (!a.filter) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int tk = tbase + 8 * nt;   // even: the pair (tk, tk + 1) is 8-byte aligned
+          if (tk + 1 < kvl[hr]) {
+            *reinterpret_cast<float2*>(srow[hr] + tk) = make_float2(sc[nt][2 * hr], sc[nt][2 * hr + 1]);
+          } else if (tk < kvl[hr]) {
+            srow[hr][tk] = sc[nt][2 * hr];
+          }
+          if ((tk & smask) == 0 && tk < kvl[hr]) prow[hr][tk >> a.sample_shift] = sc[nt][2 * hr];
+        }
+      continue;
+    }
+    // the filtered form: the lane's scores whose keys reach its lists' thresholds go to the lists'
+    // candidate buffers.  The 4 lanes of a quad share a list row and take their slots, in lane
+    // order, from the quad's pool; the last lane refills the pool kCandChunk slots at a time with
+    // one atomic on the list's counter, so that the round trip is rare.
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      uint32_t f = 0u;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int tk = tbase + 8 * nt;
+        f |= (uint32_t)(tk < kvl[hr] && score_key(sc[nt][2 * hr]) >= lo_k[hr]) << (2 * nt);
+        f |= (uint32_t)(tk + 1 < kvl[hr] && score_key(sc[nt][2 * hr + 1]) >= lo_k[hr]) << (2 * nt + 1);
+      }
+      if (__ballot_sync(0xFFFFFFFFu, f != 0u) == 0u) continue;
+      const int c = __popc(f);
+      int x = c;   // inclusive prefix over the quad
+      int y = __shfl_up_sync(0xFFFFFFFFu, x, 1);
+      if ((lane & 3) >= 1) x += y;
+      y = __shfl_up_sync(0xFFFFFFFFu, x, 2);
+      if ((lane & 3) >= 2) x += y;
+      const uint32_t tot = (uint32_t)__shfl_sync(0xFFFFFFFFu, x, lane | 3);
+      const uint32_t room = pool_end[hr] - pool_next[hr];
+      uint32_t fresh = 0u, want = 0u;
+      if (tot > room) {
+        want = (tot - room + kCandChunk - 1) / kCandChunk * kCandChunk;
+        if ((lane & 3) == 3) fresh = atomicAdd(ccnt[hr], want);
+      }
+      fresh = __shfl_sync(0xFFFFFFFFu, fresh, lane | 3);
+      uint32_t i = (uint32_t)(x - c);   // this lane's first rank in the quad
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (!((f >> e) & 1u)) continue;
+        const int nt = e >> 1;
+        const uint32_t slot = i < room ? pool_next[hr] + i : fresh + (i - room);
+        if (slot < (uint32_t)kTopkCandCap)
+          cbuf[hr][slot] = make_uint2(score_key(sc[nt][2 * hr + (e & 1)]), (uint32_t)(tbase + 8 * nt + (e & 1)));
+        ++i;
+      }
+      if (tot > room) {
+        pool_next[hr] = fresh + (tot - room);
+        pool_end[hr] = fresh + want;
+      } else {
+        pool_next[hr] += tot;
+      }
+    }
+  }
+  if (a.filter && (lane & 3) == 3) {
+    // the pools' unused slots become holes: an index no list has, which the selection skips
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr)
+      for (uint32_t slot = pool_next[hr]; slot < pool_end[hr] && slot < (uint32_t)kTopkCandCap; ++slot)
+        cbuf[hr][slot] = make_uint2(0u, kCandHole);
   }
 }
 
@@ -336,6 +416,180 @@ __global__ void __launch_bounds__(kTcThreads, kTcCtasPerSm)
   }
 }
 
+// Sequence b, visible length L and kept count k = min(k_t, L) of list th (token t = th / Hq).
+__device__ __forceinline__ void list_len_k(const TopkArgs& a, int th, int& b, int& L, int& k) {
+  const int t = th / a.qv.hq;
+  if (a.qv.q_indptr == nullptr) {
+    b = t;
+  } else {
+    int lo = 0, hi = a.kv.batch;   // largest b with q_indptr[b] <= t
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(a.qv.q_indptr + mid) <= t) lo = mid; else hi = mid;
+    }
+    b = lo;
+  }
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, false);
+  L = 0;
+  if (t >= si.t0 && t < si.t0 + si.n) L = kv_len_of(a.qv, si, t - si.t0);
+  int kreq = a.k_max;
+  if (a.k_per_token != nullptr) {
+    kreq = __ldg(a.k_per_token + t);
+    kreq = kreq < 0 ? 0 : (kreq > a.k_max ? a.k_max : kreq);
+  }
+  k = kreq < L ? kreq : L;
+}
+__device__ __forceinline__ void list_len_k(const TopkArgs& a, int th, int& L, int& k) {
+  int b;
+  list_len_k(a, th, b, L, k);
+}
+
+// ---------------------------------------------------------------------------
+// Candidate filter of the exact indexer: sample pre-pass and per-list thresholds
+// ---------------------------------------------------------------------------
+// Before the scoring kernel, topk_sample_kernel scores every 2^sample_shift-th token of every
+// list (bf16 queries), and topk_threshold_kernel turns each list's sample into a threshold key
+// lo (as the selection's sampled fast path would).  The scoring kernel then appends every score
+// at or above lo to the list's candidate buffer besides writing the full score row, and the
+// selection works on the candidates alone when they hold the top-k (see select_candidates).
+constexpr int kSmpWarps = 4;
+constexpr int kSmpRows = 16 * kSmpWarps;   // sample rows per CTA: 16 per warp (the mma M)
+
+// grid (ceil(max samples / kSmpRows), Hkv x list groups, batch).  Warp w of CTA x scores sample
+// rows j = kSmpRows x + 16 w .. + 15 (token j 2^shift) of (b, g) against the CTA's <= 16 lists:
+// D(16 rows x 8 lists) = K(16 x 128) . Q^T per group of 8 lists, 8 k-steps of mma.m16n8k16, the
+// K fragments loaded straight from the cache rows (bf16 x bf16 products are exact in fp32).
+__global__ void __launch_bounds__(32 * kSmpWarps) topk_sample_kernel(TopkArgs a) {
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, false);
+  const int G = a.qv.hq / a.kv.hkv;
+  int nlists = si.n * G - lg * a.lists_per_cta;
+  if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
+  pdl_launch_dependents();
+  if (nlists <= 0) return;
+  const int shift = a.sample_shift;
+  const int j0 = (blockIdx.x * kSmpWarps + warp) * 16;
+  if ((int64_t)j0 << shift >= si.len) return;
+  const int tr = lane >> 2, kq = 2 * (lane & 3);
+  // B operand (q, bf16): lists 8 grp + tr, dims [16 ks + kq, +1] and [+8, +9]
+  uint32_t bq[2][8][2];
+#pragma unroll
+  for (int grp = 0; grp < 2; ++grp) {
+    const int m = 8 * grp + tr;
+    const uint32_t* qrow = nullptr;
+    if (m < nlists) {
+      const int mg = lg * a.lists_per_cta + m;
+      const int jt = mg / G;
+      qrow = reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(a.qv.q) +
+                                               ((int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G)) * kHeadDim);
+    }
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      bq[grp][ks][0] = qrow != nullptr ? __ldg(qrow + 8 * ks + kq / 2) : 0u;
+      bq[grp][ks][1] = qrow != nullptr ? __ldg(qrow + 8 * ks + kq / 2 + 4) : 0u;
+    }
+  }
+  // the two sample rows of this lane (A rows tr and tr + 8)
+  uint32_t rr[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t tok = (int64_t)(j0 + tr + 8 * h) << shift;
+    rr[h] = tok < si.len ? kv_row(a.kv, b, g, (int)tok) : kInvalidRow;
+    if (tok < si.len && rr[h] == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
+  }
+  uint32_t af[8][4];
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t* kr = reinterpret_cast<const uint32_t*>(a.kv.k + (int64_t)(rr[h] != kInvalidRow ? rr[h] : 0) * kHeadDim);
+      af[ks][h] = rr[h] != kInvalidRow ? __ldg(kr + 8 * ks + kq / 2) : 0u;
+      af[ks][2 + h] = rr[h] != kInvalidRow ? __ldg(kr + 8 * ks + kq / 2 + 4) : 0u;
+    }
+  }
+#pragma unroll
+  for (int grp = 0; grp < 2; ++grp) {
+    if (8 * grp >= nlists) break;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) mma_bf16(d, af[ks], bq[grp][ks][0], bq[grp][ks][1]);
+    // D: (row tr, lists 8 grp + kq, + 1) = d0, d1; (row tr + 8, the same lists) = d2, d3
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int m = 8 * grp + kq + u;
+      if (m >= nlists) continue;
+      const int mg = lg * a.lists_per_cta + m;
+      const int jt = mg / G;
+      const int kvl = kv_len_of(a.qv, si, jt);
+      float* prow = a.samples + ((int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G)) * a.sample_stride;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = j0 + tr + 8 * h;
+        if (rr[h] != kInvalidRow && ((int64_t)j << shift) < kvl) prow[j] = d[2 * h + u];
+      }
+    }
+  }
+  (void)FULL;
+}
+
+// Threshold keys: one warp per list.  From the list's sample (ns = ceil(L / 2^shift) scores) it
+// finds, bit by bit from the top, the r-th largest sample key with its low 10 bits cleared, r
+// the expected count above the k-th score plus 4 standard deviations plus 4 -- with
+// overwhelming probability at least k of the list's scores lie at or above it.  Lists of at most
+// kTopkCandCap tokens take every score (lo = 0); a list the filter cannot serve (k = 0, k = L,
+// too many expected candidates, or more samples than the warp holds) gets lo = 0xFFFFFFFF,
+// which no score reaches, and the selection takes its other paths.
+constexpr int kThrWarps = 8;
+constexpr int kThrMaxSamples = 2048;   // 64 per lane
+
+__global__ void __launch_bounds__(32 * kThrWarps) topk_threshold_kernel(TopkArgs a, int num_lists) {
+  constexpr unsigned FULL = 0xFFFFFFFFu;
+  const int lane = threadIdx.x & 31;
+  const int th = blockIdx.x * kThrWarps + (threadIdx.x >> 5);
+  if (th >= num_lists) return;
+  int L, k;
+  list_len_k(a, th, L, k);
+  pdl_wait();   // the sample pre-pass wrote this list's samples
+  pdl_launch_dependents();
+  uint32_t lo = 0xFFFFFFFFu;
+  const int ns = (L + (1 << a.sample_shift) - 1) >> a.sample_shift;
+  if (k > 0 && k < L && a.filter == 1) {
+    if (L <= kTopkCandCap) {
+      lo = 0u;
+    } else {
+      const float mean = (float)ns * (float)k / (float)L;
+      const int r = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
+      if (ns <= kThrMaxSamples && r < ns && (int64_t)r * L <= (int64_t)kTopkCandCap * ns * 3 / 4) {
+        const float* samp = a.samples + (int64_t)th * a.sample_stride;
+        uint32_t key[kThrMaxSamples / 32];
+#pragma unroll
+        for (int i = 0; i < kThrMaxSamples / 32; ++i) {
+          const int j = 32 * i + lane;
+          key[i] = j < ns ? score_key(__ldcg(samp + j)) : 0u;
+        }
+        uint32_t prefix = 0u;
+        for (int bit = 31; bit >= 10; --bit) {
+          const uint32_t trial = prefix | (1u << bit);
+          int c = 0;
+#pragma unroll
+          for (int i = 0; i < kThrMaxSamples / 32; ++i) c += key[i] >= trial;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(FULL, c, o);
+          if (c >= r) prefix = trial;
+        }
+        lo = prefix;
+      }
+    }
+  }
+  if (lane == 0) {
+    a.lo_key[th] = lo;
+    a.meta[th] = make_int2(L, k);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Selection
 // ---------------------------------------------------------------------------
@@ -388,11 +642,6 @@ __device__ __forceinline__ void load16(const float* row, int i0, int L, float* f
     float4 v = (i < L) ? __ldcg(reinterpret_cast<const float4*>(row + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
     f[4 * j] = v.x; f[4 * j + 1] = v.y; f[4 * j + 2] = v.z; f[4 * j + 3] = v.w;
   }
-}
-
-// The score of an order-preserving key (inverse of score_key; -0 comes back as +0).
-__device__ __forceinline__ float key_score(uint32_t key) {
-  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 // Warp 0 only: in hist[0, nb) find the bin d (scanning from the top) with count(bins above d)
@@ -678,41 +927,187 @@ __device__ bool select_fast(SelectSmem& S, const float* row, const float* samp, 
   return true;
 }
 
+// Lists up to this many tokens can take the candidate path: its ordered output marks the kept
+// indices in a bitmap that reuses the 16 KB of keep masks.
+constexpr int kCandBitmapTokens = kSelWarps * kSelMaskIters * 32 * 16;
+static_assert(kCandBitmapTokens == 131072, "bitmap of the candidate path");
+static_assert(kCandBitmapTokens <= 2 * kSelBins * 32, "the tie bitmap reuses both histograms");
+static_assert(kTopkCandCap <= kFastCap, "candidate keys and indices share the fast path's buffer");
+
+// The candidate path: the scoring kernel appended, in no particular order, the (key, index) of
+// every score at or above the list's threshold into `slots` reserved slots (at most
+// kTopkCandCap), some of them holes.  With at least k of them, the candidates contain the whole
+// top-k and every score equal to the k-th; with fewer the function returns false having
+// written nothing, and the caller takes the list's score row.  Three radix rounds give
+// the k-th key T and the number need_eq of keys equal to T to keep.  Keys > T are marked in a
+// bitmap of the list's tokens and keys == T in a second one; a block scan over the tie bitmap
+// keeps the need_eq lowest-index ties, a second scan gives every thread its output offset, and
+// the kept indices are written in ascending order.
+__device__ bool select_candidates(SelectSmem& S, const uint2* cand, int slots, int L, int k, int32_t* out, int k_max) {
+  uint32_t* ckey = S.cand;
+  uint32_t* cidx = S.cand + kFastCap;
+  uint32_t* above = reinterpret_cast<uint32_t*>(&S.keep[0][0][0]);   // keys > T
+  uint32_t* tied = &S.hist[0][0];                                      // keys == T (after the rounds)
+  const int lane = threadIdx.x & 31;
+  const int words = (L + 31) >> 5;
+  for (int i = threadIdx.x; i < kSelBins; i += kSelectThreads) S.hist[0][i] = 0u;
+  for (int i = threadIdx.x; i < words; i += kSelectThreads) above[i] = 0u;
+  if (threadIdx.x == 0) S.ncand = 0;
+  __syncthreads();
+  // the reserved slots, without the holes the scoring kernel's pools left
+  for (int i0 = 0; i0 < slots; i0 += kSelectThreads) {
+    const int i = i0 + threadIdx.x;
+    const uint2 v = i < slots ? __ldcg(cand + i) : make_uint2(0u, kCandHole);
+    const bool ok = v.y < (uint32_t)L;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, ok);
+    int base = 0;
+    if (lane == 0 && m != 0u) base = atomicAdd(&S.ncand, __popc(m));
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    if (ok) {
+      const int pos = base + __popc(m & ((1u << lane) - 1u));
+      ckey[pos] = v.x;
+      cidx[pos] = v.y;
+    }
+  }
+  __syncthreads();
+  const int cnt = S.ncand;
+  if (cnt < k) {        // fewer than k scores reached the threshold: the caller takes the row
+    __syncthreads();    // every thread has read ncand before the shared memory is reused
+    return false;
+  }
+  radix_round(S, ckey, cnt, 11, 21, true, 0u, k, 0);
+  uint32_t prefix = (uint32_t)S.found_bin;
+  int need = k - S.found_above;
+  radix_round(S, ckey, cnt, 11, 10, false, prefix, need, 1);
+  prefix = (prefix << 11) | (uint32_t)S.found_bin;
+  need -= S.found_above;
+  radix_round(S, ckey, cnt, 10, 0, false, prefix, need, 0);
+  const uint32_t T = (prefix << 10) | (uint32_t)S.found_bin;
+  const int need_eq = need - S.found_above;   // 1 <= need_eq <= the number of keys equal to T
+  // every thread has read the rounds' results (radix_round ends in a barrier): reuse hist
+  for (int i = threadIdx.x; i < words; i += kSelectThreads) tied[i] = 0u;
+  __syncthreads();
+  for (int i = threadIdx.x; i < cnt; i += kSelectThreads) {
+    const uint32_t key = ckey[i], x = cidx[i];
+    if (x >= (uint32_t)L) continue;
+    if (key > T) atomicOr(&above[x >> 5], 1u << (x & 31));
+    else if (key == T) atomicOr(&tied[x >> 5], 1u << (x & 31));
+  }
+  __syncthreads();
+  // thread j owns words [8 j, 8 j + 8): the ties before it decide how many of its own it keeps
+  constexpr int kWordsPer = kCandBitmapTokens / 32 / kSelectThreads;
+  const int w0 = threadIdx.x * kWordsPer;
+  int my_ties = 0, my_above = 0;
+#pragma unroll
+  for (int w = 0; w < kWordsPer; ++w) {
+    if (w0 + w < words) {
+      my_ties += __popc(tied[w0 + w]);
+      my_above += __popc(above[w0 + w]);
+    }
+  }
+  int total;
+  const int ties_before = block_exclusive_scan<kSelectThreads>(my_ties, S.scan_tmp, &total);
+  int keep_ties = need_eq - ties_before;
+  keep_ties = keep_ties < 0 ? 0 : (keep_ties > my_ties ? my_ties : keep_ties);
+  int pos = block_exclusive_scan<kSelectThreads>(my_above + keep_ties, S.scan_tmp, &total);
+#pragma unroll
+  for (int w = 0; w < kWordsPer; ++w) {
+    if (w0 + w >= words) break;
+    uint32_t tb = tied[w0 + w];
+    uint32_t kept_tb = 0u;
+    while (tb != 0u && keep_ties > 0) {   // the lowest-index ties first
+      const uint32_t low = tb & (0u - tb);
+      kept_tb |= low;
+      tb ^= low;
+      --keep_ties;
+    }
+    uint32_t bits = above[w0 + w] | kept_tb;
+    while (bits != 0u) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1u;
+      if (pos < k) out[pos] = (w0 + w) * 32 + bit;
+      ++pos;
+    }
+  }
+  for (int i = k + threadIdx.x; i < k_max; i += kSelectThreads) out[i] = -1;
+  return true;
+}
+
+// The filtered scoring kernel writes no score rows.  A list the candidate path cannot serve (its
+// threshold kept fewer than k scores or more than kTopkCandCap) gets its row recomputed here by
+// the selection CTA -- one thread per token, an fp32 dot
+// product of the bf16 query with the token's bf16 key row -- and then takes the row paths.
+__device__ void rescore_row(const TopkArgs& a, int th, int b, int L, float* row, float* qs) {
+  const int h = th % a.qv.hq;
+  const int g = h / (a.qv.hq / a.kv.hkv);
+  const uint16_t* q = static_cast<const uint16_t*>(a.qv.q) + (int64_t)th * kHeadDim;
+  if (threadIdx.x < kHeadDim) qs[threadIdx.x] = __uint_as_float((uint32_t)__ldg(q + threadIdx.x) << 16);
+  __syncthreads();
+  for (int tok = threadIdx.x; tok < L; tok += kSelectThreads) {
+    const uint32_t r = kv_row(a.kv, b, g, tok);
+    float s = 0.f;
+    if (r != kInvalidRow) {
+      const uint4* kr = reinterpret_cast<const uint4*>(a.kv.k + (int64_t)r * kHeadDim);
+#pragma unroll 4
+      for (int c = 0; c < kHeadDim / 8; ++c) {
+        const uint4 v = __ldg(kr + c);
+        const float* qc = qs + 8 * c;
+        s = fmaf(bf16lo(v.x), qc[0], s);
+        s = fmaf(bf16hi(v.x), qc[1], s);
+        s = fmaf(bf16lo(v.y), qc[2], s);
+        s = fmaf(bf16hi(v.y), qc[3], s);
+        s = fmaf(bf16lo(v.z), qc[4], s);
+        s = fmaf(bf16hi(v.z), qc[5], s);
+        s = fmaf(bf16lo(v.w), qc[6], s);
+        s = fmaf(bf16hi(v.w), qc[7], s);
+      }
+    } else {
+      flag_status(a.status, TSD_DEV_BAD_PAGE);
+    }
+    row[tok] = s;
+  }
+  __threadfence();   // the row paths read it back through L2
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
   const int th = blockIdx.x;
-  const int t = th / a.qv.hq;
-
-  // sequence of token t
-  int b;
-  if (a.qv.q_indptr == nullptr) {
-    b = t;
+  int b = -1, L, k;
+  // launched as a dependent of the scoring kernel: its scores (or candidates) are read only once
+  // that kernel has completed.  The filtered form takes the list's (kv_len, k) from the
+  // threshold kernel, which finished before the scoring kernel did; the unfiltered form works
+  // them out from the call's inputs before the wait.
+  if (a.filter) {
+    pdl_wait();
+    const int2 m = __ldcg(a.meta + th);
+    L = m.x;
+    k = m.y;
   } else {
-    int lo = 0, hi = a.kv.batch;   // largest b with q_indptr[b] <= t
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (__ldg(a.qv.q_indptr + mid) <= t) lo = mid; else hi = mid;
-    }
-    b = lo;
+    list_len_k(a, th, b, L, k);
+    pdl_wait();
   }
-  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, false);
-  int L = 0;
-  if (t >= si.t0 && t < si.t0 + si.n) L = kv_len_of(a.qv, si, t - si.t0);
-  int kreq = a.k_max;
-  if (a.k_per_token != nullptr) {
-    kreq = __ldg(a.k_per_token + t);
-    kreq = kreq < 0 ? 0 : (kreq > a.k_max ? a.k_max : kreq);
-  }
-  const int k = kreq < L ? kreq : L;
+  pdl_launch_dependents();
   int32_t* out = a.out_idx + (int64_t)th * a.k_max;
   float* osc = a.out_scores != nullptr ? a.out_scores + (int64_t)th * a.k_max : nullptr;
   if (a.out_count != nullptr && threadIdx.x == 0) a.out_count[th] = k;
   const float* row = a.scores + (int64_t)th * a.score_stride;
-  // launched as a dependent of the scoring kernel: everything above read only the call's
-  // inputs; the scores are read only once that kernel has completed
-  pdl_wait();
-  pdl_launch_dependents();
+
+  if (a.filter) {
+    // the scoring kernel appended this list's scores at or above its threshold; take the count
+    // and leave the counter zero for the next call, whatever path runs below
+    __shared__ int s_cand;
+    if (threadIdx.x == 0) {
+      s_cand = (int)a.cand_cnt[th];
+      a.cand_cnt[th] = 0u;
+    }
+    __syncthreads();
+    const int cnt = s_cand;
+    if (k > 0 && k < L && L <= kCandBitmapTokens && cnt >= k && cnt <= kTopkCandCap && osc == nullptr &&
+        select_candidates(S, a.cand + (int64_t)th * kTopkCandCap, cnt, L, k, out, a.k_max))
+      return;
+  }
 
   if (k == L || k == 0) {   // every visible token is kept, or none
     for (int i = threadIdx.x; i < a.k_max; i += kSelectThreads) {
@@ -720,6 +1115,12 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
       if (osc != nullptr) osc[i] = i < k ? __ldcg(row + i) + 0.f : -CUDART_INF_F;
     }
     return;
+  }
+  if (a.filter) {   // the filtered scoring kernel wrote no score row: recompute this one
+    __shared__ float s_q[kHeadDim];
+    int L2, k2;
+    if (b < 0) list_len_k(a, th, b, L2, k2);   // the list's sequence
+    rescore_row(a, th, b, L, a.scores + (int64_t)th * a.score_stride, s_q);
   }
   if (L >= kFastMinL &&
       select_fast(S, row, a.samples + (int64_t)th * a.sample_stride, a.sample_shift, L, k, out, osc, a.k_max))
@@ -885,6 +1286,17 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
     configured = true;
   }
   dim3 g1(nwin, hkv * a.list_groups, batch);
+  if (a.filter) {
+    // the candidate filter: sample pre-pass, then the thresholds (a programmatic dependent)
+    const int64_t max_ns = (a.kv.max_seq_len + (1LL << a.sample_shift) - 1) >> a.sample_shift;
+    dim3 g0((unsigned)((max_ns + kSmpRows - 1) / kSmpRows), hkv * a.list_groups, batch);
+    topk_sample_kernel<<<g0, 32 * kSmpWarps, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = launch_dependent(topk_threshold_kernel, dim3((unsigned)((num_lists + kThrWarps - 1) / kThrWarps)),
+                           dim3(32 * kThrWarps), 0, stream, a, num_lists);
+    if (e != cudaSuccess) return e;
+  }
   if (score_on_tcgen05()) {
     if (a.qv.q_f32) {
       topk_score_tc_kernel<true><<<g1, kTcThreads, TcLayout<true>::bytes, stream>>>(a, maps);
@@ -893,6 +1305,10 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
     }
   } else if (a.qv.q_f32) {
     topk_score_kernel<true><<<g1, kScThreads, ScLayout<true, kScStages>::bytes, stream>>>(a, maps);
+  } else if (a.filter) {   // a programmatic dependent of the thresholds: its consumers wait for lo
+    cudaError_t e = launch_dependent(topk_score_kernel<false>, g1, dim3(kScThreads),
+                                     (size_t)ScLayout<false, kScStages>::bytes, stream, a, maps);
+    if (e != cudaSuccess) return e;
   } else {
     topk_score_kernel<false><<<g1, kScThreads, ScLayout<false, kScStages>::bytes, stream>>>(a, maps);
   }
