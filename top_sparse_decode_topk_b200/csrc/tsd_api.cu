@@ -375,6 +375,13 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   a.list_groups = p.list_groups;
   a.window = p.window;
   a.status = static_cast<uint32_t*>(ws);
+  if (a.filter) {
+    // the pre-pass: about six CTAs per SM in all, each group's 16-row sample tiles split evenly
+    const int64_t groups = sh.batch * sh.hkv * p.list_groups;
+    const int64_t tiles = (((int64_t)sh.max_seq_len + (1LL << a.sample_shift) - 1) >> a.sample_shift) / 16 + 1;
+    int64_t splits = (6LL * current_sm_count() + groups - 1) / groups;
+    a.prepass_splits = (int)(splits < 1 ? 1 : (splits > tiles ? tiles : splits));
+  }
   KvMaps maps;
   st = make_kv_maps(cache, &maps);
   if (st != TSD_OK) return st;

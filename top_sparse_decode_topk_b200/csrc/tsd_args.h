@@ -45,7 +45,8 @@ struct TopkArgs {
   uint32_t* lo_key;       // [T][Hq] candidate threshold keys (filter)
   uint2* cand;            // [T][Hq][kTopkCandCap] (key, index) candidates (filter)
   uint32_t* cand_cnt;     // [T][Hq] candidate slots reserved (zero region; the selection clears it)
-  int2* meta;             // [T][Hq] (kv_len, k) of each list (filter: threshold kernel -> selection)
+  int2* meta;             // [T][Hq] (kv_len, k) of each list (filter: pre-pass -> selection)
+  int32_t prepass_splits; // filter: CTAs sharing one (sequence, kv head, list group)'s sample tiles
   int32_t lists_per_cta;
   int32_t list_groups;
   int32_t window;

@@ -245,13 +245,19 @@ __device__ __forceinline__ void q_frag(const unsigned char* qt, int ks, int lane
 
 // S(16 queries x 16 tokens) of one warp: tokens [16 w, 16 w + 16) of the tile in stage K.
 // S[nt][0..1] = (query lane/4, tokens 8 nt + 2 (lane%4) + {0,1}); S[nt][2..3] = query lane/4 + 8.
-template <bool QF32>
+// With SPLIT the even and odd k-steps accumulate separately and are added at the end, which
+// halves the chain of dependent MMAs (the scores then round in that order).
+template <bool QF32, bool SPLIT = false>
 __device__ __forceinline__ void qk_tile(const unsigned char* qhi, const unsigned char* qlo, const unsigned char* ktile,
                                         int w, int lane, float S[2][4]) {
+  float T[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) S[nt][i] = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      S[nt][i] = 0.f;
+      T[nt][i] = 0.f;
+    }
   const int i4 = lane >> 3, rr = lane & 7;
   const int tokrow = 16 * w + ((i4 >> 1) << 3) + rr;
   const uint32_t kbase = smem_u32(ktile);
@@ -262,13 +268,20 @@ __device__ __forceinline__ void qk_tile(const unsigned char* qhi, const unsigned
     ldsm_x4(kbase + (ks >> 2) * kHalfBytes + sw128(tokrow, chunk), b00, b01, b10, b11);
     uint32_t a[4];
     q_frag(qhi, ks, lane, a);
-    mma_bf16(S[0], a, b00, b01);
-    mma_bf16(S[1], a, b10, b11);
+    float (*D)[4] = (SPLIT && (ks & 1)) ? T : S;
+    mma_bf16(D[0], a, b00, b01);
+    mma_bf16(D[1], a, b10, b11);
     if (QF32) {
       q_frag(qlo, ks, lane, a);
-      mma_bf16(S[0], a, b00, b01);
-      mma_bf16(S[1], a, b10, b11);
+      mma_bf16(D[0], a, b00, b01);
+      mma_bf16(D[1], a, b10, b11);
     }
+  }
+  if (SPLIT) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) S[nt][i] += T[nt][i];
   }
 }
 

@@ -130,9 +130,10 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
     }
   }
   const int smask = (1 << a.sample_shift) - 1;
-  // candidate filter: this lane's lists' threshold keys and candidate buffers (the test is on
-  // the order-preserving key, so that every score the full-row selection ranks above lo is kept)
-  uint32_t lo_k[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
+  // candidate filter: this lane's lists' thresholds and candidate buffers.  A score is appended
+  // unless it is below lo_f, the float whose key is lo: every score whose key reaches lo, plus
+  // NaNs whatever their key (the selection drops the keys below lo).
+  float lo_f[2] = {CUDART_INF_F, CUDART_INF_F};
   uint32_t* ccnt[2] = {nullptr, nullptr};
   uint2* cbuf[2] = {nullptr, nullptr};
   uint32_t pool_next[2] = {0u, 0u}, pool_end[2] = {0u, 0u};   // the quad's reserved, unused slots
@@ -145,7 +146,9 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
         const int mg = lg * a.lists_per_cta + m;
         const int j = mg / G;
         const int64_t list = (int64_t)(si.t0 + j) * a.qv.hq + g * G + (mg - j * G);
-        lo_k[hr] = __ldcg(a.lo_key + list);
+        const uint32_t lo = __ldcg(a.lo_key + list);
+        // keys above +inf's are positive NaNs, keys below -inf's negative ones
+        lo_f[hr] = lo >= 0xFF800000u ? CUDART_INF_F : (lo <= 0x007FFFFFu ? -CUDART_INF_F : key_score(lo));
         ccnt[hr] = a.cand_cnt + list;
         cbuf[hr] = a.cand + list * kTopkCandCap;
       }
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
   for (int tile = 0; tile < ntiles; ++tile) {
     if (!consume_wait<kScStages>(full, abort_flag, tile, lane, a.status)) break;
     float sc[2][4];
-    qk_tile<QF32>(qhi, qlo, stages + (size_t)(tile % kScStages) * kTileBytesKV, warp, lane, sc);
+    qk_tile<QF32, true>(qhi, qlo, stages + (size_t)(tile % kScStages) * kTileBytesKV, warp, lane, sc);
     // the fragments are in registers: release the stage to the producer before the stores
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[tile % kScStages]);
@@ -178,41 +181,51 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
     // candidate buffers.  The 4 lanes of a quad share a list row and take their slots, in lane
     // order, from the quad's pool; the last lane refills the pool kCandChunk slots at a time with
     // one atomic on the list's counter, so that the round trip is rare.
+    uint32_t f[2] = {0u, 0u};
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
-      uint32_t f = 0u;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int tk = tbase + 8 * nt;
-        f |= (uint32_t)(tk < kvl[hr] && score_key(sc[nt][2 * hr]) >= lo_k[hr]) << (2 * nt);
-        f |= (uint32_t)(tk + 1 < kvl[hr] && score_key(sc[nt][2 * hr + 1]) >= lo_k[hr]) << (2 * nt + 1);
+      for (int e = 0; e < 4; ++e) f[hr] |= (uint32_t)!(sc[e >> 1][2 * hr + (e & 1)] < lo_f[hr]) << e;
+      if (tbase + 9 >= kvl[hr]) {   // the tile's tail: drop the tokens at or past kv_len
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (tbase + 8 * (e >> 1) + (e & 1) >= kvl[hr]) f[hr] &= ~(1u << e);
       }
-      if (__ballot_sync(0xFFFFFFFFu, f != 0u) == 0u) continue;
-      const int c = __popc(f);
-      int x = c;   // inclusive prefix over the quad
-      int y = __shfl_up_sync(0xFFFFFFFFu, x, 1);
-      if ((lane & 3) >= 1) x += y;
-      y = __shfl_up_sync(0xFFFFFFFFu, x, 2);
-      if ((lane & 3) >= 2) x += y;
-      const uint32_t tot = (uint32_t)__shfl_sync(0xFFFFFFFFu, x, lane | 3);
+    }
+    if (__ballot_sync(0xFFFFFFFFu, (f[0] | f[1]) != 0u) == 0u) continue;
+    // both rows' counts in one word: inclusive prefix over the quad, and the quad's totals
+    const uint32_t cpk = (uint32_t)__popc(f[0]) | ((uint32_t)__popc(f[1]) << 16);
+    uint32_t x = cpk;
+    uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, 1);
+    if ((lane & 3) >= 1) x += y;
+    y = __shfl_up_sync(0xFFFFFFFFu, x, 2);
+    if ((lane & 3) >= 2) x += y;
+    const uint32_t tpk = __shfl_sync(0xFFFFFFFFu, x, lane | 3);
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const uint32_t tot = (tpk >> (16 * hr)) & 0xFFFFu;
       const uint32_t room = pool_end[hr] - pool_next[hr];
+      const bool grow = tot > room;   // the same in the quad's 4 lanes
       uint32_t fresh = 0u, want = 0u;
-      if (tot > room) {
-        want = (tot - room + kCandChunk - 1) / kCandChunk * kCandChunk;
-        if ((lane & 3) == 3) fresh = atomicAdd(ccnt[hr], want);
+      if (__any_sync(0xFFFFFFFFu, grow)) {
+        if (grow) {
+          want = (tot - room + kCandChunk - 1) / kCandChunk * kCandChunk;
+          if ((lane & 3) == 3) fresh = atomicAdd(ccnt[hr], want);
+        }
+        fresh = __shfl_sync(0xFFFFFFFFu, fresh, lane | 3);
       }
-      fresh = __shfl_sync(0xFFFFFFFFu, fresh, lane | 3);
-      uint32_t i = (uint32_t)(x - c);   // this lane's first rank in the quad
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (!((f >> e) & 1u)) continue;
-        const int nt = e >> 1;
+      uint32_t i = ((x >> (16 * hr)) & 0xFFFFu) - ((cpk >> (16 * hr)) & 0xFFFFu);   // first rank in the quad
+      uint32_t bits = f[hr];
+      while (bits != 0u) {
+        const int e = __ffs(bits) - 1;
+        bits &= bits - 1u;
         const uint32_t slot = i < room ? pool_next[hr] + i : fresh + (i - room);
+        const float v = e == 0 ? sc[0][2 * hr] : (e == 1 ? sc[0][2 * hr + 1] : (e == 2 ? sc[1][2 * hr] : sc[1][2 * hr + 1]));
         if (slot < (uint32_t)kTopkCandCap)
-          cbuf[hr][slot] = make_uint2(score_key(sc[nt][2 * hr + (e & 1)]), (uint32_t)(tbase + 8 * nt + (e & 1)));
+          cbuf[hr][slot] = make_uint2(score_key(v), (uint32_t)(tbase + 8 * (e >> 1) + (e & 1)));
         ++i;
       }
-      if (tot > room) {
+      if (grow) {
         pool_next[hr] = fresh + (tot - room);
         pool_end[hr] = fresh + want;
       } else {
@@ -445,34 +458,85 @@ __device__ __forceinline__ void list_len_k(const TopkArgs& a, int th, int& L, in
 }
 
 // ---------------------------------------------------------------------------
-// Candidate filter of the exact indexer: sample pre-pass and per-list thresholds
+// Candidate filter of the exact indexer: the pre-pass
 // ---------------------------------------------------------------------------
-// Before the scoring kernel, topk_sample_kernel scores every 2^sample_shift-th token of every
-// list (bf16 queries), and topk_threshold_kernel turns each list's sample into a threshold key
-// lo (as the selection's sampled fast path would).  The scoring kernel then appends every score
-// at or above lo to the list's candidate buffer besides writing the full score row, and the
-// selection works on the candidates alone when they hold the top-k (see select_candidates).
-constexpr int kSmpWarps = 4;
-constexpr int kSmpRows = 16 * kSmpWarps;   // sample rows per CTA: 16 per warp (the mma M)
+// Before the scoring kernel, topk_prepass_kernel scores every 2^sample_shift-th token of every
+// list (bf16 queries) and turns each list's sample into a threshold key lo, as the selection's
+// sampled fast path would.  The scoring kernel then appends every score whose key reaches lo to
+// the list's candidate buffer instead of writing the score row, and the selection works on the
+// candidates alone (see select_candidates).
+//
+// Grid (splits, Hkv x list groups, batch), kPpWarps warps per CTA.  The splits of a (sequence,
+// kv head, list group) share its sample tiles; each writes its samples, and the last to arrive
+// on the group's counter -- the candidate counter of the group's first list, which the scoring
+// kernel needs zero only after this kernel has completed -- computes the group's thresholds
+// and leaves the counter zero.
+constexpr int kPpWarps = 8;
+constexpr int kThrMaxSamples = 2048;   // 64 per lane
 
-// grid (ceil(max samples / kSmpRows), Hkv x list groups, batch).  Warp w of CTA x scores sample
-// rows j = kSmpRows x + 16 w .. + 15 (token j 2^shift) of (b, g) against the CTA's <= 16 lists:
-// D(16 rows x 8 lists) = K(16 x 128) . Q^T per group of 8 lists, 8 k-steps of mma.m16n8k16, the
-// K fragments loaded straight from the cache rows (bf16 x bf16 products are exact in fp32).
-__global__ void __launch_bounds__(32 * kSmpWarps) topk_sample_kernel(TopkArgs a) {
+// Threshold key of one list from its ns sample scores (one warp): bit by bit from the top, the
+// r-th largest sample key with its low 16 bits cleared, r the expected count above the k-th
+// score plus 4 standard deviations plus 4 -- with overwhelming probability at least k of the
+// list's scores reach it.  Lists of at most kTopkCandCap tokens take every score (lo = 0); a
+// list the filter cannot serve (k = 0, k = L, too many expected candidates, or more samples than
+// the warp holds) gets lo = 0xFFFFFFFF, which only the largest NaN key reaches, and the
+// selection takes its other paths.
+__device__ uint32_t list_threshold(const float* samp, int L, int k, int shift, bool enabled, int lane) {
   constexpr unsigned FULL = 0xFFFFFFFFu;
+  if (!(k > 0 && k < L && enabled)) return 0xFFFFFFFFu;
+  if (L <= kTopkCandCap) return 0u;
+  const int ns = (L + (1 << shift) - 1) >> shift;
+  const float mean = (float)ns * (float)k / (float)L;
+  const int r = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
+  if (!(ns <= kThrMaxSamples && r < ns && (int64_t)r * L <= (int64_t)kTopkCandCap * ns * 3 / 4)) return 0xFFFFFFFFu;
+  uint32_t key[kThrMaxSamples / 32];
+#pragma unroll
+  for (int i = 0; i < kThrMaxSamples / 32; ++i) {
+    const int j = 32 * i + lane;
+    key[i] = j < ns ? score_key(__ldcg(samp + j)) : 0u;
+  }
+  // 16 bits (sign, exponent, 7 mantissa bits): the threshold then sits at most 2^-7 of its
+  // value below the sample's r-th largest, which adds few candidates; eight partial counts keep
+  // the chains of dependent adds short
+  uint32_t prefix = 0u;
+  for (int bit = 31; bit >= 16; --bit) {
+    const uint32_t trial = prefix | (1u << bit);
+    int c8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < kThrMaxSamples / 32; ++i) c8[i & 7] += key[i] >= trial;
+    int c = ((c8[0] + c8[1]) + (c8[2] + c8[3])) + ((c8[4] + c8[5]) + (c8[6] + c8[7]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(FULL, c, o);
+    if (c >= r) prefix = trial;
+  }
+  return prefix;
+}
+
+// kept count k = min(k_t, L) of query token t with visible length L
+__device__ __forceinline__ int list_k(const TopkArgs& a, int t, int L) {
+  int kreq = a.k_max;
+  if (a.k_per_token != nullptr) {
+    kreq = __ldg(a.k_per_token + t);
+    kreq = kreq < 0 ? 0 : (kreq > a.k_max ? a.k_max : kreq);
+  }
+  return kreq < L ? kreq : L;
+}
+
+__global__ void __launch_bounds__(32 * kPpWarps, 2) topk_prepass_kernel(TopkArgs a) {
   const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
   const int b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();   // the scoring kernel may launch; its consumers wait for this grid
   const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, false);
   const int G = a.qv.hq / a.kv.hkv;
   int nlists = si.n * G - lg * a.lists_per_cta;
   if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
-  pdl_launch_dependents();
-  if (nlists <= 0) return;
+  if (nlists <= 0) return;   // the same in every split of the group: no thresholds to make
   const int shift = a.sample_shift;
-  const int j0 = (blockIdx.x * kSmpWarps + warp) * 16;
-  if ((int64_t)j0 << shift >= si.len) return;
+  const int64_t max_ns = ((int64_t)a.kv.max_seq_len + (1 << shift) - 1) >> shift;
+  const int per_split = (int)(((max_ns + 15) / 16 + gridDim.x - 1) / gridDim.x);   // 16-row tiles
+  const int ns_seq = (int)(((int64_t)si.len + (1 << shift) - 1) >> shift);
+  const int tile_end = min((int)blockIdx.x * per_split + per_split, (ns_seq + 15) / 16);
   const int tr = lane >> 2, kq = 2 * (lane & 3);
   // B operand (q, bf16): lists 8 grp + tr, dims [16 ks + kq, +1] and [+8, +9]
   uint32_t bq[2][8][2];
@@ -492,104 +556,78 @@ __global__ void __launch_bounds__(32 * kSmpWarps) topk_sample_kernel(TopkArgs a)
       bq[grp][ks][1] = qrow != nullptr ? __ldg(qrow + 8 * ks + kq / 2 + 4) : 0u;
     }
   }
-  // the two sample rows of this lane (A rows tr and tr + 8)
-  uint32_t rr[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int64_t tok = (int64_t)(j0 + tr + 8 * h) << shift;
-    rr[h] = tok < si.len ? kv_row(a.kv, b, g, (int)tok) : kInvalidRow;
-    if (tok < si.len && rr[h] == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
-  }
-  uint32_t af[8][4];
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
+  // the two sample rows of this lane in tile t (A rows tr and tr + 8); a bad page is flagged
+  auto rows_of = [&](int t, uint32_t* rr) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint32_t* kr = reinterpret_cast<const uint32_t*>(a.kv.k + (int64_t)(rr[h] != kInvalidRow ? rr[h] : 0) * kHeadDim);
-      af[ks][h] = rr[h] != kInvalidRow ? __ldg(kr + 8 * ks + kq / 2) : 0u;
-      af[ks][2 + h] = rr[h] != kInvalidRow ? __ldg(kr + 8 * ks + kq / 2 + 4) : 0u;
+      const int64_t tok = (int64_t)(t * 16 + tr + 8 * h) << shift;
+      rr[h] = t < tile_end && tok < si.len ? kv_row(a.kv, b, g, (int)tok) : kInvalidRow;
+      if (t < tile_end && tok < si.len && rr[h] == kInvalidRow) flag_status(a.status, TSD_DEV_BAD_PAGE);
     }
-  }
+  };
+  uint32_t rnext[2];
+  rows_of((int)blockIdx.x * per_split + warp, rnext);
+  for (int tile = (int)blockIdx.x * per_split + warp; tile < tile_end; tile += kPpWarps) {
+    const int j0 = tile * 16;
+    const uint32_t rr[2] = {rnext[0], rnext[1]};
+    rows_of(tile + kPpWarps, rnext);   // the next tile's page lookups overlap this tile's loads
+    uint32_t af[8][4];
 #pragma unroll
-  for (int grp = 0; grp < 2; ++grp) {
-    if (8 * grp >= nlists) break;
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) mma_bf16(d, af[ks], bq[grp][ks][0], bq[grp][ks][1]);
-    // D: (row tr, lists 8 grp + kq, + 1) = d0, d1; (row tr + 8, the same lists) = d2, d3
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int m = 8 * grp + kq + u;
-      if (m >= nlists) continue;
-      const int mg = lg * a.lists_per_cta + m;
-      const int jt = mg / G;
-      const int kvl = kv_len_of(a.qv, si, jt);
-      float* prow = a.samples + ((int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G)) * a.sample_stride;
+    for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int j = j0 + tr + 8 * h;
-        if (rr[h] != kInvalidRow && ((int64_t)j << shift) < kvl) prow[j] = d[2 * h + u];
+        const uint32_t* kr = reinterpret_cast<const uint32_t*>(a.kv.k + (int64_t)(rr[h] != kInvalidRow ? rr[h] : 0) * kHeadDim);
+        af[ks][h] = rr[h] != kInvalidRow ? __ldg(kr + 8 * ks + kq / 2) : 0u;
+        af[ks][2 + h] = rr[h] != kInvalidRow ? __ldg(kr + 8 * ks + kq / 2 + 4) : 0u;
+      }
+    }
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+      if (8 * grp >= nlists) break;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) mma_bf16(d, af[ks], bq[grp][ks][0], bq[grp][ks][1]);
+      // D: (row tr, lists 8 grp + kq, + 1) = d0, d1; (row tr + 8, the same lists) = d2, d3
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int m = 8 * grp + kq + u;
+        if (m >= nlists) continue;
+        const int mg = lg * a.lists_per_cta + m;
+        const int jt = mg / G;
+        const int kvl = kv_len_of(a.qv, si, jt);
+        float* prow = a.samples + ((int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G)) * a.sample_stride;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int j = j0 + tr + 8 * h;
+          if (rr[h] != kInvalidRow && ((int64_t)j << shift) < kvl) prow[j] = d[2 * h + u];
+        }
       }
     }
   }
-  (void)FULL;
-}
-
-// Threshold keys: one warp per list.  From the list's sample (ns = ceil(L / 2^shift) scores) it
-// finds, bit by bit from the top, the r-th largest sample key with its low 10 bits cleared, r
-// the expected count above the k-th score plus 4 standard deviations plus 4 -- with
-// overwhelming probability at least k of the list's scores lie at or above it.  Lists of at most
-// kTopkCandCap tokens take every score (lo = 0); a list the filter cannot serve (k = 0, k = L,
-// too many expected candidates, or more samples than the warp holds) gets lo = 0xFFFFFFFF,
-// which no score reaches, and the selection takes its other paths.
-constexpr int kThrWarps = 8;
-constexpr int kThrMaxSamples = 2048;   // 64 per lane
-
-__global__ void __launch_bounds__(32 * kThrWarps) topk_threshold_kernel(TopkArgs a, int num_lists) {
-  constexpr unsigned FULL = 0xFFFFFFFFu;
-  const int lane = threadIdx.x & 31;
-  const int th = blockIdx.x * kThrWarps + (threadIdx.x >> 5);
-  if (th >= num_lists) return;
-  int L, k;
-  list_len_k(a, th, L, k);
-  pdl_wait();   // the sample pre-pass wrote this list's samples
-  pdl_launch_dependents();
-  uint32_t lo = 0xFFFFFFFFu;
-  const int ns = (L + (1 << a.sample_shift) - 1) >> a.sample_shift;
-  if (k > 0 && k < L && a.filter == 1) {
-    if (L <= kTopkCandCap) {
-      lo = 0u;
-    } else {
-      const float mean = (float)ns * (float)k / (float)L;
-      const int r = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
-      if (ns <= kThrMaxSamples && r < ns && (int64_t)r * L <= (int64_t)kTopkCandCap * ns * 3 / 4) {
-        const float* samp = a.samples + (int64_t)th * a.sample_stride;
-        uint32_t key[kThrMaxSamples / 32];
-#pragma unroll
-        for (int i = 0; i < kThrMaxSamples / 32; ++i) {
-          const int j = 32 * i + lane;
-          key[i] = j < ns ? score_key(__ldcg(samp + j)) : 0u;
-        }
-        uint32_t prefix = 0u;
-        for (int bit = 31; bit >= 10; --bit) {
-          const uint32_t trial = prefix | (1u << bit);
-          int c = 0;
-#pragma unroll
-          for (int i = 0; i < kThrMaxSamples / 32; ++i) c += key[i] >= trial;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(FULL, c, o);
-          if (c >= r) prefix = trial;
-        }
-        lo = prefix;
-      }
+  // arrive; the last split of the group makes its thresholds
+  const int j_first = (lg * a.lists_per_cta) / G;
+  const int64_t first_list = (int64_t)(si.t0 + j_first) * a.qv.hq + g * G + (lg * a.lists_per_cta - j_first * G);
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(a.cand_cnt + first_list, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) a.cand_cnt[first_list] = 0u;
+  for (int m = warp; m < nlists; m += kPpWarps) {
+    const int mg = lg * a.lists_per_cta + m;
+    const int jt = mg / G;
+    const int64_t list = (int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G);
+    const int L = kv_len_of(a.qv, si, jt);
+    const int k = list_k(a, si.t0 + jt, L);
+    const uint32_t lo = list_threshold(a.samples + list * a.sample_stride, L, k, shift, a.filter == 1, lane);
+    if (lane == 0) {
+      a.lo_key[list] = lo;
+      a.meta[list] = make_int2(L, k);
     }
   }
-  if (lane == 0) {
-    a.lo_key[th] = lo;
-    a.meta[th] = make_int2(L, k);
-  }
 }
-
 // ---------------------------------------------------------------------------
 // Selection
 // ---------------------------------------------------------------------------
@@ -935,15 +973,16 @@ static_assert(kCandBitmapTokens <= 2 * kSelBins * 32, "the tie bitmap reuses bot
 static_assert(kTopkCandCap <= kFastCap, "candidate keys and indices share the fast path's buffer");
 
 // The candidate path: the scoring kernel appended, in no particular order, the (key, index) of
-// every score at or above the list's threshold into `slots` reserved slots (at most
-// kTopkCandCap), some of them holes.  With at least k of them, the candidates contain the whole
+// every score whose key reaches the list's threshold lo (and of NaN scores, whose keys below lo
+// are dropped here) into `slots` reserved slots (at most kTopkCandCap), some of them holes.  With at least k of them, the candidates contain the whole
 // top-k and every score equal to the k-th; with fewer the function returns false having
 // written nothing, and the caller takes the list's score row.  Three radix rounds give
 // the k-th key T and the number need_eq of keys equal to T to keep.  Keys > T are marked in a
 // bitmap of the list's tokens and keys == T in a second one; a block scan over the tie bitmap
 // keeps the need_eq lowest-index ties, a second scan gives every thread its output offset, and
 // the kept indices are written in ascending order.
-__device__ bool select_candidates(SelectSmem& S, const uint2* cand, int slots, int L, int k, int32_t* out, int k_max) {
+__device__ bool select_candidates(SelectSmem& S, const uint2* cand, int slots, uint32_t lo, int L, int k, int32_t* out,
+                                  int k_max) {
   uint32_t* ckey = S.cand;
   uint32_t* cidx = S.cand + kFastCap;
   uint32_t* above = reinterpret_cast<uint32_t*>(&S.keep[0][0][0]);   // keys > T
@@ -954,11 +993,11 @@ __device__ bool select_candidates(SelectSmem& S, const uint2* cand, int slots, i
   for (int i = threadIdx.x; i < words; i += kSelectThreads) above[i] = 0u;
   if (threadIdx.x == 0) S.ncand = 0;
   __syncthreads();
-  // the reserved slots, without the holes the scoring kernel's pools left
+  // the reserved slots' keys >= lo, without the holes the scoring kernel's pools left
   for (int i0 = 0; i0 < slots; i0 += kSelectThreads) {
     const int i = i0 + threadIdx.x;
     const uint2 v = i < slots ? __ldcg(cand + i) : make_uint2(0u, kCandHole);
-    const bool ok = v.y < (uint32_t)L;
+    const bool ok = v.y < (uint32_t)L && v.x >= lo;
     const uint32_t m = __ballot_sync(0xFFFFFFFFu, ok);
     int base = 0;
     if (lane == 0 && m != 0u) base = atomicAdd(&S.ncand, __popc(m));
@@ -1105,7 +1144,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
     __syncthreads();
     const int cnt = s_cand;
     if (k > 0 && k < L && L <= kCandBitmapTokens && cnt >= k && cnt <= kTopkCandCap && osc == nullptr &&
-        select_candidates(S, a.cand + (int64_t)th * kTopkCandCap, cnt, L, k, out, a.k_max))
+        select_candidates(S, a.cand + (int64_t)th * kTopkCandCap, cnt, __ldcg(a.lo_key + th), L, k, out, a.k_max))
       return;
   }
 
@@ -1286,15 +1325,10 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
     configured = true;
   }
   dim3 g1(nwin, hkv * a.list_groups, batch);
-  if (a.filter) {
-    // the candidate filter: sample pre-pass, then the thresholds (a programmatic dependent)
-    const int64_t max_ns = (a.kv.max_seq_len + (1LL << a.sample_shift) - 1) >> a.sample_shift;
-    dim3 g0((unsigned)((max_ns + kSmpRows - 1) / kSmpRows), hkv * a.list_groups, batch);
-    topk_sample_kernel<<<g0, 32 * kSmpWarps, 0, stream>>>(a);
+  if (a.filter) {   // the candidate filter's pre-pass: samples and thresholds
+    const dim3 g0((unsigned)a.prepass_splits, hkv * a.list_groups, batch);
+    topk_prepass_kernel<<<g0, 32 * kPpWarps, 0, stream>>>(a);
     cudaError_t e = cudaGetLastError();
-    if (e == cudaSuccess)
-      e = launch_dependent(topk_threshold_kernel, dim3((unsigned)((num_lists + kThrWarps - 1) / kThrWarps)),
-                           dim3(32 * kThrWarps), 0, stream, a, num_lists);
     if (e != cudaSuccess) return e;
   }
   if (score_on_tcgen05()) {
@@ -1305,7 +1339,7 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
     }
   } else if (a.qv.q_f32) {
     topk_score_kernel<true><<<g1, kScThreads, ScLayout<true, kScStages>::bytes, stream>>>(a, maps);
-  } else if (a.filter) {   // a programmatic dependent of the thresholds: its consumers wait for lo
+  } else if (a.filter) {   // a programmatic dependent of the pre-pass: its consumers wait for lo
     cudaError_t e = launch_dependent(topk_score_kernel<false>, g1, dim3(kScThreads),
                                      (size_t)ScLayout<false, kScStages>::bytes, stream, a, maps);
     if (e != cudaSuccess) return e;
