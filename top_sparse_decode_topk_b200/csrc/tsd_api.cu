@@ -368,6 +368,9 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   a.lo_key = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_lo);
   a.cand = reinterpret_cast<uint2*>(static_cast<char*>(ws) + lay.off_cand);
   a.meta = reinterpret_cast<int2*>(static_cast<char*>(ws) + lay.off_meta);
+  a.queue = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + lay.off_queue);
+  a.queue_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16);
+  a.queue_done = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 20);
   a.cand_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 256);
   // scoring streams K in the dense path's tiles, with its own occupancy
   const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kScoreCtasPerSm, kMaxWindowScore);
@@ -381,6 +384,8 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
     const int64_t tiles = (((int64_t)sh.max_seq_len + (1LL << a.sample_shift) - 1) >> a.sample_shift) / 16 + 1;
     int64_t splits = (6LL * current_sm_count() + groups - 1) / groups;
     a.prepass_splits = (int)(splits < 1 ? 1 : (splits > tiles ? tiles : splits));
+    const int64_t qc = 2LL * current_sm_count();   // the selection's CTAs per SM
+    a.queue_ctas = (int)(qc < sh.tokens * sh.hq ? qc : sh.tokens * sh.hq);
   }
   KvMaps maps;
   st = make_kv_maps(cache, &maps);

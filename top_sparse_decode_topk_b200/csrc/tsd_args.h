@@ -47,6 +47,10 @@ struct TopkArgs {
   uint32_t* cand_cnt;     // [T][Hq] candidate slots reserved (zero region; the selection clears it)
   int2* meta;             // [T][Hq] (kv_len, k) of each list (filter: pre-pass -> selection)
   int32_t prepass_splits; // filter: CTAs sharing one (sequence, kv head, list group)'s sample tiles
+  int32_t* queue;         // filter: [T][Hq] lists the candidate kernel left to the row paths
+  uint32_t* queue_cnt;    // filter: their number (zero region; the last queue CTA clears it)
+  uint32_t* queue_done;   // filter: queue CTAs finished (zero region; cleared with queue_cnt)
+  int32_t queue_ctas;     // filter: CTAs of the queue pass
   int32_t lists_per_cta;
   int32_t list_groups;
   int32_t window;

@@ -3,9 +3,11 @@
 // Workspace layout (bytes from the start; every region 256-byte aligned):
 //   [0, 256)              header: device status word (uint32) at offset 0; the persistent
 //                         sparse kernel's task and done counters (uint32) at offsets 4 and 8;
-//                         the rest reserved
+//                         the filtered indexer's queue count and queue-CTA counter (uint32) at
+//                         offsets 16 and 20; the rest reserved
 //   counters              uint32, one per list (token x q head): arrival counters of the
-//                         split-K merge (zero between calls)
+//                         split-K merge, or the filtered indexer's candidate counters (and the
+//                         pre-pass's arrival counters); zero between calls
 //   -- everything above is the "zero region": it must be zero when a call starts and every
 //      call leaves it zero --
 //   decode partials       float2 [T][Hq][nsplit] (running max, running sum; base-2 units)
@@ -13,6 +15,7 @@
 //   top-k scores          float  [T][Hq][score_stride] (fp32 q.K of every visible token)
 //   top-k score samples   float  [T][Hq][sample_stride]: every 2^sample_shift-th token's score
 //                         (its strided sample for the selection's threshold)
+//   filtered indexer      thresholds, candidates, (kv_len, k) and the queue (TopkLayout)
 #pragma once
 
 #include <stddef.h>
@@ -225,7 +228,8 @@ struct TopkLayout {
   int64_t sample_stride;
   size_t off_lo;      // uint32 [T][Hq]: each list's candidate threshold key
   size_t off_cand;    // uint2 [T][Hq][kTopkCandCap]: (key, index) candidates
-  size_t off_meta;    // int2 [T][Hq]: each list's (kv_len, k), written by the threshold kernel
+  size_t off_meta;    // int2 [T][Hq]: each list's (kv_len, k), written by the pre-pass
+  size_t off_queue;   // int32 [T][Hq]: lists the candidate kernel leaves to the row paths
   size_t total;
 };
 
@@ -240,7 +244,8 @@ inline TopkLayout topk_layout(const Shapes& s) {
   l.off_lo = l.off_samples + align256((size_t)s.tokens * s.hq * l.sample_stride * sizeof(float));
   l.off_cand = l.off_lo + align256((size_t)s.tokens * s.hq * sizeof(uint32_t));
   l.off_meta = l.off_cand + align256((size_t)s.tokens * s.hq * kTopkCandCap * 2 * sizeof(uint32_t));
-  l.total = l.off_meta + align256((size_t)s.tokens * s.hq * 2 * sizeof(int32_t));
+  l.off_queue = l.off_meta + align256((size_t)s.tokens * s.hq * 2 * sizeof(int32_t));
+  l.total = l.off_queue + align256((size_t)s.tokens * s.hq * sizeof(int32_t));
   return l;
 }
 

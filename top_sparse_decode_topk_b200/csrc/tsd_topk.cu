@@ -83,14 +83,20 @@ __global__ void __launch_bounds__(kScThreads, kScCtasPerSm) topk_score_kernel(To
   const int G = a.qv.hq / a.kv.hkv;
   int nlists = si.n * G - lg * a.lists_per_cta;
   if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
-  if (nlists <= 0) return;
   const int tok0 = win * a.window;
   const int tok_end = min(tok0 + a.window, si.len);
-  if (tok_end <= tok0) return;
+  const bool idle = nlists <= 0 || tok_end <= tok0;
+  // Under the filter the kernels after this one read what the pre-pass wrote once this grid has
+  // completed, so every CTA waits for the pre-pass before it exits (the consumers below do).
+  if (idle) {
+    if (a.filter) pdl_wait();
+    return;
+  }
   const int ntiles = (tok_end - tok0 + kTileTok - 1) / kTileTok;
   const bool use_tma = a.kv.page_table == nullptr || a.kv.page_shift >= 3;
   if (smem_u32(stages) & 1023u) {
     if (threadIdx.x == 0) flag_status(a.status, TSD_DEV_TIMEOUT);
+    if (a.filter) pdl_wait();
     return;
   }
   if (threadIdx.x == 0) {
@@ -484,7 +490,7 @@ constexpr int kThrMaxSamples = 2048;   // 64 per lane
 __device__ uint32_t list_threshold(const float* samp, int L, int k, int shift, bool enabled, int lane) {
   constexpr unsigned FULL = 0xFFFFFFFFu;
   if (!(k > 0 && k < L && enabled)) return 0xFFFFFFFFu;
-  if (L <= kTopkCandCap) return 0u;
+  if (L <= kTopkCandCap / 2) return 0u;   // leaves room for the pools' holes
   const int ns = (L + (1 << shift) - 1) >> shift;
   const float mean = (float)ns * (float)k / (float)L;
   const int r = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
@@ -687,7 +693,8 @@ __device__ __forceinline__ void load16(const float* row, int i0, int L, float* f
 // the contiguous bins [nb - (l + 1) per, nb - l per), read in a rotated order so that the 32
 // lanes hit 32 different banks; a lane scan finds the lane whose range crosses `need`, and
 // the 32 lanes then split that range (per / 32 bins each) for a second scan.
-__device__ __forceinline__ void warp_find_bin(SelectSmem& S, const uint32_t* hist, int nb, int need) {
+template <class SM>
+__device__ __forceinline__ void warp_find_bin(SM& S, const uint32_t* hist, int nb, int need) {
   constexpr unsigned FULL = 0xFFFFFFFFu;
   const int lane = threadIdx.x & 31;
   const int per = nb >> 5;
@@ -965,91 +972,150 @@ __device__ bool select_fast(SelectSmem& S, const float* row, const float* samp, 
   return true;
 }
 
-// Lists up to this many tokens can take the candidate path: its ordered output marks the kept
-// indices in a bitmap that reuses the 16 KB of keep masks.
-constexpr int kCandBitmapTokens = kSelWarps * kSelMaskIters * 32 * 16;
-static_assert(kCandBitmapTokens == 131072, "bitmap of the candidate path");
+// ---------------------------------------------------------------------------
+// The candidate path of the filtered indexer (topk_cand_kernel)
+// ---------------------------------------------------------------------------
+// One CTA per list.  The scoring kernel appended, in no particular order, the
+// (key, index) of every score not below the list's threshold into `slots` reserved slots (at
+// most kTopkCandCap), some of them holes; the keys below lo (NaN scores) and the holes are
+// skipped here.  With at least k valid candidates they hold the whole top-k and every score
+// equal to the k-th.  Three radix rounds over the candidates, read from L2 each time, give the
+// k-th key T and the number need_eq of keys equal to T to keep.  Keys > T are marked in a bitmap
+// of the list's tokens and keys == T in a second one; a block scan over the tie bitmap keeps
+// the need_eq lowest-index ties, a second scan gives every thread its output offset, and the
+// kept indices are written in ascending order.  A list with fewer than k valid candidates, or
+// more than fit, goes into the queue that topk_select_kernel works off over recomputed rows.
+constexpr int kCandBitmapTokens = 131072;   // longest list the bitmaps cover
+constexpr int kCsUnroll = 8;                  // candidate loads in flight per thread
+template <int NT>
+struct CandSmem {
+  uint32_t hist[2][kSelBins];               // radix histograms; after the rounds, the tie bitmap
+  uint32_t above[kCandBitmapTokens / 32];   // keys > T
+  int scan_tmp[NT / 32 + 1];
+  int found_bin, found_above, nvalid, slots;
+};
 static_assert(kCandBitmapTokens <= 2 * kSelBins * 32, "the tie bitmap reuses both histograms");
-static_assert(kTopkCandCap <= kFastCap, "candidate keys and indices share the fast path's buffer");
+static_assert(sizeof(CandSmem<1024>) <= 48 * 1024, "static shared memory of the candidate kernel");
 
-// The candidate path: the scoring kernel appended, in no particular order, the (key, index) of
-// every score whose key reaches the list's threshold lo (and of NaN scores, whose keys below lo
-// are dropped here) into `slots` reserved slots (at most kTopkCandCap), some of them holes.  With at least k of them, the candidates contain the whole
-// top-k and every score equal to the k-th; with fewer the function returns false having
-// written nothing, and the caller takes the list's score row.  Three radix rounds give
-// the k-th key T and the number need_eq of keys equal to T to keep.  Keys > T are marked in a
-// bitmap of the list's tokens and keys == T in a second one; a block scan over the tie bitmap
-// keeps the need_eq lowest-index ties, a second scan gives every thread its output offset, and
-// the kept indices are written in ascending order.
-__device__ bool select_candidates(SelectSmem& S, const uint2* cand, int slots, uint32_t lo, int L, int k, int32_t* out,
-                                  int k_max) {
-  uint32_t* ckey = S.cand;
-  uint32_t* cidx = S.cand + kFastCap;
-  uint32_t* above = reinterpret_cast<uint32_t*>(&S.keep[0][0][0]);   // keys > T
-  uint32_t* tied = &S.hist[0][0];                                      // keys == T (after the rounds)
-  const int lane = threadIdx.x & 31;
-  const int words = (L + 31) >> 5;
-  for (int i = threadIdx.x; i < kSelBins; i += kSelectThreads) S.hist[0][i] = 0u;
-  for (int i = threadIdx.x; i < words; i += kSelectThreads) above[i] = 0u;
-  if (threadIdx.x == 0) S.ncand = 0;
-  __syncthreads();
-  // the reserved slots' keys >= lo, without the holes the scoring kernel's pools left
-  for (int i0 = 0; i0 < slots; i0 += kSelectThreads) {
-    const int i = i0 + threadIdx.x;
-    const uint2 v = i < slots ? __ldcg(cand + i) : make_uint2(0u, kCandHole);
-    const bool ok = v.y < (uint32_t)L && v.x >= lo;
-    const uint32_t m = __ballot_sync(0xFFFFFFFFu, ok);
-    int base = 0;
-    if (lane == 0 && m != 0u) base = atomicAdd(&S.ncand, __popc(m));
-    base = __shfl_sync(0xFFFFFFFFu, base, 0);
-    if (ok) {
-      const int pos = base + __popc(m & ((1u << lane) - 1u));
-      ckey[pos] = v.x;
-      cidx[pos] = v.y;
+// Every valid candidate of the list (index < L, key >= lo) through f(key, index), kCsUnroll
+// loads in flight per thread.
+template <int NT, class F>
+__device__ __forceinline__ void for_candidates(const uint2* cand, int slots, uint32_t L, uint32_t lo, F f) {
+  for (int i0 = threadIdx.x; i0 < slots; i0 += NT * kCsUnroll) {
+    uint2 v[kCsUnroll];
+#pragma unroll
+    for (int u = 0; u < kCsUnroll; ++u) {
+      const int i = i0 + u * NT;
+      v[u] = i < slots ? __ldcg(cand + i) : make_uint2(0u, kCandHole);
     }
+#pragma unroll
+    for (int u = 0; u < kCsUnroll; ++u)
+      if (v[u].y < L && v[u].x >= lo) f(v[u].x, v[u].y);
   }
+}
+
+// One radix round over the valid candidates: histogram of digit (key >> shift) & (2^nb - 1)
+// among the keys whose bits above shift + nb equal prefix, then the digit of the need-th
+// largest.  Histograms alternate between S.hist[cur] and S.hist[cur ^ 1].
+template <int NT>
+__device__ void cand_round(CandSmem<NT>& S, const uint2* cand, int slots, uint32_t L, uint32_t lo, int nb, int shift,
+                           uint32_t prefix, int need, int cur) {
+  uint32_t* h = S.hist[cur];
+  uint32_t* z = S.hist[cur ^ 1];
+  for (int i = threadIdx.x; i < kSelBins; i += NT) z[i] = 0u;
+  const uint32_t mask = (1u << nb) - 1u;
+  for_candidates<NT>(cand, slots, L, lo, [&](uint32_t key, uint32_t) {
+    if ((key >> (shift + nb)) == prefix) atomicAdd(&h[(key >> shift) & mask], 1u);
+  });
   __syncthreads();
-  const int cnt = S.ncand;
-  if (cnt < k) {        // fewer than k scores reached the threshold: the caller takes the row
-    __syncthreads();    // every thread has read ncand before the shared memory is reused
-    return false;
+  if (threadIdx.x < 32) warp_find_bin(S, h, 1 << nb, need);
+  __syncthreads();
+}
+
+// NT threads per list: 1024 when the lists are few enough for one wave, else 256.
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_cand_kernel(TopkArgs a) {
+  __shared__ CandSmem<NT> S;
+  const int th = blockIdx.x;
+  pdl_wait();   // the scoring kernel (and before it the pre-pass) has completed
+  pdl_launch_dependents();
+  const int2 m = __ldcg(a.meta + th);
+  const uint32_t L = (uint32_t)m.x;
+  const int k = m.y < a.k_max ? m.y : a.k_max;
+  int32_t* out = a.out_idx + (int64_t)th * a.k_max;
+  if (threadIdx.x == 0) {
+    if (a.out_count != nullptr) a.out_count[th] = k;
+    S.slots = (int)a.cand_cnt[th];
+    a.cand_cnt[th] = 0u;   // zero again for the next call
+    S.nvalid = 0;
   }
-  radix_round(S, ckey, cnt, 11, 21, true, 0u, k, 0);
+  if (k == 0 || k == (int)L) {   // every visible token is kept, or none
+    for (int i = threadIdx.x; i < a.k_max; i += NT) out[i] = i < k ? i : -1;
+    return;
+  }
+  const uint32_t lo = __ldcg(a.lo_key + th);
+  const int words = (int)((L + 31) >> 5);
+  for (int i = threadIdx.x; i < kSelBins; i += NT) {
+    S.hist[0][i] = 0u;
+    S.hist[1][i] = 0u;
+  }
+  for (int i = threadIdx.x; i < words && i < kCandBitmapTokens / 32; i += NT) S.above[i] = 0u;
+  __syncthreads();
+  const int slots = S.slots;
+  if (slots < k || slots > kTopkCandCap || L > (uint32_t)kCandBitmapTokens) {
+    if (threadIdx.x == 0) a.queue[atomicAdd(a.queue_cnt, 1u)] = th;
+    return;
+  }
+  const uint2* cand = a.cand + (int64_t)th * kTopkCandCap;
+  // round 1 (top 11 key bits), counting the valid candidates on the way
+  int mine = 0;
+  for_candidates<NT>(cand, slots, L, lo, [&](uint32_t key, uint32_t) {
+    atomicAdd(&S.hist[0][key >> 21], 1u);
+    ++mine;
+  });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xFFFFFFFFu, mine, o);
+  if ((threadIdx.x & 31) == 0 && mine != 0) atomicAdd(&S.nvalid, mine);
+  __syncthreads();
+  if (S.nvalid < k) {   // the same in every thread; nothing was written
+    if (threadIdx.x == 0) a.queue[atomicAdd(a.queue_cnt, 1u)] = th;
+    return;
+  }
+  if (threadIdx.x < 32) warp_find_bin(S, S.hist[0], kSelBins, k);
+  __syncthreads();
   uint32_t prefix = (uint32_t)S.found_bin;
   int need = k - S.found_above;
-  radix_round(S, ckey, cnt, 11, 10, false, prefix, need, 1);
+  cand_round<NT>(S, cand, slots, L, lo, 11, 10, prefix, need, 1);
   prefix = (prefix << 11) | (uint32_t)S.found_bin;
   need -= S.found_above;
-  radix_round(S, ckey, cnt, 10, 0, false, prefix, need, 0);
+  cand_round<NT>(S, cand, slots, L, lo, 10, 0, prefix, need, 0);
   const uint32_t T = (prefix << 10) | (uint32_t)S.found_bin;
   const int need_eq = need - S.found_above;   // 1 <= need_eq <= the number of keys equal to T
-  // every thread has read the rounds' results (radix_round ends in a barrier): reuse hist
-  for (int i = threadIdx.x; i < words; i += kSelectThreads) tied[i] = 0u;
+  // every thread has read the rounds' results (cand_round ends in a barrier): reuse hist
+  uint32_t* tied = &S.hist[0][0];
+  for (int i = threadIdx.x; i < words; i += NT) tied[i] = 0u;
   __syncthreads();
-  for (int i = threadIdx.x; i < cnt; i += kSelectThreads) {
-    const uint32_t key = ckey[i], x = cidx[i];
-    if (x >= (uint32_t)L) continue;
-    if (key > T) atomicOr(&above[x >> 5], 1u << (x & 31));
+  for_candidates<NT>(cand, slots, L, lo, [&](uint32_t key, uint32_t x) {
+    if (key > T) atomicOr(&S.above[x >> 5], 1u << (x & 31));
     else if (key == T) atomicOr(&tied[x >> 5], 1u << (x & 31));
-  }
+  });
   __syncthreads();
-  // thread j owns words [8 j, 8 j + 8): the ties before it decide how many of its own it keeps
-  constexpr int kWordsPer = kCandBitmapTokens / 32 / kSelectThreads;
+  // thread j owns words [W j, W j + W): the ties before it decide how many of its own it keeps
+  constexpr int kWordsPer = kCandBitmapTokens / 32 / NT;
   const int w0 = threadIdx.x * kWordsPer;
   int my_ties = 0, my_above = 0;
 #pragma unroll
   for (int w = 0; w < kWordsPer; ++w) {
     if (w0 + w < words) {
       my_ties += __popc(tied[w0 + w]);
-      my_above += __popc(above[w0 + w]);
+      my_above += __popc(S.above[w0 + w]);
     }
   }
   int total;
-  const int ties_before = block_exclusive_scan<kSelectThreads>(my_ties, S.scan_tmp, &total);
+  const int ties_before = block_exclusive_scan<NT>(my_ties, S.scan_tmp, &total);
   int keep_ties = need_eq - ties_before;
   keep_ties = keep_ties < 0 ? 0 : (keep_ties > my_ties ? my_ties : keep_ties);
-  int pos = block_exclusive_scan<kSelectThreads>(my_above + keep_ties, S.scan_tmp, &total);
-#pragma unroll
+  int pos = block_exclusive_scan<NT>(my_above + keep_ties, S.scan_tmp, &total);
   for (int w = 0; w < kWordsPer; ++w) {
     if (w0 + w >= words) break;
     uint32_t tb = tied[w0 + w];
@@ -1060,7 +1126,7 @@ __device__ bool select_candidates(SelectSmem& S, const uint2* cand, int slots, u
       tb ^= low;
       --keep_ties;
     }
-    uint32_t bits = above[w0 + w] | kept_tb;
+    uint32_t bits = S.above[w0 + w] | kept_tb;
     while (bits != 0u) {
       const int bit = __ffs(bits) - 1;
       bits &= bits - 1u;
@@ -1068,8 +1134,7 @@ __device__ bool select_candidates(SelectSmem& S, const uint2* cand, int slots, u
       ++pos;
     }
   }
-  for (int i = k + threadIdx.x; i < k_max; i += kSelectThreads) out[i] = -1;
-  return true;
+  for (int i = k + threadIdx.x; i < a.k_max; i += NT) out[i] = -1;
 }
 
 // The filtered scoring kernel writes no score rows.  A list the candidate path cannot serve (its
@@ -1109,45 +1174,13 @@ __device__ void rescore_row(const TopkArgs& a, int th, int b, int L, float* row,
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
-  const int th = blockIdx.x;
-  int b = -1, L, k;
-  // launched as a dependent of the scoring kernel: its scores (or candidates) are read only once
-  // that kernel has completed.  The filtered form takes the list's (kv_len, k) from the
-  // threshold kernel, which finished before the scoring kernel did; the unfiltered form works
-  // them out from the call's inputs before the wait.
-  if (a.filter) {
-    pdl_wait();
-    const int2 m = __ldcg(a.meta + th);
-    L = m.x;
-    k = m.y;
-  } else {
-    list_len_k(a, th, b, L, k);
-    pdl_wait();
-  }
-  pdl_launch_dependents();
+// The selection over a list's score row: every visible token (k = L) or none (k = 0), the
+// sampled fast path, else the multi-pass radix path.  Under the candidate filter the scoring
+// kernel wrote no row, so the list's row is recomputed first.
+__device__ void select_rows(SelectSmem& S, const TopkArgs& a, int th, int b, int L, int k) {
   int32_t* out = a.out_idx + (int64_t)th * a.k_max;
   float* osc = a.out_scores != nullptr ? a.out_scores + (int64_t)th * a.k_max : nullptr;
-  if (a.out_count != nullptr && threadIdx.x == 0) a.out_count[th] = k;
   const float* row = a.scores + (int64_t)th * a.score_stride;
-
-  if (a.filter) {
-    // the scoring kernel appended this list's scores at or above its threshold; take the count
-    // and leave the counter zero for the next call, whatever path runs below
-    __shared__ int s_cand;
-    if (threadIdx.x == 0) {
-      s_cand = (int)a.cand_cnt[th];
-      a.cand_cnt[th] = 0u;
-    }
-    __syncthreads();
-    const int cnt = s_cand;
-    if (k > 0 && k < L && L <= kCandBitmapTokens && cnt >= k && cnt <= kTopkCandCap && osc == nullptr &&
-        select_candidates(S, a.cand + (int64_t)th * kTopkCandCap, cnt, __ldcg(a.lo_key + th), L, k, out, a.k_max))
-      return;
-  }
-
   if (k == L || k == 0) {   // every visible token is kept, or none
     for (int i = threadIdx.x; i < a.k_max; i += kSelectThreads) {
       out[i] = i < k ? i : -1;
@@ -1293,6 +1326,42 @@ __global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs
   }
 }
 
+// Without the filter: one CTA per list (th = blockIdx.x).  With it (queued != 0): the lists the
+// candidate kernel could not serve, taken from its queue by a grid of a few CTAs per SM; the
+// last CTA to finish leaves the queue empty for the next call.
+__global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(TopkArgs a, int queued) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  SelectSmem& S = *reinterpret_cast<SelectSmem*>(smem_raw);
+  if (queued) {
+    pdl_wait();   // the candidate kernel has queued its lists
+    pdl_launch_dependents();
+    const int n = (int)__ldcg(a.queue_cnt);
+    for (int i = blockIdx.x; i < n; i += gridDim.x) {
+      const int th = __ldcg(a.queue + i);
+      const int2 m = __ldcg(a.meta + th);
+      select_rows(S, a, th, -1, m.x, m.y);
+      __syncthreads();   // the next list reuses the shared memory
+    }
+    __shared__ int s_last;
+    if (threadIdx.x == 0) s_last = atomicAdd(a.queue_done, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (s_last && threadIdx.x == 0) {
+      *a.queue_cnt = 0u;
+      *a.queue_done = 0u;
+    }
+    return;
+  }
+  const int th = blockIdx.x;
+  int b, L, k;
+  // launched as a dependent of the scoring kernel: everything before the wait reads only the
+  // call's inputs; the scores are read only once that kernel has completed
+  list_len_k(a, th, b, L, k);
+  if (a.out_count != nullptr && threadIdx.x == 0) a.out_count[th] = k;
+  pdl_wait();
+  pdl_launch_dependents();
+  select_rows(S, a, th, b, L, k);
+}
+
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
@@ -1348,7 +1417,16 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_dependent(topk_select_kernel, dim3(num_lists), dim3(kSelectThreads), sizeof(SelectSmem), stream, a);
+  if (!a.filter)
+    return launch_dependent(topk_select_kernel, dim3(num_lists), dim3(kSelectThreads), sizeof(SelectSmem), stream, a, 0);
+  // the candidate path, then the queue of lists it could not serve
+  if (num_lists <= a.queue_ctas)   // at most two lists per SM: one wave of 1024-thread CTAs
+    e = launch_dependent(topk_cand_kernel<1024>, dim3(num_lists), dim3(1024), 0, stream, a);
+  else
+    e = launch_dependent(topk_cand_kernel<256>, dim3(num_lists), dim3(256), 0, stream, a);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(topk_select_kernel, dim3((unsigned)a.queue_ctas), dim3(kSelectThreads), sizeof(SelectSmem),
+                          stream, a, 1);
 }
 
 // The selection alone, over scores another kernel wrote into the workspace (the label indexer).
@@ -1360,7 +1438,7 @@ cudaError_t launch_topk_select_only(const TopkArgs& a, int num_lists, cudaStream
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  return launch_dependent(topk_select_kernel, dim3(num_lists), dim3(kSelectThreads), sizeof(SelectSmem), stream, a);
+  return launch_dependent(topk_select_kernel, dim3(num_lists), dim3(kSelectThreads), sizeof(SelectSmem), stream, a, 0);
 }
 
 }  // namespace tsd
