@@ -622,6 +622,10 @@ def run_native(args):
     topk_bytes = ctx_rows * 256 + q_bytes + T * Hq * k_max * 4
     index_bytes = T * Hq * k_max * 4
     hbm, peak_kind = peaks()
+    topk_plan = tsd.topk_select_plan(cache, queries, k_max)
+    topk_form = ("candidate-filtered: sample pre-pass, per-list thresholds, scoring that keeps only the "
+                 "scores reaching them, selection among those" if topk_plan["filtered"]
+                 else "full score rows, then selection over each row")
     # whole-job bytes (each rank decodes its own batch) over the slowest rank's time; the
     # roofline is per GPU: the job's bytes per GPU over that time
     job_sparse, job_dense, job_topk = sum_over_ranks([sparse_bytes, dense_bytes, topk_bytes], dev)
@@ -874,7 +878,10 @@ def run_native(args):
                      "index_bytes_not_counted": index_bytes},
         "rooflines_other": {
             "topk_select": {"achieved": round(topk_gbs, 1), "frac": round(topk_gbs / hbm, 4),
-                            "algorithmic_bytes": topk_bytes, "kernels": ["topk_score_kernel", "topk_select_kernel"]},
+                            "algorithmic_bytes": topk_bytes, "form": topk_form,
+                            "kernels": (["topk_prepass_kernel", "topk_score_kernel", "topk_cand_kernel",
+                                         "topk_select_kernel (queue pass)"] if topk_plan["filtered"]
+                                        else ["topk_score_kernel", "topk_select_kernel"])},
             "dense_decode": {"achieved": round(dense_gbs, 1), "frac": round(dense_gbs / hbm, 4),
                              "algorithmic_bytes": dense_bytes, "kernels": ["dense_decode_kernel"]},
         },
@@ -889,7 +896,7 @@ def run_native(args):
         "graph20_rotating": graph20_line,
         "sparse_leg_us_stats": sparse_stats,
         "other_workloads": others,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (topk_plan["kernels"] + 2) * args.steps,
         "clocks": cl,
     }
     if cpu is not None:

@@ -153,6 +153,17 @@ size_t tsd_sparse_decode_workspace_size(const tsd_kv_cache* cache, const tsd_que
 tsd_status tsd_sparse_decode_plan(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
                                   int32_t* persistent, int32_t* entries_per_task, int32_t* tasks_per_list);
 
+/* The form tsd_topk_select takes for these shapes and k_max (the exact indexer of the pages'
+ * section 2, "Oracle Top-K").  *filtered = 1 for the candidate-filtered form: a sample pre-pass
+ * sets a per-list threshold, the scoring kernel keeps only the scores that reach it, and the
+ * selection works on those (exact in either form; chosen for bf16 queries when the score rows
+ * would not stay in L2 and the expected candidates fit).  0 for the form over full score rows.
+ * *kernels = the kernels one call launches (4 or 2).  The environment variable TSD_TOPK_FILTER
+ * (0, 1 or rescore) overrides the choice, as it does for tsd_topk_select.  Device pointers may
+ * be NULL.  Errors: INVALID_ARGUMENT, UNSUPPORTED (as tsd_topk_select's host checks). */
+tsd_status tsd_topk_select_plan(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                int32_t* filtered, int32_t* kernels);
+
 /*
  * Sparse decode attention over per-(token, head) index lists (pages section 2,
  * "Hardware implementation"; section 3.C).  For each query token t and q head h:

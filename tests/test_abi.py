@@ -308,3 +308,38 @@ def test_sparse_decode_plan_choice(lib):
                                       ctypes.byref(n)) == tsd.TSD_ERR_INVALID_ARGUMENT
     bad = make_cache(head_dim=64)
     assert lib.tsd_sparse_decode_plan(ctypes.byref(bad), ctypes.byref(q), 655, *args) == tsd.TSD_ERR_UNSUPPORTED
+
+
+def test_topk_select_plan_choice(lib, monkeypatch):
+    """Which form of the exact indexer a call takes (host arithmetic only).  The Llama-3-8B shape
+    (256 lists x 32K tokens: 33.5 MB of score rows, which stay in L2) takes the form over score
+    rows, 2 kernels; the ragged shape (4096 lists x 128K: 2.1 GB of rows) the candidate filter, 4
+    kernels; fp32 queries, a k too large for the candidate buffer and TSD_TOPK_FILTER=0 all give
+    the row form, and TSD_TOPK_FILTER=1 forces the filter on the small shape."""
+    monkeypatch.delenv("TSD_TOPK_FILTER", raising=False)
+    monkeypatch.delenv("TSD_SCORE_KERNEL", raising=False)
+    f, n = ctypes.c_int32(), ctypes.c_int32()
+    args = (ctypes.byref(f), ctypes.byref(n))
+    c, q = make_cache(), make_queries()
+    assert lib.tsd_topk_select_plan(ctypes.byref(c), ctypes.byref(q), 655, *args) == tsd.TSD_OK
+    assert (f.value, n.value) == (0, 2)
+    rc = make_cache(batch=32, max_pages=8192, num_pages=32 * 8192, max_seq_len=131072)
+    rq = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=4)
+    assert lib.tsd_topk_select_plan(ctypes.byref(rc), ctypes.byref(rq), 2622, *args) == tsd.TSD_OK
+    assert (f.value, n.value) == (1, 4)
+    rq32 = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=4, q_dtype=tsd.TSD_F32)
+    assert lib.tsd_topk_select_plan(ctypes.byref(rc), ctypes.byref(rq32), 2622, *args) == tsd.TSD_OK
+    assert (f.value, n.value) == (0, 2)
+    assert lib.tsd_topk_select_plan(ctypes.byref(rc), ctypes.byref(rq), 13107, *args) == tsd.TSD_OK
+    assert (f.value, n.value) == (0, 2)
+    monkeypatch.setenv("TSD_TOPK_FILTER", "0")
+    assert lib.tsd_topk_select_plan(ctypes.byref(rc), ctypes.byref(rq), 2622, *args) == tsd.TSD_OK
+    assert (f.value, n.value) == (0, 2)
+    monkeypatch.setenv("TSD_TOPK_FILTER", "1")
+    assert lib.tsd_topk_select_plan(ctypes.byref(c), ctypes.byref(q), 655, *args) == tsd.TSD_OK
+    assert (f.value, n.value) == (1, 4)
+    assert lib.tsd_topk_select_plan(ctypes.byref(c), ctypes.byref(q), 0, *args) == tsd.TSD_ERR_INVALID_ARGUMENT
+    assert lib.tsd_topk_select_plan(ctypes.byref(c), ctypes.byref(q), 655, None,
+                                    ctypes.byref(n)) == tsd.TSD_ERR_INVALID_ARGUMENT
+    bad = make_cache(head_dim=64)
+    assert lib.tsd_topk_select_plan(ctypes.byref(bad), ctypes.byref(q), 655, *args) == tsd.TSD_ERR_UNSUPPORTED

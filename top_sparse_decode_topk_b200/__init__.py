@@ -89,6 +89,8 @@ EXPORTS = {
                                         ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                         ctypes.c_void_p]),
     "tsd_read_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "tsd_topk_select_plan": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
+                                            ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)]),
     "tsd_sparse_decode_plan": (ctypes.c_int, [ctypes.POINTER(_KvCacheC), ctypes.POINTER(_QueriesC), ctypes.c_int32,
                                               ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                                               ctypes.POINTER(ctypes.c_int32)]),
@@ -520,6 +522,17 @@ def sparse_decode(cache: KVCache, queries: Queries, idx, out=None, out_dtype=Non
                                               k_max, out.data_ptr(), odt, lp, ws.data_ptr(), ws.numel(), sp),
                "tsd_sparse_decode_weighted")
     return _finish(out, host_out, lse, host_lse, s)
+
+
+def topk_select_plan(cache: KVCache, queries: Queries, k_max: int) -> dict:
+    """The form topk_select would take (tsd_topk_select_plan): whether the candidate filter
+    runs, and how many kernels one call launches."""
+    lib = load_library()
+    cs, qs = cache.c_struct(), queries.c_struct()
+    f, n = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib.tsd_topk_select_plan(ctypes.byref(cs), ctypes.byref(qs), int(k_max), ctypes.byref(f), ctypes.byref(n)),
+           "tsd_topk_select_plan")
+    return {"filtered": bool(f.value), "kernels": int(n.value)}
 
 
 def sparse_decode_plan(cache: KVCache, queries: Queries, k_max: int) -> dict:

@@ -328,6 +328,32 @@ static bool score_on_tcgen05_host() {
   return e != nullptr && strcmp(e, "tcgen05") == 0;
 }
 
+// The form of the exact indexer for a call: 0 unfiltered, 1 candidate-filtered, 2 filtered with
+// every threshold disabled (TSD_TOPK_FILTER=rescore).
+static int topk_filter_choice(const Shapes& sh, bool q_f32, bool with_scores, int32_t k_max) {
+  const TopkLayout lay = topk_layout(sh);
+  const int fm = filter_mode();
+  const double row_bytes = (double)sh.tokens * sh.hq * (double)lay.score_stride * sizeof(float);
+  const bool can = !q_f32 && !with_scores && !score_on_tcgen05_host();
+  if (fm == kFilterRescore) return can ? 2 : 0;
+  if (fm == kFilterOn) return can && filter_fits(k_max, lay.sample_shift + 1) ? 1 : 0;
+  if (fm == kFilterAuto)
+    return can && filter_fits(k_max, lay.sample_shift + 1) && row_bytes > kFilterMinRowBytes ? 1 : 0;
+  return 0;
+}
+
+tsd_status tsd_topk_select_plan(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
+                                int32_t* filtered, int32_t* kernels) {
+  Shapes sh;
+  if (k_max < 1 || filtered == nullptr || kernels == nullptr || queries == nullptr) return TSD_ERR_INVALID_ARGUMENT;
+  const tsd_status st = sizes_for(cache, queries, &sh);
+  if (st != TSD_OK) return st;
+  const int f = topk_filter_choice(sh, queries->q_dtype == TSD_F32, false, k_max);
+  *filtered = f != 0 ? 1 : 0;
+  *kernels = f != 0 ? 4 : 2;
+  return TSD_OK;
+}
+
 static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
                                    const int32_t* k_per_token, int32_t* out_idx, float* out_scores,
                                    int32_t* out_count, void* ws, size_t ws_bytes, tsd_stream_t stream) {
@@ -356,14 +382,7 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   // no score rows) serves bf16 queries with the warp-MMA scoring kernel when k_max is small
   // enough for the candidates to fit; the kept scores' output (tsd_topk_select_scores), fp32
   // queries and larger k take the paths over the full score rows.
-  const int fm = filter_mode();
-  const double row_bytes = (double)sh.tokens * sh.hq * (double)lay.score_stride * sizeof(float);
-  const bool can = !qv.q_f32 && out_scores == nullptr && !score_on_tcgen05_host();
-  if (fm == kFilterRescore) a.filter = can ? 2 : 0;
-  else if (fm == kFilterOn) a.filter = can && filter_fits(k_max, lay.sample_shift + 1) ? 1 : 0;
-  else if (fm == kFilterAuto)
-    a.filter = can && filter_fits(k_max, lay.sample_shift + 1) && row_bytes > kFilterMinRowBytes ? 1 : 0;
-  else a.filter = 0;
+  a.filter = topk_filter_choice(sh, qv.q_f32, out_scores != nullptr, k_max);
   if (a.filter) a.sample_shift = lay.sample_shift + 1;   // the pre-pass samples every other sample slot
   a.lo_key = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_lo);
   a.cand = reinterpret_cast<uint2*>(static_cast<char*>(ws) + lay.off_cand);
