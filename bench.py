@@ -65,6 +65,8 @@ def parse():
                    help="with --record-traffic: the bench line of the same command run without ncu; its "
                         "sparse-decode algorithmic bytes are stored beside the captured traffic, so that the "
                         "figure can be scaled to a larger copy of the workload")
+    p.add_argument("--traffic-command", metavar="CMD",
+                   help="with --record-traffic: the ncu command that made the log, stored with the figure")
     return p.parse_args()
 
 
@@ -220,7 +222,7 @@ KERNEL_SOURCES = {
 }
 
 
-def record_traffic(csv_path: str, workload: str, plain_line: str = None):
+def record_traffic(csv_path: str, workload: str, plain_line: str = None, command: str = None):
     """Fold one ncu --csv metric log into profiles/dram_traffic.json (first launch of each kernel)."""
     alg = None
     if plain_line:
@@ -248,9 +250,10 @@ def record_traffic(csv_path: str, workload: str, plain_line: str = None):
             out = json.load(f)
     except Exception:
         out = {}
-    out["_about"] = ("DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of one captured "
-                     "launch per kernel in the first timed step of the bench, L2 flushed before it; bench.py "
-                     "uses a kernel's figure as roofline.traffic only while source_sha still matches its sources.")
+    out.setdefault("_about", "DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of one captured "
+                   "launch per kernel and workload, L2 flushed before it (the bench's own flush); bench.py uses a "
+                   "kernel's figure as roofline.traffic only while source_sha still matches the kernel's sources. "
+                   "Each entry gives the command that made it.")
     for kern, e in got.items():
         rd, wr = e.get("dram__bytes_read.sum"), e.get("dram__bytes_write.sum")
         if rd is None or wr is None:
@@ -259,6 +262,8 @@ def record_traffic(csv_path: str, workload: str, plain_line: str = None):
             "bytes_per_launch": rd + wr, "read": rd, "write": wr,
             "duration_us": round(e.get("gpu__time_duration.sum", float("nan")) / 1e3, 3),
             "sources": KERNEL_SOURCES[kern], "source_sha": source_sha(KERNEL_SOURCES[kern])}
+        if command:
+            out[kern][workload]["command"] = command
         if alg is not None and kern.startswith("sparse_"):
             out[kern][workload]["algorithmic_bytes"] = alg
     with open(path, "w") as f:
@@ -972,7 +977,7 @@ def run_reference(args):
 def main():
     args = parse()
     if args.record_traffic:
-        record_traffic(args.record_traffic, args.config, args.plain_line)
+        record_traffic(args.record_traffic, args.config, args.plain_line, args.traffic_command)
     elif args.impl == "reference":
         run_reference(args)
     else:

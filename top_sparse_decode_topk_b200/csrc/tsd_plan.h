@@ -136,8 +136,9 @@ struct DensePlan {
 
 constexpr int kDenseMaxLists = 16;
 constexpr int kDnCtasPerSm = 3;    // resident dense-decode CTAs per SM (its launch bounds)
-constexpr int kScCtasPerSm = 5;    // resident top-k scoring CTAs per SM, warp-MMA kernel (its launch bounds)
-constexpr int kScTcCtasPerSm = 5;  // the same for the tcgen05 scoring kernel
+constexpr int kScCtasPerSm = 6;    // resident top-k scoring CTAs per SM, warp-MMA kernel (its launch bounds;
+                                   // bf16 queries: fp32 queries' second query tile leaves room for 5)
+constexpr int kScTcCtasPerSm = 6;  // the same for the tcgen05 scoring kernel
 constexpr int kScoreCtasPerSm = kScCtasPerSm;
 static_assert(kScTcCtasPerSm == kScCtasPerSm, "both scoring kernels share one window plan");
 // Tokens per CTA at most.  Windows are sized on max_seq_len, so on a ragged batch (lengths
