@@ -126,3 +126,36 @@ def test_step_llama3_8b_sampled():
     w, cache, queries = _setup(W.CONFIGS["llama3_8b"], seed=0)
     pairs = PT.sample_pairs(w, 8, full_seqs=(0,), seed=3)
     _check(w, cache, queries, 655, pairs, torch.bfloat16)
+
+
+@pytest.mark.parametrize("per_token", [False, True])
+def test_step_with_the_candidate_filter_forced(monkeypatch, per_token):
+    """The step with the exact indexer's candidate filter forced on (TSD_TOPK_FILTER=1): its
+    pre-pass arrival counters, candidate counters and queue must be left zero by every replay,
+    so that the second replay of the graph agrees with the oracle as the first did."""
+    import torch
+    monkeypatch.setenv("TSD_TOPK_FILTER", "1")
+    if per_token:
+        cfg = W.DecodeConfig(name="step_ragged_small", batch=4, num_q_heads=8, num_kv_heads=2,
+                             seq_len_range=(3000, 20000), tokens_per_seq=4, k_frac_ceil=0.02, planted=True,
+                             causal=True)
+        w, cache, queries = _setup(cfg, seed=4)
+        k = None
+    else:
+        w, cache, queries = _setup(SMALL, lens=[6000, 300, 2500], seed=1)
+        k = 100
+    kpt = w.k_per_token(k)
+    assert tsd.topk_select_plan(cache, queries, int(kpt.max()))["filtered"]
+    pairs = [(t, h) for t in range(len(w.kv_len)) for h in range(w.cfg.num_q_heads)]
+    _check(w, cache, queries, k, pairs, torch.float32)
+
+
+def test_step_ragged_8_sampled():
+    """The ragged batch with 8 sequences, where the filter runs by default (537 MB of score rows
+    would not stay in L2)."""
+    import torch
+    w, cache, queries = _setup(W.CONFIGS["ragged_8"], seed=0)
+    kpt = w.k_per_token(None)
+    assert tsd.topk_select_plan(cache, queries, int(kpt.max()))["filtered"]
+    pairs = PT.sample_pairs(w, 8, full_seqs=(0,), seed=5)
+    _check(w, cache, queries, None, pairs, torch.bfloat16)

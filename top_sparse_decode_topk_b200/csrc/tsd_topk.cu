@@ -984,9 +984,9 @@ __device__ bool select_fast(SelectSmem& S, const float* row, const float* samp, 
 // skipped here.  With at least k valid candidates they hold the whole top-k and every score
 // equal to the k-th.  Three radix rounds over the candidates, read from L2 each time, give the
 // k-th key T and the number need_eq of keys equal to T to keep.  Keys > T are marked in a bitmap
-// of the list's tokens and keys == T in a second one; a block scan over the tie bitmap keeps
-// the need_eq lowest-index ties, a second scan gives every thread its output offset, and the
-// kept indices are written in ascending order.  A list with fewer than k valid candidates, or
+// of the list's tokens and keys == T in a second one; warp-owned word ranges, read 32 words at a
+// time, give the tie ranks (the need_eq lowest-index ties are kept) and the output ranks, and
+// the kept indices are written in ascending order.  A list with fewer than k valid candidates, or
 // more than fit, goes into the queue that topk_select_kernel works off over recomputed rows.
 constexpr int kCandBitmapTokens = 131072;   // longest list the bitmaps cover
 constexpr int kCsUnroll = 8;                  // candidate loads in flight per thread
@@ -994,7 +994,8 @@ template <int NT>
 struct CandSmem {
   uint32_t hist[2][kSelBins];               // radix histograms; after the rounds, the tie bitmap
   uint32_t above[kCandBitmapTokens / 32];   // keys > T
-  int scan_tmp[NT / 32 + 1];
+  int scan_tmp[NT / 32 + 1];   // block scans; the warps' counts of keys > T in the ordered output
+  int warp_ties[NT / 32];       // the warps' counts of keys == T in the ordered output
   int found_bin, found_above, nvalid, slots;
 };
 static_assert(kCandBitmapTokens <= 2 * kSelBins * 32, "the tie bitmap reuses both histograms");
@@ -1103,39 +1104,79 @@ __global__ void __launch_bounds__(NT) topk_cand_kernel(TopkArgs a) {
     else if (key == T) atomicOr(&tied[x >> 5], 1u << (x & 31));
   });
   __syncthreads();
-  // thread j owns words [W j, W j + W): the ties before it decide how many of its own it keeps
-  constexpr int kWordsPer = kCandBitmapTokens / 32 / NT;
-  const int w0 = threadIdx.x * kWordsPer;
-  int my_ties = 0, my_above = 0;
-#pragma unroll
-  for (int w = 0; w < kWordsPer; ++w) {
-    if (w0 + w < words) {
-      my_ties += __popc(tied[w0 + w]);
-      my_above += __popc(S.above[w0 + w]);
+  // Ordered output.  Warp w owns words [w WPW, (w + 1) WPW) and reads them 32 at a time, lane l
+  // taking word 32 r + l of round r, so the reads are conflict-free and ascending in (r, l).
+  // Pass 1 counts each warp's keys > T and ties; pass 2 walks the rounds again with warp scans:
+  // a tie is kept while its rank among all ties is below need_eq (the lowest indices first),
+  // and every kept token's index goes to its rank among the kept ones.
+  constexpr int NW = NT / 32;
+  constexpr int WPW = kCandBitmapTokens / 32 / NW;   // words per warp
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wbase = warp * WPW;
+  int n_above = 0, n_tied = 0;
+#pragma unroll 4
+  for (int r = 0; r < WPW / 32; ++r) {
+    const int wi = wbase + 32 * r + lane;
+    if (wi < words) {
+      n_above += __popc(S.above[wi]);
+      n_tied += __popc(tied[wi]);
     }
   }
-  int total;
-  const int ties_before = block_exclusive_scan<NT>(my_ties, S.scan_tmp, &total);
-  int keep_ties = need_eq - ties_before;
-  keep_ties = keep_ties < 0 ? 0 : (keep_ties > my_ties ? my_ties : keep_ties);
-  int pos = block_exclusive_scan<NT>(my_above + keep_ties, S.scan_tmp, &total);
-  for (int w = 0; w < kWordsPer; ++w) {
-    if (w0 + w >= words) break;
-    uint32_t tb = tied[w0 + w];
-    uint32_t kept_tb = 0u;
-    while (tb != 0u && keep_ties > 0) {   // the lowest-index ties first
-      const uint32_t low = tb & (0u - tb);
-      kept_tb |= low;
-      tb ^= low;
-      --keep_ties;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    n_above += __shfl_xor_sync(0xFFFFFFFFu, n_above, o);
+    n_tied += __shfl_xor_sync(0xFFFFFFFFu, n_tied, o);
+  }
+  if (lane == 0) {
+    S.scan_tmp[warp] = n_above;
+    S.warp_ties[warp] = n_tied;
+  }
+  __syncthreads();
+  int tie_run = 0, out_run = 0;   // ties and kept tokens of the warps before this one
+  for (int v = 0; v < warp; ++v) {
+    const int kt = min(max(need_eq - tie_run, 0), S.warp_ties[v]);
+    out_run += S.scan_tmp[v] + kt;
+    tie_run += S.warp_ties[v];
+  }
+  for (int r = 0; r < WPW / 32; ++r) {
+    const int wbr = wbase + 32 * r;
+    if (wbr >= words) break;   // the same in every lane of the warp
+    const int wi = wbr + lane;
+    const uint32_t ab = wi < words ? S.above[wi] : 0u;
+    uint32_t tb = wi < words ? tied[wi] : 0u;
+    // ties: this lane's rank among all ties, then how many of its own it keeps
+    const int nt = __popc(tb);
+    int ti = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+      if (lane >= o) ti += y;
     }
-    uint32_t bits = S.above[w0 + w] | kept_tb;
+    const int t_rank = tie_run + ti - nt;
+    int keep = min(max(need_eq - t_rank, 0), nt);
+    uint32_t kept = 0u;
+    while (keep-- > 0) {   // the lowest-index ties first
+      const uint32_t low = tb & (0u - tb);
+      kept |= low;
+      tb ^= low;
+    }
+    uint32_t bits = ab | kept;
+    const int nb = __popc(bits);
+    int oi = nb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, oi, o);
+      if (lane >= o) oi += y;
+    }
+    int pos = out_run + oi - nb;
     while (bits != 0u) {
       const int bit = __ffs(bits) - 1;
       bits &= bits - 1u;
-      if (pos < k) out[pos] = (w0 + w) * 32 + bit;
+      if (pos < k) out[pos] = wi * 32 + bit;
       ++pos;
     }
+    out_run += __shfl_sync(0xFFFFFFFFu, oi, 31);
+    tie_run += __shfl_sync(0xFFFFFFFFu, ti, 31);
   }
   for (int i = k + threadIdx.x; i < a.k_max; i += NT) out[i] = -1;
 }
