@@ -131,6 +131,13 @@ size_t tsd_topk_workspace_size(const tsd_kv_cache* cache, const tsd_queries* que
  *            then -1 up to k_max.
  * out_count: device int32 [T][Hq] or NULL; receives k_t.
  * k_max >= 1.  Errors: INVALID_ARGUMENT, UNSUPPORTED, WORKSPACE_TOO_SMALL, CUDA.
+ * Two forms give the same lists (tsd_topk_select_plan says which a call takes): the scores of
+ * every visible token written to the workspace and selected from there, or -- bf16 queries,
+ * score rows too large to stay in L2, k small enough -- a candidate filter: a strided sample of
+ * every list sets a threshold below which no top-k score can lie (with overwhelming
+ * probability; a list whose sample misled it is recomputed in full, so the result is exact
+ * either way), the scoring keeps only the scores that reach it, and the selection works on
+ * those.  The workspace (tsd_topk_workspace_size) holds both forms' buffers.
  */
 tsd_status tsd_topk_select(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max,
                            const int32_t* k_per_token, int32_t* out_idx, int32_t* out_count,

@@ -314,7 +314,7 @@ static int filter_mode() {
 // L2 and the filter's pre-pass costs more than it saves.
 constexpr double kFilterMinRowBytes = 64.0 * 1024 * 1024;
 
-// Whether a list of any length with k <= k_max passes the threshold kernel's size test when its
+// Whether a list of any length with k <= k_max passes the pre-pass's size test when its
 // sample takes every 2^shift-th token: with m = k_max / 2^shift the expected sample count above
 // the k-th score is at most m + 1, and r = ceil(m + 1 + 4 sqrt(m + 1) + 4) samples at stride
 // 2^shift stand for at most r 2^shift candidates, which must stay within 3/4 of the buffer.

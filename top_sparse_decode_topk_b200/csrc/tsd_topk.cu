@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kScThreads, QF32 ? 5 : kScCtasPerSm) topk_scor
   uint2* cbuf[2] = {nullptr, nullptr};
   uint32_t pool_next[2] = {0u, 0u}, pool_end[2] = {0u, 0u};   // the quad's reserved, unused slots
   if (a.filter) {
-    pdl_wait();   // the threshold kernel wrote lo
+    pdl_wait();   // the pre-pass wrote lo
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const int m = (lane >> 2) + 8 * hr;
@@ -473,7 +473,7 @@ __device__ __forceinline__ void list_len_k(const TopkArgs& a, int th, int& L, in
 // list (bf16 queries) and turns each list's sample into a threshold key lo, as the selection's
 // sampled fast path would.  The scoring kernel then appends every score whose key reaches lo to
 // the list's candidate buffer instead of writing the score row, and the selection works on the
-// candidates alone (see select_candidates).
+// candidates alone (see topk_cand_kernel).
 //
 // Grid (splits, Hkv x list groups, batch), kPpWarps warps per CTA.  The splits of a (sequence,
 // kv head, list group) share its sample tiles; each writes its samples, and the last to arrive
