@@ -133,3 +133,48 @@ def test_label_pipeline_decode(small):
                 same.append((t, h))
     assert len(same) >= 0.95 * gidx.shape[0] * gidx.shape[1]
     PT.check_decode(inp, oidx, out.cpu().numpy(), lse.cpu().numpy(), same, SM_SCALE, out_is_bf16=False)
+
+
+ONE_TOKEN = W.DecodeConfig(name="label_one_token", batch=3, num_q_heads=8, num_kv_heads=2, seq_len=20000,
+                           tokens_per_seq=1, ks=(200,), planted=True, causal=True)
+
+
+@pytest.mark.parametrize("cfg_lens", [(SMALL, SMALL_LENS, 3), (ONE_TOKEN, [20000, 9000, 3000], 4)],
+                         ids=["8_lists_per_group", "4_lists_per_group"])
+@pytest.mark.parametrize("r", [8, 16])
+def test_label_topk_candidate_filter(monkeypatch, cfg_lens, r):
+    """The label indexer's candidate filter (forced on with TSD_TOPK_FILTER=1), its row
+    recomputation (TSD_TOPK_FILTER=rescore) and the row form (=0), each against the oracle's
+    exact top-k of the label scores; the filtered and row forms score every token the same way,
+    so their lists must agree index for index.  Groups of 4 lists take the scoring kernel that
+    keeps the queries in registers, groups of 8 the general one."""
+    import torch
+    cfg, lens, seed = cfg_lens
+    w = W.make_workload(cfg, seed=seed, seq_lens=lens)
+    dw = W.to_device(w, "cuda")
+    cache = tsd.KVCache(dw.k, dw.v, dw.seq_lens, max_seq_len=cfg.max_seq_len, page_table=dw.page_table)
+    multi = cfg.tokens_per_seq > 1
+    queries = tsd.Queries(dw.q, q_indptr=dw.q_indptr if multi else None, max_tokens_per_seq=cfg.tokens_per_seq,
+                          causal=True, sm_scale=SM_SCALE)
+    inp = PT.OracleInputs(w)
+    chans = _test_channels(cfg.num_kv_heads, r, seed=30 + r)
+    index = tsd.label_cache_build(cache, torch.from_numpy(chans).cuda())
+    G = cfg.group
+    for k in (100, 400):
+        runs = {}
+        for mode in ("1", "rescore", "0"):
+            monkeypatch.setenv("TSD_TOPK_FILTER", mode)
+            gidx, gcnt = tsd.topk_select_label(cache, index, queries, k)
+            torch.cuda.synchronize()
+            gidx, gcnt = gidx.cpu().numpy(), gcnt.cpu().numpy()
+            for t in range(len(w.kv_len)):
+                b, L = int(w.token_seq[t]), int(w.kv_len[t])
+                for h in range(cfg.num_q_heads):
+                    K, _ = inp.kv(b, h // G)
+                    s = oracle.label_scores(inp.q(t, h), K[:L], chans[h // G])
+                    ok, why = oracle.topk_sets_agree(gidx[t, h], s, k, PT.TOPK_BAND)
+                    assert ok, (mode, r, k, t, h, why)
+                    assert int(gcnt[t, h]) == min(k, L)
+            runs[mode] = gidx
+        assert np.array_equal(runs["1"], runs["0"]), (r, k)
+    assert tsd.read_device_status() == 0

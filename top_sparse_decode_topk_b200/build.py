@@ -26,7 +26,7 @@ LIBS = {
     "libtsd.so": ["tsd_api.cu", "tsd_decode.cu", "tsd_topk.cu", "tsd_label.cu", "tsd_stochastic.cu", "tsd_cp.cu", "tsd_static_ws.cu"],
     "libtsd_workload.so": ["workload_fill.cu"],
 }
-HEADERS = ["tsd_common.cuh", "tsd_plan.h", "tsd_args.h", "tsd_kvtile.cuh", "tsd_umma.cuh"]
+HEADERS = ["tsd_common.cuh", "tsd_plan.h", "tsd_args.h", "tsd_kvtile.cuh", "tsd_umma.cuh", "tsd_filter.cuh"]
 
 
 def nvcc() -> str:

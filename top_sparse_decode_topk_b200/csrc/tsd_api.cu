@@ -766,8 +766,27 @@ tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k,
   a.samples = reinterpret_cast<float*>(static_cast<char*>(ws) + lay.off_samples);
   a.sample_stride = lay.sample_stride;
   a.sample_shift = lay.sample_shift;
-  a.filter = 0;
+  // The candidate filter runs here only when TSD_TOPK_FILTER forces it ("1" or "rescore"): on
+  // the ragged batch at 50x it measured slower than the row form (label top-k 1798 against
+  // 1209 us), its per-warp candidate pools refilling with a global atomic every 8 candidates
+  // of each of 16 lists.  The label scores are fp32 sums over bf16 label rows whatever the
+  // query dtype.
+  a.filter = filter_mode() > kFilterOff ? topk_filter_choice(sh, false, false, k_max) : 0;
+  if (a.filter) a.sample_shift = lay.sample_shift + 1;
   a.cand_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 256);
+  a.lo_key = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.off_lo);
+  a.cand = reinterpret_cast<uint2*>(static_cast<char*>(ws) + lay.off_cand);
+  a.meta = reinterpret_cast<int2*>(static_cast<char*>(ws) + lay.off_meta);
+  a.queue = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + lay.off_queue);
+  a.queue_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16);
+  a.queue_done = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 20);
+  {
+    const int64_t qc = 2LL * current_sm_count();
+    a.queue_ctas = (int)(qc < sh.tokens * sh.hq ? qc : sh.tokens * sh.hq);
+  }
+  a.label = static_cast<const uint16_t*>(label_k);
+  a.channels = channels;
+  a.label_r = r;
   const DensePlan p = plan_dense(sh, (int64_t)current_sm_count() * kDnCtasPerSm, kMaxWindowScore);
   a.lists_per_cta = p.lists_per_cta;
   a.list_groups = p.list_groups;

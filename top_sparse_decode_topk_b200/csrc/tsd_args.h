@@ -51,6 +51,9 @@ struct TopkArgs {
   uint32_t* queue_cnt;    // filter: their number (zero region; the last queue CTA clears it)
   uint32_t* queue_done;   // filter: queue CTAs finished (zero region; cleared with queue_cnt)
   int32_t queue_ctas;     // filter: CTAs of the queue pass
+  const uint16_t* label;    // label indexer: [rows][label_r] bf16 label cache (NULL: the exact indexer)
+  const int32_t* channels;  // label indexer: [Hkv][label_r] channel ids
+  int32_t label_r;          // label indexer: channels per kv head
   int32_t lists_per_cta;
   int32_t list_groups;
   int32_t window;

@@ -24,6 +24,7 @@
 
 #include "tsd_args.h"
 #include "tsd_common.cuh"
+#include "tsd_filter.cuh"
 
 namespace tsd {
 
@@ -141,9 +142,92 @@ __global__ void label_build_kernel(KvView kv, const int32_t* channels, int r, in
 // memory per list.  NL = 4: at most 4 lists (one decode token of a GQA group of 4, as in the
 // Llama-3-8B shape), whose query pairs, bounds and score rows live in registers, the list loop
 // unrolled; 2 tokens per lane per step keep the registers within two CTAs per SM.
-template <int R, int NL>
-__global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, const uint16_t* label,
+// ---------------------------------------------------------------------------
+// Candidate filter of the label indexer (as the exact indexer's, in tsd_topk.cu)
+// ---------------------------------------------------------------------------
+// label_prepass_kernel scores every 2^sample_shift-th token of every list on the label channels
+// and turns each list's sample into a threshold; label_score_kernel then appends the scores that
+// reach it instead of writing score rows, and the exact indexer's candidate kernel and queue
+// pass select from there.  A warp appends the candidates of one list and one token step with a
+// ballot; its slots come from a pool of kLblChunk that lane 0 refills with one atomic on the
+// list's counter.  Unused pool slots become holes (index 0xFFFFFFFF) when the CTA ends.
+constexpr uint32_t kLblChunk = 8;
+
+// Grid (Hkv x list groups, batch), kLblThreads threads: thread i scores samples i, i + 256, ...
+// of the group's lists, then warp w makes the thresholds of lists w, w + 8, ...
+template <int R>
+__global__ void __launch_bounds__(kLblThreads) label_prepass_kernel(TopkArgs a) {
+  __shared__ float qs[16][R];
+  const int g = blockIdx.x / a.list_groups, lg = blockIdx.x % a.list_groups;
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();   // the scoring kernel may launch; it waits for this grid
+  const SeqInfo si = seq_info(a.kv, a.qv, b, a.status, false);
+  const int G = a.qv.hq / a.kv.hkv;
+  int nlists = si.n * G - lg * a.lists_per_cta;
+  if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
+  if (nlists <= 0) return;
+  for (int e = threadIdx.x; e < 16 * R; e += kLblThreads) {
+    const int m = e / R, j = e - (e / R) * R;
+    float v = 0.f;
+    if (m < nlists) {
+      const int mg = lg * a.lists_per_cta + m;
+      const int jt = mg / G;
+      int c = __ldg(a.channels + (int64_t)g * R + j);
+      if (c < 0 || c >= kHeadDim) c = 0;   // the scoring kernel flags it
+      const int64_t qe = ((int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G)) * kHeadDim + c;
+      v = a.qv.q_f32 ? __ldg(reinterpret_cast<const float*>(a.qv.q) + qe)
+                     : __uint_as_float((uint32_t)__ldg(reinterpret_cast<const uint16_t*>(a.qv.q) + qe) << 16);
+    }
+    qs[m][j] = v;
+  }
+  __syncthreads();
+  const int shift = a.sample_shift;
+  const int ns_seq = (int)(((int64_t)si.len + (1 << shift) - 1) >> shift);
+  for (int j = threadIdx.x; j < ns_seq; j += kLblThreads) {
+    const int tok = j << shift;
+    const uint32_t row = kv_row(a.kv, b, g, tok);
+    if (row == kInvalidRow) continue;   // the scoring kernel flags it
+    float lv[R];
+    const uint4* src = reinterpret_cast<const uint4*>(a.label + (int64_t)row * R);
+#pragma unroll
+    for (int c = 0; c < R / 8; ++c) {
+      const uint4 v = __ldg(src + c);
+      lv[8 * c + 0] = bf16lo(v.x); lv[8 * c + 1] = bf16hi(v.x);
+      lv[8 * c + 2] = bf16lo(v.y); lv[8 * c + 3] = bf16hi(v.y);
+      lv[8 * c + 4] = bf16lo(v.z); lv[8 * c + 5] = bf16hi(v.z);
+      lv[8 * c + 6] = bf16lo(v.w); lv[8 * c + 7] = bf16hi(v.w);
+    }
+    for (int m = 0; m < nlists; ++m) {
+      const int mg = lg * a.lists_per_cta + m;
+      const int jt = mg / G;
+      if (tok >= kv_len_of(a.qv, si, jt)) continue;
+      float sc = 0.f;
+#pragma unroll
+      for (int c = 0; c < R; ++c) sc = fmaf(qs[m][c], lv[c], sc);
+      a.samples[((int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G)) * a.sample_stride + j] = sc;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  for (int m = warp; m < nlists; m += kLblThreads / 32) {
+    const int mg = lg * a.lists_per_cta + m;
+    const int jt = mg / G;
+    const int64_t list = (int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G);
+    const int L = kv_len_of(a.qv, si, jt);
+    const int k = list_k(a, si.t0 + jt, L);
+    const uint32_t lo = list_threshold(a.samples + list * a.sample_stride, L, k, shift, a.filter == 1, lane);
+    if (lane == 0) {
+      a.lo_key[list] = lo;
+      a.meta[list] = make_int2(L, k);
+    }
+  }
+}
+
+template <int R, int NL, bool FILT>
+__global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(TopkArgs a, const uint16_t* label,
                                                                   const int32_t* channels) {
+  // FILT: the filtered form, instantiated apart so that the row form keeps its registers
   __shared__ __align__(16) float qs[16][R];
   __shared__ int kvl[16];
   __shared__ int64_t srow[16];
@@ -155,10 +239,17 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
   const int G = a.qv.hq / a.kv.hkv;
   int nlists = si.n * G - lg * a.lists_per_cta;
   if (nlists > a.lists_per_cta) nlists = a.lists_per_cta;
-  if (nlists <= 0) return;
   const int tok0 = win * a.window;
   const int tok_end = min(tok0 + a.window, si.len);
-  if (tok_end <= tok0) return;
+  if (nlists <= 0 || tok_end <= tok0) {
+    // under the filter the kernels after this one read what the pre-pass wrote once this grid
+    // has completed, so every CTA waits for the pre-pass before it exits
+    if (FILT) pdl_wait();
+    return;
+  }
+  __shared__ float s_lof[16];              // filter: each list's threshold as a float
+  __shared__ int64_t s_list[16];           // filter: each list's index (t Hq + h)
+  __shared__ uint32_t s_pool[kLblThreads / 32][16][2];   // filter, many lists: each warp's pools
   for (int e = threadIdx.x; e < 16 * R; e += kLblThreads) {
     const int m = e / R, j = e - (e / R) * R;
     float v = 0.f;
@@ -184,6 +275,26 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
   }
   __syncthreads();
   pdl_launch_dependents();   // the selection may launch; it waits for this kernel's scores
+  if (FILT) {
+    pdl_wait();   // the pre-pass wrote the thresholds
+    if (threadIdx.x < 16) {
+      const int m = threadIdx.x;
+      float lf = CUDART_INF_F;
+      int64_t list = 0;
+      if (m < nlists) {
+        const int mg = lg * a.lists_per_cta + m;
+        const int jt = mg / G;
+        list = (int64_t)(si.t0 + jt) * a.qv.hq + g * G + (mg - jt * G);
+        const uint32_t lo = __ldcg(a.lo_key + list);
+        // keys above +inf's are positive NaNs, keys below -inf's negative ones
+        lf = lo >= 0xFF800000u ? CUDART_INF_F : (lo <= 0x007FFFFFu ? -CUDART_INF_F : key_score(lo));
+      }
+      s_lof[m] = lf;
+      s_list[m] = list;
+    }
+    for (int i = threadIdx.x; i < (kLblThreads / 32) * 16 * 2; i += kLblThreads) (&s_pool[0][0][0])[i] = 0u;
+    __syncthreads();
+  }
   // Each warp walks steps of kLblStep consecutive tokens (lane l takes tokens 32 u + l of the
   // step), the CTA's warps taking consecutive steps.  With pages of 4 tokens or more, a step's
   // tokens lie in at most 32 pages: lane l holds the page-table entry of the step's l-th page,
@@ -212,6 +323,15 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
       srr[m] = m < nlists ? srow[m] : 0;
       prr[m] = m < nlists ? prow[m] : 0;
     }
+  }
+  float lof[NR];          // NL > 0, filter: thresholds, lists and the warp's pools
+  int64_t lst[NR];
+  uint32_t pn[NR], pe[NR];
+#pragma unroll
+  for (int m = 0; m < NR; ++m) {
+    lof[m] = FILT && NL > 0 ? s_lof[m] : CUDART_INF_F;
+    lst[m] = FILT && NL > 0 ? s_list[m] : 0;
+    pn[m] = pe[m] = 0u;
   }
   const bool paged = a.kv.page_table != nullptr;
   const int shift = a.kv.page_shift;
@@ -257,7 +377,7 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int tok = st0 + 32 * u + lane;
-      if (row[u] == kInvalidRow) continue;
+      const bool valid = row[u] != kInvalidRow;
       // channel pairs (2i, 2i + 1) as packed fp32x2: one fma.rn.f32x2 per pair, the even
       // channels summed in the low lane and the odd ones in the high lane
       unsigned long long k2[R / 2];
@@ -276,7 +396,11 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
 #pragma unroll
           for (int j = 0; j < R / 2; ++j) acc = ffma2(qr[m][j], k2[j], acc);
           const float sc = f32x2_sum(acc);
-          if (tok < kvr[m]) {
+          if constexpr (FILT) {   // every lane takes part: the append is warp-collective
+            const bool cand = valid && tok < kvr[m] && !(sc < lof[m]);
+            warp_append(cand, sc, (uint32_t)tok, pn[m], pe[m], a.cand_cnt + lst[m], a.cand + lst[m] * kTopkCandCap,
+                        lane, kLblChunk);
+          } else if (valid && tok < kvr[m]) {
             a.scores[srr[m] + tok] = sc;
             if (sampled) a.samples[prr[m] + (tok >> a.sample_shift)] = sc;
           }
@@ -292,7 +416,18 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
             acc = ffma2(qq.y, k2[2 * j + 1], acc);
           }
           const float sc = f32x2_sum(acc);
-          if (tok < kvl[m]) {
+          if constexpr (FILT) {
+            uint32_t p0 = s_pool[warp][m][0], p1 = s_pool[warp][m][1];
+            const bool cand = valid && tok < kvl[m] && !(sc < s_lof[m]);
+            warp_append(cand, sc, (uint32_t)tok, p0, p1, a.cand_cnt + s_list[m], a.cand + s_list[m] * kTopkCandCap,
+                        lane, kLblChunk);
+            __syncwarp();
+            if (lane == 0) {
+              s_pool[warp][m][0] = p0;
+              s_pool[warp][m][1] = p1;
+            }
+            __syncwarp();
+          } else if (valid && tok < kvl[m]) {
             a.scores[srow[m] + tok] = sc;
             if (sampled) a.samples[prow[m] + (tok >> a.sample_shift)] = sc;
           }
@@ -300,6 +435,27 @@ __global__ void __launch_bounds__(kLblThreads) label_score_kernel(TopkArgs a, co
       }
     }
     pg = pg_next;
+  }
+  if (FILT && lane == 0) {
+    // the pools' unused slots become holes: an index no list has, which the selection skips
+    for (int m = 0; m < nlists; ++m) {
+      uint32_t p0, p1;
+      if constexpr (NL > 0) {
+        p0 = 0u;
+        p1 = 0u;
+#pragma unroll
+        for (int mm = 0; mm < NL; ++mm)
+          if (mm == m) {
+            p0 = pn[mm];
+            p1 = pe[mm];
+          }
+      } else {
+        p0 = s_pool[warp][m][0];
+        p1 = s_pool[warp][m][1];
+      }
+      uint2* buf = a.cand + s_list[m] * kTopkCandCap;
+      for (uint32_t slot = p0; slot < p1 && slot < (uint32_t)kTopkCandCap; ++slot) buf[slot] = make_uint2(0u, 0xFFFFFFFFu);
+    }
   }
 }
 
@@ -332,25 +488,45 @@ cudaError_t launch_label_build(const KvView& kv, const int32_t* channels, int r,
 }
 
 cudaError_t launch_topk_select_only(const TopkArgs& a, int num_lists, cudaStream_t stream);
+cudaError_t launch_topk_candidates(const TopkArgs& a, int num_lists, cudaStream_t stream);
 
 cudaError_t launch_label_topk(const TopkArgs& a, const uint16_t* label, const int32_t* channels, int r, int nwin,
                               int batch, int hkv, int num_lists, cudaStream_t stream) {
   dim3 grid(nwin, hkv * a.list_groups, batch);
   const bool few = a.lists_per_cta <= 4;   // the lists' queries fit in registers (r <= 16)
+  cudaError_t e = cudaSuccess;
+  if (a.filter) {   // the candidate filter's pre-pass: label-score samples and thresholds
+    const dim3 g0(hkv * a.list_groups, batch);
+    switch (r) {
+      case 8: label_prepass_kernel<8><<<g0, kLblThreads, 0, stream>>>(a); break;
+      case 16: label_prepass_kernel<16><<<g0, kLblThreads, 0, stream>>>(a); break;
+      case 32: label_prepass_kernel<32><<<g0, kLblThreads, 0, stream>>>(a); break;
+      default: return cudaErrorInvalidValue;
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // under the filter a programmatic dependent of the pre-pass, whose thresholds it waits for
+  auto score = [&](auto kernel) -> cudaError_t {
+    if (a.filter) return launch_dependent(kernel, grid, dim3(kLblThreads), 0, stream, a, label, channels);
+    kernel<<<grid, kLblThreads, 0, stream>>>(a, label, channels);
+    return cudaGetLastError();
+  };
+  const bool f = a.filter != 0;
   switch (r) {
     case 8:
-      if (few) label_score_kernel<8, 4><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
-      else label_score_kernel<8, 0><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
+      if (few) e = f ? score(label_score_kernel<8, 4, true>) : score(label_score_kernel<8, 4, false>);
+      else e = f ? score(label_score_kernel<8, 0, true>) : score(label_score_kernel<8, 0, false>);
       break;
     case 16:
-      if (few) label_score_kernel<16, 4><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
-      else label_score_kernel<16, 0><<<grid, kLblThreads, 0, stream>>>(a, label, channels);
+      if (few) e = f ? score(label_score_kernel<16, 4, true>) : score(label_score_kernel<16, 4, false>);
+      else e = f ? score(label_score_kernel<16, 0, true>) : score(label_score_kernel<16, 0, false>);
       break;
-    case 32: label_score_kernel<32, 0><<<grid, kLblThreads, 0, stream>>>(a, label, channels); break;
+    case 32: e = f ? score(label_score_kernel<32, 0, true>) : score(label_score_kernel<32, 0, false>); break;
     default: return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.filter) return launch_topk_candidates(a, num_lists, stream);
   return launch_topk_select_only(a, num_lists, stream);
 }
 

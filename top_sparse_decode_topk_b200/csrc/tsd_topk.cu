@@ -26,6 +26,7 @@
 #include "tsd_args.h"
 #include "tsd_common.cuh"
 #include "tsd_kvtile.cuh"
+#include "tsd_filter.cuh"
 #include "tsd_umma.cuh"
 
 namespace tsd {
@@ -481,55 +482,6 @@ __device__ __forceinline__ void list_len_k(const TopkArgs& a, int th, int& L, in
 // kernel needs zero only after this kernel has completed -- computes the group's thresholds
 // and leaves the counter zero.
 constexpr int kPpWarps = 8;
-constexpr int kThrMaxSamples = 2048;   // 64 per lane
-
-// Threshold key of one list from its ns sample scores (one warp): bit by bit from the top, the
-// r-th largest sample key with its low 16 bits cleared, r the expected count above the k-th
-// score plus 4 standard deviations plus 4 -- with overwhelming probability at least k of the
-// list's scores reach it.  Lists of at most kTopkCandCap tokens take every score (lo = 0); a
-// list the filter cannot serve (k = 0, k = L, too many expected candidates, or more samples than
-// the warp holds) gets lo = 0xFFFFFFFF, which only the largest NaN key reaches, and the
-// selection takes its other paths.
-__device__ uint32_t list_threshold(const float* samp, int L, int k, int shift, bool enabled, int lane) {
-  constexpr unsigned FULL = 0xFFFFFFFFu;
-  if (!(k > 0 && k < L && enabled)) return 0xFFFFFFFFu;
-  if (L <= kTopkCandCap / 2) return 0u;   // leaves room for the pools' holes
-  const int ns = (L + (1 << shift) - 1) >> shift;
-  const float mean = (float)ns * (float)k / (float)L;
-  const int r = (int)ceilf(mean + 4.f * sqrtf(mean) + 4.f);
-  if (!(ns <= kThrMaxSamples && r < ns && (int64_t)r * L <= (int64_t)kTopkCandCap * ns * 3 / 4)) return 0xFFFFFFFFu;
-  uint32_t key[kThrMaxSamples / 32];
-#pragma unroll
-  for (int i = 0; i < kThrMaxSamples / 32; ++i) {
-    const int j = 32 * i + lane;
-    key[i] = j < ns ? score_key(__ldcg(samp + j)) : 0u;
-  }
-  // 16 bits (sign, exponent, 7 mantissa bits): the threshold then sits at most 2^-7 of its
-  // value below the sample's r-th largest, which adds few candidates; eight partial counts keep
-  // the chains of dependent adds short
-  uint32_t prefix = 0u;
-  for (int bit = 31; bit >= 16; --bit) {
-    const uint32_t trial = prefix | (1u << bit);
-    int c8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-    for (int i = 0; i < kThrMaxSamples / 32; ++i) c8[i & 7] += key[i] >= trial;
-    int c = ((c8[0] + c8[1]) + (c8[2] + c8[3])) + ((c8[4] + c8[5]) + (c8[6] + c8[7]));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(FULL, c, o);
-    if (c >= r) prefix = trial;
-  }
-  return prefix;
-}
-
-// kept count k = min(k_t, L) of query token t with visible length L
-__device__ __forceinline__ int list_k(const TopkArgs& a, int t, int L) {
-  int kreq = a.k_max;
-  if (a.k_per_token != nullptr) {
-    kreq = __ldg(a.k_per_token + t);
-    kreq = kreq < 0 ? 0 : (kreq > a.k_max ? a.k_max : kreq);
-  }
-  return kreq < L ? kreq : L;
-}
 
 __global__ void __launch_bounds__(32 * kPpWarps, 2) topk_prepass_kernel(TopkArgs a) {
   const int g = blockIdx.y / a.list_groups, lg = blockIdx.y % a.list_groups;
@@ -1221,6 +1173,35 @@ __device__ void rescore_row(const TopkArgs& a, int th, int b, int L, float* row,
 // The selection over a list's score row: every visible token (k = L) or none (k = 0), the
 // sampled fast path, else the multi-pass radix path.  Under the candidate filter the scoring
 // kernel wrote no row, so the list's row is recomputed first.
+// The same for the label indexer: the list's label scores, sum over its kv head's label channels
+// of q[c] * label[row][c] in fp32, one thread per token.
+__device__ void rescore_label_row(const TopkArgs& a, int th, int b, int L, float* row, float* qs) {
+  const int h = th % a.qv.hq;
+  const int g = h / (a.qv.hq / a.kv.hkv);
+  const int R = a.label_r;
+  if (threadIdx.x < R) {
+    int c = __ldg(a.channels + (int64_t)g * R + threadIdx.x);
+    if (c < 0 || c >= kHeadDim) c = 0;   // the scoring kernel flags it
+    const int64_t qe = (int64_t)th * kHeadDim + c;
+    qs[threadIdx.x] = a.qv.q_f32 ? __ldg(static_cast<const float*>(a.qv.q) + qe)
+                                 : __uint_as_float((uint32_t)__ldg(static_cast<const uint16_t*>(a.qv.q) + qe) << 16);
+  }
+  __syncthreads();
+  for (int tok = threadIdx.x; tok < L; tok += kSelectThreads) {
+    const uint32_t r = kv_row(a.kv, b, g, tok);
+    float s = 0.f;
+    if (r != kInvalidRow) {
+      const uint16_t* lr = a.label + (int64_t)r * R;
+      for (int c = 0; c < R; ++c) s = fmaf(qs[c], __uint_as_float((uint32_t)__ldg(lr + c) << 16), s);
+    } else {
+      flag_status(a.status, TSD_DEV_BAD_PAGE);
+    }
+    row[tok] = s;
+  }
+  __threadfence();   // the row paths read it back through L2
+  __syncthreads();
+}
+
 __device__ void select_rows(SelectSmem& S, const TopkArgs& a, int th, int b, int L, int k) {
   int32_t* out = a.out_idx + (int64_t)th * a.k_max;
   float* osc = a.out_scores != nullptr ? a.out_scores + (int64_t)th * a.k_max : nullptr;
@@ -1236,7 +1217,8 @@ __device__ void select_rows(SelectSmem& S, const TopkArgs& a, int th, int b, int
     __shared__ float s_q[kHeadDim];
     int L2, k2;
     if (b < 0) list_len_k(a, th, b, L2, k2);   // the list's sequence
-    rescore_row(a, th, b, L, a.scores + (int64_t)th * a.score_stride, s_q);
+    if (a.label != nullptr) rescore_label_row(a, th, b, L, a.scores + (int64_t)th * a.score_stride, s_q);
+    else rescore_row(a, th, b, L, a.scores + (int64_t)th * a.score_stride, s_q);
   }
   if (L >= kFastMinL &&
       select_fast(S, row, a.samples + (int64_t)th * a.sample_stride, a.sample_shift, L, k, out, osc, a.k_max))
@@ -1417,6 +1399,26 @@ static bool score_on_tcgen05() {
   return e != nullptr && strcmp(e, "tcgen05") == 0;
 }
 
+// The filtered forms' selection (exact and label indexers): the candidate kernel, then the queue
+// of lists it could not serve, each a programmatic dependent of the kernel before.
+cudaError_t launch_topk_candidates(const TopkArgs& a, int num_lists, cudaStream_t stream) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e =
+        cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SelectSmem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  cudaError_t e;
+  if (num_lists <= a.queue_ctas)   // at most two lists per SM: one wave of 1024-thread CTAs
+    e = launch_dependent(topk_cand_kernel<1024>, dim3(num_lists), dim3(1024), 0, stream, a);
+  else
+    e = launch_dependent(topk_cand_kernel<256>, dim3(num_lists), dim3(256), 0, stream, a);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(topk_select_kernel, dim3((unsigned)a.queue_ctas), dim3(kSelectThreads), sizeof(SelectSmem),
+                          stream, a, 1);
+}
+
 cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int batch, int hkv, int num_lists,
                         cudaStream_t stream) {
   static bool configured = false;
@@ -1463,14 +1465,7 @@ cudaError_t launch_topk(const TopkArgs& a, const KvMaps& maps, int nwin, int bat
   if (e != cudaSuccess) return e;
   if (!a.filter)
     return launch_dependent(topk_select_kernel, dim3(num_lists), dim3(kSelectThreads), sizeof(SelectSmem), stream, a, 0);
-  // the candidate path, then the queue of lists it could not serve
-  if (num_lists <= a.queue_ctas)   // at most two lists per SM: one wave of 1024-thread CTAs
-    e = launch_dependent(topk_cand_kernel<1024>, dim3(num_lists), dim3(1024), 0, stream, a);
-  else
-    e = launch_dependent(topk_cand_kernel<256>, dim3(num_lists), dim3(256), 0, stream, a);
-  if (e != cudaSuccess) return e;
-  return launch_dependent(topk_select_kernel, dim3((unsigned)a.queue_ctas), dim3(kSelectThreads), sizeof(SelectSmem),
-                          stream, a, 1);
+  return launch_topk_candidates(a, num_lists, stream);
 }
 
 // The selection alone, over scores another kernel wrote into the workspace (the label indexer).
