@@ -767,10 +767,8 @@ tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k,
   a.sample_stride = lay.sample_stride;
   a.sample_shift = lay.sample_shift;
   // The candidate filter runs here only when TSD_TOPK_FILTER forces it ("1" or "rescore"): on
-  // the ragged batch at 50x it measured slower than the row form (label top-k 1798 against
-  // 1209 us), its per-warp candidate pools refilling with a global atomic every 8 candidates
-  // of each of 16 lists.  The label scores are fp32 sums over bf16 label rows whatever the
-  // query dtype.
+  // the ragged batch at 50x it measured slower than the row form (label top-k 1779 against
+  // 1200 us).  The label scores are fp32 sums over bf16 label rows whatever the query dtype.
   a.filter = filter_mode() > kFilterOff ? topk_filter_choice(sh, false, false, k_max) : 0;
   if (a.filter) a.sample_shift = lay.sample_shift + 1;
   a.cand_cnt = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 256);

@@ -148,10 +148,35 @@ __global__ void label_build_kernel(KvView kv, const int32_t* channels, int r, in
 // label_prepass_kernel scores every 2^sample_shift-th token of every list on the label channels
 // and turns each list's sample into a threshold; label_score_kernel then appends the scores that
 // reach it instead of writing score rows, and the exact indexer's candidate kernel and queue
-// pass select from there.  A warp appends the candidates of one list and one token step with a
-// ballot; its slots come from a pool of kLblChunk that lane 0 refills with one atomic on the
-// list's counter.  Unused pool slots become holes (index 0xFFFFFFFF) when the CTA ends.
-constexpr uint32_t kLblChunk = 8;
+// pass select from there.  A warp stages the candidates of one list and one token step in the
+// CTA's shared-memory buffer with a ballot and one shared atomic; when the CTA ends, one global
+// atomic per list reserves the list's range and the CTA copies its candidates out.  Candidates
+// that find the buffer full go straight to the list's buffer.
+constexpr uint32_t kLblStage = 4096;   // staged candidates per CTA (32 KB)
+constexpr uint32_t kLblStageHole = 0xFFFFFFFFu;
+
+// Warp-collective: lanes with `cand` stage (key(sc), tok | m << 24) for list m.
+__device__ __forceinline__ void stage_append(bool cand, float sc, uint32_t tok, int m, uint2* st, uint32_t* nst,
+                                             uint32_t* lcnt, uint32_t* gcnt, uint2* gbuf, int lane) {
+  const uint32_t bal = __ballot_sync(0xFFFFFFFFu, cand);
+  if (bal == 0u) return;
+  const uint32_t n = __popc(bal);
+  uint32_t base = 0u;
+  if (lane == 0) base = atomicAdd(nst, n);
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  const uint32_t i = __popc(bal & ((1u << lane) - 1u));
+  if (base + n <= kLblStage) {
+    if (cand) st[base + i] = make_uint2(score_key(sc), tok | ((uint32_t)m << 24));
+    if (lane == 0) atomicAdd(lcnt + m, n);
+    return;
+  }
+  // the buffer is full: the slots this call took inside it become holes, the candidates go out
+  if (cand && base + i < kLblStage) st[base + i] = make_uint2(0u, kLblStageHole);
+  uint32_t g = 0u;
+  if (lane == 0) g = atomicAdd(gcnt, n);
+  g = __shfl_sync(0xFFFFFFFFu, g, 0);
+  if (cand && g + i < (uint32_t)kTopkCandCap) gbuf[g + i] = make_uint2(score_key(sc), tok);
+}
 
 // Grid (Hkv x list groups, batch), kLblThreads threads: thread i scores samples i, i + 256, ...
 // of the group's lists, then warp w makes the thresholds of lists w, w + 8, ...
@@ -224,8 +249,14 @@ __global__ void __launch_bounds__(kLblThreads) label_prepass_kernel(TopkArgs a) 
   }
 }
 
+// resident CTAs per SM: the row form's counts as measured (r = 8 with many lists in 64 registers,
+// r = 16 with many lists in 80, the rest in 128); the filtered form, with its 34 KB of staged
+// candidates, two
+constexpr int label_score_min_ctas(int R, int NL, bool filt) {
+  return filt ? 2 : (NL == 0 && R == 8 ? 4 : (NL == 0 && R == 16 ? 3 : 2));
+}
 template <int R, int NL, bool FILT>
-__global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(TopkArgs a, const uint16_t* label,
+__global__ void __launch_bounds__(kLblThreads, label_score_min_ctas(R, NL, FILT)) label_score_kernel(TopkArgs a, const uint16_t* label,
                                                                   const int32_t* channels) {
   // FILT: the filtered form, instantiated apart so that the row form keeps its registers
   __shared__ __align__(16) float qs[16][R];
@@ -249,7 +280,10 @@ __global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(
   }
   __shared__ float s_lof[16];              // filter: each list's threshold as a float
   __shared__ int64_t s_list[16];           // filter: each list's index (t Hq + h)
-  __shared__ uint32_t s_pool[kLblThreads / 32][16][2];   // filter, many lists: each warp's pools
+  __shared__ uint2 s_stage[kLblStage];     // filter: the CTA's staged candidates
+  __shared__ uint32_t s_nst;               // filter: staged slots taken
+  __shared__ uint32_t s_lcnt[16];          // filter: staged candidates per list, then a running index
+  __shared__ uint32_t s_lbase[16];         // filter: each list's reserved range
   for (int e = threadIdx.x; e < 16 * R; e += kLblThreads) {
     const int m = e / R, j = e - (e / R) * R;
     float v = 0.f;
@@ -291,8 +325,9 @@ __global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(
       }
       s_lof[m] = lf;
       s_list[m] = list;
+      s_lcnt[m] = 0u;
     }
-    for (int i = threadIdx.x; i < (kLblThreads / 32) * 16 * 2; i += kLblThreads) (&s_pool[0][0][0])[i] = 0u;
+    if (threadIdx.x == 0) s_nst = 0u;
     __syncthreads();
   }
   // Each warp walks steps of kLblStep consecutive tokens (lane l takes tokens 32 u + l of the
@@ -324,15 +359,9 @@ __global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(
       prr[m] = m < nlists ? prow[m] : 0;
     }
   }
-  float lof[NR];          // NL > 0, filter: thresholds, lists and the warp's pools
-  int64_t lst[NR];
-  uint32_t pn[NR], pe[NR];
+  float lof[NR];          // NL > 0, filter: the thresholds
 #pragma unroll
-  for (int m = 0; m < NR; ++m) {
-    lof[m] = FILT && NL > 0 ? s_lof[m] : CUDART_INF_F;
-    lst[m] = FILT && NL > 0 ? s_list[m] : 0;
-    pn[m] = pe[m] = 0u;
-  }
+  for (int m = 0; m < NR; ++m) lof[m] = FILT && NL > 0 ? s_lof[m] : CUDART_INF_F;
   const bool paged = a.kv.page_table != nullptr;
   const int shift = a.kv.page_shift;
   const int pmask = (1 << shift) - 1;
@@ -378,6 +407,7 @@ __global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(
     for (int u = 0; u < U; ++u) {
       const int tok = st0 + 32 * u + lane;
       const bool valid = row[u] != kInvalidRow;
+      if (!FILT && !valid) continue;   // the filtered form's appends are warp-collective: no early out
       // channel pairs (2i, 2i + 1) as packed fp32x2: one fma.rn.f32x2 per pair, the even
       // channels summed in the low lane and the odd ones in the high lane
       unsigned long long k2[R / 2];
@@ -398,9 +428,9 @@ __global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(
           const float sc = f32x2_sum(acc);
           if constexpr (FILT) {   // every lane takes part: the append is warp-collective
             const bool cand = valid && tok < kvr[m] && !(sc < lof[m]);
-            warp_append(cand, sc, (uint32_t)tok, pn[m], pe[m], a.cand_cnt + lst[m], a.cand + lst[m] * kTopkCandCap,
-                        lane, kLblChunk);
-          } else if (valid && tok < kvr[m]) {
+            stage_append(cand, sc, (uint32_t)tok, m, s_stage, &s_nst, s_lcnt, a.cand_cnt + s_list[m],
+                         a.cand + s_list[m] * kTopkCandCap, lane);
+          } else if (tok < kvr[m]) {   // the row form: invalid rows left above
             a.scores[srr[m] + tok] = sc;
             if (sampled) a.samples[prr[m] + (tok >> a.sample_shift)] = sc;
           }
@@ -417,17 +447,10 @@ __global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(
           }
           const float sc = f32x2_sum(acc);
           if constexpr (FILT) {
-            uint32_t p0 = s_pool[warp][m][0], p1 = s_pool[warp][m][1];
             const bool cand = valid && tok < kvl[m] && !(sc < s_lof[m]);
-            warp_append(cand, sc, (uint32_t)tok, p0, p1, a.cand_cnt + s_list[m], a.cand + s_list[m] * kTopkCandCap,
-                        lane, kLblChunk);
-            __syncwarp();
-            if (lane == 0) {
-              s_pool[warp][m][0] = p0;
-              s_pool[warp][m][1] = p1;
-            }
-            __syncwarp();
-          } else if (valid && tok < kvl[m]) {
+            stage_append(cand, sc, (uint32_t)tok, m, s_stage, &s_nst, s_lcnt, a.cand_cnt + s_list[m],
+                         a.cand + s_list[m] * kTopkCandCap, lane);
+          } else if (tok < kvl[m]) {
             a.scores[srow[m] + tok] = sc;
             if (sampled) a.samples[prow[m] + (tok >> a.sample_shift)] = sc;
           }
@@ -436,25 +459,22 @@ __global__ void __launch_bounds__(kLblThreads, FILT ? 2 : 1) label_score_kernel(
     }
     pg = pg_next;
   }
-  if (FILT && lane == 0) {
-    // the pools' unused slots become holes: an index no list has, which the selection skips
-    for (int m = 0; m < nlists; ++m) {
-      uint32_t p0, p1;
-      if constexpr (NL > 0) {
-        p0 = 0u;
-        p1 = 0u;
-#pragma unroll
-        for (int mm = 0; mm < NL; ++mm)
-          if (mm == m) {
-            p0 = pn[mm];
-            p1 = pe[mm];
-          }
-      } else {
-        p0 = s_pool[warp][m][0];
-        p1 = s_pool[warp][m][1];
-      }
-      uint2* buf = a.cand + s_list[m] * kTopkCandCap;
-      for (uint32_t slot = p0; slot < p1 && slot < (uint32_t)kTopkCandCap; ++slot) buf[slot] = make_uint2(0u, 0xFFFFFFFFu);
+  if (FILT) {
+    // one global atomic per list reserves its staged candidates' range; the CTA copies them out
+    __syncthreads();
+    if (threadIdx.x < nlists) {
+      const uint32_t c = s_lcnt[threadIdx.x];
+      s_lbase[threadIdx.x] = c != 0u ? atomicAdd(a.cand_cnt + s_list[threadIdx.x], c) : 0u;
+      s_lcnt[threadIdx.x] = 0u;
+    }
+    __syncthreads();
+    const uint32_t nst = s_nst < kLblStage ? s_nst : kLblStage;
+    for (uint32_t e = threadIdx.x; e < nst; e += kLblThreads) {
+      const uint2 v = s_stage[e];
+      if (v.y == kLblStageHole) continue;
+      const int m = (int)(v.y >> 24);
+      const uint32_t pos = s_lbase[m] + atomicAdd(s_lcnt + m, 1u);
+      if (pos < (uint32_t)kTopkCandCap) a.cand[s_list[m] * kTopkCandCap + pos] = make_uint2(v.x, v.y & 0xFFFFFFu);
     }
   }
 }
