@@ -343,3 +343,15 @@ def test_topk_select_plan_choice(lib, monkeypatch):
                                     ctypes.byref(n)) == tsd.TSD_ERR_INVALID_ARGUMENT
     bad = make_cache(head_dim=64)
     assert lib.tsd_topk_select_plan(ctypes.byref(bad), ctypes.byref(q), 655, *args) == tsd.TSD_ERR_UNSUPPORTED
+
+
+def test_topk_filter_not_taken_past_the_candidate_bitmap(lib, monkeypatch):
+    """Lists longer than the candidate selection's 128K-token bitmaps would all fall back to the
+    recomputed rows, so a call with a longer max_seq_len takes the form over score rows, even
+    with the filter forced."""
+    monkeypatch.setenv("TSD_TOPK_FILTER", "1")
+    f, n = ctypes.c_int32(), ctypes.c_int32()
+    c = make_cache(batch=8, max_pages=16384, num_pages=8 * 16384, max_seq_len=262144)
+    q = make_queries()
+    assert lib.tsd_topk_select_plan(ctypes.byref(c), ctypes.byref(q), 655, ctypes.byref(f), ctypes.byref(n)) == tsd.TSD_OK
+    assert (f.value, n.value) == (0, 2)

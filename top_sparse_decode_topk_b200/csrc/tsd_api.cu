@@ -334,7 +334,7 @@ static int topk_filter_choice(const Shapes& sh, bool q_f32, bool with_scores, in
   const TopkLayout lay = topk_layout(sh);
   const int fm = filter_mode();
   const double row_bytes = (double)sh.tokens * sh.hq * (double)lay.score_stride * sizeof(float);
-  const bool can = !q_f32 && !with_scores && !score_on_tcgen05_host();
+  const bool can = !q_f32 && !with_scores && !score_on_tcgen05_host() && sh.max_seq_len <= kTopkCandMaxLen;
   if (fm == kFilterRescore) return can ? 2 : 0;
   if (fm == kFilterOn) return can && filter_fits(k_max, lay.sample_shift + 1) ? 1 : 0;
   if (fm == kFilterAuto)

@@ -940,7 +940,7 @@ __device__ bool select_fast(SelectSmem& S, const float* row, const float* samp, 
 // time, give the tie ranks (the need_eq lowest-index ties are kept) and the output ranks, and
 // the kept indices are written in ascending order.  A list with fewer than k valid candidates, or
 // more than fit, goes into the queue that topk_select_kernel works off over recomputed rows.
-constexpr int kCandBitmapTokens = 131072;   // longest list the bitmaps cover
+constexpr int kCandBitmapTokens = kTopkCandMaxLen;   // longest list the bitmaps cover
 constexpr int kCsUnroll = 8;                  // candidate loads in flight per thread
 template <int NT>
 struct CandSmem {
