@@ -13,6 +13,7 @@
 #include "tsd.h"
 #include "tsd_common.cuh"
 #include "tsd_plan.h"
+#include "tsd_filter.cuh"
 
 #include "tsd_args.h"
 #include "tsd_kvtile.cuh"
@@ -188,6 +189,18 @@ tsd_status tsd_workspace_init(void* ws, size_t bytes, tsd_stream_t stream) {
   return cuda_status(cudaMemsetAsync(ws, 0, bytes, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static int topk_filter_choice(const Shapes& sh, bool q_f32, bool with_scores, int32_t k_max);
+// The top-k workspace layout, with the candidate filter's regions (thresholds, candidates,
+// (kv_len, k), queue) only when `filter`: without them those offsets all equal `total`.
+static TopkLayout topk_layout_for(const Shapes& sh, bool filter) {
+  TopkLayout l = topk_layout(sh);
+  if (!filter) l.off_cand = l.off_meta = l.off_queue = l.total = l.off_lo;
+  return l;
+}
+// Whether a top-k workspace for these shapes holds the candidate filter's regions: when the
+// filter could run for some call on them (either indexer; the query dtype aside).
+static bool topk_filter_space(const Shapes& sh, int32_t k_max) { return topk_filter_choice(sh, false, false, k_max) != 0; }
+
 size_t tsd_topk_workspace_size(const tsd_kv_cache* cache, const tsd_queries* queries, int32_t k_max) {
   KvView kv; QView qv; Shapes sh;
   if (k_max < 1) return 0;
@@ -201,7 +214,7 @@ size_t tsd_topk_workspace_size(const tsd_kv_cache* cache, const tsd_queries* que
   if (c.layout == TSD_LAYOUT_PAGED && c.page_table == nullptr) c.page_table = reinterpret_cast<const int32_t*>(dummy);
   if (q.q == nullptr) q.q = dummy;
   if (check_inputs(&c, &q, &kv, &qv, &sh) != TSD_OK) return 0;
-  return topk_layout(sh).total;
+  return topk_layout_for(sh, topk_filter_space(sh, k_max)).total;
 }
 
 // SM count of the current device: the sparse plan sizes its grid to the resident CTAs.  A
@@ -362,7 +375,7 @@ static tsd_status topk_select_impl(const tsd_kv_cache* cache, const tsd_queries*
   if (st != TSD_OK) return st;
   if (k_max < 1 || out_idx == nullptr || ws == nullptr) return TSD_ERR_INVALID_ARGUMENT;
   if (((uintptr_t)ws & 255) != 0) return TSD_ERR_INVALID_ARGUMENT;
-  const TopkLayout lay = topk_layout(sh);
+  const TopkLayout lay = topk_layout_for(sh, topk_filter_space(sh, k_max));
   if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
   TopkArgs a;
   memset(&a, 0, sizeof(a));
@@ -514,7 +527,7 @@ static bool step_layout(const tsd_kv_cache* cache, const tsd_queries* queries, i
                         StepLayout* L) {
   Shapes sh;
   if (k_max < 1 || k_max > kMaxSparseK || sizes_for(cache, queries, &sh) != TSD_OK) return false;
-  const size_t topk = topk_layout(sh).total;
+  const size_t topk = topk_layout_for(sh, topk_filter_space(sh, k_max)).total;
   const size_t dec = decode_layout(sh, sparse_plan(sh, k_max).nsplit).total;
   L->shared = align256(topk > dec ? topk : dec);
   L->off_idx = L->shared;
@@ -751,7 +764,7 @@ tsd_status tsd_topk_select_label(const tsd_kv_cache* cache, const void* label_k,
   if (k_max < 1 || out_idx == nullptr || ws == nullptr || label_k == nullptr || channels == nullptr)
     return TSD_ERR_INVALID_ARGUMENT;
   if (((uintptr_t)ws & 255) != 0 || ((uintptr_t)label_k & 15) != 0) return TSD_ERR_INVALID_ARGUMENT;
-  const TopkLayout lay = topk_layout(sh);
+  const TopkLayout lay = topk_layout_for(sh, topk_filter_space(sh, k_max));
   if (ws_bytes < lay.total) return TSD_ERR_WORKSPACE_TOO_SMALL;
   TopkArgs a;
   memset(&a, 0, sizeof(a));

@@ -13,6 +13,10 @@ namespace tsd {
 
 constexpr int kThrMaxSamples = 2048;   // 64 per lane
 
+// Longest list the candidate selection covers (its bitmaps of the list's tokens): calls whose
+// max_seq_len is longer take the unfiltered form.
+constexpr int kTopkCandMaxLen = 131072;
+
 // Threshold key of one list from its ns sample scores (one warp): bit by bit from the top, the
 // r-th largest sample key with its low 16 bits cleared, r the expected count above the k-th
 // score plus 4 standard deviations plus 4 -- with overwhelming probability at least k of the

@@ -220,9 +220,6 @@ constexpr int64_t kMaxSample = 4096;
 // Candidates of the exact indexer (tsd_topk_select): the scoring kernel also appends every
 // (key, index) at or above a list's sampled threshold, at most kTopkCandCap per list.
 constexpr int kTopkCandCap = 8192;
-// Longest list the candidate selection covers (its bitmaps of the list's tokens): calls whose
-// max_seq_len is longer take the unfiltered form.
-constexpr int kTopkCandMaxLen = 131072;
 
 struct TopkLayout {
   size_t off_scores;
