@@ -1023,7 +1023,7 @@ __global__ void __launch_bounds__(NT) topk_cand_kernel(TopkArgs a) {
     return;
   }
   const uint2* cand = a.cand + (int64_t)th * kTopkCandCap;
-  // round 1 (top 11 key bits), counting the valid candidates on the way
+  // the first radix round (top 11 key bits), counting the valid candidates on the way
   int mine = 0;
   for_candidates<NT>(cand, slots, L, lo, [&](uint32_t key, uint32_t) {
     atomicAdd(&S.hist[0][key >> 21], 1u);
