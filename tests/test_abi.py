@@ -355,3 +355,25 @@ def test_topk_filter_not_taken_past_the_candidate_bitmap(lib, monkeypatch):
     q = make_queries()
     assert lib.tsd_topk_select_plan(ctypes.byref(c), ctypes.byref(q), 655, ctypes.byref(f), ctypes.byref(n)) == tsd.TSD_OK
     assert (f.value, n.value) == (0, 2)
+
+
+def test_topk_workspace_holds_the_filter_regions_only_when_the_filter_can_run(lib, monkeypatch):
+    """The exact indexer's workspace grows by the candidate filter's regions -- a threshold key,
+    8192 (key, index) candidate slots, a (kv_len, k) pair and a queue entry per list -- only
+    for shapes and k where the filter can run: the ragged shape at k = 2622 (filtered) against
+    k = 20000 (too many candidates for the buffer); the scores and samples are the same size."""
+    monkeypatch.delenv("TSD_TOPK_FILTER", raising=False)
+    monkeypatch.delenv("TSD_SCORE_KERNEL", raising=False)
+    rc = make_cache(batch=32, max_pages=8192, num_pages=32 * 8192, max_seq_len=131072)
+    rq = make_queries(tokens=128, q_indptr=FAKE + 0x800000, max_tokens=4)
+    with_filter = lib.tsd_topk_workspace_size(ctypes.byref(rc), ctypes.byref(rq), 2622)
+    without = lib.tsd_topk_workspace_size(ctypes.byref(rc), ctypes.byref(rq), 20000)
+    lists = 128 * 32
+    a256 = lambda n: (n + 255) // 256 * 256
+    assert with_filter - without == a256(lists * 4) + a256(lists * 8192 * 8) + a256(lists * 8) + a256(lists * 4)
+    c, q = make_cache(), make_queries()   # 256 lists of 32K tokens: rows stay in L2, no filter
+    monkeypatch.setenv("TSD_TOPK_FILTER", "1")
+    forced = lib.tsd_topk_workspace_size(ctypes.byref(c), ctypes.byref(q), 655)
+    monkeypatch.delenv("TSD_TOPK_FILTER")
+    assert forced - lib.tsd_topk_workspace_size(ctypes.byref(c), ctypes.byref(q), 655) == \
+        a256(256 * 4) + a256(256 * 8192 * 8) + a256(256 * 8) + a256(256 * 4)
